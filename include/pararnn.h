@@ -1,0 +1,178 @@
+/*
+ * pararnn.h -- C ABI of the B200 (sm_100a) library that evaluates nonlinear RNNs
+ * over the whole sequence at once with Newton (DEER) or quasi-Newton iterations.
+ *
+ * Method, as the pages describe it:
+ *   - "Parallelizing non-linear sequential models over the sequence length"
+ *     (Lim et al.), summary, "Approach": the recurrence is restated as a fixed-point
+ *     problem solved by Newton's method; each iteration linearises the model with its
+ *     Jacobians and solves the resulting linear recurrence with a parallel prefix scan.
+ *   - "ParaRNN: Unlocking Parallel Training of Nonlinear RNNs for Large Language
+ *     Models", abstract: the whole sequence is one system of equations solved with
+ *     Newton's iterations and parallel reductions; GRU and LSTM adaptations.
+ *   - "Towards Scalable and Stable Parallelization of Nonlinear RNNs", Abstract:
+ *     quasi-Newton (diagonal Jacobian) variants converge comparably and cost less.
+ *   - "Para-Seq" README, "Main features": diagonal ParaGRU, CIFG/peephole ParaLSTM with
+ *     2x2 block scans, vanilla tanh RNN, dense/diagonal/2x2-block associative scans
+ *     and reverse adjoint scans; "Quick example": batch-first tensors.
+ *
+ * Conventions for every entry point
+ *   - All tensor pointers are DEVICE pointers owned by the caller, row-major,
+ *     batch-first, contiguous.  The library never frees or keeps them.
+ *   - Calls are asynchronous and ordered on the context's stream; outputs are ready
+ *     when that stream reaches the point of the call.  Device-side conditions
+ *     (non-finite values, a bounded wait that ran out) are reported through
+ *     pararnn_get_status.
+ *   - Return value: PARARNN_OK (0) or a negative PARARNN_E* code; on an error
+ *     nothing was enqueued.
+ *   - Vector paths need 16-byte aligned base pointers (PARARNN_EALIGN otherwise).
+ *   - A context owns only its device workspace (iteration bookkeeping, chunk
+ *     aggregates for the scan's look-back); it grows on demand with cudaMalloc
+ *     and is released by pararnn_destroy.  A context is not thread-safe; use one
+ *     per host thread or stream.
+ *
+ * Shapes (G = 3 gates for GRU and LSTM, 1 for the tanh RNN; n = H for the tanh RNN):
+ *   x      [B, T, in]          W   [G*H, in] (row g*H + u feeds gate g of unit u)
+ *   xproj  [B, T, G, H] fp32   bias [G*H]
+ *   GRU    state [B, T, H]      h0 [B, H]      a [3, H] = (a_z, a_r, a_c)
+ *   LSTM   state [B, T, H, 2] as (c, h) pairs; h0 [B, H, 2]; a [3, H] = (a_f, a_g, a_o);
+ *          peep [2, H] = (w_f, w_o)
+ *   tanh   state [B, T, n]      h0 [B, n]      A [n, n] (A[i][j] multiplies h_j)
+ * Output element t of the state is h_{t+1}; h0 is the state before the first step.
+ */
+#ifndef PARARNN_H
+#define PARARNN_H
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- status codes ---------------------------------------------------------------- */
+#define PARARNN_OK 0
+#define PARARNN_NOTCONVERGED 1   /* reported by get_status: the cap was reached with delta >= tol */
+#define PARARNN_EINVAL (-1)      /* null pointer, bad enum or bad shape */
+#define PARARNN_EALIGN (-2)      /* a pointer is not 16-byte aligned */
+#define PARARNN_ECUDA (-3)       /* a CUDA call or launch failed */
+#define PARARNN_ENOMEM (-4)      /* workspace allocation failed */
+#define PARARNN_ENONFINITE (-5)  /* device: an iterate or residual became NaN or Inf */
+#define PARARNN_ETIMEOUT (-6)    /* device: a bounded wait (look-back, grid barrier) ran out */
+#define PARARNN_EUNSUPPORTED (-7) /* valid request outside what this build implements */
+
+typedef enum {
+    PARARNN_GRU_DIAG = 0,        /* diagonal ParaGRU, diagonal Jacobian */
+    PARARNN_LSTM_CIFG_PEEP = 1,  /* CIFG + peephole ParaLSTM, 2x2 Jacobian per unit */
+    PARARNN_RNN_TANH_DENSE = 2,  /* vanilla tanh RNN, full n x n Jacobian (DEER) */
+    PARARNN_RNN_TANH_QUASI = 3   /* vanilla tanh RNN, diagonal of the Jacobian (quasi-DEER) */
+} pararnn_cell;
+
+typedef enum { PARARNN_SCAN_DIAG = 0, PARARNN_SCAN_BLOCK2 = 1, PARARNN_SCAN_DENSE = 2 } pararnn_scan_kind;
+
+typedef enum { PARARNN_F32 = 0, PARARNN_BF16 = 1 } pararnn_dtype;
+
+typedef struct pararnn_ctx pararnn_ctx;
+
+/* Cell description and parameters (device pointers).  Unused fields may be NULL.
+ * x/W/bias are read only when xproj is NULL ("fused projection", in <= 8): the
+ * projection W x_t + bias is then recomputed inside the solver at every iteration
+ * instead of being stored, which is cheaper for narrow inputs. */
+typedef struct {
+    int cell;              /* pararnn_cell */
+    int B, T, H;           /* batch, steps, units (tanh RNN: state size n) */
+    int in;                /* input width, fused projection only */
+    const float *a;        /* [3, H]  GRU / LSTM recurrent diagonals */
+    const float *peep;     /* [2, H]  LSTM peepholes */
+    const float *A;        /* [n, n]  tanh RNN recurrent matrix */
+    const float *x;        /* [B, T, in] fp32 (fused projection) */
+    const float *W;        /* [G*H, in] fp32 (fused projection) */
+    const float *bias;     /* [G*H] fp32 or NULL (fused projection) */
+} pararnn_params;
+
+/* Create a context on `device` that enqueues on `cuda_stream` (a cudaStream_t, or
+ * NULL for the legacy default stream).  *ctx is NULL on failure. */
+int pararnn_create(pararnn_ctx **ctx, int device, void *cuda_stream);
+/* Synchronise the context's stream, free its workspace and the context. */
+int pararnn_destroy(pararnn_ctx *ctx);
+/* Change the stream later calls enqueue on. */
+int pararnn_set_stream(pararnn_ctx *ctx, void *cuda_stream);
+
+/* Input projection, the method's one dense contraction:
+ *   xproj[m, n] = sum_k x[m, k] * W[n, k] + bias[n]      (M = B*T, N = G*H, K = in)
+ * x [M, K] and W [N, K] are both bf16 (x_dtype = PARARNN_BF16, tcgen05 tensor cores,
+ * fp32 accumulation) or both fp32 (PARARNN_F32, CUDA cores); bias fp32 [N] or NULL;
+ * xproj fp32 [M, N].  Implied by the cells of the pages: the input term W x_t does
+ * not depend on the state, so it is computed once per forward pass.
+ * bf16 needs K % 64 == 0 and N % 16 == 0 ... see the EINVAL conditions in the
+ * implementation notes below; any M is accepted. */
+int pararnn_input_proj(pararnn_ctx *ctx, const void *x, int x_dtype, const void *W,
+                       const float *bias, float *xproj, int M, int K, int N);
+
+/* Newton (DEER) / quasi-Newton forward solve of the whole sequence
+ * ("Parallelizing non-linear sequential models over the sequence length", Approach;
+ * quasi: "Towards Scalable and Stable Parallelization of Nonlinear RNNs", Abstract).
+ * From the initial guess h^(0)_t = 0 (t >= 1), each iteration k evaluates the cell and
+ * its Jacobian at every step from h^(k)_{t-1}, solves h^(k+1)_t = J_t h^(k+1)_{t-1} + b_t,
+ * b_t = f_t - J_t h^(k)_{t-1}, and stops after the first iteration whose
+ *   delta_k = max over all state elements |h^(k+1) - h^(k)|
+ * is < tol (strict; tol <= 0 runs exactly max_iters iterations), or at max_iters.
+ *   xproj      [B, T, G, H] projected inputs (bias included), or NULL to use p->x/W/bias
+ *   h0         initial state, or NULL for zeros
+ *   h_out      [B, T, H] (LSTM [B, T, H, 2]; tanh [B, T, n]) receives the final iterate
+ *   iters_out  device int: number of Newton updates applied (counting the one whose
+ *              delta fell below tol); max_iters = 0 leaves h_out = 0 and writes 0
+ *   final_delta_out  device float or NULL: delta of the last iteration
+ *   residual_out     device float or NULL: max |h_t - f(h_{t-1}, x_t)| at the result
+ * Supported: GRU and LSTM any H; tanh RNN with n <= 64.  B, T >= 1. */
+int pararnn_newton_forward(pararnn_ctx *ctx, const float *xproj, const pararnn_params *p,
+                           const float *h0, float *h_out, int max_iters, float tol,
+                           int *iters_out, float *final_delta_out, float *residual_out);
+
+/* Standalone linear recurrence by a chunked parallel scan
+ * ("Para-Seq" README, Main features: dense, diagonal and 2x2 block associative scans,
+ * plus reverse adjoint scans).
+ *   forward (reverse = 0):  out_t = J_t out_{t-1} + b_t,        out_{-1} = h0 (or 0)
+ *   reverse (reverse = 1):  out_t = b_t + J_{t+1}^T out_{t+1},  out_{T-1} = b_{T-1} + h0 (or 0)
+ * kind DIAG:   J, b, out [B, T, N];             h0 [B, N]
+ * kind BLOCK2: J [B, T, N, 2, 2] (row-major 2x2), b, out [B, T, N, 2]; h0 [B, N, 2]
+ * kind DENSE:  J [B, T, N, N] (J[i][j] multiplies out_j), b, out [B, T, N]; h0 [B, N]; N <= 64 */
+int pararnn_linear_scan(pararnn_ctx *ctx, int kind, const float *J, const float *b,
+                        const float *h0, float *h_out, int B, int T, int N, int reverse);
+
+/* Adjoint backward at the states h returned by pararnn_newton_forward, for
+ * L = sum_t <grad_h_t, h_t> ("Para-Seq" README, Main features: adjoint backward with
+ * reverse adjoint scans; DEER summary, Surprising findings: the backward pass is one
+ * linear solve).  With every Jacobian evaluated at the given states:
+ *   lambda_t = grad_h_t + J_{t+1}^T lambda_{t+1},  lambda_{T-1} = grad_h_{T-1}
+ *   grad_xproj_t = (df_t/dp_t)^T lambda_t;  grad_params = sum_{b,t} (df_t/dtheta)^T lambda_t;
+ *   grad_h0 = J_0^T lambda_0.
+ * GRU and LSTM, xproj path only (p->x unused).
+ *   grad_h      like h (LSTM: (dL/dc, dL/dh) pairs)
+ *   grad_xproj  [B, T, 3, H]
+ *   grad_params GRU [3, H] = d/d(a_z, a_r, a_c); LSTM [5, H] = d/d(a_f, a_g, a_o, w_f, w_o)
+ *               (overwritten; summed with float atomics, so the summation order varies)
+ *   grad_h0     like h0, or NULL */
+int pararnn_adjoint_backward(pararnn_ctx *ctx, const float *xproj, const pararnn_params *p,
+                             const float *h0, const float *h, const float *grad_h,
+                             float *grad_xproj, float *grad_params, float *grad_h0);
+
+/* Synchronise the context's stream and report (then clear) device-side conditions:
+ * *device_status = PARARNN_OK, PARARNN_ENONFINITE or PARARNN_ETIMEOUT (first seen). */
+int pararnn_get_status(pararnn_ctx *ctx, int *device_status);
+
+/* Static text for a status code. */
+const char *pararnn_strerror(int status);
+
+/* Diagnostics.
+ * knob 1: bounded-wait limit in nanoseconds (default 1e9).
+ * knob 2: tile index whose look-back publication is withheld (-1 = none); used
+ *         only by the failure-detection test to make a successor's wait run out.
+ * knob 3: device pointer (float*) receiving delta_k of every Newton iteration, with
+ *         knob 4 its capacity (0 disables). */
+int pararnn_debug_set(pararnn_ctx *ctx, int knob, long long value);
+
+/* Number of kernels the last call launched on the stream. */
+int pararnn_last_launch_count(pararnn_ctx *ctx);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* PARARNN_H */

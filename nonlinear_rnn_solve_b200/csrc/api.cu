@@ -1,0 +1,306 @@
+// api.cu -- the C ABI declared in include/pararnn.h: argument checks, the context's
+// device workspace, and stream-ordered launches of the sm_100a kernels.
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include <algorithm>
+
+#include "../../include/pararnn.h"
+#include "common.cuh"
+#include "internal.h"
+
+struct pararnn_ctx {
+    int device = 0;
+    cudaStream_t stream = nullptr;
+    int num_sms = 0;
+    void *ws = nullptr;        // workspace: control block, flags, aggregates, side buffers
+    size_t ws_bytes = 0;
+    int *sticky = nullptr;     // sticky device status word
+    prn::DbgHost dbg;
+    int last_launches = 0;
+};
+
+namespace {
+
+struct DeviceGuard {
+    int prev = -1;
+    bool ok = true;
+    explicit DeviceGuard(int dev) {
+        if (cudaGetDevice(&prev) != cudaSuccess) { ok = false; return; }
+        if (prev != dev && cudaSetDevice(dev) != cudaSuccess) ok = false;
+    }
+    ~DeviceGuard() {
+        int cur = -1;
+        if (prev >= 0 && cudaGetDevice(&cur) == cudaSuccess && cur != prev) cudaSetDevice(prev);
+    }
+};
+
+bool misaligned(const void *p) { return p && ((uintptr_t)p & 15u); }
+
+size_t up256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+// Make the workspace at least `need` bytes (grows, never shrinks).
+int ensure_ws(pararnn_ctx *ctx, size_t need) {
+    if (ctx->ws_bytes >= need) return PARARNN_OK;
+    if (ctx->ws) {
+        if (cudaStreamSynchronize(ctx->stream) != cudaSuccess) return PARARNN_ECUDA;
+        cudaFree(ctx->ws);
+        ctx->ws = nullptr;
+        ctx->ws_bytes = 0;
+    }
+    size_t sz = std::max(need, (size_t)1 << 20);
+    if (cudaMalloc(&ctx->ws, sz) != cudaSuccess) {
+        cudaGetLastError();
+        return PARARNN_ENOMEM;
+    }
+    if (cudaMemset(ctx->ws, 0, sz) != cudaSuccess) return PARARNN_ECUDA;
+    ctx->ws_bytes = sz;
+    return PARARNN_OK;
+}
+
+// Carve the workspace for a plan, zero the control block and the flags on the stream.
+int prepare(pararnn_ctx *ctx, const prn::Plan &plan, prn::Work *w) {
+    const size_t ctl_b = up256(sizeof(prn::Ctl));
+    const size_t fl_b = up256(plan.flags_bytes), ag_b = up256(plan.agg_bytes), in_b = up256(plan.inc_bytes),
+                 sd_b = up256(plan.side_bytes);
+    int rc = ensure_ws(ctx, ctl_b + fl_b + ag_b + in_b + sd_b);
+    if (rc) return rc;
+    char *base = static_cast<char *>(ctx->ws);
+    w->ctl = reinterpret_cast<prn::Ctl *>(base);
+    w->flags = reinterpret_cast<unsigned *>(base + ctl_b);
+    w->agg = reinterpret_cast<float *>(base + ctl_b + fl_b);
+    w->inc = reinterpret_cast<float *>(base + ctl_b + fl_b + ag_b);
+    w->side = reinterpret_cast<float *>(base + ctl_b + fl_b + ag_b + in_b);
+    w->sticky = ctx->sticky;
+    if (cudaMemsetAsync(base, 0, ctl_b + fl_b, ctx->stream) != cudaSuccess) return PARARNN_ECUDA;
+    return PARARNN_OK;
+}
+
+int cuda_rc(cudaError_t e) {
+    if (e == cudaSuccess) return PARARNN_OK;
+    cudaGetLastError();
+    return PARARNN_ECUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int pararnn_create(pararnn_ctx **out, int device, void *cuda_stream) {
+    if (!out) return PARARNN_EINVAL;
+    *out = nullptr;
+    int ndev = 0;
+    if (cudaGetDeviceCount(&ndev) != cudaSuccess || device < 0 || device >= ndev) {
+        cudaGetLastError();
+        return ndev > 0 ? PARARNN_EINVAL : PARARNN_ECUDA;
+    }
+    DeviceGuard g(device);
+    if (!g.ok) return PARARNN_ECUDA;
+    pararnn_ctx *ctx = new pararnn_ctx();
+    ctx->device = device;
+    ctx->stream = static_cast<cudaStream_t>(cuda_stream);
+    if (cudaDeviceGetAttribute(&ctx->num_sms, cudaDevAttrMultiProcessorCount, device) != cudaSuccess ||
+        cudaMalloc(&ctx->sticky, 256) != cudaSuccess || cudaMemset(ctx->sticky, 0, 256) != cudaSuccess) {
+        cudaGetLastError();
+        if (ctx->sticky) cudaFree(ctx->sticky);
+        delete ctx;
+        return PARARNN_ECUDA;
+    }
+    *out = ctx;
+    return PARARNN_OK;
+}
+
+int pararnn_destroy(pararnn_ctx *ctx) {
+    if (!ctx) return PARARNN_EINVAL;
+    DeviceGuard g(ctx->device);
+    cudaStreamSynchronize(ctx->stream);
+    if (ctx->ws) cudaFree(ctx->ws);
+    if (ctx->sticky) cudaFree(ctx->sticky);
+    delete ctx;
+    return PARARNN_OK;
+}
+
+int pararnn_set_stream(pararnn_ctx *ctx, void *cuda_stream) {
+    if (!ctx) return PARARNN_EINVAL;
+    ctx->stream = static_cast<cudaStream_t>(cuda_stream);
+    return PARARNN_OK;
+}
+
+int pararnn_newton_forward(pararnn_ctx *ctx, const float *xproj, const pararnn_params *p, const float *h0,
+                           float *h_out, int max_iters, float tol, int *iters_out, float *final_delta_out,
+                           float *residual_out) {
+    if (!ctx || !p || !h_out || !iters_out) return PARARNN_EINVAL;
+    if (p->B < 1 || p->T < 1 || p->H < 1 || max_iters < 0) return PARARNN_EINVAL;
+    if (!(tol == tol)) return PARARNN_EINVAL;
+    const bool fused = xproj == nullptr;
+    if (fused && (!p->x || !p->W || p->in < 1 || p->in > 8)) return PARARNN_EINVAL;
+    if (misaligned(xproj) || misaligned(h_out) || misaligned(h0) || (fused && misaligned(p->x)))
+        return PARARNN_EALIGN;
+    DeviceGuard g(ctx->device);
+    if (!g.ok) return PARARNN_ECUDA;
+    ctx->last_launches = 0;
+    prn::Plan plan;
+    prn::Work w;
+    int rc;
+    if (p->cell == PARARNN_GRU_DIAG || p->cell == PARARNN_LSTM_CIFG_PEEP) {
+        const int lstm = p->cell == PARARNN_LSTM_CIFG_PEEP;
+        if (!p->a || (lstm && !p->peep)) return PARARNN_EINVAL;
+        prn::NewtonDiagReq r{lstm, p->B, p->T, p->H, p->in, xproj, p->x, p->W, p->bias, p->a, p->peep, h0, h_out,
+                             max_iters, tol, iters_out, final_delta_out, residual_out};
+        if (prn::newton_diag_plan(r, ctx->num_sms, &plan)) return PARARNN_ECUDA;
+        if ((rc = prepare(ctx, plan, &w))) return rc;
+        if (max_iters == 0) {
+            const size_t n = (size_t)p->B * p->T * p->H * (lstm ? 2 : 1);
+            if (cudaMemsetAsync(h_out, 0, n * sizeof(float), ctx->stream) != cudaSuccess) return PARARNN_ECUDA;
+        }
+        rc = cuda_rc(prn::newton_diag_launch(r, plan, w, ctx->dbg, ctx->stream));
+    } else if (p->cell == PARARNN_RNN_TANH_DENSE || p->cell == PARARNN_RNN_TANH_QUASI) {
+        if (!p->A) return PARARNN_EINVAL;
+        if (p->H > 64) return PARARNN_EUNSUPPORTED;
+        prn::NewtonTanhReq r{p->cell == PARARNN_RNN_TANH_QUASI, p->B, p->T, p->H, p->in, xproj, p->x, p->W,
+                             p->bias, p->A, h0, h_out, max_iters, tol, iters_out, final_delta_out, residual_out};
+        int prc = prn::newton_tanh_plan(r, ctx->num_sms, &plan);
+        if (prc == 1) return PARARNN_EUNSUPPORTED;
+        if (prc) return PARARNN_ECUDA;
+        if ((rc = prepare(ctx, plan, &w))) return rc;
+        if (max_iters == 0) {
+            const size_t n = (size_t)p->B * p->T * p->H;
+            if (cudaMemsetAsync(h_out, 0, n * sizeof(float), ctx->stream) != cudaSuccess) return PARARNN_ECUDA;
+        }
+        rc = cuda_rc(prn::newton_tanh_launch(r, plan, w, ctx->dbg, ctx->stream));
+    } else {
+        return PARARNN_EINVAL;
+    }
+    if (rc == PARARNN_OK) ctx->last_launches = 1;
+    return rc;
+}
+
+int pararnn_linear_scan(pararnn_ctx *ctx, int kind, const float *J, const float *b, const float *h0, float *h_out,
+                        int B, int T, int N, int reverse) {
+    if (!ctx || !J || !b || !h_out) return PARARNN_EINVAL;
+    if (B < 1 || T < 1 || N < 1 || (reverse != 0 && reverse != 1)) return PARARNN_EINVAL;
+    if (kind != PARARNN_SCAN_DIAG && kind != PARARNN_SCAN_BLOCK2 && kind != PARARNN_SCAN_DENSE)
+        return PARARNN_EINVAL;
+    if (kind == PARARNN_SCAN_DENSE && N > 64) return PARARNN_EUNSUPPORTED;
+    if (misaligned(J) || misaligned(b) || misaligned(h0) || misaligned(h_out)) return PARARNN_EALIGN;
+    DeviceGuard g(ctx->device);
+    if (!g.ok) return PARARNN_ECUDA;
+    ctx->last_launches = 0;
+    prn::ScanReq r{kind, B, T, N, reverse, J, b, h0, h_out};
+    prn::Plan plan;
+    prn::Work w;
+    int rc;
+    if (kind == PARARNN_SCAN_DENSE) {
+        int prc = prn::scan_dense_plan(r, ctx->num_sms, &plan);
+        if (prc == 1) return PARARNN_EUNSUPPORTED;
+        if (prc) return PARARNN_ECUDA;
+        if ((rc = prepare(ctx, plan, &w))) return rc;
+        rc = cuda_rc(prn::scan_dense_launch(r, plan, w, ctx->dbg, ctx->stream));
+    } else {
+        if (prn::scan_diag_plan(r, ctx->num_sms, &plan)) return PARARNN_ECUDA;
+        if ((rc = prepare(ctx, plan, &w))) return rc;
+        rc = cuda_rc(prn::scan_diag_launch(r, plan, w, ctx->dbg, ctx->stream));
+    }
+    if (rc == PARARNN_OK) ctx->last_launches = 1;
+    return rc;
+}
+
+int pararnn_adjoint_backward(pararnn_ctx *ctx, const float *xproj, const pararnn_params *p, const float *h0,
+                             const float *h, const float *grad_h, float *grad_xproj, float *grad_params,
+                             float *grad_h0) {
+    if (!ctx || !p || !xproj || !h || !grad_h || !grad_xproj || !grad_params) return PARARNN_EINVAL;
+    if (p->B < 1 || p->T < 1 || p->H < 1) return PARARNN_EINVAL;
+    if (p->cell != PARARNN_GRU_DIAG && p->cell != PARARNN_LSTM_CIFG_PEEP) return PARARNN_EUNSUPPORTED;
+    const int lstm = p->cell == PARARNN_LSTM_CIFG_PEEP;
+    if (!p->a || (lstm && !p->peep)) return PARARNN_EINVAL;
+    if (misaligned(xproj) || misaligned(h) || misaligned(grad_h) || misaligned(grad_xproj) || misaligned(h0) ||
+        misaligned(grad_h0))
+        return PARARNN_EALIGN;
+    DeviceGuard g(ctx->device);
+    if (!g.ok) return PARARNN_ECUDA;
+    ctx->last_launches = 0;
+    prn::AdjointReq r{lstm, p->B, p->T, p->H, xproj, p->a, p->peep, h0, h, grad_h, grad_xproj, grad_params, grad_h0};
+    prn::Plan plan;
+    prn::Work w;
+    int rc;
+    if (prn::adjoint_plan(r, ctx->num_sms, &plan)) return PARARNN_ECUDA;
+    if ((rc = prepare(ctx, plan, &w))) return rc;
+    const size_t np = (size_t)(lstm ? 5 : 3) * p->H;
+    if (cudaMemsetAsync(grad_params, 0, np * sizeof(float), ctx->stream) != cudaSuccess) return PARARNN_ECUDA;
+    rc = cuda_rc(prn::adjoint_launch(r, plan, w, ctx->dbg, ctx->stream));
+    if (rc == PARARNN_OK) ctx->last_launches = 1;
+    return rc;
+}
+
+int pararnn_input_proj(pararnn_ctx *ctx, const void *x, int x_dtype, const void *W, const float *bias,
+                       float *xproj, int M, int K, int N) {
+    if (!ctx || !x || !W || !xproj || M < 1 || K < 1 || N < 1) return PARARNN_EINVAL;
+    if (x_dtype != PARARNN_F32 && x_dtype != PARARNN_BF16) return PARARNN_EINVAL;
+    if (misaligned(x) || misaligned(W) || misaligned(xproj) || misaligned(bias)) return PARARNN_EALIGN;
+    int chk = prn::proj_check(x_dtype, M, K, N);
+    if (chk) return chk;
+    DeviceGuard g(ctx->device);
+    if (!g.ok) return PARARNN_ECUDA;
+    ctx->last_launches = 0;
+    int launches = 0;
+    int rc = cuda_rc(prn::proj_launch(x_dtype, x, W, bias, xproj, M, K, N, ctx->num_sms, ctx->stream, &launches));
+    if (rc == PARARNN_OK) ctx->last_launches = launches;
+    return rc;
+}
+
+int pararnn_get_status(pararnn_ctx *ctx, int *device_status) {
+    if (!ctx || !device_status) return PARARNN_EINVAL;
+    DeviceGuard g(ctx->device);
+    if (!g.ok) return PARARNN_ECUDA;
+    if (cudaStreamSynchronize(ctx->stream) != cudaSuccess) return cuda_rc(cudaGetLastError());
+    int v = 0;
+    if (cudaMemcpy(&v, ctx->sticky, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return PARARNN_ECUDA;
+    if (cudaMemset(ctx->sticky, 0, sizeof(int)) != cudaSuccess) return PARARNN_ECUDA;
+    if (v & prn::kStTimeout)
+        *device_status = PARARNN_ETIMEOUT;
+    else if (v & prn::kStNonfinite)
+        *device_status = PARARNN_ENONFINITE;
+    else if (v & prn::kStNotConverged)
+        *device_status = PARARNN_NOTCONVERGED;
+    else
+        *device_status = PARARNN_OK;
+    return PARARNN_OK;
+}
+
+const char *pararnn_strerror(int s) {
+    switch (s) {
+        case PARARNN_OK: return "ok";
+        case PARARNN_NOTCONVERGED: return "not converged: iteration cap reached with delta >= tol";
+        case PARARNN_EINVAL: return "invalid argument (null pointer, enum or shape)";
+        case PARARNN_EALIGN: return "pointer not 16-byte aligned";
+        case PARARNN_ECUDA: return "CUDA error";
+        case PARARNN_ENOMEM: return "workspace allocation failed";
+        case PARARNN_ENONFINITE: return "non-finite iterate or residual";
+        case PARARNN_ETIMEOUT: return "bounded device wait ran out";
+        case PARARNN_EUNSUPPORTED: return "unsupported configuration";
+        default: return "unknown status";
+    }
+}
+
+int pararnn_debug_set(pararnn_ctx *ctx, int knob, long long value) {
+    if (!ctx) return PARARNN_EINVAL;
+    switch (knob) {
+        case 1:
+            if (value <= 0) return PARARNN_EINVAL;
+            ctx->dbg.wait_ns = (unsigned long long)value;
+            return PARARNN_OK;
+        case 2: ctx->dbg.skip_tile = value; return PARARNN_OK;
+        case 3: ctx->dbg.delta_log = reinterpret_cast<float *>((uintptr_t)value); return PARARNN_OK;
+        case 4:
+            if (value < 0) return PARARNN_EINVAL;
+            ctx->dbg.delta_log_cap = (int)value;
+            return PARARNN_OK;
+        default: return PARARNN_EINVAL;
+    }
+}
+
+int pararnn_last_launch_count(pararnn_ctx *ctx) { return ctx ? ctx->last_launches : 0; }
+
+}  // extern "C"

@@ -1,0 +1,350 @@
+// common.cuh -- device building blocks shared by the sm_100a kernels of the library:
+// iteration bookkeeping, bounded waits, a grid barrier for persistent cooperative
+// kernels, affine scan elements and the chunked scan (CTA scan + decoupled look-back).
+//
+// The linear recurrence h_t = J_t h_{t-1} + b_t that every Newton iteration solves
+// ("Parallelizing non-linear sequential models over the sequence length", Approach:
+// the linear recurrence is solved with an associative prefix scan) is a composition
+// of affine maps x -> J x + b.  Composition is associative, so a chunk of steps
+// reduces to one affine map, and chunks combine in any grouping.
+#pragma once
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace prn {
+
+constexpr int kThreads = 256;
+
+// ------------------------------------------------------------------ status / control
+enum : int { kStNonfinite = 1, kStTimeout = 2, kStNotConverged = 4 };
+enum : unsigned { kFlagAgg = 1u, kFlagInc = 2u };
+
+// Per-call control block (zeroed by the host before every launch).
+struct Ctl {
+    unsigned bar_count;
+    unsigned bar_gen;
+    unsigned delta_bits[3];  // ring of per-iteration max|delta| (float bits, >= 0)
+    unsigned res_bits;       // residual max (float bits)
+    int abort;               // set on a timeout: every wait gives up at once
+    int pad[9];
+};
+
+// Debug / test controls passed by value in every kernel's arguments.
+struct Dbg {
+    unsigned long long wait_ns;  // bounded-wait limit
+    long long skip_tile;         // tile whose look-back publication is withheld (-1 none)
+    float *delta_log;            // per-iteration delta (may be null)
+    int delta_log_cap;
+};
+
+__device__ __forceinline__ unsigned long long gtimer() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+__device__ __forceinline__ unsigned ld_acquire(const unsigned *p) {
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_release(unsigned *p, unsigned v) {
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ int ld_relaxed_int(const int *p) {
+    int v;
+    asm volatile("ld.relaxed.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void raise_status(int *sticky, Ctl *ctl, int bit, bool abort) {
+    atomicOr(sticky, bit);
+    if (abort) atomicExch(&ctl->abort, 1);
+}
+
+// Grid-wide barrier for a cooperative (co-resident) grid.  Every wait is bounded:
+// it gives up when the per-call abort flag is set or after dbg.wait_ns, raising
+// kStTimeout.  Returns false when the kernel must stop.
+__device__ __forceinline__ bool grid_sync(Ctl *ctl, int *sticky, const Dbg &dbg) {
+    __shared__ int s_ok;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int ok = 1;
+        unsigned gen = ld_acquire(&ctl->bar_gen);
+        __threadfence();
+        unsigned arrived = atomicAdd(&ctl->bar_count, 1u);
+        if (arrived == gridDim.x - 1) {
+            atomicExch(&ctl->bar_count, 0u);
+            __threadfence();
+            st_release(&ctl->bar_gen, gen + 1);
+        } else {
+            unsigned long long t0 = gtimer();
+            while (ld_acquire(&ctl->bar_gen) == gen) {
+                if (ld_relaxed_int(&ctl->abort)) { ok = 0; break; }
+                if (gtimer() - t0 > dbg.wait_ns) {
+                    raise_status(sticky, ctl, kStTimeout, true);
+                    ok = 0;
+                    break;
+                }
+                __nanosleep(64);
+            }
+        }
+        if (ld_relaxed_int(&ctl->abort)) ok = 0;
+        __threadfence();
+        s_ok = ok;
+    }
+    __syncthreads();
+    return s_ok != 0;
+}
+
+// ------------------------------------------------------------------ math
+// Logistic function and tanh from the exponential: s(u) = 1 / (1 + e^-u),
+// tanh(u) = 2 s(2u) - 1 (textbook identities), with the hardware exp2-based
+// __expf and a fast reciprocal.  Absolute error stays near 1e-7, far inside the
+// 1e-4 state tolerance; both are deterministic, so Newton converges to the fixed
+// point of exactly this cell.
+__device__ __forceinline__ float sigm(float u) { return __fdividef(1.0f, 1.0f + __expf(-u)); }
+__device__ __forceinline__ float tanh_(float u) { return fmaf(2.0f, sigm(2.0f * u), -1.0f); }
+
+__device__ __forceinline__ bool finitef(float v) { return fabsf(v) <= 3.402823466e38f; }
+
+// ------------------------------------------------------------------ affine elements
+// Aff<S>: x -> a x + d with x an S-vector (S = 1 diagonal, S = 2 for 2x2 blocks).
+template <int S> struct Aff;
+template <> struct Aff<1> {
+    float a, d;
+    __device__ __forceinline__ static Aff ident() { return {1.f, 0.f}; }
+    __device__ __forceinline__ static Aff cst(const float *v) { return {0.f, v[0]}; }
+    __device__ __forceinline__ void apply(const float *x, float *y) const { y[0] = fmaf(a, x[0], d); }
+    __device__ __forceinline__ Aff shfl_up(unsigned off) const {
+        return {__shfl_up_sync(0xffffffffu, a, off), __shfl_up_sync(0xffffffffu, d, off)};
+    }
+    __device__ __forceinline__ Aff shfl_down(unsigned off) const {
+        return {__shfl_down_sync(0xffffffffu, a, off), __shfl_down_sync(0xffffffffu, d, off)};
+    }
+    __device__ __forceinline__ void store_cg(float *p) const { __stcg(reinterpret_cast<float2 *>(p), make_float2(a, d)); }
+    __device__ __forceinline__ static Aff load_cg(const float *p) {
+        float2 v = __ldcg(reinterpret_cast<const float2 *>(p));
+        return {v.x, v.y};
+    }
+    static constexpr int kFloats = 2;
+};
+template <> struct Aff<2> {
+    float a00, a01, a10, a11, d0, d1;
+    __device__ __forceinline__ static Aff ident() { return {1.f, 0.f, 0.f, 1.f, 0.f, 0.f}; }
+    __device__ __forceinline__ static Aff cst(const float *v) { return {0.f, 0.f, 0.f, 0.f, v[0], v[1]}; }
+    __device__ __forceinline__ void apply(const float *x, float *y) const {
+        float y0 = fmaf(a00, x[0], fmaf(a01, x[1], d0));
+        float y1 = fmaf(a10, x[0], fmaf(a11, x[1], d1));
+        y[0] = y0;
+        y[1] = y1;
+    }
+    __device__ __forceinline__ Aff shfl_up(unsigned off) const {
+        const unsigned m = 0xffffffffu;
+        return {__shfl_up_sync(m, a00, off), __shfl_up_sync(m, a01, off), __shfl_up_sync(m, a10, off),
+                __shfl_up_sync(m, a11, off), __shfl_up_sync(m, d0, off), __shfl_up_sync(m, d1, off)};
+    }
+    __device__ __forceinline__ Aff shfl_down(unsigned off) const {
+        const unsigned m = 0xffffffffu;
+        return {__shfl_down_sync(m, a00, off), __shfl_down_sync(m, a01, off), __shfl_down_sync(m, a10, off),
+                __shfl_down_sync(m, a11, off), __shfl_down_sync(m, d0, off), __shfl_down_sync(m, d1, off)};
+    }
+    __device__ __forceinline__ void store_cg(float *p) const {
+        float2 *q = reinterpret_cast<float2 *>(p);
+        __stcg(q, make_float2(a00, a01));
+        __stcg(q + 1, make_float2(a10, a11));
+        __stcg(q + 2, make_float2(d0, d1));
+    }
+    __device__ __forceinline__ static Aff load_cg(const float *p) {
+        const float2 *q = reinterpret_cast<const float2 *>(p);
+        float2 u = __ldcg(q), v = __ldcg(q + 1), w = __ldcg(q + 2);
+        return {u.x, u.y, v.x, v.y, w.x, w.y};
+    }
+    static constexpr int kFloats = 6;
+};
+
+// outer o inner: apply `inner` first, then `outer`.
+__device__ __forceinline__ Aff<1> compose(const Aff<1> &inner, const Aff<1> &outer) {
+    return {outer.a * inner.a, fmaf(outer.a, inner.d, outer.d)};
+}
+__device__ __forceinline__ Aff<2> compose(const Aff<2> &i, const Aff<2> &o) {
+    Aff<2> r;
+    r.a00 = fmaf(o.a00, i.a00, o.a01 * i.a10);
+    r.a01 = fmaf(o.a00, i.a01, o.a01 * i.a11);
+    r.a10 = fmaf(o.a10, i.a00, o.a11 * i.a10);
+    r.a11 = fmaf(o.a10, i.a01, o.a11 * i.a11);
+    r.d0 = fmaf(o.a00, i.d0, fmaf(o.a01, i.d1, o.d0));
+    r.d1 = fmaf(o.a10, i.d0, fmaf(o.a11, i.d1, o.d1));
+    return r;
+}
+// Element for one step of a recurrence, from a Jacobian (S x S row-major) and an offset.
+template <int S> __device__ __forceinline__ Aff<S> make_aff(const float *J, const float *d);
+template <> __device__ __forceinline__ Aff<1> make_aff<1>(const float *J, const float *d) { return {J[0], d[0]}; }
+template <> __device__ __forceinline__ Aff<2> make_aff<2>(const float *J, const float *d) {
+    return {J[0], J[1], J[2], J[3], d[0], d[1]};
+}
+
+// ------------------------------------------------------------------ chunked scan
+// Look-back workspace of one launch: a flag per tile (epoch << 2 | kFlagAgg/kFlagInc),
+// the tile aggregate per channel (published first) and the tile's inclusive value
+// per channel (the carried state at its last step, published once known).
+template <int S> struct LookBack {
+    unsigned *flags;  // [ntiles]
+    float *agg;       // [ntiles][C][Aff<S>::kFloats]
+    float *inc;       // [ntiles][C][S]
+};
+
+template <int S, int C> struct ScanSmem {
+    static constexpr int NW = kThreads / 32;
+    Aff<S> wtot[NW][C];  // per-warp totals (scan order)
+    float carry[C][S];   // carry entering the tile, per channel
+};
+
+// Inclusive composition, in scan order, of the per-thread elements of one tile.
+// Threads are laid out tid = s * C + c (s = scan position, c = channel); C divides 32.
+// On return: `excl` is the composition of the elements before this thread's
+// position (identity for s = 0) and `total` (valid in warp 0, lanes c < C) is the
+// tile's aggregate for channel c.
+template <int S, int C>
+__device__ __forceinline__ void cta_scan(const Aff<S> &e, ScanSmem<S, C> &sm, Aff<S> &excl, Aff<S> &total) {
+    static_assert(32 % C == 0, "C must divide 32");
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    Aff<S> inc = e;
+#pragma unroll
+    for (int off = C; off < 32; off <<= 1) {
+        Aff<S> o = inc.shfl_up(off);
+        if (lane >= off) inc = compose(o, inc);
+    }
+    Aff<S> wex = inc.shfl_up(C);
+    if (lane < C) wex = Aff<S>::ident();
+    if (lane >= 32 - C) sm.wtot[warp][lane - (32 - C)] = inc;
+    __syncthreads();
+    const int c = lane % C;
+    Aff<S> pre = Aff<S>::ident();
+    for (int w = 0; w < warp; ++w) pre = compose(pre, sm.wtot[w][c]);
+    excl = compose(pre, wex);
+    if (warp == 0 && lane < C) {
+        Aff<S> t = Aff<S>::ident();
+#pragma unroll
+        for (int w = 0; w < ScanSmem<S, C>::NW; ++w) t = compose(t, sm.wtot[w][lane]);
+        total = t;
+    }
+}
+
+// Decoupled look-back, run by warp 0 with lane = i * C + c (window slot i, channel c).
+// Publishes the tile aggregate, walks predecessors (tile - nseq, tile - 2 nseq, ...)
+// in windows of 32 / C, composes their aggregates until an inclusive value (or the
+// start of the sequence, whose carry is `base`), publishes this tile's inclusive
+// value and leaves the carry entering the tile in sm.carry.
+// Every wait is bounded (abort flag, dbg.wait_ns).  Returns false on a timeout.
+template <int S, int C>
+__device__ bool look_back(const LookBack<S> &lb, ScanSmem<S, C> &sm, const Aff<S> &total, long tile,
+                          int chunk, long nseq, unsigned epoch, const float *base /* [S] for lanes c<C */,
+                          Ctl *ctl, int *sticky, const Dbg &dbg) {
+    constexpr int WIN = 32 / C;
+    const int lane = threadIdx.x & 31, i = lane / C, c = lane % C;
+    const bool publish = (dbg.skip_tile != tile);
+    float carry[S];
+    bool ok = true;
+    if (chunk == 0) {
+        if (lane < C) {
+#pragma unroll
+            for (int q = 0; q < S; ++q) carry[q] = base[q];
+        }
+    } else {
+        if (lane < C && publish) total.store_cg(lb.agg + (tile * C + c) * Aff<S>::kFloats);
+        __threadfence();
+        __syncwarp();
+        if (lane == 0 && publish) st_release(lb.flags + tile, (epoch << 2) | kFlagAgg);
+        Aff<S> acc = Aff<S>::ident();  // composition of everything between here and the window
+        long pred = tile - nseq;
+        int pchunk = chunk - 1;
+        bool done = false;
+        while (!done) {
+            const int my_chunk = pchunk - i;
+            const long my_tile = pred - (long)i * nseq;
+            unsigned st = 3u;  // 3 = sequence start
+            if (my_chunk >= 0) {
+                unsigned long long t0 = 0;
+                int polls = 0;
+                for (;;) {
+                    unsigned f = ld_acquire(lb.flags + my_tile);
+                    if ((f >> 2) == epoch) { st = f & 3u; break; }
+                    if (ld_relaxed_int(&ctl->abort)) { ok = false; break; }
+                    if (++polls == 8) t0 = gtimer();
+                    if (polls > 8 && gtimer() - t0 > dbg.wait_ns) {
+                        raise_status(sticky, ctl, kStTimeout, true);
+                        ok = false;
+                        break;
+                    }
+                    if (polls > 8) __nanosleep(32);
+                }
+            }
+            __syncwarp();
+            if (__any_sync(0xffffffffu, !ok)) { ok = false; break; }
+            Aff<S> v;
+            if (st == 3u) {
+                v = Aff<S>::cst(base);
+            } else if (st == kFlagInc) {
+                float iv[S];
+#pragma unroll
+                for (int q = 0; q < S; ++q) iv[q] = __ldcg(lb.inc + (my_tile * C + c) * S + q);
+                v = Aff<S>::cst(iv);
+            } else {
+                v = Aff<S>::load_cg(lb.agg + (my_tile * C + c) * Aff<S>::kFloats);
+            }
+            const unsigned stop = __ballot_sync(0xffffffffu, st != kFlagAgg);
+            const int first = stop ? (__ffs(stop) - 1) / C : WIN;  // first slot with a known value
+            if (i > first) v = Aff<S>::ident();
+            // reduce the window: slot 0 is the nearest predecessor (applied last)
+#pragma unroll
+            for (int off = C; off < 32; off <<= 1) {
+                Aff<S> o = v.shfl_down(off);
+                if (lane + off < 32) v = compose(o, v);
+            }
+            acc = compose(v, acc);
+            if (stop) {
+                float z[S];
+#pragma unroll
+                for (int q = 0; q < S; ++q) z[q] = 0.f;
+                acc.apply(z, carry);  // acc is a constant map here
+                done = true;
+            } else {
+                pred -= (long)WIN * nseq;
+                pchunk -= WIN;
+            }
+        }
+    }
+    if (ok) {
+        if (lane < C) {
+            float incv[S];
+            total.apply(carry, incv);
+            if (publish) {
+#pragma unroll
+                for (int q = 0; q < S; ++q) __stcg(lb.inc + (tile * C + c) * S + q, incv[q]);
+            }
+#pragma unroll
+            for (int q = 0; q < S; ++q) sm.carry[c][q] = carry[q];
+        }
+        __threadfence();
+        __syncwarp();
+        if (lane == 0 && publish) st_release(lb.flags + tile, (epoch << 2) | kFlagInc);
+    }
+    return ok;
+}
+
+// Block-wide max of a non-negative float (NaN propagates as a NaN bit pattern).
+__device__ __forceinline__ unsigned block_max_bits(float v, unsigned *s_red) {
+    unsigned b = isnan(v) ? 0x7fc00000u : __float_as_uint(fabsf(v));
+#pragma unroll
+    for (int off = 16; off; off >>= 1) b = max(b, __shfl_xor_sync(0xffffffffu, b, off));
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    if (lane == 0) s_red[warp] = b;
+    __syncthreads();
+    unsigned r = 0;
+    if (threadIdx.x == 0)
+        for (int w = 0; w < kThreads / 32; ++w) r = max(r, s_red[w]);
+    __syncthreads();
+    return r;  // valid in thread 0
+}
+
+}  // namespace prn

@@ -1,0 +1,101 @@
+// internal.h -- host-side interfaces between the C ABI (api.cu) and the kernel files.
+#pragma once
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace prn {
+
+struct Ctl;
+struct Dbg;
+
+// Workspace carved by the host for one launch.
+struct Work {
+    Ctl *ctl;          // per-call control block (zeroed before the launch)
+    int *sticky;       // sticky device status (cleared by get_status)
+    unsigned *flags;   // look-back flags [ntiles]
+    float *agg;        // tile aggregates
+    float *inc;        // tile inclusive values
+    float *side;       // Newton: last state of every tile, two parities
+};
+
+// Sizes a launch needs, in bytes, given the geometry (filled by plan_* functions).
+struct Plan {
+    long ntiles = 0;
+    int grid = 0;
+    size_t flags_bytes = 0, agg_bytes = 0, inc_bytes = 0, side_bytes = 0;
+    const void *kernel = nullptr;  // for the launch
+    int variant = 0;
+};
+
+struct DbgHost {
+    unsigned long long wait_ns = 1000000000ull;
+    long long skip_tile = -1;
+    float *delta_log = nullptr;
+    int delta_log_cap = 0;
+};
+
+// ---- Newton forward, diagonal / 2x2-block cells (GRU, LSTM) -----------------------
+struct NewtonDiagReq {
+    int cell;  // 0 GRU, 1 LSTM
+    int B, T, H, in;
+    const float *xproj, *x, *W, *bias, *a, *peep, *h0;
+    float *h;
+    int max_iters;
+    float tol;
+    int *iters_out;
+    float *delta_out, *residual_out;
+};
+int newton_diag_plan(const NewtonDiagReq &r, int num_sms, Plan *plan);
+cudaError_t newton_diag_launch(const NewtonDiagReq &r, const Plan &plan, const Work &w,
+                               const DbgHost &dbg, cudaStream_t st);
+
+// ---- Newton forward, tanh RNN (dense DEER and quasi-DEER) -------------------------
+struct NewtonTanhReq {
+    int quasi;
+    int B, T, n, in;
+    const float *xproj, *x, *W, *bias, *A, *h0;
+    float *h;
+    int max_iters;
+    float tol;
+    int *iters_out;
+    float *delta_out, *residual_out;
+};
+int newton_tanh_plan(const NewtonTanhReq &r, int num_sms, Plan *plan);
+cudaError_t newton_tanh_launch(const NewtonTanhReq &r, const Plan &plan, const Work &w,
+                               const DbgHost &dbg, cudaStream_t st);
+
+// ---- standalone linear scan -------------------------------------------------------
+struct ScanReq {
+    int kind;  // 0 diag, 1 block2, 2 dense
+    int B, T, N, reverse;
+    const float *J, *b, *h0;
+    float *out;
+};
+int scan_diag_plan(const ScanReq &r, int num_sms, Plan *plan);   // kinds diag, block2
+cudaError_t scan_diag_launch(const ScanReq &r, const Plan &plan, const Work &w, const DbgHost &dbg,
+                             cudaStream_t st);
+int scan_dense_plan(const ScanReq &r, int num_sms, Plan *plan);  // kind dense
+cudaError_t scan_dense_launch(const ScanReq &r, const Plan &plan, const Work &w, const DbgHost &dbg,
+                              cudaStream_t st);
+
+// ---- adjoint backward (GRU, LSTM) --------------------------------------------------
+struct AdjointReq {
+    int cell;  // 0 GRU, 1 LSTM
+    int B, T, H;
+    const float *xproj, *a, *peep, *h0, *h, *g;
+    float *grad_xproj, *grad_params, *grad_h0;
+};
+int adjoint_plan(const AdjointReq &r, int num_sms, Plan *plan);
+cudaError_t adjoint_launch(const AdjointReq &r, const Plan &plan, const Work &w, const DbgHost &dbg,
+                           cudaStream_t st);
+
+// ---- input projection ---------------------------------------------------------------
+int proj_check(int x_dtype, int M, int K, int N);
+cudaError_t proj_launch(int x_dtype, const void *x, const void *W, const float *bias, float *y, int M,
+                        int K, int N, int num_sms, cudaStream_t st, int *launches);
+
+// Helpers.
+int occupancy_grid(const void *kernel, int threads, size_t smem, int num_sms, long ntiles);
+
+}  // namespace prn

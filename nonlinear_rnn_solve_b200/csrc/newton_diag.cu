@@ -1,0 +1,412 @@
+// newton_diag.cu -- fused Newton (DEER) forward for cells whose Jacobian is diagonal
+// (ParaGRU) or 2x2 block diagonal (ParaLSTM).
+//
+// "Parallelizing non-linear sequential models over the sequence length", Approach:
+// each Newton iteration linearises the recurrence with its Jacobians and solves the
+// linear recurrence with an associative prefix scan.  Here one persistent cooperative
+// kernel runs every iteration:
+//
+//   for k = 0, 1, ...:                                    (device-side loop)
+//     for each tile [T-chunk x C channels] of this CTA:
+//       read h^(k) and the projected inputs once; evaluate f, J and the residual
+//       r_t = f(h^(k)_{t-1}) - h^(k)_t in registers (J and r never reach HBM);
+//       scan the update delta_t = J_t delta_{t-1} + r_t, delta_{-1} = 0: thread-serial
+//       over L steps, warp shuffles, shared memory, then decoupled look-back across
+//       T-chunks;  write h^(k+1) = h^(k) + delta in place;
+//     max |delta| -> grid barrier -> every CTA takes the same stop decision.
+//
+// The update in delta form is the b-form step h^(k+1)_t = J_t h^(k+1)_{t-1} + b_t,
+// b_t = f_t - J_t h^(k)_{t-1}, minus h^(k)_t on both sides; it is equal in exact
+// arithmetic and keeps fp32 rounding proportional to the (vanishing) update.
+//
+// In-place update without a second state buffer: a tile reads its own steps of h^(k)
+// plus h^(k)_{t0-1} of the tile before it; the latter is read from a small side
+// buffer written in the previous iteration, so no tile ever reads a step another
+// tile may already have overwritten.
+#include <algorithm>
+
+#include "cells.cuh"
+#include "common.cuh"
+#include "internal.h"
+
+namespace prn {
+
+struct NewtonDiagArgs {
+    int B, T, H, in;
+    const float *xproj, *x, *W, *bias, *a, *peep, *h0;
+    float *h;
+    int max_iters;
+    float tol;
+    int *iters_out;
+    float *delta_out, *residual_out;
+    Ctl *ctl;
+    int *sticky;
+    unsigned *flags;
+    float *agg, *inc, *side;
+    Dbg dbg;
+};
+
+// Projected inputs p (3 gates) of unit h at (b, t).
+// IN = 0: read xproj [B, T, 3, H].  IN > 0: recompute W x_t + bias with IN inputs.
+// IN = -1: same with the runtime width (<= 8).
+template <int IN> struct Proj {
+    static constexpr int MAXIN = IN > 0 ? IN : 8;
+    float w[3][MAXIN], bz[3];
+    const float *x;
+    int T, in;
+    __device__ __forceinline__ void load(const NewtonDiagArgs &A, int h) {
+        x = A.x;
+        T = A.T;
+        in = IN > 0 ? IN : A.in;
+#pragma unroll
+        for (int g = 0; g < 3; ++g) {
+            bz[g] = A.bias ? __ldg(A.bias + g * A.H + h) : 0.f;
+#pragma unroll
+            for (int i = 0; i < MAXIN; ++i)
+                w[g][i] = (i < in) ? __ldg(A.W + (size_t)(g * A.H + h) * in + i) : 0.f;
+        }
+    }
+    __device__ __forceinline__ void get(int b, int t, int, float p[3]) const {
+        const float *xr = x + ((size_t)b * T + t) * in;
+        float xv[MAXIN];
+        if (IN == 2) {
+            float2 v = *reinterpret_cast<const float2 *>(xr);
+            xv[0] = v.x;
+            xv[1 % MAXIN] = v.y;
+        } else if (IN == 4) {
+            float4 v = *reinterpret_cast<const float4 *>(xr);
+            xv[0] = v.x;
+            xv[1 % MAXIN] = v.y;
+            xv[2 % MAXIN] = v.z;
+            xv[3 % MAXIN] = v.w;
+        } else {
+#pragma unroll
+            for (int i = 0; i < MAXIN; ++i) xv[i] = (i < in) ? xr[i] : 0.f;
+        }
+#pragma unroll
+        for (int g = 0; g < 3; ++g) {
+            float acc = bz[g];
+#pragma unroll
+            for (int i = 0; i < MAXIN; ++i) acc = fmaf(w[g][i], xv[i], acc);
+            p[g] = acc;
+        }
+    }
+};
+template <> struct Proj<0> {
+    const float *xp;
+    int T, H;
+    __device__ __forceinline__ void load(const NewtonDiagArgs &A, int) {
+        xp = A.xproj;
+        T = A.T;
+        H = A.H;
+    }
+    __device__ __forceinline__ void get(int b, int t, int h, float p[3]) const {
+        const float *q = xp + ((size_t)b * T + t) * 3 * H + h;
+        p[0] = q[0];
+        p[1] = q[H];
+        p[2] = q[2 * H];
+    }
+};
+
+template <int S>
+__device__ __forceinline__ void load_state(const float *hbuf, size_t idx, float *v) {
+    if (S == 1) {
+        v[0] = hbuf[idx];
+    } else {
+        float2 u = *reinterpret_cast<const float2 *>(hbuf + idx * 2);
+        v[0] = u.x;
+        v[S - 1] = u.y;
+    }
+}
+template <int S>
+__device__ __forceinline__ void store_state(float *hbuf, size_t idx, const float *v) {
+    if (S == 1) {
+        hbuf[idx] = v[0];
+    } else {
+        *reinterpret_cast<float2 *>(hbuf + idx * 2) = make_float2(v[0], v[S - 1]);
+    }
+}
+
+template <class Cell, int C, int L, int IN>
+__global__ void __launch_bounds__(kThreads, 2) newton_diag_kernel(const NewtonDiagArgs A) {
+    constexpr int S = Cell::S;
+    constexpr int SUB = kThreads / C;
+    constexpr int TCH = SUB * L;
+    __shared__ ScanSmem<S, C> sm;
+    __shared__ unsigned s_red[kThreads / 32];
+    __shared__ int s_fail;
+    const int tid = threadIdx.x, c = tid % C, s = tid / C;
+    const int nct = (A.H + C - 1) / C;
+    const long nseq = (long)A.B * nct;
+    const int nchunk = (A.T + TCH - 1) / TCH;
+    const long ntiles = nseq * nchunk;
+    const size_t side_stride = (size_t)ntiles * C * S;
+    LookBack<S> lb{A.flags, A.agg, A.inc};
+    if (tid == 0) s_fail = 0;
+
+    int iters = 0;
+    float last_delta = 0.f;
+    bool stop_all = false;
+    for (int k = 0; k < A.max_iters; ++k) {
+        const unsigned epoch = (unsigned)k + 1u;
+        if (blockIdx.x == 0 && tid == 0) A.ctl->delta_bits[(k + 1) % 3] = 0u;
+        const float *side_in = A.side + (size_t)(k & 1) * side_stride;
+        float *side_out = A.side + (size_t)((k + 1) & 1) * side_stride;
+        float my_max = 0.f;
+        for (long tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+            const int chunk = (int)(tile / nseq);
+            const long seq = tile - (long)chunk * nseq;
+            const int b = (int)(seq / nct);
+            const int h = (int)(seq % nct) * C + c;
+            const bool cv = h < A.H;
+            const int hh = cv ? h : 0;
+            const int t0 = chunk * TCH + s * L;
+            Cell cell;
+            cell.load(A.a, A.peep, A.H, hh);
+            Proj<IN> pj;
+            pj.load(A, hh);
+
+            // state entering step t0 (iterate k)
+            float hp[S];
+#pragma unroll
+            for (int q = 0; q < S; ++q) hp[q] = 0.f;
+            if (t0 == 0) {
+                if (A.h0) load_state<S>(A.h0, (size_t)b * A.H + hh, hp);
+            } else if (k > 0) {
+                if (s == 0) {
+#pragma unroll
+                    for (int q = 0; q < S; ++q) hp[q] = side_in[((tile - nseq) * C + c) * S + q];
+                } else if (t0 - 1 < A.T) {
+                    load_state<S>(A.h, ((size_t)b * A.T + (t0 - 1)) * A.H + hh, hp);
+                }
+            }
+            float Jr[L][S * S], rr[L][S], hc[L][S];
+#pragma unroll
+            for (int i = 0; i < L; ++i) {
+                const int t = t0 + i;
+                const bool v = cv && t < A.T;
+                float p[3];
+                pj.get(b, v ? t : 0, hh, p);
+                float cur[S];
+#pragma unroll
+                for (int q = 0; q < S; ++q) cur[q] = 0.f;
+                if (k > 0 && v) load_state<S>(A.h, ((size_t)b * A.T + t) * A.H + hh, cur);
+                float f[S], J[S * S];
+                cell.eval(p, hp, f, J);
+#pragma unroll
+                for (int q = 0; q < S; ++q) {
+                    rr[i][q] = v ? f[q] - cur[q] : 0.f;
+                    hc[i][q] = cur[q];
+                    hp[q] = cur[q];
+                }
+#pragma unroll
+                for (int q = 0; q < S * S; ++q) Jr[i][q] = v ? J[q] : ((q % (S + 1)) == 0 ? 1.f : 0.f);
+            }
+            Aff<S> e = Aff<S>::ident();
+#pragma unroll
+            for (int i = 0; i < L; ++i) e = compose(e, make_aff<S>(Jr[i], rr[i]));
+            Aff<S> excl, total;
+            cta_scan<S, C>(e, sm, excl, total);
+            if (tid < 32) {
+                float base[S];
+#pragma unroll
+                for (int q = 0; q < S; ++q) base[q] = 0.f;  // delta entering t = 0 is 0
+                if (!look_back<S, C>(lb, sm, total, tile, chunk, nseq, epoch, base, A.ctl, A.sticky, A.dbg))
+                    if ((tid & 31) == 0) s_fail = 1;
+            }
+            __syncthreads();
+            if (s_fail) return;  // a bounded wait ran out; the status says so
+            float d[S];
+            excl.apply(sm.carry[c], d);
+#pragma unroll
+            for (int i = 0; i < L; ++i) {
+                const int t = t0 + i;
+                float nd[S];
+                const Aff<S> el = make_aff<S>(Jr[i], rr[i]);
+                el.apply(d, nd);
+                float hn[S];
+#pragma unroll
+                for (int q = 0; q < S; ++q) {
+                    d[q] = nd[q];
+                    hn[q] = hc[i][q] + nd[q];
+                    const float ad = fabsf(nd[q]);
+                    my_max = (ad > my_max || isnan(nd[q])) ? ad : my_max;
+                }
+                if (cv && t < A.T) store_state<S>(A.h, ((size_t)b * A.T + t) * A.H + hh, hn);
+                if (i == L - 1 && s == SUB - 1 && cv && chunk < nchunk - 1) {
+#pragma unroll
+                    for (int q = 0; q < S; ++q) side_out[(tile * C + c) * S + q] = hn[q];
+                }
+            }
+            __syncthreads();
+        }
+        const unsigned bits = block_max_bits(my_max, s_red);
+        if (tid == 0) atomicMax(&A.ctl->delta_bits[k % 3], bits);
+        if (!grid_sync(A.ctl, A.sticky, A.dbg)) return;
+        const unsigned dbits = ld_acquire(&A.ctl->delta_bits[k % 3]);
+        last_delta = __uint_as_float(dbits);
+        iters = k + 1;
+        if (blockIdx.x == 0 && tid == 0 && A.dbg.delta_log && k < A.dbg.delta_log_cap)
+            A.dbg.delta_log[k] = last_delta;
+        if (dbits >= 0x7f800000u) {
+            if (blockIdx.x == 0 && tid == 0) atomicOr(A.sticky, kStNonfinite);
+            stop_all = true;
+            break;
+        }
+        if (last_delta < A.tol) break;
+    }
+
+    // Final residual max |h_t - f(h_{t-1})| at the returned iterate.
+    if (A.residual_out && !stop_all) {
+        float my_res = 0.f;
+        for (long tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+            const int chunk = (int)(tile / nseq);
+            const long seq = tile - (long)chunk * nseq;
+            const int b = (int)(seq / nct);
+            const int h = (int)(seq % nct) * C + c;
+            if (h >= A.H) continue;
+            const int t0 = chunk * TCH + s * L;
+            Cell cell;
+            cell.load(A.a, A.peep, A.H, h);
+            Proj<IN> pj;
+            pj.load(A, h);
+            float hp[S];
+#pragma unroll
+            for (int q = 0; q < S; ++q) hp[q] = 0.f;
+            if (t0 == 0) {
+                if (A.h0) load_state<S>(A.h0, (size_t)b * A.H + h, hp);
+            } else if (t0 - 1 < A.T) {
+                load_state<S>(A.h, ((size_t)b * A.T + (t0 - 1)) * A.H + h, hp);
+            }
+#pragma unroll
+            for (int i = 0; i < L; ++i) {
+                const int t = t0 + i;
+                if (t >= A.T) break;
+                float p[3], cur[S], f[S], J[S * S];
+                pj.get(b, t, h, p);
+                load_state<S>(A.h, ((size_t)b * A.T + t) * A.H + h, cur);
+                cell.eval(p, hp, f, J);
+#pragma unroll
+                for (int q = 0; q < S; ++q) {
+                    const float ad = fabsf(cur[q] - f[q]);
+                    my_res = (ad > my_res || isnan(ad)) ? ad : my_res;
+                    hp[q] = cur[q];
+                }
+            }
+        }
+        const unsigned bits = block_max_bits(my_res, s_red);
+        if (tid == 0) atomicMax(&A.ctl->res_bits, bits);
+        if (!grid_sync(A.ctl, A.sticky, A.dbg)) return;
+        if (blockIdx.x == 0 && tid == 0) {
+            const unsigned rb = ld_acquire(&A.ctl->res_bits);
+            *A.residual_out = __uint_as_float(rb);
+            if (rb >= 0x7f800000u) atomicOr(A.sticky, kStNonfinite);
+        }
+    }
+    if (blockIdx.x == 0 && tid == 0) {
+        *A.iters_out = iters;
+        if (A.delta_out) *A.delta_out = last_delta;
+        if (!stop_all && A.tol > 0.f && iters == A.max_iters && !(last_delta < A.tol))
+            atomicOr(A.sticky, kStNotConverged);
+    }
+}
+
+// ------------------------------------------------------------------ host dispatch
+namespace {
+
+int pick_C(int H) {
+    if (H >= 32) return 32;
+    int c = 1;
+    while (c < H) c <<= 1;
+    return c;
+}
+
+template <class Cell, int C, int IN> const void *kernel_for() {
+    constexpr int L = Cell::S == 1 ? 16 : 8;
+    return reinterpret_cast<const void *>(&newton_diag_kernel<Cell, C, L, IN>);
+}
+
+template <class Cell, int IN> const void *kernel_by_C(int C) {
+    switch (C) {
+        case 1: return kernel_for<Cell, 1, IN>();
+        case 2: return kernel_for<Cell, 2, IN>();
+        case 4: return kernel_for<Cell, 4, IN>();
+        case 8: return kernel_for<Cell, 8, IN>();
+        case 16: return kernel_for<Cell, 16, IN>();
+        default: return kernel_for<Cell, 32, IN>();
+    }
+}
+
+template <class Cell> const void *kernel_by_in(int C, bool fused, int in) {
+    if (!fused) return kernel_by_C<Cell, 0>(C);
+    if (in == 2) return kernel_by_C<Cell, 2>(C);
+    if (in == 4) return kernel_by_C<Cell, 4>(C);
+    return kernel_by_C<Cell, -1>(C);
+}
+
+}  // namespace
+
+int newton_diag_plan(const NewtonDiagReq &r, int num_sms, Plan *plan) {
+    const int S = r.cell == 1 ? 2 : 1;
+    const int L = S == 1 ? 16 : 8;
+    const int C = pick_C(r.H);
+    const int TCH = (kThreads / C) * L;
+    const long nct = (r.H + C - 1) / C;
+    const long nseq = (long)r.B * nct;
+    const long nchunk = (r.T + TCH - 1) / TCH;
+    plan->ntiles = nseq * nchunk;
+    const bool fused = r.xproj == nullptr;
+    plan->kernel = r.cell == 1 ? kernel_by_in<LstmCell>(C, fused, r.in) : kernel_by_in<GruCell>(C, fused, r.in);
+    plan->variant = C;
+    plan->flags_bytes = (size_t)plan->ntiles * sizeof(unsigned);
+    plan->agg_bytes = (size_t)plan->ntiles * C * (S == 1 ? 2 : 6) * sizeof(float);
+    plan->inc_bytes = (size_t)plan->ntiles * C * S * sizeof(float);
+    plan->side_bytes = 2 * (size_t)plan->ntiles * C * S * sizeof(float);
+    plan->grid = occupancy_grid(plan->kernel, kThreads, 0, num_sms, plan->ntiles);
+    return plan->grid > 0 ? 0 : -1;
+}
+
+cudaError_t newton_diag_launch(const NewtonDiagReq &r, const Plan &plan, const Work &w, const DbgHost &dbg,
+                               cudaStream_t st) {
+    NewtonDiagArgs A;
+    A.B = r.B;
+    A.T = r.T;
+    A.H = r.H;
+    A.in = r.in;
+    A.xproj = r.xproj;
+    A.x = r.x;
+    A.W = r.W;
+    A.bias = r.bias;
+    A.a = r.a;
+    A.peep = r.peep;
+    A.h0 = r.h0;
+    A.h = r.h;
+    A.max_iters = r.max_iters;
+    A.tol = r.tol;
+    A.iters_out = r.iters_out;
+    A.delta_out = r.delta_out;
+    A.residual_out = r.residual_out;
+    A.ctl = w.ctl;
+    A.sticky = w.sticky;
+    A.flags = w.flags;
+    A.agg = w.agg;
+    A.inc = w.inc;
+    A.side = w.side;
+    A.dbg.wait_ns = dbg.wait_ns;
+    A.dbg.skip_tile = dbg.skip_tile;
+    A.dbg.delta_log = dbg.delta_log;
+    A.dbg.delta_log_cap = dbg.delta_log_cap;
+    void *args[] = {&A};
+    return cudaLaunchCooperativeKernel(plan.kernel, dim3(plan.grid), dim3(kThreads), args, 0, st);
+}
+
+int occupancy_grid(const void *kernel, int threads, size_t smem, int num_sms, long ntiles) {
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, smem) != cudaSuccess) return -1;
+    if (per_sm <= 0) return -1;
+    long g = (long)per_sm * num_sms;
+    if (ntiles < g) g = ntiles;
+    return (int)std::max<long>(g, 1);
+}
+
+}  // namespace prn

@@ -1,0 +1,66 @@
+"""Output allocation around the C ABI (marshalling only; the work runs in libpararnn.so).
+
+Each function allocates its outputs with torch on the inputs' device, calls one
+entry point of ``include/pararnn.h`` on the context's stream, and returns tensors.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import (PARARNN_GRU_DIAG, PARARNN_LSTM_CIFG_PEEP, PARARNN_RNN_TANH_DENSE,
+               PARARNN_RNN_TANH_QUASI, make_params, pararnn_adjoint_backward,
+               pararnn_input_proj, pararnn_linear_scan, pararnn_newton_forward)
+
+CELLS = {"gru": PARARNN_GRU_DIAG, "lstm": PARARNN_LSTM_CIFG_PEEP,
+         "tanh": PARARNN_RNN_TANH_DENSE, "tanh_quasi": PARARNN_RNN_TANH_QUASI}
+
+
+def state_shape(cell, B, T, H):
+    return (B, T, H, 2) if cell == "lstm" else (B, T, H)
+
+
+def newton_forward(ctx, cell, B, T, H, *, xproj=None, x=None, W=None, bias=None, a=None,
+                   peep=None, A=None, h0=None, max_iters=None, tol=1e-6, residual=False,
+                   h_out=None):
+    """Newton / quasi-Newton solve.  Returns dict(h, iters, delta, residual) (device tensors)."""
+    dev = (xproj if xproj is not None else x).device
+    inp = 0 if x is None else x.shape[-1]
+    prm = make_params(CELLS[cell], B, T, H, inp, a=a, peep=peep, A=A,
+                      x=x if xproj is None else None, W=W if xproj is None else None,
+                      bias=bias if xproj is None else None)
+    if h_out is None:
+        h_out = torch.empty(state_shape(cell, B, T, H), device=dev, dtype=torch.float32)
+    iters = torch.zeros(1, device=dev, dtype=torch.int32)
+    delta = torch.zeros(1, device=dev, dtype=torch.float32)
+    res = torch.zeros(1, device=dev, dtype=torch.float32) if residual else None
+    pararnn_newton_forward(ctx, xproj, prm, h0, h_out, T if max_iters is None else max_iters, tol,
+                           iters, delta, res)
+    return {"h": h_out, "iters": iters, "delta": delta, "residual": res}
+
+
+def input_proj(ctx, x, W, bias=None):
+    """xproj = x W^T + bias with x [..., K] and W [N, K] (both bf16 or both fp32)."""
+    N = W.shape[0]
+    out = torch.empty(*x.shape[:-1], N, device=x.device, dtype=torch.float32)
+    pararnn_input_proj(ctx, x, W, bias, out)
+    return out
+
+
+def linear_scan(ctx, kind, J, b, h0=None, reverse=False):
+    from . import PARARNN_SCAN_BLOCK2, PARARNN_SCAN_DENSE, PARARNN_SCAN_DIAG
+    k = {"diag": PARARNN_SCAN_DIAG, "block2": PARARNN_SCAN_BLOCK2, "dense": PARARNN_SCAN_DENSE}[kind]
+    B, T, N = b.shape[:3]
+    out = torch.empty_like(b)
+    pararnn_linear_scan(ctx, k, J, b, h0, out, B, T, N, reverse)
+    return out
+
+
+def adjoint_backward(ctx, cell, B, T, H, *, xproj, a, peep=None, h0=None, h, grad_h):
+    """Adjoint gradients at states h.  Returns (grad_xproj, grad_params, grad_h0)."""
+    dev = xproj.device
+    prm = make_params(CELLS[cell], B, T, H, 0, a=a, peep=peep)
+    gx = torch.empty(B, T, 3, H, device=dev, dtype=torch.float32)
+    gp = torch.empty(5 if cell == "lstm" else 3, H, device=dev, dtype=torch.float32)
+    gh0 = torch.empty((B, H, 2) if cell == "lstm" else (B, H), device=dev, dtype=torch.float32)
+    pararnn_adjoint_backward(ctx, xproj, prm, h0, h, grad_h, gx, gp, gh0)
+    return gx, gp, gh0

@@ -1,0 +1,77 @@
+"""Host-side checks of the C ABI (no GPU needed, no compute calls).
+
+The library must load, export every entry point include/pararnn.h declares, and
+reject bad arguments with status codes before touching the device.
+"""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import nonlinear_rnn_solve_b200 as prn
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "pararnn.h")
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(pararnn_[a-z_0-9]+)\s*\(", src)))
+
+
+def test_library_builds_and_loads():
+    from nonlinear_rnn_solve_b200 import build
+    path = build.build()
+    assert os.path.exists(path)
+    assert prn.lib() is not None
+
+
+def test_every_declared_symbol_is_exported():
+    names = declared_functions()
+    assert len(names) >= 10
+    L = prn.lib()
+    missing = [n for n in names if not hasattr(L, n)]
+    assert not missing, missing
+    out = subprocess.run(["nm", "-D", "--defined-only", prn.LIB_PATH], capture_output=True, text=True).stdout
+    for n in names:
+        assert re.search(rf"\bT {n}$", out, flags=re.M), n
+    assert sorted(prn.EXPORTED) == names
+
+
+def test_strerror_covers_codes():
+    for code in [0, 1, -1, -2, -3, -4, -5, -6, -7]:
+        assert prn.strerror(code) != "unknown status"
+    assert prn.strerror(12345) == "unknown status"
+
+
+def test_null_context_and_pointers_are_rejected():
+    L = prn.lib()
+    EINVAL = prn.PARARNN_EINVAL
+    p = prn.pararnn_params()
+    assert L.pararnn_create(None, 0, None) == EINVAL
+    assert L.pararnn_destroy(None) == EINVAL
+    assert L.pararnn_set_stream(None, None) == EINVAL
+    assert L.pararnn_newton_forward(None, None, ctypes.byref(p), None, None, 1, 1e-6, None, None, None) == EINVAL
+    assert L.pararnn_linear_scan(None, 0, None, None, None, None, 1, 1, 1, 0) == EINVAL
+    assert L.pararnn_adjoint_backward(None, None, ctypes.byref(p), None, None, None, None, None, None) == EINVAL
+    assert L.pararnn_input_proj(None, None, 0, None, None, None, 1, 1, 1) == EINVAL
+    st = ctypes.c_int()
+    assert L.pararnn_get_status(None, ctypes.byref(st)) == EINVAL
+    assert L.pararnn_debug_set(None, 1, 5) == EINVAL
+    assert L.pararnn_last_launch_count(None) == 0
+
+
+@pytest.mark.skipif(os.path.exists("/dev/nvidia0"), reason="a GPU is present")
+def test_create_without_gpu_fails_cleanly():
+    ctx = ctypes.c_void_p()
+    rc = prn.lib().pararnn_create(ctypes.byref(ctx), 0, None)
+    assert rc < 0 and not ctx.value
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    with pytest.raises(TypeError):
+        prn._p(torch.zeros(4))

@@ -20,6 +20,7 @@ struct pararnn_ctx {
     int *sticky = nullptr;     // sticky device status word
     prn::DbgHost dbg;
     int last_launches = 0;
+    unsigned long long epoch_next = 0;  // look-back epochs handed out so far
 };
 
 namespace {
@@ -60,21 +61,28 @@ int ensure_ws(pararnn_ctx *ctx, size_t need) {
     return PARARNN_OK;
 }
 
-// Carve the workspace for a plan, zero the control block and the flags on the stream.
+// Carve the workspace for a plan and zero the control block on the stream.  Layout:
+// [control block | look-back aggregates | look-back inclusive values | side buffers].
+// Look-back words carry the epoch that wrote them; every launch takes a fresh epoch
+// range, and when the 32-bit range would wrap the look-back words are zeroed.
 int prepare(pararnn_ctx *ctx, const prn::Plan &plan, prn::Work *w) {
     const size_t ctl_b = up256(sizeof(prn::Ctl));
-    const size_t fl_b = up256(plan.flags_bytes), ag_b = up256(plan.agg_bytes), in_b = up256(plan.inc_bytes),
-                 sd_b = up256(plan.side_bytes);
-    int rc = ensure_ws(ctx, ctl_b + fl_b + ag_b + in_b + sd_b);
+    const size_t ag_b = up256(plan.agg_words * 8), in_b = up256(plan.inc_words * 8), sd_b = up256(plan.side_bytes);
+    int rc = ensure_ws(ctx, ctl_b + ag_b + in_b + sd_b);
     if (rc) return rc;
     char *base = static_cast<char *>(ctx->ws);
     w->ctl = reinterpret_cast<prn::Ctl *>(base);
-    w->flags = reinterpret_cast<unsigned *>(base + ctl_b);
-    w->agg = reinterpret_cast<float *>(base + ctl_b + fl_b);
-    w->inc = reinterpret_cast<float *>(base + ctl_b + fl_b + ag_b);
-    w->side = reinterpret_cast<float *>(base + ctl_b + fl_b + ag_b + in_b);
+    w->agg = reinterpret_cast<unsigned long long *>(base + ctl_b);
+    w->inc = reinterpret_cast<unsigned long long *>(base + ctl_b + ag_b);
+    w->side = reinterpret_cast<float *>(base + ctl_b + ag_b + in_b);
     w->sticky = ctx->sticky;
-    if (cudaMemsetAsync(base, 0, ctl_b + fl_b, ctx->stream) != cudaSuccess) return PARARNN_ECUDA;
+    if (ctx->epoch_next + plan.epochs + 2 >= 0xffffffffull) {
+        if (cudaMemsetAsync(base + ctl_b, 0, ctx->ws_bytes - ctl_b, ctx->stream) != cudaSuccess) return PARARNN_ECUDA;
+        ctx->epoch_next = 0;
+    }
+    w->epoch0 = (unsigned)ctx->epoch_next;
+    ctx->epoch_next += plan.epochs;
+    if (cudaMemsetAsync(base, 0, ctl_b, ctx->stream) != cudaSuccess) return PARARNN_ECUDA;
     return PARARNN_OK;
 }
 
@@ -132,7 +140,7 @@ int pararnn_newton_forward(pararnn_ctx *ctx, const float *xproj, const pararnn_p
                            float *h_out, int max_iters, float tol, int *iters_out, float *final_delta_out,
                            float *residual_out) {
     if (!ctx || !p || !h_out || !iters_out) return PARARNN_EINVAL;
-    if (p->B < 1 || p->T < 1 || p->H < 1 || max_iters < 0) return PARARNN_EINVAL;
+    if (p->B < 1 || p->T < 1 || p->H < 1 || max_iters < 0 || max_iters > (1 << 30)) return PARARNN_EINVAL;
     if (!(tol == tol)) return PARARNN_EINVAL;
     const bool fused = xproj == nullptr;
     if (fused && (!p->x || !p->W || p->in < 1 || p->in > 8)) return PARARNN_EINVAL;

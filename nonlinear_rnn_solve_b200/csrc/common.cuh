@@ -17,7 +17,7 @@ constexpr int kThreads = 256;
 
 // ------------------------------------------------------------------ status / control
 enum : int { kStNonfinite = 1, kStTimeout = 2, kStNotConverged = 4 };
-enum : unsigned { kFlagAgg = 1u, kFlagInc = 2u };
+enum : unsigned { kFlagAgg = 1u, kFlagInc = 2u };  // look-back states
 
 // Per-call control block (zeroed by the host before every launch).
 struct Ctl {
@@ -121,11 +121,8 @@ template <> struct Aff<1> {
     __device__ __forceinline__ Aff shfl_down(unsigned off) const {
         return {__shfl_down_sync(0xffffffffu, a, off), __shfl_down_sync(0xffffffffu, d, off)};
     }
-    __device__ __forceinline__ void store_cg(float *p) const { __stcg(reinterpret_cast<float2 *>(p), make_float2(a, d)); }
-    __device__ __forceinline__ static Aff load_cg(const float *p) {
-        float2 v = __ldcg(reinterpret_cast<const float2 *>(p));
-        return {v.x, v.y};
-    }
+    __device__ __forceinline__ void to_floats(float *v) const { v[0] = a; v[1] = d; }
+    __device__ __forceinline__ static Aff from_floats(const float *v) { return {v[0], v[1]}; }
     static constexpr int kFloats = 2;
 };
 template <> struct Aff<2> {
@@ -148,17 +145,10 @@ template <> struct Aff<2> {
         return {__shfl_down_sync(m, a00, off), __shfl_down_sync(m, a01, off), __shfl_down_sync(m, a10, off),
                 __shfl_down_sync(m, a11, off), __shfl_down_sync(m, d0, off), __shfl_down_sync(m, d1, off)};
     }
-    __device__ __forceinline__ void store_cg(float *p) const {
-        float2 *q = reinterpret_cast<float2 *>(p);
-        __stcg(q, make_float2(a00, a01));
-        __stcg(q + 1, make_float2(a10, a11));
-        __stcg(q + 2, make_float2(d0, d1));
+    __device__ __forceinline__ void to_floats(float *v) const {
+        v[0] = a00; v[1] = a01; v[2] = a10; v[3] = a11; v[4] = d0; v[5] = d1;
     }
-    __device__ __forceinline__ static Aff load_cg(const float *p) {
-        const float2 *q = reinterpret_cast<const float2 *>(p);
-        float2 u = __ldcg(q), v = __ldcg(q + 1), w = __ldcg(q + 2);
-        return {u.x, u.y, v.x, v.y, w.x, w.y};
-    }
+    __device__ __forceinline__ static Aff from_floats(const float *v) { return {v[0], v[1], v[2], v[3], v[4], v[5]}; }
     static constexpr int kFloats = 6;
 };
 
@@ -184,14 +174,30 @@ template <> __device__ __forceinline__ Aff<2> make_aff<2>(const float *J, const 
 }
 
 // ------------------------------------------------------------------ chunked scan
-// Look-back workspace of one launch: a flag per tile (epoch << 2 | kFlagAgg/kFlagInc),
-// the tile aggregate per channel (published first) and the tile's inclusive value
-// per channel (the carried state at its last step, published once known).
+// Look-back workspace: every published float travels in one 64-bit word together
+// with the 32-bit epoch of the iteration that wrote it, so a reader that sees the
+// current epoch in a word also sees that word's value (single-copy atomic 64-bit
+// access): no fences and no separate flag are needed.  Epochs are unique per
+// context across launches (the host hands out a fresh range for every launch), so
+// words left by earlier launches or iterations never match.
+//   agg [ntiles][C][Aff<S>::kFloats]  tile aggregate per channel (published first)
+//   inc [ntiles][C][S]                carried state at the tile's last step
 template <int S> struct LookBack {
-    unsigned *flags;  // [ntiles]
-    float *agg;       // [ntiles][C][Aff<S>::kFloats]
-    float *inc;       // [ntiles][C][S]
+    unsigned long long *agg;
+    unsigned long long *inc;
 };
+
+__device__ __forceinline__ unsigned long long pack_tag(float v, unsigned epoch) {
+    return ((unsigned long long)__float_as_uint(v) << 32) | epoch;
+}
+__device__ __forceinline__ void st_relaxed_u64(unsigned long long *p, unsigned long long v) {
+    asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+__device__ __forceinline__ unsigned long long ld_relaxed_u64(const unsigned long long *p) {
+    unsigned long long v;
+    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
 
 template <int S, int C> struct ScanSmem {
     static constexpr int NW = kThreads / 32;
@@ -238,23 +244,24 @@ __device__ __forceinline__ void cta_scan(const Aff<S> &e, ScanSmem<S, C> &sm, Af
 // Every wait is bounded (abort flag, dbg.wait_ns).  Returns false on a timeout.
 template <int S, int C>
 __device__ bool look_back(const LookBack<S> &lb, ScanSmem<S, C> &sm, const Aff<S> &total, long tile,
-                          int chunk, long nseq, unsigned epoch, const float *base /* [S] for lanes c<C */,
+                          int chunk, long nseq, unsigned epoch, const float *base /* [S], channel c */,
                           Ctl *ctl, int *sticky, const Dbg &dbg) {
     constexpr int WIN = 32 / C;
+    constexpr int KF = Aff<S>::kFloats;
     const int lane = threadIdx.x & 31, i = lane / C, c = lane % C;
     const bool publish = (dbg.skip_tile != tile);
     float carry[S];
     bool ok = true;
     if (chunk == 0) {
-        if (lane < C) {
 #pragma unroll
-            for (int q = 0; q < S; ++q) carry[q] = base[q];
-        }
+        for (int q = 0; q < S; ++q) carry[q] = base[q];
     } else {
-        if (lane < C && publish) total.store_cg(lb.agg + (tile * C + c) * Aff<S>::kFloats);
-        __threadfence();
-        __syncwarp();
-        if (lane == 0 && publish) st_release(lb.flags + tile, (epoch << 2) | kFlagAgg);
+        if (lane < C && publish) {
+            float tv[KF];
+            total.to_floats(tv);
+#pragma unroll
+            for (int q = 0; q < KF; ++q) st_relaxed_u64(lb.agg + (tile * C + c) * KF + q, pack_tag(tv[q], epoch));
+        }
         Aff<S> acc = Aff<S>::ident();  // composition of everything between here and the window
         long pred = tile - nseq;
         int pchunk = chunk - 1;
@@ -262,36 +269,51 @@ __device__ bool look_back(const LookBack<S> &lb, ScanSmem<S, C> &sm, const Aff<S
         while (!done) {
             const int my_chunk = pchunk - i;
             const long my_tile = pred - (long)i * nseq;
-            unsigned st = 3u;  // 3 = sequence start
+            unsigned st = 3u;  // 3: start of the sequence
+            float iv[S], av[KF];
             if (my_chunk >= 0) {
                 unsigned long long t0 = 0;
                 int polls = 0;
                 for (;;) {
-                    unsigned f = ld_acquire(lb.flags + my_tile);
-                    if ((f >> 2) == epoch) { st = f & 3u; break; }
-                    if (ld_relaxed_int(&ctl->abort)) { ok = false; break; }
-                    if (++polls == 8) t0 = gtimer();
-                    if (polls > 8 && gtimer() - t0 > dbg.wait_ns) {
-                        raise_status(sticky, ctl, kStTimeout, true);
-                        ok = false;
-                        break;
+                    unsigned long long wi[S], wa[KF];
+#pragma unroll
+                    for (int q = 0; q < S; ++q) wi[q] = ld_relaxed_u64(lb.inc + (my_tile * C + c) * S + q);
+#pragma unroll
+                    for (int q = 0; q < KF; ++q) wa[q] = ld_relaxed_u64(lb.agg + (my_tile * C + c) * KF + q);
+                    bool inc_ok = true, agg_ok = true;
+#pragma unroll
+                    for (int q = 0; q < S; ++q) {
+                        inc_ok &= (unsigned)wi[q] == epoch;
+                        iv[q] = __uint_as_float((unsigned)(wi[q] >> 32));
                     }
-                    if (polls > 8) __nanosleep(32);
+#pragma unroll
+                    for (int q = 0; q < KF; ++q) {
+                        agg_ok &= (unsigned)wa[q] == epoch;
+                        av[q] = __uint_as_float((unsigned)(wa[q] >> 32));
+                    }
+                    if (inc_ok) { st = kFlagInc; break; }
+                    if (agg_ok) { st = kFlagAgg; break; }
+                    if (ld_relaxed_int(&ctl->abort)) { ok = false; break; }
+                    if (++polls == 4) t0 = gtimer();
+                    if (polls > 4) {
+                        if (gtimer() - t0 > dbg.wait_ns) {
+                            raise_status(sticky, ctl, kStTimeout, true);
+                            ok = false;
+                            break;
+                        }
+                        __nanosleep(20);
+                    }
                 }
             }
             __syncwarp();
             if (__any_sync(0xffffffffu, !ok)) { ok = false; break; }
             Aff<S> v;
-            if (st == 3u) {
+            if (st == 3u)
                 v = Aff<S>::cst(base);
-            } else if (st == kFlagInc) {
-                float iv[S];
-#pragma unroll
-                for (int q = 0; q < S; ++q) iv[q] = __ldcg(lb.inc + (my_tile * C + c) * S + q);
+            else if (st == kFlagInc)
                 v = Aff<S>::cst(iv);
-            } else {
-                v = Aff<S>::load_cg(lb.agg + (my_tile * C + c) * Aff<S>::kFloats);
-            }
+            else
+                v = Aff<S>::from_floats(av);
             const unsigned stop = __ballot_sync(0xffffffffu, st != kFlagAgg);
             const int first = stop ? (__ffs(stop) - 1) / C : WIN;  // first slot with a known value
             if (i > first) v = Aff<S>::ident();
@@ -314,20 +336,15 @@ __device__ bool look_back(const LookBack<S> &lb, ScanSmem<S, C> &sm, const Aff<S
             }
         }
     }
-    if (ok) {
-        if (lane < C) {
-            float incv[S];
-            total.apply(carry, incv);
-            if (publish) {
+    if (ok && lane < C) {
+        float incv[S];
+        total.apply(carry, incv);
+        if (publish) {
 #pragma unroll
-                for (int q = 0; q < S; ++q) __stcg(lb.inc + (tile * C + c) * S + q, incv[q]);
-            }
-#pragma unroll
-            for (int q = 0; q < S; ++q) sm.carry[c][q] = carry[q];
+            for (int q = 0; q < S; ++q) st_relaxed_u64(lb.inc + (tile * C + c) * S + q, pack_tag(incv[q], epoch));
         }
-        __threadfence();
-        __syncwarp();
-        if (lane == 0 && publish) st_release(lb.flags + tile, (epoch << 2) | kFlagInc);
+#pragma unroll
+        for (int q = 0; q < S; ++q) sm.carry[c][q] = carry[q];
     }
     return ok;
 }

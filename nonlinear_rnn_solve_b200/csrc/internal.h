@@ -11,20 +11,23 @@ struct Dbg;
 
 // Workspace carved by the host for one launch.
 struct Work {
-    Ctl *ctl;          // per-call control block (zeroed before the launch)
-    int *sticky;       // sticky device status (cleared by get_status)
-    unsigned *flags;   // look-back flags [ntiles]
-    float *agg;        // tile aggregates
-    float *inc;        // tile inclusive values
-    float *side;       // Newton: last state of every tile, two parities
+    Ctl *ctl;                  // per-call control block (zeroed before the launch)
+    int *sticky;               // sticky device status (cleared by get_status)
+    unsigned long long *agg;   // look-back: tile aggregates, epoch-tagged words
+    unsigned long long *inc;   // look-back: tile inclusive values, epoch-tagged words
+    float *side;               // Newton: last state of every tile, two parities
+    unsigned epoch0;           // this launch uses epochs epoch0 + 1 .. epoch0 + plan.epochs
 };
 
-// Sizes a launch needs, in bytes, given the geometry (filled by plan_* functions).
+// What a launch needs (filled by the *_plan functions).
 struct Plan {
     long ntiles = 0;
     int grid = 0;
-    size_t flags_bytes = 0, agg_bytes = 0, inc_bytes = 0, side_bytes = 0;
+    int C = 0;                     // channels per tile
+    size_t agg_words = 0, inc_words = 0, side_bytes = 0;
+    unsigned epochs = 2;           // look-back epochs the launch may consume
     const void *kernel = nullptr;  // for the launch
+    int dyn_smem = 0;
     int variant = 0;
 };
 
@@ -47,6 +50,7 @@ struct NewtonDiagReq {
     float *delta_out, *residual_out;
 };
 int newton_diag_plan(const NewtonDiagReq &r, int num_sms, Plan *plan);
+int newton_staged_plan(const NewtonDiagReq &r, int num_sms, Plan *plan);  // 1: shape not covered
 cudaError_t newton_diag_launch(const NewtonDiagReq &r, const Plan &plan, const Work &w,
                                const DbgHost &dbg, cudaStream_t st);
 

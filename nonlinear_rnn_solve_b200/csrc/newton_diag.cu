@@ -28,104 +28,9 @@
 #include "cells.cuh"
 #include "common.cuh"
 #include "internal.h"
+#include "newton_common.cuh"
 
 namespace prn {
-
-struct NewtonDiagArgs {
-    int B, T, H, in;
-    const float *xproj, *x, *W, *bias, *a, *peep, *h0;
-    float *h;
-    int max_iters;
-    float tol;
-    int *iters_out;
-    float *delta_out, *residual_out;
-    Ctl *ctl;
-    int *sticky;
-    unsigned *flags;
-    float *agg, *inc, *side;
-    Dbg dbg;
-};
-
-// Projected inputs p (3 gates) of unit h at (b, t).
-// IN = 0: read xproj [B, T, 3, H].  IN > 0: recompute W x_t + bias with IN inputs.
-// IN = -1: same with the runtime width (<= 8).
-template <int IN> struct Proj {
-    static constexpr int MAXIN = IN > 0 ? IN : 8;
-    float w[3][MAXIN], bz[3];
-    const float *x;
-    int T, in;
-    __device__ __forceinline__ void load(const NewtonDiagArgs &A, int h) {
-        x = A.x;
-        T = A.T;
-        in = IN > 0 ? IN : A.in;
-#pragma unroll
-        for (int g = 0; g < 3; ++g) {
-            bz[g] = A.bias ? __ldg(A.bias + g * A.H + h) : 0.f;
-#pragma unroll
-            for (int i = 0; i < MAXIN; ++i)
-                w[g][i] = (i < in) ? __ldg(A.W + (size_t)(g * A.H + h) * in + i) : 0.f;
-        }
-    }
-    __device__ __forceinline__ void get(int b, int t, int, float p[3]) const {
-        const float *xr = x + ((size_t)b * T + t) * in;
-        float xv[MAXIN];
-        if (IN == 2) {
-            float2 v = *reinterpret_cast<const float2 *>(xr);
-            xv[0] = v.x;
-            xv[1 % MAXIN] = v.y;
-        } else if (IN == 4) {
-            float4 v = *reinterpret_cast<const float4 *>(xr);
-            xv[0] = v.x;
-            xv[1 % MAXIN] = v.y;
-            xv[2 % MAXIN] = v.z;
-            xv[3 % MAXIN] = v.w;
-        } else {
-#pragma unroll
-            for (int i = 0; i < MAXIN; ++i) xv[i] = (i < in) ? xr[i] : 0.f;
-        }
-#pragma unroll
-        for (int g = 0; g < 3; ++g) {
-            float acc = bz[g];
-#pragma unroll
-            for (int i = 0; i < MAXIN; ++i) acc = fmaf(w[g][i], xv[i], acc);
-            p[g] = acc;
-        }
-    }
-};
-template <> struct Proj<0> {
-    const float *xp;
-    int T, H;
-    __device__ __forceinline__ void load(const NewtonDiagArgs &A, int) {
-        xp = A.xproj;
-        T = A.T;
-        H = A.H;
-    }
-    __device__ __forceinline__ void get(int b, int t, int h, float p[3]) const {
-        const float *q = xp + ((size_t)b * T + t) * 3 * H + h;
-        p[0] = q[0];
-        p[1] = q[H];
-        p[2] = q[2 * H];
-    }
-};
-
-template <int S>
-__device__ __forceinline__ void load_state(const float *hbuf, size_t idx, float *v) {
-    if (S == 1) {
-        v[0] = hbuf[idx];
-    } else {
-        float2 u = *reinterpret_cast<const float2 *>(hbuf + idx * 2);
-        v[0] = u.x;
-        v[S - 1] = u.y;
-    }
-}
-template <int S>
-__device__ __forceinline__ void store_state(float *hbuf, size_t idx, const float *v) {
-    if (S == 1) {
-        hbuf[idx] = v[0];
-    } else {
-        *reinterpret_cast<float2 *>(hbuf + idx * 2) = make_float2(v[0], v[S - 1]);
-    }
-}
 
 template <class Cell, int C, int L, int IN>
 __global__ void __launch_bounds__(kThreads, 2) newton_diag_kernel(const NewtonDiagArgs A) {
@@ -141,14 +46,14 @@ __global__ void __launch_bounds__(kThreads, 2) newton_diag_kernel(const NewtonDi
     const int nchunk = (A.T + TCH - 1) / TCH;
     const long ntiles = nseq * nchunk;
     const size_t side_stride = (size_t)ntiles * C * S;
-    LookBack<S> lb{A.flags, A.agg, A.inc};
+    LookBack<S> lb{A.agg, A.inc};
     if (tid == 0) s_fail = 0;
 
     int iters = 0;
     float last_delta = 0.f;
     bool stop_all = false;
     for (int k = 0; k < A.max_iters; ++k) {
-        const unsigned epoch = (unsigned)k + 1u;
+        const unsigned epoch = A.epoch0 + (unsigned)k + 1u;
         if (blockIdx.x == 0 && tid == 0) A.ctl->delta_bits[(k + 1) % 3] = 0u;
         const float *side_in = A.side + (size_t)(k & 1) * side_stride;
         float *side_out = A.side + (size_t)((k + 1) & 1) * side_stride;
@@ -257,52 +162,8 @@ __global__ void __launch_bounds__(kThreads, 2) newton_diag_kernel(const NewtonDi
     }
 
     // Final residual max |h_t - f(h_{t-1})| at the returned iterate.
-    if (A.residual_out && !stop_all) {
-        float my_res = 0.f;
-        for (long tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
-            const int chunk = (int)(tile / nseq);
-            const long seq = tile - (long)chunk * nseq;
-            const int b = (int)(seq / nct);
-            const int h = (int)(seq % nct) * C + c;
-            if (h >= A.H) continue;
-            const int t0 = chunk * TCH + s * L;
-            Cell cell;
-            cell.load(A.a, A.peep, A.H, h);
-            Proj<IN> pj;
-            pj.load(A, h);
-            float hp[S];
-#pragma unroll
-            for (int q = 0; q < S; ++q) hp[q] = 0.f;
-            if (t0 == 0) {
-                if (A.h0) load_state<S>(A.h0, (size_t)b * A.H + h, hp);
-            } else if (t0 - 1 < A.T) {
-                load_state<S>(A.h, ((size_t)b * A.T + (t0 - 1)) * A.H + h, hp);
-            }
-#pragma unroll
-            for (int i = 0; i < L; ++i) {
-                const int t = t0 + i;
-                if (t >= A.T) break;
-                float p[3], cur[S], f[S], J[S * S];
-                pj.get(b, t, h, p);
-                load_state<S>(A.h, ((size_t)b * A.T + t) * A.H + h, cur);
-                cell.eval(p, hp, f, J);
-#pragma unroll
-                for (int q = 0; q < S; ++q) {
-                    const float ad = fabsf(cur[q] - f[q]);
-                    my_res = (ad > my_res || isnan(ad)) ? ad : my_res;
-                    hp[q] = cur[q];
-                }
-            }
-        }
-        const unsigned bits = block_max_bits(my_res, s_red);
-        if (tid == 0) atomicMax(&A.ctl->res_bits, bits);
-        if (!grid_sync(A.ctl, A.sticky, A.dbg)) return;
-        if (blockIdx.x == 0 && tid == 0) {
-            const unsigned rb = ld_acquire(&A.ctl->res_bits);
-            *A.residual_out = __uint_as_float(rb);
-            if (rb >= 0x7f800000u) atomicOr(A.sticky, kStNonfinite);
-        }
-    }
+    if (A.residual_out && !stop_all)
+        if (!residual_pass<Cell, C, L, IN>(A, s_red)) return;
     if (blockIdx.x == 0 && tid == 0) {
         *A.iters_out = iters;
         if (A.delta_out) *A.delta_out = last_delta;
@@ -347,6 +208,8 @@ template <class Cell> const void *kernel_by_in(int C, bool fused, int in) {
 }  // namespace
 
 int newton_diag_plan(const NewtonDiagReq &r, int num_sms, Plan *plan) {
+    const int staged = newton_staged_plan(r, num_sms, plan);
+    if (staged <= 0) return staged;
     const int S = r.cell == 1 ? 2 : 1;
     const int L = S == 1 ? 16 : 8;
     const int C = pick_C(r.H);
@@ -358,10 +221,12 @@ int newton_diag_plan(const NewtonDiagReq &r, int num_sms, Plan *plan) {
     const bool fused = r.xproj == nullptr;
     plan->kernel = r.cell == 1 ? kernel_by_in<LstmCell>(C, fused, r.in) : kernel_by_in<GruCell>(C, fused, r.in);
     plan->variant = C;
-    plan->flags_bytes = (size_t)plan->ntiles * sizeof(unsigned);
-    plan->agg_bytes = (size_t)plan->ntiles * C * (S == 1 ? 2 : 6) * sizeof(float);
-    plan->inc_bytes = (size_t)plan->ntiles * C * S * sizeof(float);
+    plan->C = C;
+    plan->dyn_smem = 0;
+    plan->agg_words = (size_t)plan->ntiles * C * (S == 1 ? 2 : 6);
+    plan->inc_words = (size_t)plan->ntiles * C * S;
     plan->side_bytes = 2 * (size_t)plan->ntiles * C * S * sizeof(float);
+    plan->epochs = (unsigned)r.max_iters + 1u;
     plan->grid = occupancy_grid(plan->kernel, kThreads, 0, num_sms, plan->ntiles);
     return plan->grid > 0 ? 0 : -1;
 }
@@ -388,16 +253,16 @@ cudaError_t newton_diag_launch(const NewtonDiagReq &r, const Plan &plan, const W
     A.residual_out = r.residual_out;
     A.ctl = w.ctl;
     A.sticky = w.sticky;
-    A.flags = w.flags;
     A.agg = w.agg;
     A.inc = w.inc;
     A.side = w.side;
+    A.epoch0 = w.epoch0;
     A.dbg.wait_ns = dbg.wait_ns;
     A.dbg.skip_tile = dbg.skip_tile;
     A.dbg.delta_log = dbg.delta_log;
     A.dbg.delta_log_cap = dbg.delta_log_cap;
     void *args[] = {&A};
-    return cudaLaunchCooperativeKernel(plan.kernel, dim3(plan.grid), dim3(kThreads), args, 0, st);
+    return cudaLaunchCooperativeKernel(plan.kernel, dim3(plan.grid), dim3(kThreads), args, plan.dyn_smem, st);
 }
 
 int occupancy_grid(const void *kernel, int threads, size_t smem, int num_sms, long ntiles) {

@@ -20,8 +20,8 @@ struct ScanArgs {
     float *out;
     Ctl *ctl;
     int *sticky;
-    unsigned *flags;
-    float *agg, *inc;
+    unsigned long long *agg, *inc;
+    unsigned epoch0;
     Dbg dbg;
 };
 
@@ -64,7 +64,7 @@ __global__ void __launch_bounds__(kThreads, 2) scan_kernel(const ScanArgs A) {
     const long nseq = (long)A.B * nct;
     const int nchunk = (A.T + TCH - 1) / TCH;
     const long ntiles = nseq * nchunk;
-    LookBack<S> lb{A.flags, A.agg, A.inc};
+    LookBack<S> lb{A.agg, A.inc};
     if (tid == 0) s_fail = 0;
     for (long tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
         const int chunk = (int)(tile / nseq);  // position in scan order
@@ -103,7 +103,7 @@ __global__ void __launch_bounds__(kThreads, 2) scan_kernel(const ScanArgs A) {
 #pragma unroll
                 for (int q = 0; q < S; ++q) base[q] = A.h0[((size_t)b * A.N + nn) * S + q];
             }
-            if (!look_back<S, C>(lb, sm, total, tile, chunk, nseq, 1u, base, A.ctl, A.sticky, A.dbg))
+            if (!look_back<S, C>(lb, sm, total, tile, chunk, nseq, A.epoch0 + 1u, base, A.ctl, A.sticky, A.dbg))
                 if ((tid & 31) == 0) s_fail = 1;
         }
         __syncthreads();
@@ -155,10 +155,11 @@ int scan_diag_plan(const ScanReq &r, int num_sms, Plan *plan) {
     plan->ntiles = nseq * ((r.T + TCH - 1) / TCH);
     plan->kernel = S == 1 ? scan_kernel_by_C<1, 16>(C) : scan_kernel_by_C<2, 8>(C);
     plan->variant = C;
-    plan->flags_bytes = (size_t)plan->ntiles * sizeof(unsigned);
-    plan->agg_bytes = (size_t)plan->ntiles * C * (S == 1 ? 2 : 6) * sizeof(float);
-    plan->inc_bytes = (size_t)plan->ntiles * C * S * sizeof(float);
+    plan->C = C;
+    plan->agg_words = (size_t)plan->ntiles * C * (S == 1 ? 2 : 6);
+    plan->inc_words = (size_t)plan->ntiles * C * S;
     plan->side_bytes = 0;
+    plan->epochs = 2;
     plan->grid = occupancy_grid(plan->kernel, kThreads, 0, num_sms, plan->ntiles);
     return plan->grid > 0 ? 0 : -1;
 }
@@ -176,9 +177,9 @@ cudaError_t scan_diag_launch(const ScanReq &r, const Plan &plan, const Work &w, 
     A.out = r.out;
     A.ctl = w.ctl;
     A.sticky = w.sticky;
-    A.flags = w.flags;
     A.agg = w.agg;
     A.inc = w.inc;
+    A.epoch0 = w.epoch0;
     A.dbg.wait_ns = dbg.wait_ns;
     A.dbg.skip_tile = dbg.skip_tile;
     A.dbg.delta_log = nullptr;

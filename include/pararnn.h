@@ -172,6 +172,35 @@ int pararnn_debug_set(pararnn_ctx *ctx, int knob, long long value);
 /* Number of kernels the last call launched on the stream. */
 int pararnn_last_launch_count(pararnn_ctx *ctx);
 
+/* ---- Allocation-free variant (no counterpart in the pages) ------------------------
+ * pararnn_linear_scan_noalloc computes exactly what pararnn_linear_scan computes for
+ * kind PARARNN_SCAN_DIAG or PARARNN_SCAN_BLOCK2, for callers that cannot call
+ * cudaMalloc: programs whose device memory belongs to another allocator, loops that
+ * must not pay the implicit device synchronisation of an allocation, services that
+ * must not meet out-of-memory after start-up.  It takes no context and allocates
+ * nothing: its scratch (control block and look-back words) is one static device
+ * array of PARARNN_NOALLOC_SCRATCH_BYTES that every device loading the library keeps
+ * until the process exits.
+ *   - Runs on the calling thread's current device, on `cuda_stream` (NULL = legacy
+ *     default stream).  Inputs and outputs are caller-owned device memory as for
+ *     pararnn_linear_scan.
+ *   - The first call on a device resolves the array's device address
+ *     (cudaGetSymbolAddress) and clears it; make that first call before any stream
+ *     capture.
+ *   - All calls share the one array and it keeps the last call's contents: calls that
+ *     overlap on the GPU (other streams, other host threads on the same device) race
+ *     and must be serialised by the caller.
+ *   - status_out: optional device int, set to 0 by the call; non-zero afterwards means a
+ *     bounded wait of the scan ran out (the output is then not valid).
+ *   - Returns PARARNN_ESCRATCH, before enqueuing anything, when the problem's scratch
+ *     exceeds the array: diag needs about 24 bytes per tile channel, i.e. roughly
+ *     B*N*T/128*24 bytes for N >= 32 (B*N*T up to ~89 million) and B*T/4096*24 bytes for
+ *     N = 1; block2 about B*N*T bytes for N >= 32. */
+#define PARARNN_ESCRATCH (-8)
+#define PARARNN_NOALLOC_SCRATCH_BYTES (16u << 20)
+int pararnn_linear_scan_noalloc(int kind, const float *J, const float *b, const float *h0, float *h_out,
+                                int B, int T, int N, int reverse, int *status_out, void *cuda_stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -24,6 +24,7 @@ PARARNN_ENOMEM = -4
 PARARNN_ENONFINITE = -5
 PARARNN_ETIMEOUT = -6
 PARARNN_EUNSUPPORTED = -7
+PARARNN_ESCRATCH = -8
 
 PARARNN_GRU_DIAG = 0
 PARARNN_LSTM_CIFG_PEEP = 1
@@ -41,6 +42,7 @@ EXPORTED = [
     "pararnn_create", "pararnn_destroy", "pararnn_set_stream", "pararnn_input_proj",
     "pararnn_newton_forward", "pararnn_linear_scan", "pararnn_adjoint_backward",
     "pararnn_get_status", "pararnn_strerror", "pararnn_debug_set", "pararnn_last_launch_count",
+    "pararnn_linear_scan_noalloc",
 ]
 
 
@@ -83,6 +85,7 @@ def lib() -> ctypes.CDLL:
         L.pararnn_strerror.restype = ctypes.c_char_p
         L.pararnn_debug_set.argtypes = [vp, i, ctypes.c_longlong]
         L.pararnn_last_launch_count.argtypes = [vp]
+        L.pararnn_linear_scan_noalloc.argtypes = [i, vp, vp, vp, vp, i, i, i, i, vp, vp]
         for name in EXPORTED:
             if getattr(L, name).restype is None and name != "pararnn_strerror":
                 getattr(L, name).restype = i
@@ -195,6 +198,16 @@ def pararnn_debug_set(ctx, knob: int, value: int) -> None:
 
 def pararnn_last_launch_count(ctx) -> int:
     return int(lib().pararnn_last_launch_count(ctx))
+
+
+def pararnn_linear_scan_noalloc(kind, J, b, h0, h_out, B, T, N, reverse=False, status_out=None,
+                                stream=None) -> None:
+    """Allocation-free diag / block2 scan (see include/pararnn.h); current device and stream."""
+    f32 = torch.float32
+    _check(lib().pararnn_linear_scan_noalloc(int(kind), _p(J, f32), _p(b, f32), _p(h0, f32),
+                                             _p(h_out, f32), int(B), int(T), int(N), int(bool(reverse)),
+                                             _p(status_out, torch.int32), _stream_handle(stream)),
+           "pararnn_linear_scan_noalloc")
 
 
 # ------------------------------------------------------------------ convenience

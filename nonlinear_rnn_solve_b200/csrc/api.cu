@@ -288,6 +288,7 @@ const char *pararnn_strerror(int s) {
         case PARARNN_ENONFINITE: return "non-finite iterate or residual";
         case PARARNN_ETIMEOUT: return "bounded device wait ran out";
         case PARARNN_EUNSUPPORTED: return "unsupported configuration";
+        case PARARNN_ESCRATCH: return "problem exceeds the static scratch of the allocation-free entry point";
         default: return "unknown status";
     }
 }

@@ -1,13 +1,781 @@
-// dense.cu -- placeholder entry points for the tanh RNN (dense DEER / quasi-DEER) and
-// the dense standalone scan; replaced by the real kernels.
+// dense.cu -- the vanilla tanh RNN h_t = tanh(A h_{t-1} + U x_t + b), solved with full
+// DEER (dense n x n Jacobians) or quasi-DEER (their diagonal), and the standalone dense
+// linear scan.
+//
+// "Para-Seq" README, Main features: ParaRNN is a vanilla tanh RNN with DEER modes;
+// dense associative scans.  "Parallelizing non-linear sequential models over the
+// sequence length", Surprising findings / Limitations: the explicit Jacobian products
+// cost O(n^3) per step, memory O(n^2).  "Towards Scalable and Stable Parallelization
+// of Nonlinear RNNs", Abstract: quasi-Newton keeps only the diagonal of the Jacobian.
+//
+// Full DEER: J_t = diag(1 - f_t^2) A.  A tile [T-chunk x all n units] of one sequence
+// forms f, d_t = 1 - f_t^2 and the residual r_t = f_t - h^(k)_t for every step in
+// parallel (the matvec A h^(k)_{t-1} reads the previous iterate staged in shared
+// memory), then walks its steps once to build the chunk map
+//   delta_out = P delta_in + D,   P = J_L ... J_1  (n^3 per step, the DEER cost),
+// takes delta_in from the preceding tile's published value (an inclusive chain),
+// publishes its own, and re-walks delta_t = J_t delta_{t-1} + r_t to write h^(k+1).
+// Quasi-DEER: the Jacobian is diagonal, so the diagonal scan of the ParaGRU path is
+// reused with the matvec in the cell evaluation.
+#include <algorithm>
+
+#include "common.cuh"
 #include "internal.h"
+
 namespace prn {
-int newton_tanh_plan(const NewtonTanhReq &, int, Plan *) { return 1; }
-cudaError_t newton_tanh_launch(const NewtonTanhReq &, const Plan &, const Work &, const DbgHost &, cudaStream_t) {
-    return cudaErrorNotSupported;
+
+struct TanhArgs {
+    int B, T, n, in;
+    const float *xproj, *x, *W, *bias, *A, *h0;
+    float *h;
+    int max_iters;
+    float tol;
+    int *iters_out;
+    float *delta_out, *residual_out;
+    Ctl *ctl;
+    int *sticky;
+    unsigned long long *agg, *inc;
+    float *side;
+    unsigned epoch0;
+    Dbg dbg;
+};
+
+// Spin until a 64-bit look-back word carries `epoch`; bounded like every wait.
+__device__ __forceinline__ bool wait_word(const unsigned long long *p, unsigned epoch, float *v, Ctl *ctl,
+                                          int *sticky, const Dbg &dbg) {
+    unsigned long long t0 = 0;
+    for (int polls = 0;; ++polls) {
+        const unsigned long long w = ld_relaxed_u64(p);
+        if ((unsigned)w == epoch) {
+            *v = __uint_as_float((unsigned)(w >> 32));
+            return true;
+        }
+        if (ld_relaxed_int(&ctl->abort)) return false;
+        if (polls == 4) t0 = gtimer();
+        if (polls > 4) {
+            if (gtimer() - t0 > dbg.wait_ns) {
+                raise_status(sticky, ctl, kStTimeout, true);
+                return false;
+            }
+            __nanosleep(32);
+        }
+    }
 }
-int scan_dense_plan(const ScanReq &, int, Plan *) { return 1; }
-cudaError_t scan_dense_launch(const ScanReq &, const Plan &, const Work &, const DbgHost &, cudaStream_t) {
-    return cudaErrorNotSupported;
+
+// Shared-memory layout of a tanh tile (N = padded state size, TCH steps).
+template <int N, int TCH> struct TanhSmem {
+    static constexpr int AS = N + 4;  // padded row stride (keeps float4 alignment)
+    float AT[N * AS];                 // AT[k][i] = A[i][k]
+    float hs[(TCH + 1) * N];          // h^(k) for steps t0-1 .. t0+TCH-1 (row 0 = t0-1)
+    float xin[TCH * 8];               // raw inputs of the tile (fused projection)
+    float Wt[8 * N];                  // Wt[q][i] = W[i][q]
+    float bz[N];
+};
+
+// Projected input and cell output of (step row tr, unit i) of the tile:
+// u = A h_{t-1} + p_t, with p_t from xproj or from the staged raw inputs.
+template <int N, int TCH>
+__device__ __forceinline__ float tanh_preact(const TanhArgs &A, const TanhSmem<N, TCH> &sm, int b, int t, int tr,
+                                             int i) {
+    float u;
+    if (A.xproj) {
+        u = A.xproj[((size_t)b * A.T + t) * A.n + i];
+    } else {
+        u = sm.bz[i];
+        for (int q = 0; q < A.in; ++q) u = fmaf(sm.Wt[q * N + i], sm.xin[tr * 8 + q], u);
+    }
+    const float *hp = sm.hs + tr * N;  // h^(k)_{t-1}
+#pragma unroll 16
+    for (int k = 0; k < N; ++k) u = fmaf(sm.AT[k * TanhSmem<N, TCH>::AS + i], hp[k], u);
+    return u;
 }
+
+// Stage A^T, W^T, bias once per CTA (zero-padded to N).
+template <int N, int TCH> __device__ void tanh_stage_params(const TanhArgs &A, TanhSmem<N, TCH> &sm) {
+    constexpr int AS = TanhSmem<N, TCH>::AS;
+    for (int e = threadIdx.x; e < N * N; e += kThreads) {
+        const int i = e / N, k = e % N;  // A[i][k]
+        sm.AT[k * AS + i] = (i < A.n && k < A.n) ? A.A[(size_t)i * A.n + k] : 0.f;
+    }
+    for (int e = threadIdx.x; e < 8 * N; e += kThreads) {
+        const int q = e / N, i = e % N;
+        sm.Wt[e] = (!A.xproj && q < A.in && i < A.n) ? A.W[(size_t)i * A.in + q] : 0.f;
+    }
+    for (int i = threadIdx.x; i < N; i += kThreads) sm.bz[i] = (!A.xproj && A.bias && i < A.n) ? A.bias[i] : 0.f;
+}
+
+// Stage the tile's inputs and states: hs rows 0..TCH (states t0-1 .. t0+TCH-1 of
+// iterate k; h0 before t = 0; zeros for k = 0) and raw inputs.
+template <int N, int TCH>
+__device__ void tanh_stage_tile(const TanhArgs &A, TanhSmem<N, TCH> &sm, int b, int t0, int k, const float *prev_side,
+                                bool residual_mode) {
+    for (int e = threadIdx.x; e < (TCH + 1) * N; e += kThreads) {
+        const int r = e / N, i = e % N, t = t0 + r - 1;  // state h_{t+1} in output indexing = index t
+        float v = 0.f;
+        if (i < A.n) {
+            if (t < 0) {
+                v = A.h0 ? A.h0[(size_t)b * A.n + i] : 0.f;
+            } else if (t < A.T && (k > 0 || residual_mode)) {
+                v = (r == 0 && prev_side) ? prev_side[i] : A.h[((size_t)b * A.T + t) * A.n + i];
+            }
+        }
+        sm.hs[e] = v;
+    }
+    if (!A.xproj) {
+        for (int e = threadIdx.x; e < TCH * 8; e += kThreads) {
+            const int r = e / 8, q = e % 8, t = t0 + r;
+            sm.xin[e] = (q < A.in && t < A.T) ? A.x[((size_t)b * A.T + t) * A.in + q] : 0.f;
+        }
+    }
+}
+
+// ------------------------------------------------------------------ full DEER
+template <int N> struct DeerCfg {
+    static constexpr int TCH = N >= 64 ? 64 : (N >= 32 ? 128 : 256);
+    static constexpr int BR = N >= 16 ? N / 16 : 1;   // register block of the chain product
+    static constexpr int TG = N / BR;                  // thread grid side (16, or 8 for N = 8)
+};
+
+template <int N> struct DeerExtra {
+    static constexpr int TCH = DeerCfg<N>::TCH;
+    float d[TCH * N];       // 1 - f^2
+    float r[TCH * N];       // f - h^(k)
+    float P[2][N * N];      // chain product, double buffered
+    float D[2][N];          // chain offset
+    float carry[N];
+    float dl[2][N];         // re-walk delta, double buffered
+};
+
+template <int N>
+__global__ void __launch_bounds__(kThreads, 1) tanh_deer_kernel(const TanhArgs A) {
+    constexpr int TCH = DeerCfg<N>::TCH, BR = DeerCfg<N>::BR, TG = DeerCfg<N>::TG;
+    constexpr int AS = TanhSmem<N, TCH>::AS;
+    extern __shared__ __align__(16) unsigned char smraw[];
+    TanhSmem<N, TCH> &sm = *reinterpret_cast<TanhSmem<N, TCH> *>(smraw);
+    DeerExtra<N> &sx = *reinterpret_cast<DeerExtra<N> *>(smraw + ((sizeof(TanhSmem<N, TCH>) + 15) & ~size_t(15)));
+    __shared__ unsigned s_red[kThreads / 32];
+    __shared__ int s_fail;
+    const int tid = threadIdx.x;
+    const int nchunk = (A.T + TCH - 1) / TCH;
+    const long nseq = A.B;
+    const long ntiles = nseq * nchunk;
+    if (tid == 0) s_fail = 0;
+    tanh_stage_params<N, TCH>(A, sm);
+    int iters = 0;
+    float last_delta = 0.f;
+    bool stop_all = false;
+    for (int k = 0; k < A.max_iters; ++k) {
+        const unsigned epoch = A.epoch0 + (unsigned)k + 1u;
+        if (blockIdx.x == 0 && tid == 0) A.ctl->delta_bits[(k + 1) % 3] = 0u;
+        const float *side_in = A.side + (size_t)(k & 1) * ntiles * N;
+        float *side_out = A.side + (size_t)((k + 1) & 1) * ntiles * N;
+        float my_max = 0.f;
+        for (long tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+            const int chunk = (int)(tile / nseq);
+            const int b = (int)(tile - (long)chunk * nseq);
+            const int t0 = chunk * TCH;
+            const int steps = min(TCH, A.T - t0);
+            __syncthreads();
+            tanh_stage_tile<N, TCH>(A, sm, b, t0, k, (k > 0 && chunk > 0) ? side_in + (tile - nseq) * N : nullptr,
+                                    false);
+            __syncthreads();
+            // d_t, r_t for every (step, unit)
+            for (int e = tid; e < TCH * N; e += kThreads) {
+                const int tr = e / N, i = e % N, t = t0 + tr;
+                float dv = 0.f, rv = 0.f;
+                if (tr < steps && i < A.n) {
+                    const float f = tanh_(tanh_preact<N, TCH>(A, sm, b, t, tr, i));
+                    dv = 1.f - f * f;
+                    rv = f - sm.hs[(tr + 1) * N + i];
+                }
+                sx.d[e] = dv;
+                sx.r[e] = rv;
+            }
+            // chain: P = I, D = 0, then P <- diag(d_t) A P, D <- diag(d_t) A D + r_t
+            for (int e = tid; e < N * N; e += kThreads) sx.P[0][e] = (e / N == e % N) ? 1.f : 0.f;
+            if (tid < N) sx.D[0][tid] = 0.f;
+            __syncthreads();
+            int cur = 0;
+            for (int tr = 0; tr < steps; ++tr) {
+                const float *Pi = sx.P[cur];
+                float *Po = sx.P[cur ^ 1];
+                const float *dv = sx.d + tr * N;
+                if (tid < TG * TG) {
+                    const int i0 = (tid / TG) * BR, j0 = (tid % TG) * BR;
+                    float acc[BR][BR];
+#pragma unroll
+                    for (int a = 0; a < BR; ++a)
+#pragma unroll
+                        for (int c = 0; c < BR; ++c) acc[a][c] = 0.f;
+#pragma unroll 8
+                    for (int kk = 0; kk < N; ++kk) {
+                        float av[BR], pv[BR];
+#pragma unroll
+                        for (int a = 0; a < BR; ++a) av[a] = sm.AT[kk * AS + i0 + a];
+#pragma unroll
+                        for (int c = 0; c < BR; ++c) pv[c] = Pi[kk * N + j0 + c];
+#pragma unroll
+                        for (int a = 0; a < BR; ++a)
+#pragma unroll
+                            for (int c = 0; c < BR; ++c) acc[a][c] = fmaf(av[a], pv[c], acc[a][c]);
+                    }
+#pragma unroll
+                    for (int a = 0; a < BR; ++a)
+#pragma unroll
+                        for (int c = 0; c < BR; ++c) Po[(i0 + a) * N + j0 + c] = dv[i0 + a] * acc[a][c];
+                }
+                if (tid >= kThreads - N) {
+                    const int i = tid - (kThreads - N);
+                    float acc = 0.f;
+                    for (int kk = 0; kk < N; ++kk) acc = fmaf(sm.AT[kk * AS + i], sx.D[cur][kk], acc);
+                    sx.D[cur ^ 1][i] = fmaf(dv[i], acc, sx.r[tr * N + i]);
+                }
+                __syncthreads();
+                cur ^= 1;
+            }
+            // inclusive chain across tiles: delta_in from the preceding tile
+            if (tid < N) {
+                float cv = 0.f;
+                if (chunk > 0 && !wait_word(A.inc + (tile - nseq) * N + tid, epoch, &cv, A.ctl, A.sticky, A.dbg))
+                    s_fail = 1;
+                sx.carry[tid] = cv;
+            }
+            __syncthreads();
+            if (s_fail) return;
+            if (tid < N) {
+                float acc = sx.D[cur][tid];
+                for (int j = 0; j < N; ++j) acc = fmaf(sx.P[cur][tid * N + j], sx.carry[j], acc);
+                if (A.dbg.skip_tile != tile) st_relaxed_u64(A.inc + tile * N + tid, pack_tag(acc, epoch));
+                sx.dl[0][tid] = sx.carry[tid];
+            }
+            __syncthreads();
+            // re-walk: delta_t = diag(d_t) A delta_{t-1} + r_t, h^(k+1) = h^(k) + delta
+            int dc = 0;
+            for (int tr = 0; tr < steps; ++tr) {
+                if (tid < 4 * N) {
+                    const int i = tid >> 2, q = tid & 3;
+                    float acc = 0.f;
+                    for (int kk = q; kk < N; kk += 4) acc = fmaf(sm.AT[kk * AS + i], sx.dl[dc][kk], acc);
+                    acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+                    acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+                    if (q == 0) {
+                        const float nd = fmaf(sx.d[tr * N + i], acc, sx.r[tr * N + i]);
+                        sx.dl[dc ^ 1][i] = nd;
+                        if (i < A.n) {
+                            const float hn = sm.hs[(tr + 1) * N + i] + nd;
+                            const float ad = fabsf(nd);
+                            my_max = (ad > my_max || isnan(nd)) ? ad : my_max;
+                            A.h[((size_t)b * A.T + t0 + tr) * A.n + i] = hn;
+                            if (tr == TCH - 1 && chunk < nchunk - 1) side_out[tile * N + i] = hn;
+                        }
+                    }
+                }
+                __syncthreads();
+                dc ^= 1;
+            }
+        }
+        const unsigned bits = block_max_bits(my_max, s_red);
+        if (tid == 0) atomicMax(&A.ctl->delta_bits[k % 3], bits);
+        if (!grid_sync(A.ctl, A.sticky, A.dbg)) return;
+        const unsigned dbits = ld_acquire(&A.ctl->delta_bits[k % 3]);
+        last_delta = __uint_as_float(dbits);
+        iters = k + 1;
+        if (blockIdx.x == 0 && tid == 0 && A.dbg.delta_log && k < A.dbg.delta_log_cap) A.dbg.delta_log[k] = last_delta;
+        if (dbits >= 0x7f800000u) {
+            if (blockIdx.x == 0 && tid == 0) atomicOr(A.sticky, kStNonfinite);
+            stop_all = true;
+            break;
+        }
+        if (last_delta < A.tol) break;
+    }
+    if (A.residual_out && !stop_all) {
+        float my_res = 0.f;
+        for (long tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+            const int chunk = (int)(tile / nseq);
+            const int b = (int)(tile - (long)chunk * nseq);
+            const int t0 = chunk * TCH;
+            const int steps = min(TCH, A.T - t0);
+            __syncthreads();
+            tanh_stage_tile<N, TCH>(A, sm, b, t0, 1, nullptr, true);
+            __syncthreads();
+            for (int e = tid; e < TCH * N; e += kThreads) {
+                const int tr = e / N, i = e % N;
+                if (tr < steps && i < A.n) {
+                    const float f = tanh_(tanh_preact<N, TCH>(A, sm, b, t0 + tr, tr, i));
+                    const float ad = fabsf(sm.hs[(tr + 1) * N + i] - f);
+                    my_res = (ad > my_res || isnan(ad)) ? ad : my_res;
+                }
+            }
+        }
+        const unsigned bits = block_max_bits(my_res, s_red);
+        if (tid == 0) atomicMax(&A.ctl->res_bits, bits);
+        if (!grid_sync(A.ctl, A.sticky, A.dbg)) return;
+        if (blockIdx.x == 0 && tid == 0) {
+            const unsigned rb = ld_acquire(&A.ctl->res_bits);
+            *A.residual_out = __uint_as_float(rb);
+            if (rb >= 0x7f800000u) atomicOr(A.sticky, kStNonfinite);
+        }
+    }
+    if (blockIdx.x == 0 && tid == 0) {
+        *A.iters_out = iters;
+        if (A.delta_out) *A.delta_out = last_delta;
+        if (!stop_all && A.tol > 0.f && iters == A.max_iters && !(last_delta < A.tol))
+            atomicOr(A.sticky, kStNotConverged);
+    }
+}
+
+// ------------------------------------------------------------------ quasi-DEER
+// CTA scan for C = 64 channels (two warps per sub-chunk row): tid = s * 64 + c.
+struct Scan64Smem {
+    Aff<1> w[kThreads / 64][64];
+    ScanSmem<1, 32> half[2];
+};
+
+template <int N> struct QuasiCfg {
+    static constexpr int C = N;                 // channels per tile = padded state size
+    static constexpr int SUB = kThreads / C;
+    static constexpr int L = 16;
+    static constexpr int TCH = SUB * L;
+};
+
+template <int N>
+__global__ void __launch_bounds__(kThreads, 2) tanh_quasi_kernel(const TanhArgs A) {
+    constexpr int C = QuasiCfg<N>::C, SUB = QuasiCfg<N>::SUB, L = QuasiCfg<N>::L, TCH = QuasiCfg<N>::TCH;
+    constexpr int AS = TanhSmem<N, TCH>::AS;
+    extern __shared__ __align__(16) unsigned char smraw[];
+    TanhSmem<N, TCH> &sm = *reinterpret_cast<TanhSmem<N, TCH> *>(smraw);
+    __shared__ ScanSmem<1, (C <= 32 ? C : 32)> ss;
+    __shared__ Scan64Smem s64;
+    __shared__ unsigned s_red[kThreads / 32];
+    __shared__ int s_fail;
+    const int tid = threadIdx.x, c = tid % C, s = tid / C;
+    const int nchunk = (A.T + TCH - 1) / TCH;
+    const long nseq = A.B;
+    const long ntiles = nseq * nchunk;
+    LookBack<1> lb{A.agg, A.inc};
+    if (tid == 0) s_fail = 0;
+    tanh_stage_params<N, TCH>(A, sm);
+    int iters = 0;
+    float last_delta = 0.f;
+    bool stop_all = false;
+    for (int k = 0; k < A.max_iters; ++k) {
+        const unsigned epoch = A.epoch0 + (unsigned)k + 1u;
+        if (blockIdx.x == 0 && tid == 0) A.ctl->delta_bits[(k + 1) % 3] = 0u;
+        const float *side_in = A.side + (size_t)(k & 1) * ntiles * C;
+        float *side_out = A.side + (size_t)((k + 1) & 1) * ntiles * C;
+        float my_max = 0.f;
+        for (long tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+            const int chunk = (int)(tile / nseq);
+            const int b = (int)(tile - (long)chunk * nseq);
+            const int t0 = chunk * TCH;
+            __syncthreads();
+            tanh_stage_tile<N, TCH>(A, sm, b, t0, k, (k > 0 && chunk > 0) ? side_in + (tile - nseq) * C : nullptr,
+                                    false);
+            __syncthreads();
+            const bool cv = c < A.n;
+            const float aii = sm.AT[c * AS + c];
+            float Jr[L], rr[L], hc[L];
+#pragma unroll
+            for (int i = 0; i < L; ++i) {
+                const int tr = s * L + i, t = t0 + tr;
+                const bool v = cv && t < A.T;
+                const float f = cv ? tanh_(tanh_preact<N, TCH>(A, sm, b, v ? t : t0, tr, c)) : 0.f;
+                const float cur = sm.hs[(tr + 1) * N + c];
+                Jr[i] = v ? (1.f - f * f) * aii : 1.f;
+                rr[i] = v ? f - cur : 0.f;
+                hc[i] = cur;
+            }
+            Aff<1> e = Aff<1>::ident();
+#pragma unroll
+            for (int i = 0; i < L; ++i) e = compose(e, Aff<1>{Jr[i], rr[i]});
+            Aff<1> excl, total;
+            const float zero[1] = {0.f};
+            float carry_c;
+            if (C <= 32) {
+                cta_scan<1, (C <= 32 ? C : 32)>(e, ss, excl, total);
+                if (tid < 32) {
+                    if (!look_back<1, (C <= 32 ? C : 32)>(lb, ss, total, tile, chunk, nseq, epoch, zero, A.ctl,
+                                                          A.sticky, A.dbg))
+                        if ((tid & 31) == 0) s_fail = 1;
+                }
+                __syncthreads();
+                if (s_fail) return;
+                carry_c = ss.carry[c % (C <= 32 ? C : 32)][0];
+            } else {
+                s64.w[s][c] = e;
+                __syncthreads();
+                Aff<1> pre = Aff<1>::ident();
+                for (int w = 0; w < s; ++w) pre = compose(pre, s64.w[w][c]);
+                excl = pre;
+                if (tid < 64) {
+                    Aff<1> t = Aff<1>::ident();
+#pragma unroll
+                    for (int w = 0; w < SUB; ++w) t = compose(t, s64.w[w][tid]);
+                    const int half = tid >> 5;
+                    if (!look_back<1, 32>(lb, s64.half[half], t, 2 * tile + half, chunk, 2 * nseq, epoch, zero, A.ctl,
+                                          A.sticky, A.dbg))
+                        if ((tid & 31) == 0) s_fail = 1;
+                }
+                __syncthreads();
+                if (s_fail) return;
+                carry_c = s64.half[c >> 5].carry[c & 31][0];
+            }
+            float d = fmaf(excl.a, carry_c, excl.d);
+#pragma unroll
+            for (int i = 0; i < L; ++i) {
+                const int tr = s * L + i, t = t0 + tr;
+                d = fmaf(Jr[i], d, rr[i]);
+                const float hn = hc[i] + d;
+                if (cv && t < A.T) {
+                    const float ad = fabsf(d);
+                    my_max = (ad > my_max || isnan(d)) ? ad : my_max;
+                    A.h[((size_t)b * A.T + t) * A.n + c] = hn;
+                    if (tr == TCH - 1 && chunk < nchunk - 1) side_out[tile * C + c] = hn;
+                }
+            }
+        }
+        const unsigned bits = block_max_bits(my_max, s_red);
+        if (tid == 0) atomicMax(&A.ctl->delta_bits[k % 3], bits);
+        if (!grid_sync(A.ctl, A.sticky, A.dbg)) return;
+        const unsigned dbits = ld_acquire(&A.ctl->delta_bits[k % 3]);
+        last_delta = __uint_as_float(dbits);
+        iters = k + 1;
+        if (blockIdx.x == 0 && tid == 0 && A.dbg.delta_log && k < A.dbg.delta_log_cap) A.dbg.delta_log[k] = last_delta;
+        if (dbits >= 0x7f800000u) {
+            if (blockIdx.x == 0 && tid == 0) atomicOr(A.sticky, kStNonfinite);
+            stop_all = true;
+            break;
+        }
+        if (last_delta < A.tol) break;
+    }
+    if (A.residual_out && !stop_all) {
+        float my_res = 0.f;
+        for (long tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+            const int chunk = (int)(tile / nseq);
+            const int b = (int)(tile - (long)chunk * nseq);
+            const int t0 = chunk * TCH;
+            __syncthreads();
+            tanh_stage_tile<N, TCH>(A, sm, b, t0, 1, nullptr, true);
+            __syncthreads();
+            for (int e = tid; e < TCH * N; e += kThreads) {
+                const int tr = e / N, i = e % N;
+                if (t0 + tr < A.T && i < A.n) {
+                    const float f = tanh_(tanh_preact<N, TCH>(A, sm, b, t0 + tr, tr, i));
+                    const float ad = fabsf(sm.hs[(tr + 1) * N + i] - f);
+                    my_res = (ad > my_res || isnan(ad)) ? ad : my_res;
+                }
+            }
+        }
+        const unsigned bits = block_max_bits(my_res, s_red);
+        if (tid == 0) atomicMax(&A.ctl->res_bits, bits);
+        if (!grid_sync(A.ctl, A.sticky, A.dbg)) return;
+        if (blockIdx.x == 0 && tid == 0) {
+            const unsigned rb = ld_acquire(&A.ctl->res_bits);
+            *A.residual_out = __uint_as_float(rb);
+            if (rb >= 0x7f800000u) atomicOr(A.sticky, kStNonfinite);
+        }
+    }
+    if (blockIdx.x == 0 && tid == 0) {
+        *A.iters_out = iters;
+        if (A.delta_out) *A.delta_out = last_delta;
+        if (!stop_all && A.tol > 0.f && iters == A.max_iters && !(last_delta < A.tol))
+            atomicOr(A.sticky, kStNotConverged);
+    }
+}
+
+// ------------------------------------------------------------------ dense linear scan
+// out_t = M_t out_{t-1} + b_t along the scan order, M_t = J_t (forward) or J_{t+1}^T
+// (reverse, identity at the last step).  Per tile: the chunk map (P, D) by one walk,
+// the inclusive chain across tiles, then a re-walk writing out_t.
+struct DScanArgs {
+    int B, T, n, reverse;
+    const float *J, *b, *h0;
+    float *out;
+    Ctl *ctl;
+    int *sticky;
+    unsigned long long *inc;
+    unsigned epoch0;
+    Dbg dbg;
+};
+
+template <int N> struct DScanSmem {
+    static constexpr int MS = N + 4;
+    float MT[2][N * MS];  // MT[k][i] = M_t[i][k], double buffered per step
+    float P[2][N * N];
+    float D[2][N];
+    float carry[N];
+    float v[2][N];
+};
+
+// Stage MT for scan step t (time index) of sequence b into buffer mt.
+template <int N>
+__device__ __forceinline__ void dscan_stage_M(const DScanArgs &A, float *mt, int b, int t) {
+    constexpr int MS = DScanSmem<N>::MS;
+    const size_t row = (size_t)b * A.T;
+    for (int e = threadIdx.x; e < N * N; e += kThreads) {
+        const int i = e / N, k = e % N;
+        float v;
+        if (!A.reverse) {  // M = J_t, stored MT[k][i] = J_t[i][k]
+            v = (i < A.n && k < A.n) ? A.J[((row + t) * A.n + i) * A.n + k] : 0.f;
+            mt[k * MS + i] = v;
+        } else if (t + 1 < A.T) {  // M = J_{t+1}^T, MT[k][i] = J_{t+1}[k][i]; read row-major (k = row)
+            v = (i < A.n && k < A.n) ? A.J[((row + t + 1) * A.n + i) * A.n + k] : 0.f;
+            mt[i * MS + k] = v;
+        } else {
+            mt[i * MS + k] = (i == k && i < A.n) ? 1.f : 0.f;
+        }
+    }
+}
+
+template <int N>
+__global__ void __launch_bounds__(kThreads, 1) dense_scan_kernel(const DScanArgs A) {
+    constexpr int TCH = DeerCfg<N>::TCH, BR = DeerCfg<N>::BR, TG = DeerCfg<N>::TG, MS = DScanSmem<N>::MS;
+    extern __shared__ __align__(16) unsigned char smraw[];
+    DScanSmem<N> &sm = *reinterpret_cast<DScanSmem<N> *>(smraw);
+    __shared__ int s_fail;
+    const int tid = threadIdx.x;
+    const int nchunk = (A.T + TCH - 1) / TCH;
+    const long nseq = A.B;
+    const long ntiles = nseq * nchunk;
+    const unsigned epoch = A.epoch0 + 1u;
+    if (tid == 0) s_fail = 0;
+    for (long tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+        const int chunk = (int)(tile / nseq);  // scan order
+        const int b = (int)(tile - (long)chunk * nseq);
+        const int tch = A.reverse ? nchunk - 1 - chunk : chunk;
+        const int tbeg = tch * TCH;
+        const int steps = min(TCH, A.T - tbeg);
+        auto time_of = [&](int i) { return A.reverse ? tbeg + steps - 1 - i : tbeg + i; };
+        for (int e = tid; e < N * N; e += kThreads) sm.P[0][e] = (e / N == e % N) ? 1.f : 0.f;
+        if (tid < N) sm.D[0][tid] = 0.f;
+        __syncthreads();
+        dscan_stage_M<N>(A, sm.MT[0], b, time_of(0));
+        __syncthreads();
+        int cur = 0;
+        for (int i = 0; i < steps; ++i) {
+            const int t = time_of(i);
+            if (i + 1 < steps) dscan_stage_M<N>(A, sm.MT[(i + 1) & 1], b, time_of(i + 1));
+            const float *mt = sm.MT[i & 1];
+            if (tid < TG * TG) {
+                const int i0 = (tid / TG) * BR, j0 = (tid % TG) * BR;
+                float acc[BR][BR];
+#pragma unroll
+                for (int a = 0; a < BR; ++a)
+#pragma unroll
+                    for (int c = 0; c < BR; ++c) acc[a][c] = 0.f;
+#pragma unroll 8
+                for (int kk = 0; kk < N; ++kk) {
+                    float av[BR], pv[BR];
+#pragma unroll
+                    for (int a = 0; a < BR; ++a) av[a] = mt[kk * MS + i0 + a];
+#pragma unroll
+                    for (int c = 0; c < BR; ++c) pv[c] = sm.P[cur][kk * N + j0 + c];
+#pragma unroll
+                    for (int a = 0; a < BR; ++a)
+#pragma unroll
+                        for (int c = 0; c < BR; ++c) acc[a][c] = fmaf(av[a], pv[c], acc[a][c]);
+                }
+#pragma unroll
+                for (int a = 0; a < BR; ++a)
+#pragma unroll
+                    for (int c = 0; c < BR; ++c) sm.P[cur ^ 1][(i0 + a) * N + j0 + c] = acc[a][c];
+            }
+            if (tid >= kThreads - N) {
+                const int r = tid - (kThreads - N);
+                float acc = (r < A.n) ? A.b[((size_t)b * A.T + t) * A.n + r] : 0.f;
+                for (int kk = 0; kk < N; ++kk) acc = fmaf(mt[kk * MS + r], sm.D[cur][kk], acc);
+                sm.D[cur ^ 1][r] = acc;
+            }
+            __syncthreads();
+            cur ^= 1;
+        }
+        if (tid < N) {
+            float cv = 0.f;
+            if (chunk == 0) {
+                cv = (A.h0 && tid < A.n) ? A.h0[(size_t)b * A.n + tid] : 0.f;
+            } else if (!wait_word(A.inc + (tile - nseq) * N + tid, epoch, &cv, A.ctl, A.sticky, A.dbg)) {
+                s_fail = 1;
+            }
+            sm.carry[tid] = cv;
+        }
+        __syncthreads();
+        if (s_fail) return;
+        if (tid < N) {
+            float acc = sm.D[cur][tid];
+            for (int j = 0; j < N; ++j) acc = fmaf(sm.P[cur][tid * N + j], sm.carry[j], acc);
+            if (A.dbg.skip_tile != tile) st_relaxed_u64(A.inc + tile * N + tid, pack_tag(acc, epoch));
+            sm.v[0][tid] = sm.carry[tid];
+        }
+        __syncthreads();
+        dscan_stage_M<N>(A, sm.MT[0], b, time_of(0));
+        __syncthreads();
+        int vc = 0;
+        for (int i = 0; i < steps; ++i) {
+            const int t = time_of(i);
+            if (i + 1 < steps) dscan_stage_M<N>(A, sm.MT[(i + 1) & 1], b, time_of(i + 1));
+            const float *mt = sm.MT[i & 1];
+            if (tid < 4 * N) {
+                const int r = tid >> 2, q = tid & 3;
+                float acc = 0.f;
+                for (int kk = q; kk < N; kk += 4) acc = fmaf(mt[kk * MS + r], sm.v[vc][kk], acc);
+                acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+                acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+                if (q == 0) {
+                    if (r < A.n) acc += A.b[((size_t)b * A.T + t) * A.n + r];
+                    sm.v[vc ^ 1][r] = acc;
+                    if (r < A.n) A.out[((size_t)b * A.T + t) * A.n + r] = acc;
+                }
+            }
+            __syncthreads();
+            vc ^= 1;
+        }
+    }
+}
+
+// ------------------------------------------------------------------ host side
+namespace {
+
+int pad_n(int n) {
+    int N = 8;
+    while (N < n) N <<= 1;
+    return N;
+}
+
+template <class K> int set_smem(K kern, size_t bytes) {
+    return cudaFuncSetAttribute(reinterpret_cast<const void *>(kern), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)bytes) == cudaSuccess
+               ? 0
+               : -1;
+}
+
+template <int N> size_t deer_smem() {
+    return ((sizeof(TanhSmem<N, DeerCfg<N>::TCH>) + 15) & ~size_t(15)) + sizeof(DeerExtra<N>);
+}
+template <int N> size_t quasi_smem() { return sizeof(TanhSmem<N, QuasiCfg<N>::TCH>); }
+
+template <int N> int tanh_plan_n(const NewtonTanhReq &r, int num_sms, Plan *plan) {
+    if (r.quasi) {
+        constexpr int TCH = QuasiCfg<N>::TCH;
+        auto kern = &tanh_quasi_kernel<N>;
+        const size_t sm = quasi_smem<N>();
+        if (set_smem(kern, sm)) return -1;
+        plan->kernel = reinterpret_cast<const void *>(kern);
+        plan->dyn_smem = (int)sm;
+        plan->ntiles = (long)r.B * ((r.T + TCH - 1) / TCH);
+        plan->C = N;
+        plan->agg_words = (size_t)plan->ntiles * N * 2 * (N > 32 ? 1 : 1);
+        plan->inc_words = (size_t)plan->ntiles * N;
+    } else {
+        constexpr int TCH = DeerCfg<N>::TCH;
+        auto kern = &tanh_deer_kernel<N>;
+        const size_t sm = deer_smem<N>();
+        if (set_smem(kern, sm)) return -1;
+        plan->kernel = reinterpret_cast<const void *>(kern);
+        plan->dyn_smem = (int)sm;
+        plan->ntiles = (long)r.B * ((r.T + TCH - 1) / TCH);
+        plan->C = N;
+        plan->agg_words = 0;
+        plan->inc_words = (size_t)plan->ntiles * N;
+    }
+    plan->side_bytes = 2 * (size_t)plan->ntiles * N * sizeof(float);
+    plan->epochs = (unsigned)r.max_iters + 1u;
+    plan->variant = N;
+    plan->grid = occupancy_grid(plan->kernel, kThreads, plan->dyn_smem, num_sms, plan->ntiles);
+    return plan->grid > 0 ? 0 : -1;
+}
+
+}  // namespace
+
+int newton_tanh_plan(const NewtonTanhReq &r, int num_sms, Plan *plan) {
+    if (r.n > 64) return 1;
+    if (!r.xproj && (r.in < 1 || r.in > 8)) return 1;
+    switch (pad_n(r.n)) {
+        case 8: return tanh_plan_n<8>(r, num_sms, plan);
+        case 16: return tanh_plan_n<16>(r, num_sms, plan);
+        case 32: return tanh_plan_n<32>(r, num_sms, plan);
+        default: return tanh_plan_n<64>(r, num_sms, plan);
+    }
+}
+
+cudaError_t newton_tanh_launch(const NewtonTanhReq &r, const Plan &plan, const Work &w, const DbgHost &dbg,
+                               cudaStream_t st) {
+    TanhArgs A;
+    A.B = r.B;
+    A.T = r.T;
+    A.n = r.n;
+    A.in = r.in;
+    A.xproj = r.xproj;
+    A.x = r.x;
+    A.W = r.W;
+    A.bias = r.bias;
+    A.A = r.A;
+    A.h0 = r.h0;
+    A.h = r.h;
+    A.max_iters = r.max_iters;
+    A.tol = r.tol;
+    A.iters_out = r.iters_out;
+    A.delta_out = r.delta_out;
+    A.residual_out = r.residual_out;
+    A.ctl = w.ctl;
+    A.sticky = w.sticky;
+    A.agg = w.agg;
+    A.inc = w.inc;
+    A.side = w.side;
+    A.epoch0 = w.epoch0;
+    A.dbg.wait_ns = dbg.wait_ns;
+    A.dbg.skip_tile = dbg.skip_tile;
+    A.dbg.delta_log = dbg.delta_log;
+    A.dbg.delta_log_cap = dbg.delta_log_cap;
+    void *args[] = {&A};
+    return cudaLaunchCooperativeKernel(plan.kernel, dim3(plan.grid), dim3(kThreads), args, plan.dyn_smem, st);
+}
+
+int scan_dense_plan(const ScanReq &r, int num_sms, Plan *plan) {
+    if (r.N > 64) return 1;
+    const int N = pad_n(r.N);
+    size_t sm = 0;
+    const void *kern = nullptr;
+    int TCH = 0;
+    switch (N) {
+        case 8: kern = reinterpret_cast<const void *>(&dense_scan_kernel<8>); sm = sizeof(DScanSmem<8>); TCH = DeerCfg<8>::TCH; break;
+        case 16: kern = reinterpret_cast<const void *>(&dense_scan_kernel<16>); sm = sizeof(DScanSmem<16>); TCH = DeerCfg<16>::TCH; break;
+        case 32: kern = reinterpret_cast<const void *>(&dense_scan_kernel<32>); sm = sizeof(DScanSmem<32>); TCH = DeerCfg<32>::TCH; break;
+        default: kern = reinterpret_cast<const void *>(&dense_scan_kernel<64>); sm = sizeof(DScanSmem<64>); TCH = DeerCfg<64>::TCH; break;
+    }
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm) != cudaSuccess) return -1;
+    plan->kernel = kern;
+    plan->dyn_smem = (int)sm;
+    plan->ntiles = (long)r.B * ((r.T + TCH - 1) / TCH);
+    plan->C = N;
+    plan->agg_words = 0;
+    plan->inc_words = (size_t)plan->ntiles * N;
+    plan->side_bytes = 0;
+    plan->epochs = 2;
+    plan->variant = N;
+    plan->grid = occupancy_grid(plan->kernel, kThreads, plan->dyn_smem, num_sms, plan->ntiles);
+    return plan->grid > 0 ? 0 : -1;
+}
+
+cudaError_t scan_dense_launch(const ScanReq &r, const Plan &plan, const Work &w, const DbgHost &dbg, cudaStream_t st) {
+    DScanArgs A;
+    A.B = r.B;
+    A.T = r.T;
+    A.n = r.N;
+    A.reverse = r.reverse;
+    A.J = r.J;
+    A.b = r.b;
+    A.h0 = r.h0;
+    A.out = r.out;
+    A.ctl = w.ctl;
+    A.sticky = w.sticky;
+    A.inc = w.inc;
+    A.epoch0 = w.epoch0;
+    A.dbg.wait_ns = dbg.wait_ns;
+    A.dbg.skip_tile = dbg.skip_tile;
+    A.dbg.delta_log = nullptr;
+    A.dbg.delta_log_cap = 0;
+    void *args[] = {&A};
+    return cudaLaunchCooperativeKernel(plan.kernel, dim3(plan.grid), dim3(kThreads), args, plan.dyn_smem, st);
+}
+
 }  // namespace prn

@@ -53,6 +53,22 @@ def test_scan_matches_oracle(ctx, kind, reverse, shape):
     assert max_abs(host(out), ref) <= TOL
 
 
+@pytest.mark.parametrize("N", [1, 5, 8, 13, 32, 64])
+@pytest.mark.parametrize("reverse", [False, True])
+@pytest.mark.parametrize("BT", [(2, 300), (1, 1), (3, 1025)])
+def test_dense_scan_matches_oracle(ctx, N, reverse, BT):
+    B, T = BT
+    rng = np.random.Generator(np.random.PCG64(N * 1000 + T))
+    a = 0.9 * np.sqrt(3.0 / N)  # spectral radius near 0.9
+    J = rng.uniform(-a, a, (B, T, N, N)).astype(np.float32)
+    b = rng.standard_normal((B, T, N)).astype(np.float32)
+    h0 = rng.standard_normal((B, N)).astype(np.float32) if T % 2 else None
+    out = solve.linear_scan(ctx.ctx, "dense", gpu(J), gpu(b), None if h0 is None else gpu(h0), reverse=reverse)
+    torch.cuda.synchronize()
+    assert ctx.status() == 0
+    assert max_abs(host(out), oracle.linear_scan("dense", J, b, h0, reverse=reverse)) <= TOL
+
+
 def test_scan_long_sequence_many_tiles(ctx):
     """16 sequences of 2^20 steps at N = 1: 4096 tiles, full decoupled look-back."""
     B, T, N = 16, 1 << 20, 1

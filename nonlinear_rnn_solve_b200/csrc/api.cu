@@ -253,7 +253,7 @@ int pararnn_input_proj(pararnn_ctx *ctx, const void *x, int x_dtype, const void 
     if (!g.ok) return PARARNN_ECUDA;
     ctx->last_launches = 0;
     int launches = 0;
-    int rc = cuda_rc(prn::proj_launch(x_dtype, x, W, bias, xproj, M, K, N, ctx->num_sms, ctx->stream, &launches));
+    int rc = cuda_rc(prn::proj_launch(x_dtype, x, W, bias, xproj, M, K, N, ctx->num_sms, ctx->stream, &launches, ctx->sticky));
     if (rc == PARARNN_OK) ctx->last_launches = launches;
     return rc;
 }

@@ -97,7 +97,7 @@ cudaError_t adjoint_launch(const AdjointReq &r, const Plan &plan, const Work &w,
 // ---- input projection ---------------------------------------------------------------
 int proj_check(int x_dtype, int M, int K, int N);
 cudaError_t proj_launch(int x_dtype, const void *x, const void *W, const float *bias, float *y, int M,
-                        int K, int N, int num_sms, cudaStream_t st, int *launches);
+                        int K, int N, int num_sms, cudaStream_t st, int *launches, int *sticky);
 
 // Helpers.
 int occupancy_grid(const void *kernel, int threads, size_t smem, int num_sms, long ntiles);

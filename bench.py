@@ -138,6 +138,21 @@ def _dist():
     return ws, rank, local
 
 
+def rank_workload(w, rank, world):
+    """The workload one rank solves: same shape, its own independent sequences."""
+    return w.resized(seed=w.seed + 1000 * rank) if world > 1 else w
+
+
+def max_over_ranks(values, device=None):
+    """Element-wise max of per-rank timings (the job's time is its slowest rank)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
 def _cpu_oracle_sample(w, inp, max_seconds=20.0):
     """Time the fp64 oracle Newton solve on a bounded sample of the workload."""
     import oracle
@@ -238,8 +253,7 @@ def run_ours(args, w):
         dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
     dev = torch.device("cuda", local if ws > 1 else 0)
     torch.cuda.set_device(dev)
-    wr = w.resized(seed=w.seed + 1000 * rank) if ws > 1 else w
-    inp = wl.generate(wr)
+    inp = wl.generate(rank_workload(w, rank, ws))
     t = {k: torch.from_numpy(v).to(dev) for k, v in inp.items()}
     stream = torch.cuda.current_stream(dev)
     ctx = Context(dev.index, stream)
@@ -285,10 +299,7 @@ def run_ours(args, w):
     else:
         e2e_ms, h2d, d2h = _e2e(args, w, ctx, inp, dev, stream, flush, h_out)
 
-    if ws > 1:
-        tt = torch.tensor([ms, e2e_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms, e2e_ms = float(tt[0]), float(tt[1])
+    ms, e2e_ms = max_over_ranks([ms, e2e_ms], device=dev)
     units = w.elems * ws
     value = units / (ms / 1e3)
     peak, peak_kind = _peaks()

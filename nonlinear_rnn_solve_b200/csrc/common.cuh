@@ -236,117 +236,139 @@ __device__ __forceinline__ void cta_scan(const Aff<S> &e, ScanSmem<S, C> &sm, Af
     }
 }
 
-// Decoupled look-back, run by warp 0 with lane = i * C + c (window slot i, channel c).
-// Publishes the tile aggregate, walks predecessors (tile - nseq, tile - 2 nseq, ...)
-// in windows of 32 / C, composes their aggregates until an inclusive value (or the
-// start of the sequence, whose carry is `base`), publishes this tile's inclusive
-// value and leaves the carry entering the tile in sm.carry.
-// Every wait is bounded (abort flag, dbg.wait_ns).  Returns false on a timeout.
+// Decoupled look-back, in three parts, run by warp 0 with lane = i * C + c (window
+// slot i, channel c).  Every wait is bounded (abort flag, dbg.wait_ns).
+//
+// publish_agg: lanes c < C publish the tile aggregate (tiles with chunk > 0).
+template <int S, int C>
+__device__ __forceinline__ void publish_agg(const LookBack<S> &lb, const Aff<S> &total, long tile, int chunk,
+                                            unsigned epoch, const Dbg &dbg) {
+    constexpr int KF = Aff<S>::kFloats;
+    const int lane = threadIdx.x & 31;
+    if (chunk == 0 || lane >= C || dbg.skip_tile == tile) return;
+    float tv[KF];
+    total.to_floats(tv);
+#pragma unroll
+    for (int q = 0; q < KF; ++q) st_relaxed_u64(lb.agg + (tile * C + lane) * KF + q, pack_tag(tv[q], epoch));
+}
+
+// resolve_carry: the carried state entering `tile`, valid in lanes c < C.  Walks the
+// predecessors (tile - nseq, tile - 2 nseq, ...) in windows of 32 / C, composing their
+// aggregates until an inclusive value or the start of the sequence (carry `base`).
+// Returns false on a timeout / abort.
+template <int S, int C>
+__device__ bool resolve_carry(const LookBack<S> &lb, long tile, int chunk, long nseq, unsigned epoch,
+                              const float *base, float *carry, Ctl *ctl, int *sticky, const Dbg &dbg) {
+    constexpr int WIN = 32 / C;
+    constexpr int KF = Aff<S>::kFloats;
+    const int lane = threadIdx.x & 31, i = lane / C, c = lane % C;
+    if (chunk == 0) {
+#pragma unroll
+        for (int q = 0; q < S; ++q) carry[q] = base[q];
+        return true;
+    }
+    bool ok = true;
+    Aff<S> acc = Aff<S>::ident();  // composition of everything between here and the window
+    long pred = tile - nseq;
+    int pchunk = chunk - 1;
+    for (;;) {
+        const int my_chunk = pchunk - i;
+        const long my_tile = pred - (long)i * nseq;
+        unsigned st = 3u;  // 3: start of the sequence
+        float iv[S], av[KF];
+        if (my_chunk >= 0) {
+            unsigned long long t0 = 0;
+            int polls = 0;
+            for (;;) {
+                unsigned long long wi[S], wa[KF];
+#pragma unroll
+                for (int q = 0; q < S; ++q) wi[q] = ld_relaxed_u64(lb.inc + (my_tile * C + c) * S + q);
+#pragma unroll
+                for (int q = 0; q < KF; ++q) wa[q] = ld_relaxed_u64(lb.agg + (my_tile * C + c) * KF + q);
+                bool inc_ok = true, agg_ok = true;
+#pragma unroll
+                for (int q = 0; q < S; ++q) {
+                    inc_ok &= (unsigned)wi[q] == epoch;
+                    iv[q] = __uint_as_float((unsigned)(wi[q] >> 32));
+                }
+#pragma unroll
+                for (int q = 0; q < KF; ++q) {
+                    agg_ok &= (unsigned)wa[q] == epoch;
+                    av[q] = __uint_as_float((unsigned)(wa[q] >> 32));
+                }
+                if (inc_ok) { st = kFlagInc; break; }
+                if (agg_ok) { st = kFlagAgg; break; }
+                if (ld_relaxed_int(&ctl->abort)) { ok = false; break; }
+                if (++polls == 4) t0 = gtimer();
+                if (polls > 4) {
+                    if (gtimer() - t0 > dbg.wait_ns) {
+                        raise_status(sticky, ctl, kStTimeout, true);
+                        ok = false;
+                        break;
+                    }
+                    __nanosleep(20);
+                }
+            }
+        }
+        __syncwarp();
+        if (__any_sync(0xffffffffu, !ok)) return false;
+        Aff<S> v;
+        if (st == 3u)
+            v = Aff<S>::cst(base);
+        else if (st == kFlagInc)
+            v = Aff<S>::cst(iv);
+        else
+            v = Aff<S>::from_floats(av);
+        const unsigned stop = __ballot_sync(0xffffffffu, st != kFlagAgg);
+        const int first = stop ? (__ffs(stop) - 1) / C : WIN;  // first slot with a known value
+        if (i > first) v = Aff<S>::ident();
+        // reduce the window: slot 0 is the nearest predecessor (applied last)
+#pragma unroll
+        for (int off = C; off < 32; off <<= 1) {
+            Aff<S> o = v.shfl_down(off);
+            if (lane + off < 32) v = compose(o, v);
+        }
+        acc = compose(v, acc);
+        if (stop) {
+            float z[S];
+#pragma unroll
+            for (int q = 0; q < S; ++q) z[q] = 0.f;
+            acc.apply(z, carry);  // acc is a constant map here
+            return true;
+        }
+        pred -= (long)WIN * nseq;
+        pchunk -= WIN;
+    }
+}
+
+// publish_inc: lanes c < C publish the tile's inclusive value total(carry).
+template <int S, int C>
+__device__ __forceinline__ void publish_inc(const LookBack<S> &lb, const Aff<S> &total, const float *carry, long tile,
+                                            unsigned epoch, const Dbg &dbg) {
+    const int lane = threadIdx.x & 31;
+    if (lane >= C || dbg.skip_tile == tile) return;
+    float incv[S];
+    total.apply(carry, incv);
+#pragma unroll
+    for (int q = 0; q < S; ++q) st_relaxed_u64(lb.inc + (tile * C + lane) * S + q, pack_tag(incv[q], epoch));
+}
+
+// The whole look-back for one tile: publish the aggregate, resolve the carry, publish
+// the inclusive value, leave the carry in sm.carry.  Returns false on a timeout.
 template <int S, int C>
 __device__ bool look_back(const LookBack<S> &lb, ScanSmem<S, C> &sm, const Aff<S> &total, long tile,
                           int chunk, long nseq, unsigned epoch, const float *base /* [S], channel c */,
                           Ctl *ctl, int *sticky, const Dbg &dbg) {
-    constexpr int WIN = 32 / C;
-    constexpr int KF = Aff<S>::kFloats;
-    const int lane = threadIdx.x & 31, i = lane / C, c = lane % C;
-    const bool publish = (dbg.skip_tile != tile);
+    const int lane = threadIdx.x & 31;
+    publish_agg<S, C>(lb, total, tile, chunk, epoch, dbg);
     float carry[S];
-    bool ok = true;
-    if (chunk == 0) {
+    if (!resolve_carry<S, C>(lb, tile, chunk, nseq, epoch, base, carry, ctl, sticky, dbg)) return false;
+    publish_inc<S, C>(lb, total, carry, tile, epoch, dbg);
+    if (lane < C) {
 #pragma unroll
-        for (int q = 0; q < S; ++q) carry[q] = base[q];
-    } else {
-        if (lane < C && publish) {
-            float tv[KF];
-            total.to_floats(tv);
-#pragma unroll
-            for (int q = 0; q < KF; ++q) st_relaxed_u64(lb.agg + (tile * C + c) * KF + q, pack_tag(tv[q], epoch));
-        }
-        Aff<S> acc = Aff<S>::ident();  // composition of everything between here and the window
-        long pred = tile - nseq;
-        int pchunk = chunk - 1;
-        bool done = false;
-        while (!done) {
-            const int my_chunk = pchunk - i;
-            const long my_tile = pred - (long)i * nseq;
-            unsigned st = 3u;  // 3: start of the sequence
-            float iv[S], av[KF];
-            if (my_chunk >= 0) {
-                unsigned long long t0 = 0;
-                int polls = 0;
-                for (;;) {
-                    unsigned long long wi[S], wa[KF];
-#pragma unroll
-                    for (int q = 0; q < S; ++q) wi[q] = ld_relaxed_u64(lb.inc + (my_tile * C + c) * S + q);
-#pragma unroll
-                    for (int q = 0; q < KF; ++q) wa[q] = ld_relaxed_u64(lb.agg + (my_tile * C + c) * KF + q);
-                    bool inc_ok = true, agg_ok = true;
-#pragma unroll
-                    for (int q = 0; q < S; ++q) {
-                        inc_ok &= (unsigned)wi[q] == epoch;
-                        iv[q] = __uint_as_float((unsigned)(wi[q] >> 32));
-                    }
-#pragma unroll
-                    for (int q = 0; q < KF; ++q) {
-                        agg_ok &= (unsigned)wa[q] == epoch;
-                        av[q] = __uint_as_float((unsigned)(wa[q] >> 32));
-                    }
-                    if (inc_ok) { st = kFlagInc; break; }
-                    if (agg_ok) { st = kFlagAgg; break; }
-                    if (ld_relaxed_int(&ctl->abort)) { ok = false; break; }
-                    if (++polls == 4) t0 = gtimer();
-                    if (polls > 4) {
-                        if (gtimer() - t0 > dbg.wait_ns) {
-                            raise_status(sticky, ctl, kStTimeout, true);
-                            ok = false;
-                            break;
-                        }
-                        __nanosleep(20);
-                    }
-                }
-            }
-            __syncwarp();
-            if (__any_sync(0xffffffffu, !ok)) { ok = false; break; }
-            Aff<S> v;
-            if (st == 3u)
-                v = Aff<S>::cst(base);
-            else if (st == kFlagInc)
-                v = Aff<S>::cst(iv);
-            else
-                v = Aff<S>::from_floats(av);
-            const unsigned stop = __ballot_sync(0xffffffffu, st != kFlagAgg);
-            const int first = stop ? (__ffs(stop) - 1) / C : WIN;  // first slot with a known value
-            if (i > first) v = Aff<S>::ident();
-            // reduce the window: slot 0 is the nearest predecessor (applied last)
-#pragma unroll
-            for (int off = C; off < 32; off <<= 1) {
-                Aff<S> o = v.shfl_down(off);
-                if (lane + off < 32) v = compose(o, v);
-            }
-            acc = compose(v, acc);
-            if (stop) {
-                float z[S];
-#pragma unroll
-                for (int q = 0; q < S; ++q) z[q] = 0.f;
-                acc.apply(z, carry);  // acc is a constant map here
-                done = true;
-            } else {
-                pred -= (long)WIN * nseq;
-                pchunk -= WIN;
-            }
-        }
+        for (int q = 0; q < S; ++q) sm.carry[lane][q] = carry[q];
     }
-    if (ok && lane < C) {
-        float incv[S];
-        total.apply(carry, incv);
-        if (publish) {
-#pragma unroll
-            for (int q = 0; q < S; ++q) st_relaxed_u64(lb.inc + (tile * C + c) * S + q, pack_tag(incv[q], epoch));
-        }
-#pragma unroll
-        for (int q = 0; q < S; ++q) sm.carry[c][q] = carry[q];
-    }
-    return ok;
+    return true;
 }
 
 // Block-wide max of a non-negative float (NaN propagates as a NaN bit pattern).

@@ -47,16 +47,25 @@ __device__ __forceinline__ void copy_segments(float *dst, int seg, int str, cons
     }
 }
 
+// Padded stride (floats) for a per-thread segment of `seg` floats read as float4: the
+// stride in 16-byte chunks must be odd so that a quarter-warp's 128-bit reads hit
+// distinct bank groups.
+constexpr int pad_stride(int seg) { return ((seg / 4) % 2 == 0) ? seg + 4 : seg + 8; }
+
+// Shared memory the staged kernel uses beyond the input stage: per step and thread,
+// the local prefix product Q (S*S floats), the local update D (S) and h^(k) (S),
+// stored transposed ([component][step][thread]) so every access is conflict-free.
+template <int S, int L> constexpr int park_floats() { return (S * S + 2 * S) * L * kThreads; }
+
 // ---------------------------------------------------------------- long layout, H == 1
-template <class Cell, int IN> struct LongLayout {
-    static constexpr int S = Cell::S, C = 1, L = S == 1 ? 16 : 8, SUB = kThreads, TCH = SUB * L;
+template <class Cell, int IN, int LL> struct LongLayout {
+    static constexpr int S = Cell::S, C = 1, L = LL, SUB = kThreads, TCH = SUB * L;
     static constexpr int PW = IN == 0 ? 3 : IN;     // input floats per step
-    static constexpr int SEGP = L * PW, STRP = SEGP + 4;
-    static constexpr int SEGH = L * S, STRH = SEGH + 4;
+    static constexpr int SEGP = L * PW, STRP = pad_stride(SEGP);
+    static constexpr int SEGH = L * S, STRH = pad_stride(SEGH);
     static constexpr int OFFH = SUB * STRP;
     static constexpr int SMEM_FLOATS = SUB * (STRP + STRH);
     static_assert(SEGP % 4 == 0 && SEGH % 4 == 0, "segments are whole 16-byte chunks");
-    static_assert(((SEGP / 4 + 1) & 1) && ((SEGH / 4 + 1) & 1), "odd chunk stride: conflict-free float4 reads");
 
     __device__ static void issue(const NewtonDiagArgs &A, float *sm, int b, int, int tch0, bool with_h) {
         const size_t row = (size_t)b * A.T;
@@ -103,11 +112,30 @@ template <class Cell, int IN> struct LongLayout {
 #pragma unroll
         for (int q = 0; q < S; ++q) hp[q] = sm[OFFH + (s - 1) * STRH + SEGH - S + q];
     }
+    // Coalesced store of a finished tile: out[q][i][thread] (parked) -> h[b, tch0 .. +TCH).
+    __device__ static void store_tile(const NewtonDiagArgs &A, const float *out, int b, int, int tch0) {
+        const size_t row = (size_t)b * A.T;
+        const int valid = min(TCH, A.T - tch0) * S;  // floats of this tile inside the sequence
+        float *g = A.h + (row + tch0) * S;
+        for (int f = 4 * threadIdx.x; f < valid; f += 4 * kThreads) {
+            float v[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int fe = f + e, t = fe / S, q = fe % S;
+                v[e] = out[(q * L + t % L) * kThreads + t / L];
+            }
+            if (f + 4 <= valid) {
+                *reinterpret_cast<float4 *>(g + f) = make_float4(v[0], v[1], v[2], v[3]);
+            } else {
+                for (int e = 0; f + e < valid; ++e) g[f + e] = v[e];
+            }
+        }
+    }
 };
 
 // ---------------------------------------------------------------- wide layout, H % 32 == 0
-template <class Cell> struct WideLayout {
-    static constexpr int S = Cell::S, C = 32, L = S == 1 ? 16 : 8, SUB = kThreads / C, TCH = SUB * L;
+template <class Cell, int LL> struct WideLayout {
+    static constexpr int S = Cell::S, C = 32, L = LL, SUB = kThreads / C, TCH = SUB * L;
     static constexpr int PW = 3;
     static constexpr int ROWP = 3 * 32, ROWH = 32 * S;
     static constexpr int OFFH = TCH * ROWP;
@@ -153,14 +181,34 @@ template <class Cell> struct WideLayout {
 #pragma unroll
         for (int q = 0; q < S; ++q) hp[q] = sm[OFFH + (s * L - 1) * ROWH + c * S + q];
     }
+    // Coalesced store: each step is a 32 * S float row of the tile's channels.
+    __device__ static void store_tile(const NewtonDiagArgs &A, const float *out, int b, int ct, int tch0) {
+        const size_t row = (size_t)b * A.T;
+        const int steps = min(TCH, A.T - tch0);
+        for (int q = threadIdx.x; q < steps * 8 * S; q += kThreads) {
+            const int t = q / (8 * S), part = q % (8 * S);
+            float v[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int f = part * 4 + e, c = f / S, k = f % S;
+                v[e] = out[(k * L + t % L) * kThreads + (t / L) * 32 + c];
+            }
+            *reinterpret_cast<float4 *>(A.h + ((row + tch0 + t) * A.H + ct * 32) * S + part * 4) =
+                make_float4(v[0], v[1], v[2], v[3]);
+        }
+    }
 };
 
 template <class Cell, class Lay, int IN>
 __global__ void __launch_bounds__(kThreads, PRN_STAGED_MINB) newton_staged_kernel(const NewtonDiagArgs A) {
     constexpr int S = Cell::S, C = Lay::C, L = Lay::L, SUB = Lay::SUB, TCH = Lay::TCH, PW = Lay::PW;
+    constexpr int SS = S * S;
     static_assert(L % 4 == 0, "steps are read in groups of four");
     extern __shared__ __align__(16) float smem[];
+    float *const park = smem + Lay::SMEM_FLOATS;  // [SS + 2S][L][kThreads]
+    float *const parkQ = park, *const parkD = park + SS * L * kThreads, *const parkH = park + (SS + S) * L * kThreads;
     __shared__ ScanSmem<S, C> sm;
+    __shared__ float s_carry[C][S];
     __shared__ unsigned s_red[kThreads / 32];
     __shared__ int s_fail;
     const int tid = threadIdx.x, c = tid % C, s = tid / C;
@@ -202,11 +250,74 @@ __global__ void __launch_bounds__(kThreads, PRN_STAGED_MINB) newton_staged_kerne
         const float *side_in = A.side + (size_t)(k & 1) * side_stride;
         float *side_out = A.side + (size_t)((k + 1) & 1) * side_stride;
         float my_max = 0.f;
+
+        // the tile whose carry is still pending (its per-step values are parked)
+        long ptile = -1;
+        int pb = 0, pct = 0, pchunk = 0;
+        Aff<S> pexcl = Aff<S>::ident(), ptotal = Aff<S>::ident();
+
+        // Resolve the pending tile's carry (look-back), publish its inclusive value,
+        // finish its states from the parked values and store them coalesced.
+        auto finish_pending = [&]() -> bool {
+            if (tid < 32) {
+                float base[S], carry[S];
+#pragma unroll
+                for (int q = 0; q < S; ++q) base[q] = 0.f;  // delta entering t = 0 is 0
+                if (!resolve_carry<S, C>(lb, ptile, pchunk, nseq, epoch, base, carry, A.ctl, A.sticky, A.dbg)) {
+                    if (tid == 0) s_fail = 1;
+                } else {
+                    publish_inc<S, C>(lb, ptotal, carry, ptile, epoch, A.dbg);
+                    if (tid < C) {
+#pragma unroll
+                        for (int q = 0; q < S; ++q) s_carry[tid][q] = carry[q];
+                    }
+                }
+            }
+            __syncthreads();
+            if (s_fail) return false;
+            float din[S];
+            pexcl.apply(s_carry[c], din);
+            const int t0 = pchunk * TCH + s * L;
+#pragma unroll
+            for (int i = 0; i < L; ++i) {
+                float qm[SS], dv[S], hv[S];
+#pragma unroll
+                for (int q = 0; q < SS; ++q) qm[q] = parkQ[(q * L + i) * kThreads + tid];
+#pragma unroll
+                for (int q = 0; q < S; ++q) {
+                    dv[q] = parkD[(q * L + i) * kThreads + tid];
+                    hv[q] = parkH[(q * L + i) * kThreads + tid];
+                }
+                float out[S];
+#pragma unroll
+                for (int r = 0; r < S; ++r) {
+                    float d = dv[r];
+#pragma unroll
+                    for (int q = 0; q < S; ++q) d = fmaf(qm[r * S + q], din[q], d);
+                    out[r] = hv[r] + d;
+                    if (t0 + i < A.T) {
+                        const float ad = fabsf(d);
+                        my_max = (ad > my_max || isnan(d)) ? ad : my_max;
+                    }
+                    parkH[(r * L + i) * kThreads + tid] = out[r];
+                }
+                if (i == L - 1 && s == SUB - 1 && pchunk < nchunk - 1) {
+#pragma unroll
+                    for (int q = 0; q < S; ++q) side_out[(ptile * C + c) * S + q] = out[q];
+                }
+            }
+            __syncthreads();
+            Lay::store_tile(A, parkH, pb, pct, pchunk * TCH);
+            __syncthreads();
+            return true;
+        };
+
         for (long tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
             const int chunk = (int)(tile / nseq);
             const long seq = tile - (long)chunk * nseq;
             const int b = (int)(seq / nct);
-            const int h = (int)(seq % nct) * C + c;
+            const int ct = (int)(seq % nct);
+            const int h = ct * C + c;
             const int t0 = chunk * TCH + s * L;
             cp_async_wait_all();
             __syncthreads();
@@ -225,7 +336,13 @@ __global__ void __launch_bounds__(kThreads, PRN_STAGED_MINB) newton_staged_kerne
                     Lay::h_prev(smem, s, c, hp);
                 }
             }
-            float Jr[L][S * S], rr[L][S], hc[L][S];
+            // local walk with zero carry: Q_i = J_i..J_0, D_i = local update after step i
+            float Qv[L][SS], Dv[L][S], Hv[L][S];
+            float Qc[SS], Dc[S];
+#pragma unroll
+            for (int q = 0; q < SS; ++q) Qc[q] = (q % (S + 1)) == 0 ? 1.f : 0.f;
+#pragma unroll
+            for (int q = 0; q < S; ++q) Dc[q] = 0.f;
 #pragma unroll
             for (int grp = 0; grp < L / 4; ++grp) {
                 float pv[4][PW], hv[4][S];
@@ -246,18 +363,39 @@ __global__ void __launch_bounds__(kThreads, PRN_STAGED_MINB) newton_staged_kerne
                             p[g] = acc;
                         }
                     }
-                    float cur[S], f[S], J[S * S];
+                    float cur[S], f[S], J[SS];
 #pragma unroll
                     for (int q = 0; q < S; ++q) cur[q] = k > 0 ? hv[j][q] : 0.f;
                     cell.eval(p, hp, f, J);
+                    if (v) {
+                        float nQ[SS], nD[S];
 #pragma unroll
-                    for (int q = 0; q < S; ++q) {
-                        rr[i][q] = v ? f[q] - cur[q] : 0.f;
-                        hc[i][q] = cur[q];
-                        hp[q] = cur[q];
+                        for (int r = 0; r < S; ++r) {
+                            float dd = f[r] - cur[r];
+#pragma unroll
+                            for (int q = 0; q < S; ++q) dd = fmaf(J[r * S + q], Dc[q], dd);
+                            nD[r] = dd;
+#pragma unroll
+                            for (int q2 = 0; q2 < S; ++q2) {
+                                float acc = 0.f;
+#pragma unroll
+                                for (int q = 0; q < S; ++q) acc = fmaf(J[r * S + q], Qc[q * S + q2], acc);
+                                nQ[r * S + q2] = acc;
+                            }
+                        }
+#pragma unroll
+                        for (int q = 0; q < SS; ++q) Qc[q] = nQ[q];
+#pragma unroll
+                        for (int q = 0; q < S; ++q) Dc[q] = nD[q];
                     }
 #pragma unroll
-                    for (int q = 0; q < S * S; ++q) Jr[i][q] = v ? J[q] : ((q % (S + 1)) == 0 ? 1.f : 0.f);
+                    for (int q = 0; q < SS; ++q) Qv[i][q] = Qc[q];
+#pragma unroll
+                    for (int q = 0; q < S; ++q) {
+                        Dv[i][q] = Dc[q];
+                        Hv[i][q] = cur[q];
+                        hp[q] = cur[q];
+                    }
                 }
             }
             __syncthreads();  // the stage is consumed: refill it with the next tile
@@ -268,46 +406,41 @@ __global__ void __launch_bounds__(kThreads, PRN_STAGED_MINB) newton_staged_kerne
                 Lay::issue(A, smem, (int)(nsq / nct), (int)(nsq % nct), nch * TCH, k > 0);
                 cp_async_commit();
             }
-            Aff<S> e = Aff<S>::ident();
-#pragma unroll
-            for (int i = 0; i < L; ++i) e = compose(e, make_aff<S>(Jr[i], rr[i]));
+            Aff<S> e = make_aff<S>(Qc, Dc);
             Aff<S> excl, total;
             cta_scan<S, C>(e, sm, excl, total);
-            if (tid < 32) {
-                float base[S];
-#pragma unroll
-                for (int q = 0; q < S; ++q) base[q] = 0.f;  // delta entering t = 0 is 0
-                if (!look_back<S, C>(lb, sm, total, tile, chunk, nseq, epoch, base, A.ctl, A.sticky, A.dbg))
-                    if ((tid & 31) == 0) s_fail = 1;
-            }
-            __syncthreads();
-            if (s_fail) {
+            if (tid < 32) publish_agg<S, C>(lb, total, tile, chunk, epoch, A.dbg);
+            // the previous tile's look-back has had a whole tile of time to become ready
+            if (ptile >= 0 && !finish_pending()) {
                 cp_async_wait_all();
-                return;  // a bounded wait ran out; the status says so
+                return;
             }
-            float d[S];
-            excl.apply(sm.carry[c], d);
+            // park this tile's per-step values
 #pragma unroll
             for (int i = 0; i < L; ++i) {
-                const int t = t0 + i;
-                float nd[S], hn[S];
-                make_aff<S>(Jr[i], rr[i]).apply(d, nd);
+#pragma unroll
+                for (int q = 0; q < SS; ++q) parkQ[(q * L + i) * kThreads + tid] = Qv[i][q];
 #pragma unroll
                 for (int q = 0; q < S; ++q) {
-                    d[q] = nd[q];
-                    hn[q] = hc[i][q] + nd[q];
-                    const float ad = fabsf(nd[q]);
-                    my_max = (ad > my_max || isnan(nd[q])) ? ad : my_max;
-                }
-                if (t < A.T) store_state<S>(A.h, ((size_t)b * A.T + t) * A.H + h, hn);
-                if (i == L - 1 && s == SUB - 1 && chunk < nchunk - 1) {
-#pragma unroll
-                    for (int q = 0; q < S; ++q) side_out[(tile * C + c) * S + q] = hn[q];
+                    parkD[(q * L + i) * kThreads + tid] = Dv[i][q];
+                    parkH[(q * L + i) * kThreads + tid] = Hv[i][q];
                 }
             }
+            ptile = tile;
+            pb = b;
+            pct = ct;
+            pchunk = chunk;
+            pexcl = excl;
+            ptotal = total;
             if (next >= ntiles) {
-                // last tile of this iteration: prefetch this CTA's first tile for the next one
+                // last tile of this iteration: finish it now, then prefetch this CTA's
+                // first tile for the next iteration
                 __syncthreads();
+                if (!finish_pending()) {
+                    cp_async_wait_all();
+                    return;
+                }
+                ptile = -1;
                 const int nch = (int)(blockIdx.x / nseq);
                 const long nsq = blockIdx.x - (long)nch * nseq;
                 Lay::issue(A, smem, (int)(nsq / nct), (int)(nsq % nct), nch * TCH, true);
@@ -354,12 +487,14 @@ template <class K> int prepare_kernel(K *kern, int smem_bytes) {
     return 0;
 }
 
-template <class Cell, class Lay, int IN> int choose(Plan *plan, int num_sms) {
+template <class Cell, class Lay, int IN> int choose(Plan *plan, int num_sms, long B, long T, long H) {
     auto kern = &newton_staged_kernel<Cell, Lay, IN>;
-    const int smem = Lay::SMEM_FLOATS * (int)sizeof(float);
+    const int smem = (Lay::SMEM_FLOATS + park_floats<Lay::S, Lay::L>()) * (int)sizeof(float);
     if (prepare_kernel(kern, smem)) return -1;
     plan->kernel = reinterpret_cast<const void *>(kern);
     plan->dyn_smem = smem;
+    plan->C = Lay::C;
+    plan->ntiles = B * (H / Lay::C) * ((T + Lay::TCH - 1) / Lay::TCH);
     plan->grid = occupancy_grid(plan->kernel, kThreads, smem, num_sms, plan->ntiles);
     return plan->grid > 0 ? 0 : -1;
 }
@@ -368,42 +503,36 @@ template <class Cell, class Lay, int IN> int choose(Plan *plan, int num_sms) {
 
 // Staged kernels apply to H == 1 (long) or H % 32 == 0 with projected inputs (wide),
 // with 16-byte aligned per-sequence slabs.  Returns 1 when the shape is not covered.
+// Steps per thread (L) are chosen so that the input stage and the parked values of
+// two CTAs fit one SM's shared memory.
 int newton_staged_plan(const NewtonDiagReq &r, int num_sms, Plan *plan) {
     const int S = r.cell == 1 ? 2 : 1;
-    const int L = S == 1 ? 16 : 8;
     const bool fused = r.xproj == nullptr;
+    int rc;
     if (r.H == 1) {
         const int PW = fused ? r.in : 3;
         if (fused && r.in != 1 && r.in != 2 && r.in != 4) return 1;
         if (((long)r.T * PW) % 4 || ((long)r.T * S) % 4) return 1;
-        const int TCH = kThreads * L;
-        plan->ntiles = (long)r.B * ((r.T + TCH - 1) / TCH);
         plan->variant = 101;
-        int rc;
         if (S == 1) {
-            rc = !fused ? choose<GruCell, LongLayout<GruCell, 0>, 0>(plan, num_sms)
-                 : r.in == 1 ? choose<GruCell, LongLayout<GruCell, 1>, 1>(plan, num_sms)
-                 : r.in == 2 ? choose<GruCell, LongLayout<GruCell, 2>, 2>(plan, num_sms)
-                             : choose<GruCell, LongLayout<GruCell, 4>, 4>(plan, num_sms);
+            rc = !fused ? choose<GruCell, LongLayout<GruCell, 0, 8>, 0>(plan, num_sms, r.B, r.T, r.H)
+                 : r.in == 1 ? choose<GruCell, LongLayout<GruCell, 1, 16>, 1>(plan, num_sms, r.B, r.T, r.H)
+                 : r.in == 2 ? choose<GruCell, LongLayout<GruCell, 2, 16>, 2>(plan, num_sms, r.B, r.T, r.H)
+                             : choose<GruCell, LongLayout<GruCell, 4, 8>, 4>(plan, num_sms, r.B, r.T, r.H);
         } else {
-            rc = !fused ? choose<LstmCell, LongLayout<LstmCell, 0>, 0>(plan, num_sms)
-                 : r.in == 1 ? choose<LstmCell, LongLayout<LstmCell, 1>, 1>(plan, num_sms)
-                 : r.in == 2 ? choose<LstmCell, LongLayout<LstmCell, 2>, 2>(plan, num_sms)
-                             : choose<LstmCell, LongLayout<LstmCell, 4>, 4>(plan, num_sms);
+            rc = !fused ? choose<LstmCell, LongLayout<LstmCell, 0, 4>, 0>(plan, num_sms, r.B, r.T, r.H)
+                 : r.in == 1 ? choose<LstmCell, LongLayout<LstmCell, 1, 8>, 1>(plan, num_sms, r.B, r.T, r.H)
+                 : r.in == 2 ? choose<LstmCell, LongLayout<LstmCell, 2, 8>, 2>(plan, num_sms, r.B, r.T, r.H)
+                             : choose<LstmCell, LongLayout<LstmCell, 4, 4>, 4>(plan, num_sms, r.B, r.T, r.H);
         }
-        if (rc) return -1;
-        plan->C = 1;
     } else if (r.H % 32 == 0 && !fused) {
-        const int TCH = (kThreads / 32) * L;
-        plan->ntiles = (long)r.B * (r.H / 32) * ((r.T + TCH - 1) / TCH);
         plan->variant = 132;
-        int rc = S == 1 ? choose<GruCell, WideLayout<GruCell>, 0>(plan, num_sms)
-                        : choose<LstmCell, WideLayout<LstmCell>, 0>(plan, num_sms);
-        if (rc) return -1;
-        plan->C = 32;
+        rc = S == 1 ? choose<GruCell, WideLayout<GruCell, 12>, 0>(plan, num_sms, r.B, r.T, r.H)
+                    : choose<LstmCell, WideLayout<LstmCell, 8>, 0>(plan, num_sms, r.B, r.T, r.H);
     } else {
         return 1;
     }
+    if (rc) return -1;
     plan->agg_words = (size_t)plan->ntiles * plan->C * (S == 1 ? 2 : 6);
     plan->inc_words = (size_t)plan->ntiles * plan->C * S;
     plan->side_bytes = 2 * (size_t)plan->ntiles * plan->C * S * sizeof(float);

@@ -29,6 +29,10 @@ struct Plan {
     const void *kernel = nullptr;  // for the launch
     int dyn_smem = 0;
     int variant = 0;
+    int tch = 0;                   // steps per tile
+    int staged = 0;                // Newton: staged kernel (args + tensor maps)
+    int staged_tma = 0;            // staged kernel fed by TMA
+    int S = 1;                     // state components per unit
 };
 
 struct DbgHost {

@@ -1,8 +1,11 @@
 // newton_common.cuh -- pieces shared by the Newton kernels for diagonal and 2x2-block
 // cells: kernel arguments, projected-input access, state access, residual pass.
 #pragma once
+#include <cuda.h>
+
 #include "cells.cuh"
 #include "common.cuh"
+#include "internal.h"
 
 namespace prn {
 
@@ -102,6 +105,14 @@ __device__ __forceinline__ void store_state(float *hbuf, size_t idx, const float
         *reinterpret_cast<float2 *>(hbuf + idx * 2) = make_float2(v[0], v[S - 1]);
     }
 }
+
+// Tensor maps handed to the staged kernels (unused by the layouts without TMA).
+struct StagedMaps {
+    CUtensorMap x, h;
+};
+
+// Launch of a staged plan (newton_staged.cu).
+cudaError_t newton_staged_launch(const NewtonDiagArgs &A, const Plan &plan, cudaStream_t st);
 
 // Final residual r = max over every state element of |h_t - f(h_{t-1}, x_t)| at the
 // returned iterate (one read of the states and inputs), reduced over the grid.

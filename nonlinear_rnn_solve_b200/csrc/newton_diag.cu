@@ -261,6 +261,7 @@ cudaError_t newton_diag_launch(const NewtonDiagReq &r, const Plan &plan, const W
     A.dbg.skip_tile = dbg.skip_tile;
     A.dbg.delta_log = dbg.delta_log;
     A.dbg.delta_log_cap = dbg.delta_log_cap;
+    if (plan.staged) return newton_staged_launch(A, plan, st);
     void *args[] = {&A};
     return cudaLaunchCooperativeKernel(plan.kernel, dim3(plan.grid), dim3(kThreads), args, plan.dyn_smem, st);
 }

@@ -1,19 +1,21 @@
-// newton_staged.cu -- Newton (DEER) forward for ParaGRU / ParaLSTM with the tile's
-// inputs staged in shared memory by asynchronous copies (cp.async), so that the HBM
-// reads of the next tile overlap the scan, look-back and stores of the current one.
+// newton_staged.cu -- Newton (DEER) forward for ParaGRU / ParaLSTM with each tile's
+// inputs staged in shared memory ahead of use, so that the HBM reads of the next tile
+// overlap the scan, look-back and stores of the current one.
 //
 // Same method as newton_diag.cu ("Parallelizing non-linear sequential models over
 // the sequence length", Approach: linearise, then solve the linear recurrence with a
-// parallel prefix scan), specialised for the two shapes that carry the traffic:
-//   long  (H == 1): a tile is 256 threads x L consecutive steps of one sequence; each
-//         thread's segment sits in shared memory with a 16-byte pad so that its
-//         128-bit reads are free of bank conflicts;
-//   wide  (H % 32 == 0, projected inputs given): a tile is 32 channels x 8 sub-chunks
-//         of L steps; every step is a 128-byte row per gate and per state, read by a
-//         warp as one conflict-free row.
-// Copies are issued as soon as the previous tile's slab has been read into registers
-// (single stage, released early); the first tile of the next Newton iteration is
-// prefetched right after this CTA's last stores, before the grid barrier.
+// parallel prefix scan), specialised for the shapes that carry the traffic:
+//   TmaLong (H == 1, raw inputs of width <= 4): one thread streams the tile's inputs
+//         and states with 2-D TMA copies into 128-byte-swizzled shared memory; every
+//         thread reads its L consecutive steps as conflict-free 128-bit loads; results
+//         go through a swizzled staging tile and leave as coalesced 16-byte stores;
+//   CpLong (other H == 1 shapes): cp.async copies into padded per-thread segments;
+//   Wide  (H % 32 == 0, projected inputs given): a tile is 32 channels x 8 sub-chunks
+//         of L steps; every step is a 128-byte row per gate and per state.
+// A tile whose steps all lie inside the sequence takes a path without per-step guards.
+#include <cuda.h>
+#include <string.h>
+
 #include <algorithm>
 
 #include "cells.cuh"
@@ -34,6 +36,34 @@ __device__ __forceinline__ void cp_async16(float *dst, const float *src, int src
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
+__device__ __forceinline__ unsigned smem_addr(const void *p) { return (unsigned)__cvta_generic_to_shared(p); }
+__device__ __forceinline__ void mbar_init(unsigned long long *bar, unsigned count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(unsigned long long *bar, unsigned bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ bool mbar_try(unsigned long long *bar, unsigned parity) {
+    unsigned ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int x, int y,
+                                            unsigned long long *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+        "[%4];" ::"r"(smem_addr(dst)),
+        "l"(reinterpret_cast<unsigned long long>(map)), "r"(x), "r"(y), "r"(smem_addr(bar))
+        : "memory");
+}
+
 // Copy n floats (n % 4 == 0) from a 16-byte aligned global address into consecutive
 // segments of `seg` floats placed `str` floats apart; bytes at or beyond `end` are
 // zero-filled.  Consecutive threads copy consecutive 16-byte chunks (coalesced).
@@ -52,30 +82,120 @@ __device__ __forceinline__ void copy_segments(float *dst, int seg, int str, cons
 // distinct bank groups.
 constexpr int pad_stride(int seg) { return ((seg / 4) % 2 == 0) ? seg + 4 : seg + 8; }
 
-// Shared memory the staged kernel uses beyond the input stage: per step and thread,
-// the local prefix product Q (S*S floats), the local update D (S) and h^(k) (S),
-// stored transposed ([component][step][thread]) so every access is conflict-free.
-template <int S, int L> constexpr int park_floats() { return (S * S + 2 * S) * L * kThreads; }
+// ---------------------------------------------------------------- TMA long layout, H == 1
+// A slab of the tile is a run of 128-byte rows; TMA writes row r's 16-byte chunk j at
+// chunk position j ^ (r % 8) of its 1024-byte group.  Thread s's segment of `SEG` floats
+// (8, 16 or 32) is part of one row, so its 128-bit reads land on distinct bank groups
+// across each quarter-warp.
+template <int SEG> __device__ __forceinline__ float4 *swz_chunk(float *region, int s, int j) {
+    const int f = s * SEG + 4 * j;  // float offset of the chunk in the slab
+    const int row = f >> 5, lc = (f >> 2) & 7;
+    return reinterpret_cast<float4 *>(region + row * 32 + ((lc ^ (row & 7)) << 2));
+}
+__device__ __forceinline__ float swz_float(const float *region, int f) {
+    const int row = f >> 5, lc = (f >> 2) & 7;
+    return region[row * 32 + ((lc ^ (row & 7)) << 2) + (f & 3)];
+}
 
-// ---------------------------------------------------------------- long layout, H == 1
-template <class Cell, int IN, int LL> struct LongLayout {
+template <class Cell, int IN, int LL> struct TmaLong {
+    static constexpr int S = Cell::S, C = 1, L = LL, SUB = kThreads, TCH = SUB * L, PW = IN;
+    static constexpr int SEGP = L * PW, SEGH = L * S;
+    static_assert(SEGP == 8 || SEGP == 16 || SEGP == 32, "input segment must be part of one 128-byte row");
+    static_assert(SEGH == 8 || SEGH == 16 || SEGH == 32, "state segment must be part of one 128-byte row");
+    static constexpr int XFLOATS = TCH * PW, HFLOATS = TCH * S;
+    static_assert(XFLOATS / 32 <= 256 && HFLOATS / 32 <= 256, "TMA box height");
+    // regions: X | H | OUT, each a multiple of 1024 bytes
+    static constexpr int OFFH = XFLOATS, OFFO = XFLOATS + HFLOATS;
+    static constexpr int SMEM_FLOATS = XFLOATS + 2 * HFLOATS;
+    static constexpr bool kTma = true;
+
+    __device__ static void issue(const NewtonDiagArgs &A, const StagedMaps &M, float *sm, unsigned long long *bar,
+                                 int b, int, int tch0, bool with_h) {
+        const int rowx = (int)(((long)b * A.T + tch0) * PW / 32), rowh = (int)(((long)b * A.T + tch0) * S / 32);
+        mbar_expect_tx(bar, (unsigned)(XFLOATS + (with_h ? HFLOATS : 0)) * 4u);
+        tma_load_2d(sm, &M.x, 0, rowx, bar);
+        if (with_h) tma_load_2d(sm + OFFH, &M.h, 0, rowh, bar);
+    }
+    __device__ static void load_group(float *sm, int s, int, int grp, float pv[4][PW], float hv[4][S], bool with_h) {
+        float tp[4 * PW];
+#pragma unroll
+        for (int q = 0; q < PW; ++q) {
+            const float4 v = *swz_chunk<SEGP>(sm, s, grp * PW + q);
+            tp[4 * q] = v.x;
+            tp[4 * q + 1] = v.y;
+            tp[4 * q + 2] = v.z;
+            tp[4 * q + 3] = v.w;
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+#pragma unroll
+            for (int q = 0; q < PW; ++q) pv[j][q] = tp[j * PW + q];
+        if (with_h) {
+            float th[4 * S];
+#pragma unroll
+            for (int q = 0; q < S; ++q) {
+                const float4 v = *swz_chunk<SEGH>(sm + OFFH, s, grp * S + q);
+                th[4 * q] = v.x;
+                th[4 * q + 1] = v.y;
+                th[4 * q + 2] = v.z;
+                th[4 * q + 3] = v.w;
+            }
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+#pragma unroll
+                for (int q = 0; q < S; ++q) hv[j][q] = th[j * S + q];
+        }
+    }
+    __device__ static void h_prev(float *sm, int s, int, float *hp) {
+#pragma unroll
+        for (int q = 0; q < S; ++q) hp[q] = swz_float(sm + OFFH, s * SEGH - S + q);
+    }
+    // results of steps 4*grp .. 4*grp + 3 of thread s, into the staging tile
+    __device__ static void put_group(const NewtonDiagArgs &, float *sm, int s, int, int grp, const float hn[4][S], int,
+                                     int, int) {
+#pragma unroll
+        for (int q = 0; q < S; ++q) {
+            float v[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) v[e] = hn[(4 * q + e) / S][(4 * q + e) % S];
+            *swz_chunk<SEGH>(sm + OFFO, s, grp * S + q) = make_float4(v[0], v[1], v[2], v[3]);
+        }
+    }
+    // coalesced 16-byte stores of the staged results of the tile
+    __device__ static void flush(const NewtonDiagArgs &A, float *sm, int b, int, int tch0) {
+        __syncthreads();
+        const int valid = min(TCH, A.T - tch0) * S;
+        float *g = A.h + ((size_t)b * A.T + tch0) * S;
+        const float *o = sm + OFFO;
+        for (int c = threadIdx.x; 4 * c < valid; c += kThreads) {
+            const int row = c >> 3, lc = c & 7;
+            const float4 v = *reinterpret_cast<const float4 *>(o + row * 32 + ((lc ^ (row & 7)) << 2));
+            *reinterpret_cast<float4 *>(g + 4 * c) = v;
+        }
+        __syncthreads();
+    }
+};
+
+// ---------------------------------------------------------------- cp.async long layout, H == 1
+template <class Cell, int IN, int LL> struct CpLong {
     static constexpr int S = Cell::S, C = 1, L = LL, SUB = kThreads, TCH = SUB * L;
-    static constexpr int PW = IN == 0 ? 3 : IN;     // input floats per step
+    static constexpr int PW = IN == 0 ? 3 : IN;  // input floats per step
     static constexpr int SEGP = L * PW, STRP = pad_stride(SEGP);
     static constexpr int SEGH = L * S, STRH = pad_stride(SEGH);
     static constexpr int OFFH = SUB * STRP;
     static constexpr int SMEM_FLOATS = SUB * (STRP + STRH);
+    static constexpr bool kTma = false;
     static_assert(SEGP % 4 == 0 && SEGH % 4 == 0, "segments are whole 16-byte chunks");
 
-    __device__ static void issue(const NewtonDiagArgs &A, float *sm, int b, int, int tch0, bool with_h) {
+    __device__ static void issue(const NewtonDiagArgs &A, const StagedMaps &, float *sm, unsigned long long *, int b,
+                                 int, int tch0, bool with_h) {
         const size_t row = (size_t)b * A.T;
         const float *pin = IN == 0 ? A.xproj : A.x;
         copy_segments(sm, SEGP, STRP, pin + (row + tch0) * PW, TCH * PW, pin + (row + A.T) * PW);
         if (with_h) copy_segments(sm + OFFH, SEGH, STRH, A.h + (row + tch0) * S, TCH * S, A.h + (row + A.T) * S);
+        cp_async_commit();
     }
-    // four consecutive steps (grp) of thread (s, c): inputs and states from shared memory
-    __device__ static void load_group(const float *sm, int s, int, int grp, float pv[4][PW], float hv[4][S],
-                                      bool with_h) {
+    __device__ static void load_group(float *sm, int s, int, int grp, float pv[4][PW], float hv[4][S], bool with_h) {
         const float4 *pp = reinterpret_cast<const float4 *>(sm + s * STRP + grp * 4 * PW);
         float tmp[4 * PW];
 #pragma unroll
@@ -107,43 +227,31 @@ template <class Cell, int IN, int LL> struct LongLayout {
                 for (int q = 0; q < S; ++q) hv[j][q] = th[j * S + q];
         }
     }
-    // state at the step before thread s's first step (s > 0): last step of thread s - 1
-    __device__ static void h_prev(const float *sm, int s, int, float *hp) {
+    __device__ static void h_prev(float *sm, int s, int, float *hp) {
 #pragma unroll
         for (int q = 0; q < S; ++q) hp[q] = sm[OFFH + (s - 1) * STRH + SEGH - S + q];
     }
-    // Coalesced store of a finished tile: out[q][i][thread] (parked) -> h[b, tch0 .. +TCH).
-    __device__ static void store_tile(const NewtonDiagArgs &A, const float *out, int b, int, int tch0) {
-        const size_t row = (size_t)b * A.T;
-        const int valid = min(TCH, A.T - tch0) * S;  // floats of this tile inside the sequence
-        float *g = A.h + (row + tch0) * S;
-        for (int f = 4 * threadIdx.x; f < valid; f += 4 * kThreads) {
-            float v[4];
+    __device__ static void put_group(const NewtonDiagArgs &A, float *, int, int, int, const float hn[4][S], int b,
+                                     int t, int) {
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int fe = f + e, t = fe / S, q = fe % S;
-                v[e] = out[(q * L + t % L) * kThreads + t / L];
-            }
-            if (f + 4 <= valid) {
-                *reinterpret_cast<float4 *>(g + f) = make_float4(v[0], v[1], v[2], v[3]);
-            } else {
-                for (int e = 0; f + e < valid; ++e) g[f + e] = v[e];
-            }
-        }
+        for (int j = 0; j < 4; ++j)
+            if (t + j < A.T) store_state<S>(A.h, (size_t)b * A.T + t + j, hn[j]);
     }
+    __device__ static void flush(const NewtonDiagArgs &, float *, int, int, int) {}
 };
 
 // ---------------------------------------------------------------- wide layout, H % 32 == 0
-template <class Cell, int LL> struct WideLayout {
+template <class Cell, int LL> struct Wide {
     static constexpr int S = Cell::S, C = 32, L = LL, SUB = kThreads / C, TCH = SUB * L;
     static constexpr int PW = 3;
     static constexpr int ROWP = 3 * 32, ROWH = 32 * S;
     static constexpr int OFFH = TCH * ROWP;
     static constexpr int SMEM_FLOATS = TCH * (ROWP + ROWH);
+    static constexpr bool kTma = false;
 
-    __device__ static void issue(const NewtonDiagArgs &A, float *sm, int b, int ct, int tch0, bool with_h) {
+    __device__ static void issue(const NewtonDiagArgs &A, const StagedMaps &, float *sm, unsigned long long *, int b,
+                                 int ct, int tch0, bool with_h) {
         const size_t row = (size_t)b * A.T;
-        // inputs: TCH x 3 rows of 32 floats (8 chunks each)
         for (int q = threadIdx.x; q < TCH * 3 * 8; q += kThreads) {
             const int r = q >> 3, part = q & 7, t = r / 3, g = r % 3;
             const bool v = tch0 + t < A.T;
@@ -158,9 +266,9 @@ template <class Cell, int LL> struct WideLayout {
                 cp_async16(sm + OFFH + t * ROWH + part * 4, gp, v ? 16 : 0);
             }
         }
+        cp_async_commit();
     }
-    __device__ static void load_group(const float *sm, int s, int c, int grp, float pv[4][PW], float hv[4][S],
-                                      bool with_h) {
+    __device__ static void load_group(float *sm, int s, int c, int grp, float pv[4][PW], float hv[4][S], bool with_h) {
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             const int t = s * L + grp * 4 + j;
@@ -177,40 +285,75 @@ template <class Cell, int LL> struct WideLayout {
             }
         }
     }
-    __device__ static void h_prev(const float *sm, int s, int c, float *hp) {
+    __device__ static void h_prev(float *sm, int s, int c, float *hp) {
 #pragma unroll
         for (int q = 0; q < S; ++q) hp[q] = sm[OFFH + (s * L - 1) * ROWH + c * S + q];
     }
-    // Coalesced store: each step is a 32 * S float row of the tile's channels.
-    __device__ static void store_tile(const NewtonDiagArgs &A, const float *out, int b, int ct, int tch0) {
-        const size_t row = (size_t)b * A.T;
-        const int steps = min(TCH, A.T - tch0);
-        for (int q = threadIdx.x; q < steps * 8 * S; q += kThreads) {
-            const int t = q / (8 * S), part = q % (8 * S);
-            float v[4];
+    // a warp writes 32 consecutive channels of one step: already coalesced
+    __device__ static void put_group(const NewtonDiagArgs &A, float *, int, int, int, const float hn[4][S], int b,
+                                     int t, int h) {
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int f = part * 4 + e, c = f / S, k = f % S;
-                v[e] = out[(k * L + t % L) * kThreads + (t / L) * 32 + c];
-            }
-            *reinterpret_cast<float4 *>(A.h + ((row + tch0 + t) * A.H + ct * 32) * S + part * 4) =
-                make_float4(v[0], v[1], v[2], v[3]);
-        }
+        for (int j = 0; j < 4; ++j)
+            if (t + j < A.T) store_state<S>(A.h, ((size_t)b * A.T + t + j) * A.H + h, hn[j]);
     }
+    __device__ static void flush(const NewtonDiagArgs &, float *, int, int, int) {}
 };
 
+// One tile's compute phase: f, J and the residual for the thread's L steps, read from
+// the staged slab.  FULL: every step lies inside the sequence (no guards).
+template <class Cell, class Lay, int IN, bool FULL>
+__device__ __forceinline__ void tile_compute(const NewtonDiagArgs &A, float *smem, const Cell &cell, int s, int c,
+                                             int t0, int k, float *hp, const float (&wz)[3][IN > 0 ? IN : 1],
+                                             const float (&bz)[3], float (&Jr)[Lay::L][Cell::S * Cell::S],
+                                             float (&rr)[Lay::L][Cell::S], float (&hc)[Lay::L][Cell::S]) {
+    constexpr int S = Cell::S, L = Lay::L, PW = Lay::PW;
+#pragma unroll
+    for (int grp = 0; grp < L / 4; ++grp) {
+        float pv[4][PW], hv[4][S];
+        Lay::load_group(smem, s, c, grp, pv, hv, k > 0);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int i = grp * 4 + j;
+            const bool v = FULL || t0 + i < A.T;
+            float p[3];
+#pragma unroll
+            for (int g = 0; g < 3; ++g) {
+                if (IN == 0) {
+                    p[g] = pv[j][g];
+                } else {
+                    float acc = bz[g];
+#pragma unroll
+                    for (int q = 0; q < (IN > 0 ? IN : 1); ++q) acc = fmaf(wz[g][q], pv[j][q % PW], acc);
+                    p[g] = acc;
+                }
+            }
+            float cur[S], f[S], J[S * S];
+#pragma unroll
+            for (int q = 0; q < S; ++q) cur[q] = k > 0 ? hv[j][q] : 0.f;
+            cell.eval(p, hp, f, J);
+#pragma unroll
+            for (int q = 0; q < S; ++q) {
+                rr[i][q] = v ? f[q] - cur[q] : 0.f;
+                hc[i][q] = cur[q];
+                hp[q] = cur[q];
+            }
+#pragma unroll
+            for (int q = 0; q < S * S; ++q) Jr[i][q] = v ? J[q] : ((q % (S + 1)) == 0 ? 1.f : 0.f);
+        }
+    }
+}
+
 template <class Cell, class Lay, int IN>
-__global__ void __launch_bounds__(kThreads, PRN_STAGED_MINB) newton_staged_kernel(const NewtonDiagArgs A) {
-    constexpr int S = Cell::S, C = Lay::C, L = Lay::L, SUB = Lay::SUB, TCH = Lay::TCH, PW = Lay::PW;
-    constexpr int SS = S * S;
-    static_assert(L % 4 == 0, "steps are read in groups of four");
-    extern __shared__ __align__(16) float smem[];
-    float *const park = smem + Lay::SMEM_FLOATS;  // [SS + 2S][L][kThreads]
-    float *const parkQ = park, *const parkD = park + SS * L * kThreads, *const parkH = park + (SS + S) * L * kThreads;
+__global__ void __launch_bounds__(kThreads, PRN_STAGED_MINB)
+    newton_staged_kernel(const NewtonDiagArgs A, const __grid_constant__ StagedMaps M) {
+    constexpr int S = Cell::S, C = Lay::C, L = Lay::L, SUB = Lay::SUB, TCH = Lay::TCH;
+    static_assert(L % 4 == 0, "steps are handled in groups of four");
+    extern __shared__ __align__(1024) unsigned char smraw[];
+    float *const smem = reinterpret_cast<float *>(((uintptr_t)smraw + 1023) & ~(uintptr_t)1023);
     __shared__ ScanSmem<S, C> sm;
-    __shared__ float s_carry[C][S];
     __shared__ unsigned s_red[kThreads / 32];
     __shared__ int s_fail;
+    __shared__ __align__(8) unsigned long long s_bar;
     const int tid = threadIdx.x, c = tid % C, s = tid / C;
     const int nct = A.H / C;
     const long nseq = (long)A.B * nct;
@@ -218,9 +361,17 @@ __global__ void __launch_bounds__(kThreads, PRN_STAGED_MINB) newton_staged_kerne
     const long ntiles = nseq * nchunk;
     const size_t side_stride = (size_t)ntiles * C * S;
     LookBack<S> lb{A.agg, A.inc};
-    if (tid == 0) s_fail = 0;
+    unsigned bar_phase = 0;
+    if (tid == 0) {
+        s_fail = 0;
+        if (Lay::kTma) {
+            mbar_init(&s_bar, 1);
+            asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        }
+    }
+    __syncthreads();
 
-    // fused projection weights (long layout with raw inputs): p_g = bias_g + sum_q W[g][q] x_q
+    // fused projection weights (raw inputs, H == 1): p_g = bias_g + sum_q W[g][q] x_q
     float wz[3][IN > 0 ? IN : 1], bz[3];
 #pragma unroll
     for (int g = 0; g < 3; ++g) {
@@ -234,12 +385,54 @@ __global__ void __launch_bounds__(kThreads, PRN_STAGED_MINB) newton_staged_kerne
         }
     }
 
-    {
-        const int chunk = (int)(blockIdx.x / nseq);
-        const long seq = blockIdx.x - (long)chunk * nseq;
-        Lay::issue(A, smem, (int)(seq / nct), (int)(seq % nct), chunk * TCH, false);
-        cp_async_commit();
-    }
+    // Issue a tile's copies.  Data this CTA wrote with ordinary stores is made visible
+    // to the TMA (async proxy) with proxy fences after the preceding barrier.
+    auto issue = [&](long tl, bool with_h) {
+        const int ch = (int)(tl / nseq);
+        const long sq = tl - (long)ch * nseq;
+        if (Lay::kTma) {
+            if (tid == 0) {
+                asm volatile("fence.proxy.async.global;" ::: "memory");
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                Lay::issue(A, M, smem, &s_bar, (int)(sq / nct), (int)(sq % nct), ch * TCH, with_h);
+            }
+        } else {
+            Lay::issue(A, M, smem, &s_bar, (int)(sq / nct), (int)(sq % nct), ch * TCH, with_h);
+        }
+    };
+    // Wait for the staged tile (bounded).  False when the kernel must stop.
+    auto wait_stage = [&]() -> bool {
+        if (Lay::kTma) {
+            bool ok = mbar_try(&s_bar, bar_phase);
+            if (!ok) {
+                const unsigned long long t0 = gtimer();
+                while (!(ok = mbar_try(&s_bar, bar_phase))) {
+                    if (ld_relaxed_int(&A.ctl->abort)) break;
+                    if (gtimer() - t0 > A.dbg.wait_ns) {
+                        raise_status(A.sticky, A.ctl, kStTimeout, true);
+                        break;
+                    }
+                }
+            }
+            bar_phase ^= 1u;
+            return __syncthreads_and(ok) != 0;
+        }
+        cp_async_wait_all();
+        __syncthreads();
+        return true;
+    };
+    // On an abort, let a TMA copy that is still in flight land before the CTA exits
+    // (bounded like every wait).
+    auto drain = [&]() {
+        if (Lay::kTma) {
+            const unsigned long long t0 = gtimer();
+            while (!mbar_try(&s_bar, bar_phase) && gtimer() - t0 < A.dbg.wait_ns) {
+            }
+        } else {
+            cp_async_wait_all();
+        }
+    };
+    issue(blockIdx.x, false);
 
     int iters = 0;
     float last_delta = 0.f;
@@ -250,77 +443,16 @@ __global__ void __launch_bounds__(kThreads, PRN_STAGED_MINB) newton_staged_kerne
         const float *side_in = A.side + (size_t)(k & 1) * side_stride;
         float *side_out = A.side + (size_t)((k + 1) & 1) * side_stride;
         float my_max = 0.f;
-
-        // the tile whose carry is still pending (its per-step values are parked)
-        long ptile = -1;
-        int pb = 0, pct = 0, pchunk = 0;
-        Aff<S> pexcl = Aff<S>::ident(), ptotal = Aff<S>::ident();
-
-        // Resolve the pending tile's carry (look-back), publish its inclusive value,
-        // finish its states from the parked values and store them coalesced.
-        auto finish_pending = [&]() -> bool {
-            if (tid < 32) {
-                float base[S], carry[S];
-#pragma unroll
-                for (int q = 0; q < S; ++q) base[q] = 0.f;  // delta entering t = 0 is 0
-                if (!resolve_carry<S, C>(lb, ptile, pchunk, nseq, epoch, base, carry, A.ctl, A.sticky, A.dbg)) {
-                    if (tid == 0) s_fail = 1;
-                } else {
-                    publish_inc<S, C>(lb, ptotal, carry, ptile, epoch, A.dbg);
-                    if (tid < C) {
-#pragma unroll
-                        for (int q = 0; q < S; ++q) s_carry[tid][q] = carry[q];
-                    }
-                }
-            }
-            __syncthreads();
-            if (s_fail) return false;
-            float din[S];
-            pexcl.apply(s_carry[c], din);
-            const int t0 = pchunk * TCH + s * L;
-#pragma unroll
-            for (int i = 0; i < L; ++i) {
-                float qm[SS], dv[S], hv[S];
-#pragma unroll
-                for (int q = 0; q < SS; ++q) qm[q] = parkQ[(q * L + i) * kThreads + tid];
-#pragma unroll
-                for (int q = 0; q < S; ++q) {
-                    dv[q] = parkD[(q * L + i) * kThreads + tid];
-                    hv[q] = parkH[(q * L + i) * kThreads + tid];
-                }
-                float out[S];
-#pragma unroll
-                for (int r = 0; r < S; ++r) {
-                    float d = dv[r];
-#pragma unroll
-                    for (int q = 0; q < S; ++q) d = fmaf(qm[r * S + q], din[q], d);
-                    out[r] = hv[r] + d;
-                    if (t0 + i < A.T) {
-                        const float ad = fabsf(d);
-                        my_max = (ad > my_max || isnan(d)) ? ad : my_max;
-                    }
-                    parkH[(r * L + i) * kThreads + tid] = out[r];
-                }
-                if (i == L - 1 && s == SUB - 1 && pchunk < nchunk - 1) {
-#pragma unroll
-                    for (int q = 0; q < S; ++q) side_out[(ptile * C + c) * S + q] = out[q];
-                }
-            }
-            __syncthreads();
-            Lay::store_tile(A, parkH, pb, pct, pchunk * TCH);
-            __syncthreads();
-            return true;
-        };
-
+        bool my_bad = false;
         for (long tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
             const int chunk = (int)(tile / nseq);
             const long seq = tile - (long)chunk * nseq;
             const int b = (int)(seq / nct);
             const int ct = (int)(seq % nct);
             const int h = ct * C + c;
-            const int t0 = chunk * TCH + s * L;
-            cp_async_wait_all();
-            __syncthreads();
+            const int tch0 = chunk * TCH;
+            const int t0 = tch0 + s * L;
+            if (!wait_stage()) return;
             Cell cell;
             cell.load(A.a, A.peep, A.H, h);
             float hp[S];
@@ -336,121 +468,69 @@ __global__ void __launch_bounds__(kThreads, PRN_STAGED_MINB) newton_staged_kerne
                     Lay::h_prev(smem, s, c, hp);
                 }
             }
-            // local walk with zero carry: Q_i = J_i..J_0, D_i = local update after step i
-            float Qv[L][SS], Dv[L][S], Hv[L][S];
-            float Qc[SS], Dc[S];
+            float Jr[L][S * S], rr[L][S], hc[L][S];
+            if (tch0 + TCH <= A.T)
+                tile_compute<Cell, Lay, IN, true>(A, smem, cell, s, c, t0, k, hp, wz, bz, Jr, rr, hc);
+            else
+                tile_compute<Cell, Lay, IN, false>(A, smem, cell, s, c, t0, k, hp, wz, bz, Jr, rr, hc);
+            __syncthreads();  // the stage is consumed: refill it with the next tile
+            const long next = tile + gridDim.x;
+            if (next < ntiles) issue(next, k > 0);
+            Aff<S> e = Aff<S>::ident();
 #pragma unroll
-            for (int q = 0; q < SS; ++q) Qc[q] = (q % (S + 1)) == 0 ? 1.f : 0.f;
+            for (int i = 0; i < L; ++i) e = compose(e, make_aff<S>(Jr[i], rr[i]));
+            Aff<S> excl, total;
+            cta_scan<S, C>(e, sm, excl, total);
+            if (tid < 32) {
+                float base[S];
 #pragma unroll
-            for (int q = 0; q < S; ++q) Dc[q] = 0.f;
+                for (int q = 0; q < S; ++q) base[q] = 0.f;  // delta entering t = 0 is 0
+                if (!look_back<S, C>(lb, sm, total, tile, chunk, nseq, epoch, base, A.ctl, A.sticky, A.dbg))
+                    if ((tid & 31) == 0) s_fail = 1;
+            }
+            __syncthreads();
+            if (s_fail) {
+                drain();
+                return;  // a bounded wait ran out; the status says so
+            }
+            float d[S];
+            excl.apply(sm.carry[c], d);
 #pragma unroll
             for (int grp = 0; grp < L / 4; ++grp) {
-                float pv[4][PW], hv[4][S];
-                Lay::load_group(smem, s, c, grp, pv, hv, k > 0);
+                float hn[4][S];
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
                     const int i = grp * 4 + j;
-                    const bool v = t0 + i < A.T;
-                    float p[3];
-#pragma unroll
-                    for (int g = 0; g < 3; ++g) {
-                        if (IN == 0) {
-                            p[g] = pv[j][g];
-                        } else {
-                            float acc = bz[g];
-#pragma unroll
-                            for (int q = 0; q < (IN > 0 ? IN : 1); ++q) acc = fmaf(wz[g][q], pv[j][q % PW], acc);
-                            p[g] = acc;
-                        }
-                    }
-                    float cur[S], f[S], J[SS];
-#pragma unroll
-                    for (int q = 0; q < S; ++q) cur[q] = k > 0 ? hv[j][q] : 0.f;
-                    cell.eval(p, hp, f, J);
-                    if (v) {
-                        float nQ[SS], nD[S];
-#pragma unroll
-                        for (int r = 0; r < S; ++r) {
-                            float dd = f[r] - cur[r];
-#pragma unroll
-                            for (int q = 0; q < S; ++q) dd = fmaf(J[r * S + q], Dc[q], dd);
-                            nD[r] = dd;
-#pragma unroll
-                            for (int q2 = 0; q2 < S; ++q2) {
-                                float acc = 0.f;
-#pragma unroll
-                                for (int q = 0; q < S; ++q) acc = fmaf(J[r * S + q], Qc[q * S + q2], acc);
-                                nQ[r * S + q2] = acc;
-                            }
-                        }
-#pragma unroll
-                        for (int q = 0; q < SS; ++q) Qc[q] = nQ[q];
-#pragma unroll
-                        for (int q = 0; q < S; ++q) Dc[q] = nD[q];
-                    }
-#pragma unroll
-                    for (int q = 0; q < SS; ++q) Qv[i][q] = Qc[q];
+                    float nd[S];
+                    make_aff<S>(Jr[i], rr[i]).apply(d, nd);
 #pragma unroll
                     for (int q = 0; q < S; ++q) {
-                        Dv[i][q] = Dc[q];
-                        Hv[i][q] = cur[q];
-                        hp[q] = cur[q];
+                        d[q] = nd[q];
+                        hn[j][q] = hc[i][q] + nd[q];
+                        my_max = fmaxf(my_max, fabsf(nd[q]));
                     }
                 }
-            }
-            __syncthreads();  // the stage is consumed: refill it with the next tile
-            const long next = tile + gridDim.x;
-            if (next < ntiles) {
-                const int nch = (int)(next / nseq);
-                const long nsq = next - (long)nch * nseq;
-                Lay::issue(A, smem, (int)(nsq / nct), (int)(nsq % nct), nch * TCH, k > 0);
-                cp_async_commit();
-            }
-            Aff<S> e = make_aff<S>(Qc, Dc);
-            Aff<S> excl, total;
-            cta_scan<S, C>(e, sm, excl, total);
-            if (tid < 32) publish_agg<S, C>(lb, total, tile, chunk, epoch, A.dbg);
-            // the previous tile's look-back has had a whole tile of time to become ready
-            if (ptile >= 0 && !finish_pending()) {
-                cp_async_wait_all();
-                return;
-            }
-            // park this tile's per-step values
+                Lay::put_group(A, smem, s, c, grp, hn, b, t0 + grp * 4, h);
+                if (grp == L / 4 - 1 && s == SUB - 1 && chunk < nchunk - 1) {
 #pragma unroll
-            for (int i = 0; i < L; ++i) {
-#pragma unroll
-                for (int q = 0; q < SS; ++q) parkQ[(q * L + i) * kThreads + tid] = Qv[i][q];
-#pragma unroll
-                for (int q = 0; q < S; ++q) {
-                    parkD[(q * L + i) * kThreads + tid] = Dv[i][q];
-                    parkH[(q * L + i) * kThreads + tid] = Hv[i][q];
+                    for (int q = 0; q < S; ++q) side_out[(tile * C + c) * S + q] = hn[3][q];
                 }
             }
-            ptile = tile;
-            pb = b;
-            pct = ct;
-            pchunk = chunk;
-            pexcl = excl;
-            ptotal = total;
+            // a NaN or Inf anywhere in the segment reaches its last update (each update
+            // feeds the next through J), where it is caught
+#pragma unroll
+            for (int q = 0; q < S; ++q) my_bad |= !finitef(d[q]);
+            Lay::flush(A, smem, b, ct, tch0);
             if (next >= ntiles) {
-                // last tile of this iteration: finish it now, then prefetch this CTA's
-                // first tile for the next iteration
+                // last tile of this iteration: prefetch this CTA's first tile for the next
                 __syncthreads();
-                if (!finish_pending()) {
-                    cp_async_wait_all();
-                    return;
-                }
-                ptile = -1;
-                const int nch = (int)(blockIdx.x / nseq);
-                const long nsq = blockIdx.x - (long)nch * nseq;
-                Lay::issue(A, smem, (int)(nsq / nct), (int)(nsq % nct), nch * TCH, true);
-                cp_async_commit();
+                issue(blockIdx.x, true);
             }
         }
-        const unsigned bits = block_max_bits(my_max, s_red);
+        const unsigned bits = block_max_bits(my_bad ? __int_as_float(0x7fc00000) : my_max, s_red);
         if (tid == 0) atomicMax(&A.ctl->delta_bits[k % 3], bits);
         if (!grid_sync(A.ctl, A.sticky, A.dbg)) {
-            cp_async_wait_all();
+            drain();
             return;
         }
         const unsigned dbits = ld_acquire(&A.ctl->delta_bits[k % 3]);
@@ -465,7 +545,12 @@ __global__ void __launch_bounds__(kThreads, PRN_STAGED_MINB) newton_staged_kerne
         }
         if (last_delta < A.tol) break;
     }
-    cp_async_wait_all();  // a speculative prefetch may still be in flight
+    // a speculative prefetch may still be in flight
+    if (Lay::kTma) {
+        if (!wait_stage()) return;
+    } else {
+        cp_async_wait_all();
+    }
 
     if (A.residual_out && !stop_all)
         if (!residual_pass<Cell, C, L, IN>(A, s_red)) return;
@@ -480,6 +565,36 @@ __global__ void __launch_bounds__(kThreads, PRN_STAGED_MINB) newton_staged_kerne
 // ------------------------------------------------------------------ host side
 namespace {
 
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return nullptr;
+        fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+// fp32 tensor of `floats` elements viewed as rows of 32 floats; boxes of box_rows rows.
+bool map_rows(CUtensorMap *map, const float *ptr, long floats, int box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn || floats % 32) return false;
+    cuuint64_t dims[2] = {32, (cuuint64_t)(floats / 32)};
+    cuuint64_t strides[1] = {128};
+    cuuint32_t box[2] = {32, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float *>(ptr), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <class K> int prepare_kernel(K *kern, int smem_bytes) {
     if (cudaFuncSetAttribute(reinterpret_cast<const void *>(kern), cudaFuncAttributeMaxDynamicSharedMemorySize,
                              smem_bytes) != cudaSuccess)
@@ -489,11 +604,12 @@ template <class K> int prepare_kernel(K *kern, int smem_bytes) {
 
 template <class Cell, class Lay, int IN> int choose(Plan *plan, int num_sms, long B, long T, long H) {
     auto kern = &newton_staged_kernel<Cell, Lay, IN>;
-    const int smem = (Lay::SMEM_FLOATS + park_floats<Lay::S, Lay::L>()) * (int)sizeof(float);
+    const int smem = Lay::SMEM_FLOATS * (int)sizeof(float) + 1024;
     if (prepare_kernel(kern, smem)) return -1;
     plan->kernel = reinterpret_cast<const void *>(kern);
     plan->dyn_smem = smem;
     plan->C = Lay::C;
+    plan->tch = Lay::TCH;
     plan->ntiles = B * (H / Lay::C) * ((T + Lay::TCH - 1) / Lay::TCH);
     plan->grid = occupancy_grid(plan->kernel, kThreads, smem, num_sms, plan->ntiles);
     return plan->grid > 0 ? 0 : -1;
@@ -503,41 +619,71 @@ template <class Cell, class Lay, int IN> int choose(Plan *plan, int num_sms, lon
 
 // Staged kernels apply to H == 1 (long) or H % 32 == 0 with projected inputs (wide),
 // with 16-byte aligned per-sequence slabs.  Returns 1 when the shape is not covered.
-// Steps per thread (L) are chosen so that the input stage and the parked values of
-// two CTAs fit one SM's shared memory.
 int newton_staged_plan(const NewtonDiagReq &r, int num_sms, Plan *plan) {
     const int S = r.cell == 1 ? 2 : 1;
     const bool fused = r.xproj == nullptr;
     int rc;
+    plan->staged_tma = 0;
     if (r.H == 1) {
         const int PW = fused ? r.in : 3;
         if (fused && r.in != 1 && r.in != 2 && r.in != 4) return 1;
         if (((long)r.T * PW) % 4 || ((long)r.T * S) % 4) return 1;
         plan->variant = 101;
+        // TMA needs every sequence's input and state slabs to start on a 128-byte row
+        const bool tma = fused && ((long)r.T * PW) % 32 == 0 && ((long)r.T * S) % 32 == 0;
         if (S == 1) {
-            rc = !fused ? choose<GruCell, LongLayout<GruCell, 0, 8>, 0>(plan, num_sms, r.B, r.T, r.H)
-                 : r.in == 1 ? choose<GruCell, LongLayout<GruCell, 1, 16>, 1>(plan, num_sms, r.B, r.T, r.H)
-                 : r.in == 2 ? choose<GruCell, LongLayout<GruCell, 2, 16>, 2>(plan, num_sms, r.B, r.T, r.H)
-                             : choose<GruCell, LongLayout<GruCell, 4, 8>, 4>(plan, num_sms, r.B, r.T, r.H);
+            if (tma)
+                rc = r.in == 1 ? choose<GruCell, TmaLong<GruCell, 1, 16>, 1>(plan, num_sms, r.B, r.T, r.H)
+                     : r.in == 2 ? choose<GruCell, TmaLong<GruCell, 2, 16>, 2>(plan, num_sms, r.B, r.T, r.H)
+                                 : choose<GruCell, TmaLong<GruCell, 4, 8>, 4>(plan, num_sms, r.B, r.T, r.H);
+            else
+                rc = !fused ? choose<GruCell, CpLong<GruCell, 0, 16>, 0>(plan, num_sms, r.B, r.T, r.H)
+                     : r.in == 1 ? choose<GruCell, CpLong<GruCell, 1, 16>, 1>(plan, num_sms, r.B, r.T, r.H)
+                     : r.in == 2 ? choose<GruCell, CpLong<GruCell, 2, 16>, 2>(plan, num_sms, r.B, r.T, r.H)
+                                 : choose<GruCell, CpLong<GruCell, 4, 8>, 4>(plan, num_sms, r.B, r.T, r.H);
         } else {
-            rc = !fused ? choose<LstmCell, LongLayout<LstmCell, 0, 4>, 0>(plan, num_sms, r.B, r.T, r.H)
-                 : r.in == 1 ? choose<LstmCell, LongLayout<LstmCell, 1, 8>, 1>(plan, num_sms, r.B, r.T, r.H)
-                 : r.in == 2 ? choose<LstmCell, LongLayout<LstmCell, 2, 8>, 2>(plan, num_sms, r.B, r.T, r.H)
-                             : choose<LstmCell, LongLayout<LstmCell, 4, 4>, 4>(plan, num_sms, r.B, r.T, r.H);
+            if (tma)
+                rc = r.in == 1 ? choose<LstmCell, TmaLong<LstmCell, 1, 8>, 1>(plan, num_sms, r.B, r.T, r.H)
+                     : r.in == 2 ? choose<LstmCell, TmaLong<LstmCell, 2, 8>, 2>(plan, num_sms, r.B, r.T, r.H)
+                                 : choose<LstmCell, TmaLong<LstmCell, 4, 8>, 4>(plan, num_sms, r.B, r.T, r.H);
+            else
+                rc = !fused ? choose<LstmCell, CpLong<LstmCell, 0, 8>, 0>(plan, num_sms, r.B, r.T, r.H)
+                     : r.in == 1 ? choose<LstmCell, CpLong<LstmCell, 1, 8>, 1>(plan, num_sms, r.B, r.T, r.H)
+                     : r.in == 2 ? choose<LstmCell, CpLong<LstmCell, 2, 8>, 2>(plan, num_sms, r.B, r.T, r.H)
+                                 : choose<LstmCell, CpLong<LstmCell, 4, 8>, 4>(plan, num_sms, r.B, r.T, r.H);
         }
+        plan->staged_tma = tma ? 1 : 0;
     } else if (r.H % 32 == 0 && !fused) {
         plan->variant = 132;
-        rc = S == 1 ? choose<GruCell, WideLayout<GruCell, 12>, 0>(plan, num_sms, r.B, r.T, r.H)
-                    : choose<LstmCell, WideLayout<LstmCell, 8>, 0>(plan, num_sms, r.B, r.T, r.H);
+        rc = S == 1 ? choose<GruCell, Wide<GruCell, 16>, 0>(plan, num_sms, r.B, r.T, r.H)
+                    : choose<LstmCell, Wide<LstmCell, 8>, 0>(plan, num_sms, r.B, r.T, r.H);
     } else {
         return 1;
     }
     if (rc) return -1;
+    plan->S = S;
     plan->agg_words = (size_t)plan->ntiles * plan->C * (S == 1 ? 2 : 6);
     plan->inc_words = (size_t)plan->ntiles * plan->C * S;
     plan->side_bytes = 2 * (size_t)plan->ntiles * plan->C * S * sizeof(float);
     plan->epochs = (unsigned)r.max_iters + 1u;
+    plan->staged = 1;
     return 0;
+}
+
+// Launch a staged plan: build the tensor maps (TMA layouts) and pass them with the args.
+cudaError_t newton_staged_launch(const NewtonDiagArgs &A, const Plan &plan, cudaStream_t st) {
+    StagedMaps M;
+    memset(&M, 0, sizeof(M));
+    if (plan.staged_tma) {
+        const int S = plan.S;
+        const int PW = A.in;
+        const int tch = plan.tch;
+        if (!map_rows(&M.x, A.x, (long)A.B * A.T * PW, tch * PW / 32) ||
+            !map_rows(&M.h, A.h, (long)A.B * A.T * S, tch * S / 32))
+            return cudaErrorInvalidValue;
+    }
+    void *args[] = {const_cast<NewtonDiagArgs *>(&A), &M};
+    return cudaLaunchCooperativeKernel(plan.kernel, dim3(plan.grid), dim3(kThreads), args, plan.dyn_smem, st);
 }
 
 }  // namespace prn

@@ -254,8 +254,18 @@ __device__ __forceinline__ void publish_agg(const LookBack<S> &lb, const Aff<S> 
 
 // resolve_carry: the carried state entering `tile`, valid in lanes c < C.  Walks the
 // predecessors (tile - nseq, tile - 2 nseq, ...) in windows of 32 / C, composing their
-// aggregates until an inclusive value or the start of the sequence (carry `base`).
-// Returns false on a timeout / abort.
+// aggregates until a known value: an inclusive value, the start of the sequence (carry
+// `base`), or an aggregate whose matrix part is exactly zero (a constant map: nothing
+// before it can change the carry; long tiles of a contractive recurrence underflow to
+// this).  The warp polls together and never waits for slots behind the first known
+// value.  Returns false on a timeout / abort.
+template <int S> __device__ __forceinline__ bool aff_is_const(const float *v) {
+#pragma unroll
+    for (int q = 0; q < S * S; ++q)
+        if (v[q] != 0.f) return false;
+    return true;
+}
+
 template <int S, int C>
 __device__ bool resolve_carry(const LookBack<S> &lb, long tile, int chunk, long nseq, unsigned epoch,
                               const float *base, float *carry, Ctl *ctl, int *sticky, const Dbg &dbg) {
@@ -267,25 +277,28 @@ __device__ bool resolve_carry(const LookBack<S> &lb, long tile, int chunk, long 
         for (int q = 0; q < S; ++q) carry[q] = base[q];
         return true;
     }
-    bool ok = true;
     Aff<S> acc = Aff<S>::ident();  // composition of everything between here and the window
     long pred = tile - nseq;
     int pchunk = chunk - 1;
     for (;;) {
         const int my_chunk = pchunk - i;
         const long my_tile = pred - (long)i * nseq;
-        unsigned st = 3u;  // 3: start of the sequence
-        float iv[S], av[KF];
-        if (my_chunk >= 0) {
-            unsigned long long t0 = 0;
-            int polls = 0;
-            for (;;) {
+        unsigned long long t0 = 0;
+        int polls = 0;
+        Aff<S> v;
+        unsigned st;  // 0 not ready, 1 aggregate, 2 known value
+        for (;;) {
+            st = 2u;
+            if (my_chunk < 0) {
+                v = Aff<S>::cst(base);
+            } else {
                 unsigned long long wi[S], wa[KF];
 #pragma unroll
                 for (int q = 0; q < S; ++q) wi[q] = ld_relaxed_u64(lb.inc + (my_tile * C + c) * S + q);
 #pragma unroll
                 for (int q = 0; q < KF; ++q) wa[q] = ld_relaxed_u64(lb.agg + (my_tile * C + c) * KF + q);
                 bool inc_ok = true, agg_ok = true;
+                float iv[S], av[KF];
 #pragma unroll
                 for (int q = 0; q < S; ++q) {
                     inc_ok &= (unsigned)wi[q] == epoch;
@@ -296,45 +309,60 @@ __device__ bool resolve_carry(const LookBack<S> &lb, long tile, int chunk, long 
                     agg_ok &= (unsigned)wa[q] == epoch;
                     av[q] = __uint_as_float((unsigned)(wa[q] >> 32));
                 }
-                if (inc_ok) { st = kFlagInc; break; }
-                if (agg_ok) { st = kFlagAgg; break; }
-                if (ld_relaxed_int(&ctl->abort)) { ok = false; break; }
-                if (++polls == 4) t0 = gtimer();
-                if (polls > 4) {
-                    if (gtimer() - t0 > dbg.wait_ns) {
-                        raise_status(sticky, ctl, kStTimeout, true);
-                        ok = false;
-                        break;
-                    }
-                    __nanosleep(20);
+                if (inc_ok) {
+                    v = Aff<S>::cst(iv);
+                } else if (agg_ok) {
+                    v = Aff<S>::from_floats(av);
+                    st = aff_is_const<S>(av) ? 2u : 1u;
+                } else {
+                    st = 0u;
                 }
             }
-        }
-        __syncwarp();
-        if (__any_sync(0xffffffffu, !ok)) return false;
-        Aff<S> v;
-        if (st == 3u)
-            v = Aff<S>::cst(base);
-        else if (st == kFlagInc)
-            v = Aff<S>::cst(iv);
-        else
-            v = Aff<S>::from_floats(av);
-        const unsigned stop = __ballot_sync(0xffffffffu, st != kFlagAgg);
-        const int first = stop ? (__ffs(stop) - 1) / C : WIN;  // first slot with a known value
-        if (i > first) v = Aff<S>::ident();
-        // reduce the window: slot 0 is the nearest predecessor (applied last)
+            // every channel of a slot sees the same tile; a slot is known only if all
+            // its channels are (C lanes per slot)
+            const unsigned known = __ballot_sync(0xffffffffu, st == 2u);
+            const unsigned ready = __ballot_sync(0xffffffffu, st != 0u);
+            unsigned slot_known = 0, slot_ready = 0;
 #pragma unroll
-        for (int off = C; off < 32; off <<= 1) {
-            Aff<S> o = v.shfl_down(off);
-            if (lane + off < 32) v = compose(o, v);
-        }
-        acc = compose(v, acc);
-        if (stop) {
-            float z[S];
+            for (int w = 0; w < WIN; ++w) {
+                const unsigned m = (C == 32 ? 0xffffffffu : ((1u << C) - 1u)) << (w * C);
+                if ((known & m) == m) slot_known |= 1u << w;
+                if ((ready & m) == m) slot_ready |= 1u << w;
+            }
+            const int first = slot_known ? __ffs(slot_known) - 1 : WIN;
+            const int need_n = first + 1 < WIN ? first + 1 : WIN;  // slots 0 .. first must be ready
+            const unsigned need_w = need_n >= 32 ? 0xffffffffu : ((1u << need_n) - 1u);
+            if ((slot_ready & need_w) == need_w) {
+                // reduce the window up to the first known slot; slot 0 is the nearest
+                // predecessor (applied last)
+                if (i > first) v = Aff<S>::ident();
 #pragma unroll
-            for (int q = 0; q < S; ++q) z[q] = 0.f;
-            acc.apply(z, carry);  // acc is a constant map here
-            return true;
+                for (int off = C; off < 32; off <<= 1) {
+                    Aff<S> o = v.shfl_down(off);
+                    if (lane + off < 32) v = compose(o, v);
+                }
+                acc = compose(v, acc);
+                if (first < WIN) {
+                    float z[S];
+#pragma unroll
+                    for (int q = 0; q < S; ++q) z[q] = 0.f;
+                    acc.apply(z, carry);  // acc is a constant map here
+                    return true;
+                }
+                break;  // whole window of aggregates: continue with the next window
+            }
+            ++polls;  // warp-uniform
+            int bad = 0;
+            if (lane == 0) {
+                if (ld_relaxed_int(&ctl->abort)) bad = 1;
+                if (polls == 4) t0 = gtimer();
+                if (polls > 4 && gtimer() - t0 > dbg.wait_ns) {
+                    raise_status(sticky, ctl, kStTimeout, true);
+                    bad = 1;
+                }
+            }
+            if (__shfl_sync(0xffffffffu, bad, 0)) return false;
+            if (polls > 4) __nanosleep(20);
         }
         pred -= (long)WIN * nseq;
         pchunk -= WIN;

@@ -26,6 +26,9 @@
 #ifndef PRN_STAGED_MINB
 #define PRN_STAGED_MINB 2  // resident CTAs per SM the register budget is sized for
 #endif
+#ifndef PRN_LONG_GRU_L
+#define PRN_LONG_GRU_L 16  // steps per thread of the TMA-fed H = 1 ParaGRU tiles
+#endif
 
 namespace prn {
 
@@ -596,8 +599,9 @@ bool map_rows(CUtensorMap *map, const float *ptr, long floats, int box_rows) {
 }
 
 template <class K> int prepare_kernel(K *kern, int smem_bytes) {
-    if (cudaFuncSetAttribute(reinterpret_cast<const void *>(kern), cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             smem_bytes) != cudaSuccess)
+    const void *f = reinterpret_cast<const void *>(kern);
+    if (cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes) != cudaSuccess ||
+        cudaFuncSetAttribute(f, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess)
         return -1;
     return 0;
 }
@@ -634,7 +638,7 @@ int newton_staged_plan(const NewtonDiagReq &r, int num_sms, Plan *plan) {
         if (S == 1) {
             if (tma)
                 rc = r.in == 1 ? choose<GruCell, TmaLong<GruCell, 1, 16>, 1>(plan, num_sms, r.B, r.T, r.H)
-                     : r.in == 2 ? choose<GruCell, TmaLong<GruCell, 2, 16>, 2>(plan, num_sms, r.B, r.T, r.H)
+                     : r.in == 2 ? choose<GruCell, TmaLong<GruCell, 2, PRN_LONG_GRU_L>, 2>(plan, num_sms, r.B, r.T, r.H)
                                  : choose<GruCell, TmaLong<GruCell, 4, 8>, 4>(plan, num_sms, r.B, r.T, r.H);
             else
                 rc = !fused ? choose<GruCell, CpLong<GruCell, 0, 16>, 0>(plan, num_sms, r.B, r.T, r.H)

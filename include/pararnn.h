@@ -166,7 +166,9 @@ const char *pararnn_strerror(int status);
  * knob 2: tile index whose look-back publication is withheld (-1 = none); used
  *         only by the failure-detection test to make a successor's wait run out.
  * knob 3: device pointer (float*) receiving delta_k of every Newton iteration, with
- *         knob 4 its capacity (0 disables). */
+ *         knob 4 its capacity (0 disables).
+ * knob 5: non-zero makes the long-sequence Newton tiles take every carry from the
+ *         look-back, never from their own halo (tests of the look-back path). */
 int pararnn_debug_set(pararnn_ctx *ctx, int knob, long long value);
 
 /* Number of kernels the last call launched on the stream. */

@@ -306,6 +306,7 @@ int pararnn_debug_set(pararnn_ctx *ctx, int knob, long long value) {
             if (value < 0) return PARARNN_EINVAL;
             ctx->dbg.delta_log_cap = (int)value;
             return PARARNN_OK;
+        case 5: ctx->dbg.no_halo = value != 0; return PARARNN_OK;
         default: return PARARNN_EINVAL;
     }
 }

@@ -20,21 +20,34 @@ struct GruCell {
     static constexpr int S = 1;
     static constexpr int NPAR = 3;  // recurrent diagonals a_z, a_r, a_c
     float az, ar, ac;
+    float qz, qr, qc;  // the same, times pre(g)
+    // Exponent scale of gate g: s(u) = 1 / (1 + 2^(-u log2 e)), tanh(u) = 2 s(2u) - 1.
+    __host__ __device__ static constexpr float pre(int g) { return g == 2 ? -2.f * kLog2e : -kLog2e; }
     __device__ __forceinline__ void load(const float *a, const float *, int H, int h) {
         az = __ldg(a + h);
         ar = __ldg(a + H + h);
         ac = __ldg(a + 2 * H + h);
+        qz = pre(0) * az;
+        qr = pre(1) * ar;
+        qc = pre(2) * ac;
     }
-    // f and J = df/dh at previous state hp.
-    __device__ __forceinline__ void eval(const float p[3], const float *hp, float *f, float *J) const {
+    // f and J = df/dh at previous state hp, from q_g = pre(g) p_g.
+    __device__ __forceinline__ void eval_pre(const float q[3], const float *hp, float *f, float *J) const {
         const float h = hp[0];
-        const float z = sigm(fmaf(az, h, p[0]));
-        const float r = sigm(fmaf(ar, h, p[1]));
-        const float c = tanh_(fmaf(ac, r * h, p[2]));
-        f[0] = fmaf(z, c - h, h);
-        const float dz = z * (1.f - z), dr = r * (1.f - r), dc = 1.f - c * c;
-        // df/dh = (1 - z) + (c - h) dz a_z + z dc a_c (r + h dr a_r)
-        J[0] = (1.f - z) + (c - h) * dz * az + z * dc * ac * fmaf(h * dr, ar, r);
+        const float z = rcp_hw(1.f + ex2_hw(fmaf(qz, h, q[0])));
+        const float r = rcp_hw(1.f + ex2_hw(fmaf(qr, h, q[1])));
+        const float c = fmaf(2.f, rcp_hw(1.f + ex2_hw(fmaf(qc, r * h, q[2]))), -1.f);
+        const float cmh = c - h;
+        f[0] = fmaf(z, cmh, h);
+        // df/dh = (1 - z) + (c - h) dz a_z + z dc a_c (r + h dr a_r),
+        // dz = z (1 - z), dr = r (1 - r), dc = 1 - c^2
+        const float dz = fmaf(-z, z, z), dr = fmaf(-r, r, r), dc = fmaf(-c, c, 1.f);
+        const float j0 = fmaf(az, cmh * dz, 1.f - z);
+        J[0] = fmaf(ac, (z * dc) * fmaf(h * ar, dr, r), j0);
+    }
+    __device__ __forceinline__ void eval(const float p[3], const float *hp, float *f, float *J) const {
+        const float q[3] = {pre(0) * p[0], pre(1) * p[1], pre(2) * p[2]};
+        eval_pre(q, hp, f, J);
     }
     // Adjoint partials: f, J, df/dp (3) and the factors that turn df/dp into df/da:
     // df/da_z = df/dp_z * h, df/da_r = df/dp_r * h, df/da_c = df/dp_c * (r h).
@@ -58,6 +71,7 @@ struct LstmCell {
     static constexpr int S = 2;
     static constexpr int NPAR = 5;  // a_f, a_g, a_o, w_f, w_o
     float af, ag, ao, wf, wo;
+    __host__ __device__ static constexpr float pre(int) { return 1.f; }
     __device__ __forceinline__ void load(const float *a, const float *peep, int H, int h) {
         af = __ldg(a + h);
         ag = __ldg(a + H + h);
@@ -82,6 +96,9 @@ struct LstmCell {
         J[1] = dch;
         J[2] = kap * dcc;
         J[3] = fmaf(dout * ao, tc, kap * dch);
+    }
+    __device__ __forceinline__ void eval_pre(const float p[3], const float *sp, float *f, float *J) const {
+        eval(p, sp, f, J);
     }
     // dp is [2][3] = d(c', h')/d(p_f, p_g, p_o); fac = (h_{t-1}, c_{t-1}, c_t):
     // d/da_f = d/dp_f * h, d/da_g = d/dp_g * h, d/da_o = d/dp_o * h,

@@ -35,6 +35,7 @@ struct Dbg {
     long long skip_tile;         // tile whose look-back publication is withheld (-1 none)
     float *delta_log;            // per-iteration delta (may be null)
     int delta_log_cap;
+    int no_halo;                 // 1: tiles always take the carry from the look-back
 };
 
 __device__ __forceinline__ unsigned long long gtimer() {
@@ -104,6 +105,21 @@ __device__ __forceinline__ bool grid_sync(Ctl *ctl, int *sticky, const Dbg &dbg)
 // point of exactly this cell.
 __device__ __forceinline__ float sigm(float u) { return __fdividef(1.0f, 1.0f + __expf(-u)); }
 __device__ __forceinline__ float tanh_(float u) { return fmaf(2.0f, sigm(2.0f * u), -1.0f); }
+
+// 2^y and 1/y with the hardware approximations (PTX ex2.approx / rcp.approx, a few
+// ulp): with e^u = 2^(u log2 e) folded into the inputs' scale, a logistic function
+// costs one fused multiply-add, two special-function operations and one add.
+__device__ __forceinline__ float ex2_hw(float y) {
+    float r;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(y));
+    return r;
+}
+__device__ __forceinline__ float rcp_hw(float y) {
+    float r;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(y));
+    return r;
+}
+constexpr float kLog2e = 1.4426950408889634f;
 
 __device__ __forceinline__ bool finitef(float v) { return fabsf(v) <= 3.402823466e38f; }
 
@@ -199,8 +215,8 @@ __device__ __forceinline__ unsigned long long ld_relaxed_u64(const unsigned long
     return v;
 }
 
-template <int S, int C> struct ScanSmem {
-    static constexpr int NW = kThreads / 32;
+template <int S, int C, int NT = kThreads> struct ScanSmem {
+    static constexpr int NW = NT / 32;
     Aff<S> wtot[NW][C];  // per-warp totals (scan order)
     float carry[C][S];   // carry entering the tile, per channel
 };
@@ -210,8 +226,8 @@ template <int S, int C> struct ScanSmem {
 // On return: `excl` is the composition of the elements before this thread's
 // position (identity for s = 0) and `total` (valid in warp 0, lanes c < C) is the
 // tile's aggregate for channel c.
-template <int S, int C>
-__device__ __forceinline__ void cta_scan(const Aff<S> &e, ScanSmem<S, C> &sm, Aff<S> &excl, Aff<S> &total) {
+template <int S, int C, int NT = kThreads>
+__device__ __forceinline__ void cta_scan(const Aff<S> &e, ScanSmem<S, C, NT> &sm, Aff<S> &excl, Aff<S> &total) {
     static_assert(32 % C == 0, "C must divide 32");
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     Aff<S> inc = e;
@@ -231,7 +247,7 @@ __device__ __forceinline__ void cta_scan(const Aff<S> &e, ScanSmem<S, C> &sm, Af
     if (warp == 0 && lane < C) {
         Aff<S> t = Aff<S>::ident();
 #pragma unroll
-        for (int w = 0; w < ScanSmem<S, C>::NW; ++w) t = compose(t, sm.wtot[w][lane]);
+        for (int w = 0; w < ScanSmem<S, C, NT>::NW; ++w) t = compose(t, sm.wtot[w][lane]);
         total = t;
     }
 }
@@ -383,14 +399,27 @@ __device__ __forceinline__ void publish_inc(const LookBack<S> &lb, const Aff<S> 
 
 // The whole look-back for one tile: publish the aggregate, resolve the carry, publish
 // the inclusive value, leave the carry in sm.carry.  Returns false on a timeout.
-template <int S, int C>
-__device__ bool look_back(const LookBack<S> &lb, ScanSmem<S, C> &sm, const Aff<S> &total, long tile,
+// `halo` (optional, channel c): the composed map of the steps just before the tile,
+// evaluated by the tile itself; when its matrix part is exactly zero it is a constant
+// whose value is the carry, and no predecessor is read.
+template <int S, int C, int NT = kThreads>
+__device__ bool look_back(const LookBack<S> &lb, ScanSmem<S, C, NT> &sm, const Aff<S> &total, long tile,
                           int chunk, long nseq, unsigned epoch, const float *base /* [S], channel c */,
-                          Ctl *ctl, int *sticky, const Dbg &dbg) {
+                          Ctl *ctl, int *sticky, const Dbg &dbg, const Aff<S> *halo = nullptr) {
     const int lane = threadIdx.x & 31;
     publish_agg<S, C>(lb, total, tile, chunk, epoch, dbg);
     float carry[S];
-    if (!resolve_carry<S, C>(lb, tile, chunk, nseq, epoch, base, carry, ctl, sticky, dbg)) return false;
+    bool known = false;
+    if (halo != nullptr && chunk > 0) {
+        float hv[Aff<S>::kFloats];
+        halo->to_floats(hv);
+        known = __all_sync(0xffffffffu, lane >= C || aff_is_const<S>(hv));
+        if (known) {
+#pragma unroll
+            for (int q = 0; q < S; ++q) carry[q] = hv[S * S + q];
+        }
+    }
+    if (!known && !resolve_carry<S, C>(lb, tile, chunk, nseq, epoch, base, carry, ctl, sticky, dbg)) return false;
     publish_inc<S, C>(lb, total, carry, tile, epoch, dbg);
     if (lane < C) {
 #pragma unroll
@@ -400,7 +429,7 @@ __device__ bool look_back(const LookBack<S> &lb, ScanSmem<S, C> &sm, const Aff<S
 }
 
 // Block-wide max of a non-negative float (NaN propagates as a NaN bit pattern).
-__device__ __forceinline__ unsigned block_max_bits(float v, unsigned *s_red) {
+template <int NT = kThreads> __device__ __forceinline__ unsigned block_max_bits(float v, unsigned *s_red) {
     unsigned b = isnan(v) ? 0x7fc00000u : __float_as_uint(fabsf(v));
 #pragma unroll
     for (int off = 16; off; off >>= 1) b = max(b, __shfl_xor_sync(0xffffffffu, b, off));
@@ -409,7 +438,7 @@ __device__ __forceinline__ unsigned block_max_bits(float v, unsigned *s_red) {
     __syncthreads();
     unsigned r = 0;
     if (threadIdx.x == 0)
-        for (int w = 0; w < kThreads / 32; ++w) r = max(r, s_red[w]);
+        for (int w = 0; w < NT / 32; ++w) r = max(r, s_red[w]);
     __syncthreads();
     return r;  // valid in thread 0
 }

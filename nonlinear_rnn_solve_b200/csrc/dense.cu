@@ -726,6 +726,7 @@ cudaError_t newton_tanh_launch(const NewtonTanhReq &r, const Plan &plan, const W
     A.dbg.skip_tile = dbg.skip_tile;
     A.dbg.delta_log = dbg.delta_log;
     A.dbg.delta_log_cap = dbg.delta_log_cap;
+    A.dbg.no_halo = 1;
     void *args[] = {&A};
     return cudaLaunchCooperativeKernel(plan.kernel, dim3(plan.grid), dim3(kThreads), args, plan.dyn_smem, st);
 }
@@ -774,6 +775,7 @@ cudaError_t scan_dense_launch(const ScanReq &r, const Plan &plan, const Work &w,
     A.dbg.skip_tile = dbg.skip_tile;
     A.dbg.delta_log = nullptr;
     A.dbg.delta_log_cap = 0;
+    A.dbg.no_halo = 1;
     void *args[] = {&A};
     return cudaLaunchCooperativeKernel(plan.kernel, dim3(plan.grid), dim3(kThreads), args, plan.dyn_smem, st);
 }

@@ -33,6 +33,8 @@ struct Plan {
     int staged = 0;                // Newton: staged kernel (args + tensor maps)
     int staged_tma = 0;            // staged kernel fed by TMA
     int S = 1;                     // state components per unit
+    int threads = 256;             // threads per CTA
+    int halo_w = 1;                // side-buffer values per tile boundary and channel
 };
 
 struct DbgHost {
@@ -40,6 +42,7 @@ struct DbgHost {
     long long skip_tile = -1;
     float *delta_log = nullptr;
     int delta_log_cap = 0;
+    int no_halo = 0;
 };
 
 // ---- Newton forward, diagonal / 2x2-block cells (GRU, LSTM) -----------------------

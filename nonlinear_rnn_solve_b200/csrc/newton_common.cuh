@@ -116,11 +116,11 @@ cudaError_t newton_staged_launch(const NewtonDiagArgs &A, const Plan &plan, cuda
 
 // Final residual r = max over every state element of |h_t - f(h_{t-1}, x_t)| at the
 // returned iterate (one read of the states and inputs), reduced over the grid.
-// Tiles are [TCH = (256 / C) * L steps] x [C channels], as in the solver kernels.
-template <class Cell, int C, int L, int IN>
+// Tiles are [TCH = (NT / C) * L steps] x [C channels], as in the solver kernels.
+template <class Cell, int C, int L, int IN, int NT = kThreads>
 __device__ bool residual_pass(const NewtonDiagArgs &A, unsigned *s_red) {
     constexpr int S = Cell::S;
-    constexpr int TCH = (kThreads / C) * L;
+    constexpr int TCH = (NT / C) * L;
     const int tid = threadIdx.x, c = tid % C, s = tid / C;
     const int nct = (A.H + C - 1) / C;
     const long nseq = (long)A.B * nct;
@@ -162,7 +162,7 @@ __device__ bool residual_pass(const NewtonDiagArgs &A, unsigned *s_red) {
             }
         }
     }
-    const unsigned bits = block_max_bits(my_res, s_red);
+    const unsigned bits = block_max_bits<NT>(my_res, s_red);
     if (tid == 0) atomicMax(&A.ctl->res_bits, bits);
     if (!grid_sync(A.ctl, A.sticky, A.dbg)) return false;
     if (blockIdx.x == 0 && tid == 0) {

@@ -29,6 +29,15 @@
 #ifndef PRN_LONG_GRU_L
 #define PRN_LONG_GRU_L 16  // steps per thread of the TMA-fed H = 1 ParaGRU tiles
 #endif
+#ifndef PRN_LONG_NT
+#define PRN_LONG_NT 256  // threads per CTA of the TMA-fed H = 1 ParaGRU tiles
+#endif
+#ifndef PRN_LONG_MINB
+#define PRN_LONG_MINB PRN_STAGED_MINB  // resident CTAs per SM for those tiles
+#endif
+#ifndef PRN_LONG_HALO
+#define PRN_LONG_HALO 256  // steps before each H = 1 ParaGRU tile that the tile evaluates itself
+#endif
 
 namespace prn {
 
@@ -70,9 +79,10 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, i
 // Copy n floats (n % 4 == 0) from a 16-byte aligned global address into consecutive
 // segments of `seg` floats placed `str` floats apart; bytes at or beyond `end` are
 // zero-filled.  Consecutive threads copy consecutive 16-byte chunks (coalesced).
+template <int NT>
 __device__ __forceinline__ void copy_segments(float *dst, int seg, int str, const float *src, int n,
                                               const float *end) {
-    for (int f = 4 * threadIdx.x; f < n; f += 4 * kThreads) {
+    for (int f = 4 * threadIdx.x; f < n; f += 4 * NT) {
         const float *gp = src + f;
         const long rem = end - gp;
         const int bytes = rem >= 4 ? 16 : (rem > 0 ? (int)rem * 4 : 0);
@@ -100,8 +110,9 @@ __device__ __forceinline__ float swz_float(const float *region, int f) {
     return region[row * 32 + ((lc ^ (row & 7)) << 2) + (f & 3)];
 }
 
-template <class Cell, int IN, int LL> struct TmaLong {
-    static constexpr int S = Cell::S, C = 1, L = LL, SUB = kThreads, TCH = SUB * L, PW = IN;
+template <class Cell, int IN, int LL, int NT, int HL = 0> struct TmaLong {
+    static constexpr int S = Cell::S, C = 1, L = LL, SUB = NT, TCH = SUB * L, PW = IN;
+    static constexpr int HALO = HL;
     static constexpr int SEGP = L * PW, SEGH = L * S;
     static_assert(SEGP == 8 || SEGP == 16 || SEGP == 32, "input segment must be part of one 128-byte row");
     static_assert(SEGH == 8 || SEGH == 16 || SEGH == 32, "state segment must be part of one 128-byte row");
@@ -170,32 +181,35 @@ template <class Cell, int IN, int LL> struct TmaLong {
         const int valid = min(TCH, A.T - tch0) * S;
         float *g = A.h + ((size_t)b * A.T + tch0) * S;
         const float *o = sm + OFFO;
-        for (int c = threadIdx.x; 4 * c < valid; c += kThreads) {
+        for (int c = threadIdx.x; 4 * c < valid; c += NT) {
             const int row = c >> 3, lc = c & 7;
             const float4 v = *reinterpret_cast<const float4 *>(o + row * 32 + ((lc ^ (row & 7)) << 2));
             *reinterpret_cast<float4 *>(g + 4 * c) = v;
         }
-        __syncthreads();
+        // the staging tile is next written after the following tile's stage wait and
+        // scan barriers: no barrier needed here
     }
 };
 
 // ---------------------------------------------------------------- cp.async long layout, H == 1
-template <class Cell, int IN, int LL> struct CpLong {
-    static constexpr int S = Cell::S, C = 1, L = LL, SUB = kThreads, TCH = SUB * L;
+template <class Cell, int IN, int LL, int NT> struct CpLong {
+    static constexpr int S = Cell::S, C = 1, L = LL, SUB = NT, TCH = SUB * L;
     static constexpr int PW = IN == 0 ? 3 : IN;  // input floats per step
     static constexpr int SEGP = L * PW, STRP = pad_stride(SEGP);
     static constexpr int SEGH = L * S, STRH = pad_stride(SEGH);
     static constexpr int OFFH = SUB * STRP;
     static constexpr int SMEM_FLOATS = SUB * (STRP + STRH);
     static constexpr bool kTma = false;
+    static constexpr int HALO = 0;
     static_assert(SEGP % 4 == 0 && SEGH % 4 == 0, "segments are whole 16-byte chunks");
 
     __device__ static void issue(const NewtonDiagArgs &A, const StagedMaps &, float *sm, unsigned long long *, int b,
                                  int, int tch0, bool with_h) {
         const size_t row = (size_t)b * A.T;
         const float *pin = IN == 0 ? A.xproj : A.x;
-        copy_segments(sm, SEGP, STRP, pin + (row + tch0) * PW, TCH * PW, pin + (row + A.T) * PW);
-        if (with_h) copy_segments(sm + OFFH, SEGH, STRH, A.h + (row + tch0) * S, TCH * S, A.h + (row + A.T) * S);
+        copy_segments<NT>(sm, SEGP, STRP, pin + (row + tch0) * PW, TCH * PW, pin + (row + A.T) * PW);
+        if (with_h)
+            copy_segments<NT>(sm + OFFH, SEGH, STRH, A.h + (row + tch0) * S, TCH * S, A.h + (row + A.T) * S);
         cp_async_commit();
     }
     __device__ static void load_group(float *sm, int s, int, int grp, float pv[4][PW], float hv[4][S], bool with_h) {
@@ -244,25 +258,26 @@ template <class Cell, int IN, int LL> struct CpLong {
 };
 
 // ---------------------------------------------------------------- wide layout, H % 32 == 0
-template <class Cell, int LL> struct Wide {
-    static constexpr int S = Cell::S, C = 32, L = LL, SUB = kThreads / C, TCH = SUB * L;
+template <class Cell, int LL, int NT> struct Wide {
+    static constexpr int S = Cell::S, C = 32, L = LL, SUB = NT / C, TCH = SUB * L;
     static constexpr int PW = 3;
     static constexpr int ROWP = 3 * 32, ROWH = 32 * S;
     static constexpr int OFFH = TCH * ROWP;
     static constexpr int SMEM_FLOATS = TCH * (ROWP + ROWH);
     static constexpr bool kTma = false;
+    static constexpr int HALO = 0;
 
     __device__ static void issue(const NewtonDiagArgs &A, const StagedMaps &, float *sm, unsigned long long *, int b,
                                  int ct, int tch0, bool with_h) {
         const size_t row = (size_t)b * A.T;
-        for (int q = threadIdx.x; q < TCH * 3 * 8; q += kThreads) {
+        for (int q = threadIdx.x; q < TCH * 3 * 8; q += NT) {
             const int r = q >> 3, part = q & 7, t = r / 3, g = r % 3;
             const bool v = tch0 + t < A.T;
             const float *gp = A.xproj + ((row + tch0 + (v ? t : 0)) * 3 + g) * A.H + ct * 32 + part * 4;
             cp_async16(sm + r * 32 + part * 4, gp, v ? 16 : 0);
         }
         if (with_h) {
-            for (int q = threadIdx.x; q < TCH * 8 * S; q += kThreads) {
+            for (int q = threadIdx.x; q < TCH * 8 * S; q += NT) {
                 const int t = q / (8 * S), part = q % (8 * S);
                 const bool v = tch0 + t < A.T;
                 const float *gp = A.h + ((row + tch0 + (v ? t : 0)) * A.H + ct * 32) * S + part * 4;
@@ -333,7 +348,10 @@ __device__ __forceinline__ void tile_compute(const NewtonDiagArgs &A, float *sme
             float cur[S], f[S], J[S * S];
 #pragma unroll
             for (int q = 0; q < S; ++q) cur[q] = k > 0 ? hv[j][q] : 0.f;
-            cell.eval(p, hp, f, J);
+            if (IN > 0)
+                cell.eval_pre(p, hp, f, J);  // p was formed with the prescaled weights
+            else
+                cell.eval(p, hp, f, J);
 #pragma unroll
             for (int q = 0; q < S; ++q) {
                 rr[i][q] = v ? f[q] - cur[q] : 0.f;
@@ -346,23 +364,31 @@ __device__ __forceinline__ void tile_compute(const NewtonDiagArgs &A, float *sme
     }
 }
 
-template <class Cell, class Lay, int IN>
-__global__ void __launch_bounds__(kThreads, PRN_STAGED_MINB)
+template <class Cell, class Lay, int IN, int NT, int MINB>
+__global__ void __launch_bounds__(NT, MINB)
     newton_staged_kernel(const NewtonDiagArgs A, const __grid_constant__ StagedMaps M) {
     constexpr int S = Cell::S, C = Lay::C, L = Lay::L, SUB = Lay::SUB, TCH = Lay::TCH;
+    constexpr int HALO = Lay::HALO, HW = HALO > 0 ? HALO : 1;
     static_assert(L % 4 == 0, "steps are handled in groups of four");
+    static_assert(HALO == 0 || (HALO % 32 == 0 && HALO <= NT && HALO % L == 0 && IN > 0 && C == 1),
+                  "a halo is one step per thread of whole warps, covers whole segments, raw inputs, H = 1");
     extern __shared__ __align__(1024) unsigned char smraw[];
     float *const smem = reinterpret_cast<float *>(((uintptr_t)smraw + 1023) & ~(uintptr_t)1023);
-    __shared__ ScanSmem<S, C> sm;
-    __shared__ unsigned s_red[kThreads / 32];
+    __shared__ ScanSmem<S, C, NT> sm;
+    __shared__ unsigned s_red[NT / 32];
     __shared__ int s_fail;
     __shared__ __align__(8) unsigned long long s_bar;
+    __shared__ Aff<S> s_halo[HALO > 0 ? HALO / 32 : 1];
     const int tid = threadIdx.x, c = tid % C, s = tid / C;
     const int nct = A.H / C;
     const long nseq = (long)A.B * nct;
     const int nchunk = (A.T + TCH - 1) / TCH;
     const long ntiles = nseq * nchunk;
-    const size_t side_stride = (size_t)ntiles * C * S;
+    // side buffers (two parities): the last HW states that every tile but a sequence's
+    // last wrote in the previous iteration.  They are the current iterate for the
+    // successor (its halo and first step), which must not read them from h: the
+    // tile may already be overwriting them there.
+    const size_t side_stride = (size_t)ntiles * C * HW * S;
     LookBack<S> lb{A.agg, A.inc};
     unsigned bar_phase = 0;
     if (tid == 0) {
@@ -382,9 +408,10 @@ __global__ void __launch_bounds__(kThreads, PRN_STAGED_MINB)
 #pragma unroll
         for (int q = 0; q < (IN > 0 ? IN : 1); ++q) wz[g][q] = 0.f;
         if (IN > 0) {
-            bz[g] = A.bias ? __ldg(A.bias + g * A.H) : 0.f;
+            // folded into the cell's exponent scale (Cell::pre): the cell takes q = pre * p
+            bz[g] = A.bias ? Cell::pre(g) * __ldg(A.bias + g * A.H) : 0.f;
 #pragma unroll
-            for (int q = 0; q < (IN > 0 ? IN : 1); ++q) wz[g][q] = __ldg(A.W + (size_t)g * A.H * IN + q);
+            for (int q = 0; q < (IN > 0 ? IN : 1); ++q) wz[g][q] = Cell::pre(g) * __ldg(A.W + (size_t)g * A.H * IN + q);
         }
     }
 
@@ -455,9 +482,60 @@ __global__ void __launch_bounds__(kThreads, PRN_STAGED_MINB)
             const int h = ct * C + c;
             const int tch0 = chunk * TCH;
             const int t0 = tch0 + s * L;
+            // halo: thread tid < HALO evaluates step tch0 - HALO + tid (the first only
+            // supplies the state before the second); loads start before the stage wait
+            const bool use_halo = HALO > 0 && chunk > 0 && !A.dbg.no_halo;
+            float hx[IN > 0 ? IN : 1], hcur[S], hprv[S];
+            if (HALO > 0 && use_halo && tid < HALO) {
+                const float *xr = A.x + ((size_t)b * A.T + (tch0 - HALO + tid)) * (IN > 0 ? IN : 1);
+                if (IN == 2) {
+                    const float2 v = *reinterpret_cast<const float2 *>(xr);
+                    hx[0] = v.x;
+                    hx[1 % (IN > 0 ? IN : 1)] = v.y;
+                } else if (IN == 4) {
+                    const float4 v = *reinterpret_cast<const float4 *>(xr);
+                    hx[0] = v.x;
+                    hx[1 % (IN > 0 ? IN : 1)] = v.y;
+                    hx[2 % (IN > 0 ? IN : 1)] = v.z;
+                    hx[3 % (IN > 0 ? IN : 1)] = v.w;
+                } else {
+#pragma unroll
+                    for (int q = 0; q < (IN > 0 ? IN : 1); ++q) hx[q] = xr[q];
+                }
+                const float *sp = side_in + (size_t)(tile - nseq) * HW * S;
+#pragma unroll
+                for (int q = 0; q < S; ++q) {
+                    hcur[q] = k > 0 ? sp[tid * S + q] : 0.f;
+                    hprv[q] = (k > 0 && tid > 0) ? sp[(tid - 1) * S + q] : 0.f;
+                }
+            }
             if (!wait_stage()) return;
             Cell cell;
             cell.load(A.a, A.peep, A.H, h);
+            if (HALO > 0 && use_halo && tid < HALO) {
+                Aff<S> he = Aff<S>::ident();
+                if (tid > 0) {
+                    float p[3], f[S], J[S * S], r[S];
+#pragma unroll
+                    for (int g = 0; g < 3; ++g) {
+                        float acc = bz[g];
+#pragma unroll
+                        for (int q = 0; q < (IN > 0 ? IN : 1); ++q) acc = fmaf(wz[g][q], hx[q], acc);
+                        p[g] = acc;
+                    }
+                    cell.eval_pre(p, hprv, f, J);
+#pragma unroll
+                    for (int q = 0; q < S; ++q) r[q] = f[q] - hcur[q];
+                    he = make_aff<S>(J, r);
+                }
+                // ordered composition of the warp's 32 steps, into lane 0
+#pragma unroll
+                for (int off = 1; off < 32; off <<= 1) {
+                    const Aff<S> o = he.shfl_down(off);
+                    if ((tid & 31) + off < 32) he = compose(he, o);
+                }
+                if ((tid & 31) == 0) s_halo[tid >> 5] = he;  // read after cta_scan's barrier
+            }
             float hp[S];
 #pragma unroll
             for (int q = 0; q < S; ++q) hp[q] = 0.f;
@@ -466,7 +544,7 @@ __global__ void __launch_bounds__(kThreads, PRN_STAGED_MINB)
             } else if (k > 0) {
                 if (s == 0) {
 #pragma unroll
-                    for (int q = 0; q < S; ++q) hp[q] = side_in[((tile - nseq) * C + c) * S + q];
+                    for (int q = 0; q < S; ++q) hp[q] = side_in[(((tile - nseq) * C + c) * HW + HW - 1) * S + q];
                 } else {
                     Lay::h_prev(smem, s, c, hp);
                 }
@@ -476,19 +554,25 @@ __global__ void __launch_bounds__(kThreads, PRN_STAGED_MINB)
                 tile_compute<Cell, Lay, IN, true>(A, smem, cell, s, c, t0, k, hp, wz, bz, Jr, rr, hc);
             else
                 tile_compute<Cell, Lay, IN, false>(A, smem, cell, s, c, t0, k, hp, wz, bz, Jr, rr, hc);
-            __syncthreads();  // the stage is consumed: refill it with the next tile
-            const long next = tile + gridDim.x;
-            if (next < ntiles) issue(next, k > 0);
             Aff<S> e = Aff<S>::ident();
 #pragma unroll
             for (int i = 0; i < L; ++i) e = compose(e, make_aff<S>(Jr[i], rr[i]));
             Aff<S> excl, total;
-            cta_scan<S, C>(e, sm, excl, total);
+            cta_scan<S, C, NT>(e, sm, excl, total);
+            // past the scan's barrier every thread is done reading the stage: refill it
+            const long next = tile + gridDim.x;
+            if (next < ntiles) issue(next, k > 0);
             if (tid < 32) {
                 float base[S];
 #pragma unroll
                 for (int q = 0; q < S; ++q) base[q] = 0.f;  // delta entering t = 0 is 0
-                if (!look_back<S, C>(lb, sm, total, tile, chunk, nseq, epoch, base, A.ctl, A.sticky, A.dbg))
+                Aff<S> hall = Aff<S>::ident();
+                if (HALO > 0 && use_halo) {
+#pragma unroll
+                    for (int w = 0; w < HW / 32; ++w) hall = compose(hall, s_halo[w]);
+                }
+                if (!look_back<S, C, NT>(lb, sm, total, tile, chunk, nseq, epoch, base, A.ctl, A.sticky, A.dbg,
+                                         (HALO > 0 && use_halo) ? &hall : nullptr))
                     if ((tid & 31) == 0) s_fail = 1;
             }
             __syncthreads();
@@ -514,7 +598,16 @@ __global__ void __launch_bounds__(kThreads, PRN_STAGED_MINB)
                     }
                 }
                 Lay::put_group(A, smem, s, c, grp, hn, b, t0 + grp * 4, h);
-                if (grp == L / 4 - 1 && s == SUB - 1 && chunk < nchunk - 1) {
+                if (HALO > 0) {
+                    constexpr int FIRST = SUB - HALO / L;  // first thread whose steps the successor's halo covers
+                    if (s >= FIRST && chunk < nchunk - 1) {
+                        float4 *so = reinterpret_cast<float4 *>(side_out + ((size_t)tile * HW + (s - FIRST) * L + grp * 4) * S);
+#pragma unroll
+                        for (int u = 0; u < S; ++u)
+                            so[u] = make_float4(hn[(4 * u) / S][(4 * u) % S], hn[(4 * u + 1) / S][(4 * u + 1) % S],
+                                                hn[(4 * u + 2) / S][(4 * u + 2) % S], hn[(4 * u + 3) / S][(4 * u + 3) % S]);
+                    }
+                } else if (grp == L / 4 - 1 && s == SUB - 1 && chunk < nchunk - 1) {
 #pragma unroll
                     for (int q = 0; q < S; ++q) side_out[(tile * C + c) * S + q] = hn[3][q];
                 }
@@ -530,7 +623,7 @@ __global__ void __launch_bounds__(kThreads, PRN_STAGED_MINB)
                 issue(blockIdx.x, true);
             }
         }
-        const unsigned bits = block_max_bits(my_bad ? __int_as_float(0x7fc00000) : my_max, s_red);
+        const unsigned bits = block_max_bits<NT>(my_bad ? __int_as_float(0x7fc00000) : my_max, s_red);
         if (tid == 0) atomicMax(&A.ctl->delta_bits[k % 3], bits);
         if (!grid_sync(A.ctl, A.sticky, A.dbg)) {
             drain();
@@ -556,7 +649,7 @@ __global__ void __launch_bounds__(kThreads, PRN_STAGED_MINB)
     }
 
     if (A.residual_out && !stop_all)
-        if (!residual_pass<Cell, C, L, IN>(A, s_red)) return;
+        if (!residual_pass<Cell, C, L, IN, NT>(A, s_red)) return;
     if (blockIdx.x == 0 && tid == 0) {
         *A.iters_out = iters;
         if (A.delta_out) *A.delta_out = last_delta;
@@ -606,8 +699,9 @@ template <class K> int prepare_kernel(K *kern, int smem_bytes) {
     return 0;
 }
 
-template <class Cell, class Lay, int IN> int choose(Plan *plan, int num_sms, long B, long T, long H) {
-    auto kern = &newton_staged_kernel<Cell, Lay, IN>;
+template <class Cell, class Lay, int IN, int NT = kThreads, int MINB = PRN_STAGED_MINB>
+int choose(Plan *plan, int num_sms, long B, long T, long H) {
+    auto kern = &newton_staged_kernel<Cell, Lay, IN, NT, MINB>;
     const int smem = Lay::SMEM_FLOATS * (int)sizeof(float) + 1024;
     if (prepare_kernel(kern, smem)) return -1;
     plan->kernel = reinterpret_cast<const void *>(kern);
@@ -615,7 +709,9 @@ template <class Cell, class Lay, int IN> int choose(Plan *plan, int num_sms, lon
     plan->C = Lay::C;
     plan->tch = Lay::TCH;
     plan->ntiles = B * (H / Lay::C) * ((T + Lay::TCH - 1) / Lay::TCH);
-    plan->grid = occupancy_grid(plan->kernel, kThreads, smem, num_sms, plan->ntiles);
+    plan->threads = NT;
+    plan->halo_w = Lay::HALO > 0 ? Lay::HALO : 1;
+    plan->grid = occupancy_grid(plan->kernel, NT, smem, num_sms, plan->ntiles);
     return plan->grid > 0 ? 0 : -1;
 }
 
@@ -637,30 +733,33 @@ int newton_staged_plan(const NewtonDiagReq &r, int num_sms, Plan *plan) {
         const bool tma = fused && ((long)r.T * PW) % 32 == 0 && ((long)r.T * S) % 32 == 0;
         if (S == 1) {
             if (tma)
-                rc = r.in == 1 ? choose<GruCell, TmaLong<GruCell, 1, 16>, 1>(plan, num_sms, r.B, r.T, r.H)
-                     : r.in == 2 ? choose<GruCell, TmaLong<GruCell, 2, PRN_LONG_GRU_L>, 2>(plan, num_sms, r.B, r.T, r.H)
-                                 : choose<GruCell, TmaLong<GruCell, 4, 8>, 4>(plan, num_sms, r.B, r.T, r.H);
+                rc = r.in == 1
+                         ? choose<GruCell, TmaLong<GruCell, 1, 16, kThreads, PRN_LONG_HALO>, 1>(plan, num_sms, r.B, r.T, r.H)
+                     : r.in == 2 ? choose<GruCell, TmaLong<GruCell, 2, PRN_LONG_GRU_L, PRN_LONG_NT, PRN_LONG_HALO>, 2,
+                                          PRN_LONG_NT, PRN_LONG_MINB>(plan, num_sms, r.B, r.T, r.H)
+                                 : choose<GruCell, TmaLong<GruCell, 4, 8, kThreads, PRN_LONG_HALO>, 4>(plan, num_sms, r.B,
+                                                                                                      r.T, r.H);
             else
-                rc = !fused ? choose<GruCell, CpLong<GruCell, 0, 16>, 0>(plan, num_sms, r.B, r.T, r.H)
-                     : r.in == 1 ? choose<GruCell, CpLong<GruCell, 1, 16>, 1>(plan, num_sms, r.B, r.T, r.H)
-                     : r.in == 2 ? choose<GruCell, CpLong<GruCell, 2, 16>, 2>(plan, num_sms, r.B, r.T, r.H)
-                                 : choose<GruCell, CpLong<GruCell, 4, 8>, 4>(plan, num_sms, r.B, r.T, r.H);
+                rc = !fused ? choose<GruCell, CpLong<GruCell, 0, 16, kThreads>, 0>(plan, num_sms, r.B, r.T, r.H)
+                     : r.in == 1 ? choose<GruCell, CpLong<GruCell, 1, 16, kThreads>, 1>(plan, num_sms, r.B, r.T, r.H)
+                     : r.in == 2 ? choose<GruCell, CpLong<GruCell, 2, 16, kThreads>, 2>(plan, num_sms, r.B, r.T, r.H)
+                                 : choose<GruCell, CpLong<GruCell, 4, 8, kThreads>, 4>(plan, num_sms, r.B, r.T, r.H);
         } else {
             if (tma)
-                rc = r.in == 1 ? choose<LstmCell, TmaLong<LstmCell, 1, 8>, 1>(plan, num_sms, r.B, r.T, r.H)
-                     : r.in == 2 ? choose<LstmCell, TmaLong<LstmCell, 2, 8>, 2>(plan, num_sms, r.B, r.T, r.H)
-                                 : choose<LstmCell, TmaLong<LstmCell, 4, 8>, 4>(plan, num_sms, r.B, r.T, r.H);
+                rc = r.in == 1 ? choose<LstmCell, TmaLong<LstmCell, 1, 8, kThreads>, 1>(plan, num_sms, r.B, r.T, r.H)
+                     : r.in == 2 ? choose<LstmCell, TmaLong<LstmCell, 2, 8, kThreads>, 2>(plan, num_sms, r.B, r.T, r.H)
+                                 : choose<LstmCell, TmaLong<LstmCell, 4, 8, kThreads>, 4>(plan, num_sms, r.B, r.T, r.H);
             else
-                rc = !fused ? choose<LstmCell, CpLong<LstmCell, 0, 8>, 0>(plan, num_sms, r.B, r.T, r.H)
-                     : r.in == 1 ? choose<LstmCell, CpLong<LstmCell, 1, 8>, 1>(plan, num_sms, r.B, r.T, r.H)
-                     : r.in == 2 ? choose<LstmCell, CpLong<LstmCell, 2, 8>, 2>(plan, num_sms, r.B, r.T, r.H)
-                                 : choose<LstmCell, CpLong<LstmCell, 4, 8>, 4>(plan, num_sms, r.B, r.T, r.H);
+                rc = !fused ? choose<LstmCell, CpLong<LstmCell, 0, 8, kThreads>, 0>(plan, num_sms, r.B, r.T, r.H)
+                     : r.in == 1 ? choose<LstmCell, CpLong<LstmCell, 1, 8, kThreads>, 1>(plan, num_sms, r.B, r.T, r.H)
+                     : r.in == 2 ? choose<LstmCell, CpLong<LstmCell, 2, 8, kThreads>, 2>(plan, num_sms, r.B, r.T, r.H)
+                                 : choose<LstmCell, CpLong<LstmCell, 4, 8, kThreads>, 4>(plan, num_sms, r.B, r.T, r.H);
         }
         plan->staged_tma = tma ? 1 : 0;
     } else if (r.H % 32 == 0 && !fused) {
         plan->variant = 132;
-        rc = S == 1 ? choose<GruCell, Wide<GruCell, 16>, 0>(plan, num_sms, r.B, r.T, r.H)
-                    : choose<LstmCell, Wide<LstmCell, 8>, 0>(plan, num_sms, r.B, r.T, r.H);
+        rc = S == 1 ? choose<GruCell, Wide<GruCell, 16, kThreads>, 0>(plan, num_sms, r.B, r.T, r.H)
+                    : choose<LstmCell, Wide<LstmCell, 8, kThreads>, 0>(plan, num_sms, r.B, r.T, r.H);
     } else {
         return 1;
     }
@@ -668,7 +767,7 @@ int newton_staged_plan(const NewtonDiagReq &r, int num_sms, Plan *plan) {
     plan->S = S;
     plan->agg_words = (size_t)plan->ntiles * plan->C * (S == 1 ? 2 : 6);
     plan->inc_words = (size_t)plan->ntiles * plan->C * S;
-    plan->side_bytes = 2 * (size_t)plan->ntiles * plan->C * S * sizeof(float);
+    plan->side_bytes = 2 * (size_t)plan->ntiles * plan->C * plan->halo_w * S * sizeof(float);
     plan->epochs = (unsigned)r.max_iters + 1u;
     plan->staged = 1;
     return 0;
@@ -687,7 +786,7 @@ cudaError_t newton_staged_launch(const NewtonDiagArgs &A, const Plan &plan, cuda
             return cudaErrorInvalidValue;
     }
     void *args[] = {const_cast<NewtonDiagArgs *>(&A), &M};
-    return cudaLaunchCooperativeKernel(plan.kernel, dim3(plan.grid), dim3(kThreads), args, plan.dyn_smem, st);
+    return cudaLaunchCooperativeKernel(plan.kernel, dim3(plan.grid), dim3(plan.threads), args, plan.dyn_smem, st);
 }
 
 }  // namespace prn

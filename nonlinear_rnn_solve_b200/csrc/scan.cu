@@ -184,6 +184,7 @@ cudaError_t scan_diag_launch(const ScanReq &r, const Plan &plan, const Work &w, 
     A.dbg.skip_tile = dbg.skip_tile;
     A.dbg.delta_log = nullptr;
     A.dbg.delta_log_cap = 0;
+    A.dbg.no_halo = 1;
     void *args[] = {&A};
     return cudaLaunchCooperativeKernel(plan.kernel, dim3(plan.grid), dim3(kThreads), args, 0, st);
 }

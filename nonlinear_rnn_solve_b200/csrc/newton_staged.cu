@@ -381,9 +381,21 @@ __global__ void __launch_bounds__(NT, MINB)
     __shared__ Aff<S> s_halo[HALO > 0 ? HALO / 32 : 1];
     const int tid = threadIdx.x, c = tid % C, s = tid / C;
     const int nct = A.H / C;
-    const long nseq = (long)A.B * nct;
+    const int nseq = A.B * nct;  // the plan keeps tile counts below 2^31
     const int nchunk = (A.T + TCH - 1) / TCH;
-    const long ntiles = nseq * nchunk;
+    const long ntiles = (long)nseq * nchunk;
+    // tile = chunk * nseq + seq advances by gridDim.x: (chunk, seq) are stepped without
+    // dividing in the loop
+    const int step_ch = (int)(gridDim.x / (unsigned)nseq), step_sq = (int)(gridDim.x % (unsigned)nseq);
+    const int first_ch = (int)(blockIdx.x / (unsigned)nseq), first_sq = (int)(blockIdx.x % (unsigned)nseq);
+    auto advance = [&](int &ch, int &sq) {
+        ch += step_ch;
+        sq += step_sq;
+        if (sq >= nseq) {
+            sq -= nseq;
+            ++ch;
+        }
+    };
     // side buffers (two parities): the last HW states that every tile but a sequence's
     // last wrote in the previous iteration.  They are the current iterate for the
     // successor (its halo and first step), which must not read them from h: the
@@ -417,17 +429,16 @@ __global__ void __launch_bounds__(NT, MINB)
 
     // Issue a tile's copies.  Data this CTA wrote with ordinary stores is made visible
     // to the TMA (async proxy) with proxy fences after the preceding barrier.
-    auto issue = [&](long tl, bool with_h) {
-        const int ch = (int)(tl / nseq);
-        const long sq = tl - (long)ch * nseq;
+    auto issue = [&](int ch, int sq, bool with_h) {
+        const int ib = Lay::C == 1 ? sq : sq / nct, ict = Lay::C == 1 ? 0 : sq % nct;  // C == 1: H == 1
         if (Lay::kTma) {
             if (tid == 0) {
                 asm volatile("fence.proxy.async.global;" ::: "memory");
                 asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-                Lay::issue(A, M, smem, &s_bar, (int)(sq / nct), (int)(sq % nct), ch * TCH, with_h);
+                Lay::issue(A, M, smem, &s_bar, ib, ict, ch * TCH, with_h);
             }
         } else {
-            Lay::issue(A, M, smem, &s_bar, (int)(sq / nct), (int)(sq % nct), ch * TCH, with_h);
+            Lay::issue(A, M, smem, &s_bar, ib, ict, ch * TCH, with_h);
         }
     };
     // Wait for the staged tile (bounded).  False when the kernel must stop.
@@ -462,7 +473,9 @@ __global__ void __launch_bounds__(NT, MINB)
             cp_async_wait_all();
         }
     };
-    issue(blockIdx.x, false);
+    issue(first_ch, first_sq, false);
+    Cell cell;
+    if (C == 1) cell.load(A.a, A.peep, A.H, 0);  // C == 1 layouts are H == 1: one unit
 
     int iters = 0;
     float last_delta = 0.f;
@@ -474,11 +487,10 @@ __global__ void __launch_bounds__(NT, MINB)
         float *side_out = A.side + (size_t)((k + 1) & 1) * side_stride;
         float my_max = 0.f;
         bool my_bad = false;
-        for (long tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
-            const int chunk = (int)(tile / nseq);
-            const long seq = tile - (long)chunk * nseq;
-            const int b = (int)(seq / nct);
-            const int ct = (int)(seq % nct);
+        int chunk = first_ch, seq = first_sq;
+        for (long tile = blockIdx.x; tile < ntiles; tile += gridDim.x, advance(chunk, seq)) {
+            const int b = C == 1 ? seq : seq / nct;
+            const int ct = C == 1 ? 0 : seq % nct;
             const int h = ct * C + c;
             const int tch0 = chunk * TCH;
             const int t0 = tch0 + s * L;
@@ -510,8 +522,7 @@ __global__ void __launch_bounds__(NT, MINB)
                 }
             }
             if (!wait_stage()) return;
-            Cell cell;
-            cell.load(A.a, A.peep, A.H, h);
+            if (C != 1) cell.load(A.a, A.peep, A.H, h);
             if (HALO > 0 && use_halo && tid < HALO) {
                 Aff<S> he = Aff<S>::ident();
                 if (tid > 0) {
@@ -561,7 +572,11 @@ __global__ void __launch_bounds__(NT, MINB)
             cta_scan<S, C, NT>(e, sm, excl, total);
             // past the scan's barrier every thread is done reading the stage: refill it
             const long next = tile + gridDim.x;
-            if (next < ntiles) issue(next, k > 0);
+            if (next < ntiles) {
+                int nch = chunk, nsq = seq;
+                advance(nch, nsq);
+                issue(nch, nsq, k > 0);
+            }
             if (tid < 32) {
                 float base[S];
 #pragma unroll
@@ -620,7 +635,7 @@ __global__ void __launch_bounds__(NT, MINB)
             if (next >= ntiles) {
                 // last tile of this iteration: prefetch this CTA's first tile for the next
                 __syncthreads();
-                issue(blockIdx.x, true);
+                issue(first_ch, first_sq, true);
             }
         }
         const unsigned bits = block_max_bits<NT>(my_bad ? __int_as_float(0x7fc00000) : my_max, s_red);
@@ -764,6 +779,7 @@ int newton_staged_plan(const NewtonDiagReq &r, int num_sms, Plan *plan) {
         return 1;
     }
     if (rc) return -1;
+    if (plan->ntiles > 0x7fffffffL) return 1;
     plan->S = S;
     plan->agg_words = (size_t)plan->ntiles * plan->C * (S == 1 ? 2 : 6);
     plan->inc_words = (size_t)plan->ntiles * plan->C * S;

@@ -53,11 +53,12 @@ __global__ void __launch_bounds__(kThreads, 2) adjoint_kernel(const AdjArgs A) {
     const long ntiles = nseq * nchunk;
     LookBack<S> lb{A.agg, A.inc};
     if (tid == 0) s_fail = 0;
-    for (long tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
-        const int chunk = (int)(tile / nseq);  // scan order: from the end of time
-        const long seq = tile - (long)chunk * nseq;
-        const int b = (int)(seq / nct);
-        const int h = (int)(seq % nct) * C + c;
+    TileWalk tw(nseq);
+    for (long tile = blockIdx.x; tile < ntiles; tile += gridDim.x, tw.next()) {
+        const int chunk = tw.chunk;  // scan order: from the end of time
+        const int seq = tw.seq;
+        const int b = seq / nct;
+        const int h = (seq % nct) * C + c;
         const bool cv = h < A.H;
         const int hh = cv ? h : 0;
         const int tbase = (nchunk - 1 - chunk) * TCH + (SUB - 1 - s) * L;

@@ -66,6 +66,7 @@ int ensure_ws(pararnn_ctx *ctx, size_t need) {
 // Look-back words carry the epoch that wrote them; every launch takes a fresh epoch
 // range, and when the 32-bit range would wrap the look-back words are zeroed.
 int prepare(pararnn_ctx *ctx, const prn::Plan &plan, prn::Work *w) {
+    if (plan.ntiles > 0x7fffffffL) return PARARNN_EUNSUPPORTED;  // kernels number tiles in 32 bits
     const size_t ctl_b = up256(sizeof(prn::Ctl));
     const size_t ag_b = up256(plan.agg_words * 8), in_b = up256(plan.inc_words * 8), sd_b = up256(plan.side_bytes);
     int rc = ensure_ws(ctx, ctl_b + ag_b + in_b + sd_b);

@@ -189,6 +189,28 @@ template <> __device__ __forceinline__ Aff<2> make_aff<2>(const float *J, const 
     return {J[0], J[1], J[2], J[3], d[0], d[1]};
 }
 
+// ------------------------------------------------------------------ tile walk
+// Grid-stride walk over tiles numbered tile = chunk * nseq + seq (seq fastest): the
+// coordinates advance by gridDim.x tiles per step without dividing (plans keep tile
+// counts below 2^31).
+struct TileWalk {
+    int nseq, step_ch, step_sq, chunk, seq;
+    __device__ __forceinline__ explicit TileWalk(long n) : nseq((int)n) {
+        step_ch = (int)(gridDim.x / (unsigned)nseq);
+        step_sq = (int)(gridDim.x % (unsigned)nseq);
+        chunk = (int)(blockIdx.x / (unsigned)nseq);
+        seq = (int)(blockIdx.x % (unsigned)nseq);
+    }
+    __device__ __forceinline__ void next() {
+        chunk += step_ch;
+        seq += step_sq;
+        if (seq >= nseq) {
+            seq -= nseq;
+            ++chunk;
+        }
+    }
+};
+
 // ------------------------------------------------------------------ chunked scan
 // Look-back workspace: every published float travels in one 64-bit word together
 // with the 32-bit epoch of the iteration that wrote it, so a reader that sees the

@@ -170,9 +170,10 @@ __global__ void __launch_bounds__(kThreads, 1) tanh_deer_kernel(const TanhArgs A
         const float *side_in = A.side + (size_t)(k & 1) * ntiles * N;
         float *side_out = A.side + (size_t)((k + 1) & 1) * ntiles * N;
         float my_max = 0.f;
-        for (long tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
-            const int chunk = (int)(tile / nseq);
-            const int b = (int)(tile - (long)chunk * nseq);
+        TileWalk tw(nseq);
+        for (long tile = blockIdx.x; tile < ntiles; tile += gridDim.x, tw.next()) {
+            const int chunk = tw.chunk;
+            const int b = tw.seq;
             const int t0 = chunk * TCH;
             const int steps = min(TCH, A.T - t0);
             __syncthreads();
@@ -290,9 +291,10 @@ __global__ void __launch_bounds__(kThreads, 1) tanh_deer_kernel(const TanhArgs A
     }
     if (A.residual_out && !stop_all) {
         float my_res = 0.f;
-        for (long tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
-            const int chunk = (int)(tile / nseq);
-            const int b = (int)(tile - (long)chunk * nseq);
+        TileWalk tw(nseq);
+        for (long tile = blockIdx.x; tile < ntiles; tile += gridDim.x, tw.next()) {
+            const int chunk = tw.chunk;
+            const int b = tw.seq;
             const int t0 = chunk * TCH;
             const int steps = min(TCH, A.T - t0);
             __syncthreads();
@@ -364,9 +366,10 @@ __global__ void __launch_bounds__(kThreads, 2) tanh_quasi_kernel(const TanhArgs 
         const float *side_in = A.side + (size_t)(k & 1) * ntiles * C;
         float *side_out = A.side + (size_t)((k + 1) & 1) * ntiles * C;
         float my_max = 0.f;
-        for (long tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
-            const int chunk = (int)(tile / nseq);
-            const int b = (int)(tile - (long)chunk * nseq);
+        TileWalk tw(nseq);
+        for (long tile = blockIdx.x; tile < ntiles; tile += gridDim.x, tw.next()) {
+            const int chunk = tw.chunk;
+            const int b = tw.seq;
             const int t0 = chunk * TCH;
             __syncthreads();
             tanh_stage_tile<N, TCH>(A, sm, b, t0, k, (k > 0 && chunk > 0) ? side_in + (tile - nseq) * C : nullptr,
@@ -450,9 +453,10 @@ __global__ void __launch_bounds__(kThreads, 2) tanh_quasi_kernel(const TanhArgs 
     }
     if (A.residual_out && !stop_all) {
         float my_res = 0.f;
-        for (long tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
-            const int chunk = (int)(tile / nseq);
-            const int b = (int)(tile - (long)chunk * nseq);
+        TileWalk tw(nseq);
+        for (long tile = blockIdx.x; tile < ntiles; tile += gridDim.x, tw.next()) {
+            const int chunk = tw.chunk;
+            const int b = tw.seq;
             const int t0 = chunk * TCH;
             __syncthreads();
             tanh_stage_tile<N, TCH>(A, sm, b, t0, 1, nullptr, true);
@@ -539,9 +543,10 @@ __global__ void __launch_bounds__(kThreads, 1) dense_scan_kernel(const DScanArgs
     const long ntiles = nseq * nchunk;
     const unsigned epoch = A.epoch0 + 1u;
     if (tid == 0) s_fail = 0;
-    for (long tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
-        const int chunk = (int)(tile / nseq);  // scan order
-        const int b = (int)(tile - (long)chunk * nseq);
+    TileWalk tw(nseq);
+    for (long tile = blockIdx.x; tile < ntiles; tile += gridDim.x, tw.next()) {
+        const int chunk = tw.chunk;  // scan order
+        const int b = tw.seq;
         const int tch = A.reverse ? nchunk - 1 - chunk : chunk;
         const int tbeg = tch * TCH;
         const int steps = min(TCH, A.T - tbeg);

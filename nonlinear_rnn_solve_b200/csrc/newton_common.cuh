@@ -127,11 +127,12 @@ __device__ bool residual_pass(const NewtonDiagArgs &A, unsigned *s_red) {
     const int nchunk = (A.T + TCH - 1) / TCH;
     const long ntiles = nseq * nchunk;
     float my_res = 0.f;
-    for (long tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
-        const int chunk = (int)(tile / nseq);
-        const long seq = tile - (long)chunk * nseq;
-        const int b = (int)(seq / nct);
-        const int h = (int)(seq % nct) * C + c;
+    TileWalk tw(nseq);
+    for (long tile = blockIdx.x; tile < ntiles; tile += gridDim.x, tw.next()) {
+        const int chunk = tw.chunk;
+        const int seq = tw.seq;
+        const int b = seq / nct;
+        const int h = (seq % nct) * C + c;
         if (h >= A.H) continue;
         const int t0 = chunk * TCH + s * L;
         Cell cell;

@@ -58,11 +58,12 @@ __global__ void __launch_bounds__(kThreads, 2) newton_diag_kernel(const NewtonDi
         const float *side_in = A.side + (size_t)(k & 1) * side_stride;
         float *side_out = A.side + (size_t)((k + 1) & 1) * side_stride;
         float my_max = 0.f;
-        for (long tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
-            const int chunk = (int)(tile / nseq);
-            const long seq = tile - (long)chunk * nseq;
-            const int b = (int)(seq / nct);
-            const int h = (int)(seq % nct) * C + c;
+        TileWalk tw(nseq);
+        for (long tile = blockIdx.x; tile < ntiles; tile += gridDim.x, tw.next()) {
+            const int chunk = tw.chunk;
+            const int seq = tw.seq;
+            const int b = seq / nct;
+            const int h = (seq % nct) * C + c;
             const bool cv = h < A.H;
             const int hh = cv ? h : 0;
             const int t0 = chunk * TCH + s * L;

@@ -66,11 +66,12 @@ __global__ void __launch_bounds__(kThreads, 2) scan_kernel(const ScanArgs A) {
     const long ntiles = nseq * nchunk;
     LookBack<S> lb{A.agg, A.inc};
     if (tid == 0) s_fail = 0;
-    for (long tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
-        const int chunk = (int)(tile / nseq);  // position in scan order
-        const long seq = tile - (long)chunk * nseq;
-        const int b = (int)(seq / nct);
-        const int n = (int)(seq % nct) * C + c;
+    TileWalk tw(nseq);
+    for (long tile = blockIdx.x; tile < ntiles; tile += gridDim.x, tw.next()) {
+        const int chunk = tw.chunk;  // position in scan order
+        const int seq = tw.seq;
+        const int b = seq / nct;
+        const int n = (seq % nct) * C + c;
         const bool cv = n < A.N;
         const int nn = cv ? n : 0;
         // time of this thread's first step in scan order, and the direction

@@ -101,8 +101,9 @@ int pararnn_set_stream(pararnn_ctx *ctx, void *cuda_stream);
  * fp32 accumulation) or both fp32 (PARARNN_F32, CUDA cores); bias fp32 [N] or NULL;
  * xproj fp32 [M, N].  Implied by the cells of the pages: the input term W x_t does
  * not depend on the state, so it is computed once per forward pass.
- * bf16 needs K % 64 == 0 and N % 16 == 0 ... see the EINVAL conditions in the
- * implementation notes below; any M is accepted. */
+ * Shapes: any M, N >= 1; bf16 needs K % 8 == 0 (16-byte rows for the tensor-memory
+ * copies), fp32 any K; M * N <= 2^40.  x, W, bias and xproj 16-byte aligned.
+ * Returns EINVAL (null pointer, bad dtype or shape), EALIGN, or ECUDA (launch). */
 int pararnn_input_proj(pararnn_ctx *ctx, const void *x, int x_dtype, const void *W,
                        const float *bias, float *xproj, int M, int K, int N);
 

@@ -118,9 +118,10 @@ template <class Cell, int IN, int LL, int NT, int HL = 0> struct TmaLong {
     static_assert(SEGH == 8 || SEGH == 16 || SEGH == 32, "state segment must be part of one 128-byte row");
     static constexpr int XFLOATS = TCH * PW, HFLOATS = TCH * S;
     static_assert(XFLOATS / 32 <= 256 && HFLOATS / 32 <= 256, "TMA box height");
-    // regions: X | H | OUT, each a multiple of 1024 bytes
+    // regions: X | H | OUT (two, by tile parity), each a multiple of 1024 bytes
     static constexpr int OFFH = XFLOATS, OFFO = XFLOATS + HFLOATS;
-    static constexpr int SMEM_FLOATS = XFLOATS + 2 * HFLOATS;
+    static constexpr int SMEM_FLOATS = XFLOATS + 3 * HFLOATS;
+    static constexpr int OUT_STRIDE = HFLOATS;  // offset of the second staging tile
     static constexpr bool kTma = true;
 
     __device__ static void issue(const NewtonDiagArgs &A, const StagedMaps &M, float *sm, unsigned long long *bar,
@@ -175,9 +176,9 @@ template <class Cell, int IN, int LL, int NT, int HL = 0> struct TmaLong {
             *swz_chunk<SEGH>(sm + OFFO, s, grp * S + q) = make_float4(v[0], v[1], v[2], v[3]);
         }
     }
-    // coalesced 16-byte stores of the staged results of the tile
+    // coalesced 16-byte stores of the staged results of the tile (the caller puts a
+    // barrier between the put_group writes and this)
     __device__ static void flush(const NewtonDiagArgs &A, float *sm, int b, int, int tch0) {
-        __syncthreads();
         const int valid = min(TCH, A.T - tch0) * S;
         float *g = A.h + ((size_t)b * A.T + tch0) * S;
         const float *o = sm + OFFO;
@@ -186,8 +187,6 @@ template <class Cell, int IN, int LL, int NT, int HL = 0> struct TmaLong {
             const float4 v = *reinterpret_cast<const float4 *>(o + row * 32 + ((lc ^ (row & 7)) << 2));
             *reinterpret_cast<float4 *>(g + 4 * c) = v;
         }
-        // the staging tile is next written after the following tile's stage wait and
-        // scan barriers: no barrier needed here
     }
 };
 
@@ -199,6 +198,7 @@ template <class Cell, int IN, int LL, int NT> struct CpLong {
     static constexpr int SEGH = L * S, STRH = pad_stride(SEGH);
     static constexpr int OFFH = SUB * STRP;
     static constexpr int SMEM_FLOATS = SUB * (STRP + STRH);
+    static constexpr int OUT_STRIDE = 0;
     static constexpr bool kTma = false;
     static constexpr int HALO = 0;
     static_assert(SEGP % 4 == 0 && SEGH % 4 == 0, "segments are whole 16-byte chunks");
@@ -264,6 +264,7 @@ template <class Cell, int LL, int NT> struct Wide {
     static constexpr int ROWP = 3 * 32, ROWH = 32 * S;
     static constexpr int OFFH = TCH * ROWP;
     static constexpr int SMEM_FLOATS = TCH * (ROWP + ROWH);
+    static constexpr int OUT_STRIDE = 0;
     static constexpr bool kTma = false;
     static constexpr int HALO = 0;
 
@@ -374,11 +375,14 @@ __global__ void __launch_bounds__(NT, MINB)
                   "a halo is one step per thread of whole warps, covers whole segments, raw inputs, H = 1");
     extern __shared__ __align__(1024) unsigned char smraw[];
     float *const smem = reinterpret_cast<float *>(((uintptr_t)smraw + 1023) & ~(uintptr_t)1023);
-    __shared__ ScanSmem<S, C, NT> sm;
+    // scan exchange and halo totals alternate between two copies by tile parity: a
+    // warp may start the next tile while others still read this tile's copy (the tile
+    // loop has one CTA barrier per tile on the common path)
+    __shared__ ScanSmem<S, C, NT> sm2[2];
     __shared__ unsigned s_red[NT / 32];
     __shared__ int s_fail;
     __shared__ __align__(8) unsigned long long s_bar;
-    __shared__ Aff<S> s_halo[HALO > 0 ? HALO / 32 : 1];
+    __shared__ Aff<S> s_halo[2][HALO > 0 ? HALO / 32 : 1];
     const int tid = threadIdx.x, c = tid % C, s = tid / C;
     const int nct = A.H / C;
     const int nseq = A.B * nct;  // the plan keeps tile counts below 2^31
@@ -441,7 +445,10 @@ __global__ void __launch_bounds__(NT, MINB)
             Lay::issue(A, M, smem, &s_bar, ib, ict, ch * TCH, with_h);
         }
     };
-    // Wait for the staged tile (bounded).  False when the kernel must stop.
+    // Wait for the staged tile (bounded).  TMA: every thread waits on the mbarrier
+    // itself (no CTA barrier); false when the wait gave up, which the caller turns
+    // into a CTA-wide stop at the next barrier.  cp.async: each thread's copies serve
+    // other threads, so a CTA barrier follows.
     auto wait_stage = [&]() -> bool {
         if (Lay::kTma) {
             bool ok = mbar_try(&s_bar, bar_phase);
@@ -455,8 +462,8 @@ __global__ void __launch_bounds__(NT, MINB)
                     }
                 }
             }
-            bar_phase ^= 1u;
-            return __syncthreads_and(ok) != 0;
+            if (ok) bar_phase ^= 1u;  // on failure drain() waits for the pending phase
+            return ok;
         }
         cp_async_wait_all();
         __syncthreads();
@@ -488,7 +495,10 @@ __global__ void __launch_bounds__(NT, MINB)
         float my_max = 0.f;
         bool my_bad = false;
         int chunk = first_ch, seq = first_sq;
-        for (long tile = blockIdx.x; tile < ntiles; tile += gridDim.x, advance(chunk, seq)) {
+        int par = 0;                    // tile parity within the iteration
+        int fl_b = -1, fl_ct = 0, fl_t = 0;  // staged results still to be written (previous tile)
+        for (long tile = blockIdx.x; tile < ntiles; tile += gridDim.x, advance(chunk, seq), par ^= 1) {
+            ScanSmem<S, C, NT> &sm = sm2[par];
             const int b = C == 1 ? seq : seq / nct;
             const int ct = C == 1 ? 0 : seq % nct;
             const int h = ct * C + c;
@@ -521,7 +531,7 @@ __global__ void __launch_bounds__(NT, MINB)
                     hprv[q] = (k > 0 && tid > 0) ? sp[(tid - 1) * S + q] : 0.f;
                 }
             }
-            if (!wait_stage()) return;
+            if (!wait_stage()) s_fail = 1;  // acted on after the scan's barrier
             if (C != 1) cell.load(A.a, A.peep, A.H, h);
             if (HALO > 0 && use_halo && tid < HALO) {
                 Aff<S> he = Aff<S>::ident();
@@ -545,7 +555,7 @@ __global__ void __launch_bounds__(NT, MINB)
                     const Aff<S> o = he.shfl_down(off);
                     if ((tid & 31) + off < 32) he = compose(he, o);
                 }
-                if ((tid & 31) == 0) s_halo[tid >> 5] = he;  // read after cta_scan's barrier
+                if ((tid & 31) == 0) s_halo[par][tid >> 5] = he;  // read after the scan's barrier
             }
             float hp[S];
 #pragma unroll
@@ -569,34 +579,60 @@ __global__ void __launch_bounds__(NT, MINB)
 #pragma unroll
             for (int i = 0; i < L; ++i) e = compose(e, make_aff<S>(Jr[i], rr[i]));
             Aff<S> excl, total;
-            cta_scan<S, C, NT>(e, sm, excl, total);
-            // past the scan's barrier every thread is done reading the stage: refill it
+            cta_scan<S, C, NT>(e, sm, excl, total);  // the one CTA barrier of the common path
+            if (s_fail) {
+                drain();
+                return;  // a bounded wait ran out; the status says so
+            }
+            // past the barrier every thread is done reading the stage: refill it
             const long next = tile + gridDim.x;
             if (next < ntiles) {
                 int nch = chunk, nsq = seq;
                 advance(nch, nsq);
                 issue(nch, nsq, k > 0);
             }
-            if (tid < 32) {
-                float base[S];
+            // the previous tile's staged results (written before the barrier) leave now
+            if (fl_b >= 0) Lay::flush(A, smem + (par ^ 1) * Lay::OUT_STRIDE, fl_b, fl_ct, fl_t);
+            // carry entering the tile: from the halo when its composed map is constant
+            // (every thread composes the same totals, so the branch is CTA-uniform),
+            // else from the look-back by warp 0 and a second barrier
+            float carry[S];
 #pragma unroll
-                for (int q = 0; q < S; ++q) base[q] = 0.f;  // delta entering t = 0 is 0
-                Aff<S> hall = Aff<S>::ident();
-                if (HALO > 0 && use_halo) {
+            for (int q = 0; q < S; ++q) carry[q] = 0.f;  // a sequence's first tile: delta entering t = 0 is 0
+            bool known = chunk == 0;
+            if (HALO > 0 && use_halo) {
+                Aff<S> hall = s_halo[par][0];
 #pragma unroll
-                    for (int w = 0; w < HW / 32; ++w) hall = compose(hall, s_halo[w]);
-                }
-                if (!look_back<S, C, NT>(lb, sm, total, tile, chunk, nseq, epoch, base, A.ctl, A.sticky, A.dbg,
-                                         (HALO > 0 && use_halo) ? &hall : nullptr))
-                    if ((tid & 31) == 0) s_fail = 1;
+                for (int w = 1; w < HW / 32; ++w) hall = compose(hall, s_halo[par][w]);
+                float hv[Aff<S>::kFloats];
+                hall.to_floats(hv);
+                known = aff_is_const<S>(hv);
+#pragma unroll
+                for (int q = 0; q < S; ++q) carry[q] = hv[S * S + q];
             }
-            __syncthreads();
-            if (s_fail) {
-                drain();
-                return;  // a bounded wait ran out; the status says so
+            if (known) {
+                if (tid < 32) {  // keep the look-back words complete for tiles that need them
+                    publish_agg<S, C>(lb, total, tile, chunk, epoch, A.dbg);
+                    publish_inc<S, C>(lb, total, carry, tile, epoch, A.dbg);
+                }
+            } else {
+                if (tid < 32) {
+                    float base[S];
+#pragma unroll
+                    for (int q = 0; q < S; ++q) base[q] = 0.f;  // delta entering t = 0 is 0
+                    if (!look_back<S, C, NT>(lb, sm, total, tile, chunk, nseq, epoch, base, A.ctl, A.sticky, A.dbg))
+                        if ((tid & 31) == 0) s_fail = 1;
+                }
+                __syncthreads();
+                if (s_fail) {
+                    drain();
+                    return;  // a bounded wait ran out; the status says so
+                }
+#pragma unroll
+                for (int q = 0; q < S; ++q) carry[q] = sm.carry[c][q];
             }
             float d[S];
-            excl.apply(sm.carry[c], d);
+            excl.apply(carry, d);
 #pragma unroll
             for (int grp = 0; grp < L / 4; ++grp) {
                 float hn[4][S];
@@ -612,7 +648,7 @@ __global__ void __launch_bounds__(NT, MINB)
                         my_max = fmaxf(my_max, fabsf(nd[q]));
                     }
                 }
-                Lay::put_group(A, smem, s, c, grp, hn, b, t0 + grp * 4, h);
+                Lay::put_group(A, smem + par * Lay::OUT_STRIDE, s, c, grp, hn, b, t0 + grp * 4, h);
                 if (HALO > 0) {
                     constexpr int FIRST = SUB - HALO / L;  // first thread whose steps the successor's halo covers
                     if (s >= FIRST && chunk < nchunk - 1) {
@@ -631,15 +667,18 @@ __global__ void __launch_bounds__(NT, MINB)
             // feeds the next through J), where it is caught
 #pragma unroll
             for (int q = 0; q < S; ++q) my_bad |= !finitef(d[q]);
-            Lay::flush(A, smem, b, ct, tch0);
-            if (next >= ntiles) {
-                // last tile of this iteration: prefetch this CTA's first tile for the next
-                __syncthreads();
-                issue(first_ch, first_sq, true);
-            }
+            fl_b = b;
+            fl_ct = ct;
+            fl_t = tch0;
         }
+        // the last tile's staged results
+        __syncthreads();
+        if (fl_b >= 0) Lay::flush(A, smem + (par ^ 1) * Lay::OUT_STRIDE, fl_b, fl_ct, fl_t);
         const unsigned bits = block_max_bits<NT>(my_bad ? __int_as_float(0x7fc00000) : my_max, s_red);
         if (tid == 0) atomicMax(&A.ctl->delta_bits[k % 3], bits);
+        // prefetch this CTA's first tile for the next iteration: past the barriers of the
+        // block max, all of this CTA's stores to it are done (no other CTA writes it)
+        issue(first_ch, first_sq, true);
         if (!grid_sync(A.ctl, A.sticky, A.dbg)) {
             drain();
             return;

@@ -340,12 +340,138 @@ template <int N> struct QuasiCfg {
     static constexpr int TCH = SUB * L;
 };
 
+// Shared memory of a quasi-DEER tile.  Phase A evaluates the cell for the whole tile as
+// a small matrix product, U[tr][i] = sum_k A[i][k] h^(k)[tr-1][k] + p[tr][i], with each
+// thread holding a 4-step x 4-unit block in registers (two 128-bit loads feed sixteen
+// FMAs), and leaves J, r and h^(k) per (step, unit).  Phase B is the diagonal scan.
+template <int N> struct QuasiSmem {
+    static constexpr int TCH = QuasiCfg<N>::TCH;
+    static constexpr int AS = N + 4;    // row stride of AT and Wt (float4-aligned)
+    static constexpr int HS = TCH + 4;  // row stride of hT and xT (float4-aligned, >= TCH + 1)
+    float AT[N * AS];                   // AT[k][i] = A[i][k]
+    float Wt[8 * AS];                   // Wt[q][i] = W[i][q]
+    float bz[N];
+    float hT[N * HS];                   // hT[k][r] = h^(k) of unit k at step t0 - 1 + r
+    float xT[8 * HS];                   // xT[q][tr] = x of input q at step t0 + tr
+    float Js[TCH * N], rs[TCH * N], hc[TCH * N];  // per (step row, unit)
+};
+
+template <int N> __device__ void quasi_stage_params(const TanhArgs &A, QuasiSmem<N> &sm) {
+    constexpr int AS = QuasiSmem<N>::AS;
+    for (int e = threadIdx.x; e < N * N; e += kThreads) {
+        const int i = e / N, k = e % N;  // A[i][k]
+        sm.AT[k * AS + i] = (i < A.n && k < A.n) ? A.A[(size_t)i * A.n + k] : 0.f;
+    }
+    for (int e = threadIdx.x; e < 8 * N; e += kThreads) {
+        const int q = e / N, i = e % N;
+        sm.Wt[q * AS + i] = (!A.xproj && q < A.in && i < A.n) ? A.W[(size_t)i * A.in + q] : 0.f;
+    }
+    for (int i = threadIdx.x; i < N; i += kThreads) sm.bz[i] = (!A.xproj && A.bias && i < A.n) ? A.bias[i] : 0.f;
+}
+
+// Stage the tile's states (h^(k) rows t0-1 .. t0+TCH-1: h0 before t = 0, the side
+// value for the preceding tile's last step, zeros on the first iteration) and raw
+// inputs, transposed so that four consecutive steps of one unit are one 128-bit read.
+template <int N>
+__device__ void quasi_stage_tile(const TanhArgs &A, QuasiSmem<N> &sm, int b, int t0, bool have_h,
+                                 const float *prev_side) {
+    constexpr int TCH = QuasiSmem<N>::TCH, HS = QuasiSmem<N>::HS;
+    for (int e = threadIdx.x; e < (TCH + 1) * N; e += kThreads) {
+        const int r = e / N, i = e % N, t = t0 + r - 1;
+        float v = 0.f;
+        if (i < A.n) {
+            if (t < 0)
+                v = A.h0 ? A.h0[(size_t)b * A.n + i] : 0.f;
+            else if (t < A.T && have_h)
+                v = (r == 0 && prev_side) ? prev_side[i] : A.h[((size_t)b * A.T + t) * A.n + i];
+        }
+        sm.hT[i * HS + r] = v;
+    }
+    if (!A.xproj) {
+        for (int e = threadIdx.x; e < TCH * 8; e += kThreads) {
+            const int r = e / 8, q = e % 8, t = t0 + r;
+            sm.xT[q * HS + r] = (q < A.in && t < A.T) ? A.x[((size_t)b * A.T + t) * A.in + q] : 0.f;
+        }
+    }
+}
+
+// Phase A: f = tanh(A h_{t-1} + p_t) for the thread's 4 x 4 block; J = (1 - f^2) A_ii
+// (identity outside the sequence), r = f - h^(k)_t; returns max |r| over valid entries.
+template <int N>
+__device__ float quasi_phase_a(const TanhArgs &A, QuasiSmem<N> &sm, int b, int t0) {
+    constexpr int TCH = QuasiSmem<N>::TCH, AS = QuasiSmem<N>::AS, HS = QuasiSmem<N>::HS;
+    constexpr int NUB = N / 4;
+    const int ub = threadIdx.x % NUB, sb = threadIdx.x / NUB;
+    const int i0 = 4 * ub, r0 = 4 * sb;
+    float acc[4][4];
+    if (A.xproj) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int t = t0 + r0 + j;
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                acc[j][u] = (t < A.T && i0 + u < A.n) ? A.xproj[((size_t)b * A.T + t) * A.n + i0 + u] : 0.f;
+        }
+    } else {
+        const float4 bz = *reinterpret_cast<const float4 *>(sm.bz + i0);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            acc[j][0] = bz.x;
+            acc[j][1] = bz.y;
+            acc[j][2] = bz.z;
+            acc[j][3] = bz.w;
+        }
+        for (int q = 0; q < A.in; ++q) {
+            const float4 w = *reinterpret_cast<const float4 *>(sm.Wt + q * AS + i0);
+            const float4 x = *reinterpret_cast<const float4 *>(sm.xT + q * HS + r0);
+            const float xv[4] = {x.x, x.y, x.z, x.w}, wv[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+#pragma unroll
+                for (int u = 0; u < 4; ++u) acc[j][u] = fmaf(wv[u], xv[j], acc[j][u]);
+        }
+    }
+#pragma unroll 8
+    for (int k = 0; k < N; ++k) {
+        const float4 a = *reinterpret_cast<const float4 *>(sm.AT + k * AS + i0);
+        const float4 h = *reinterpret_cast<const float4 *>(sm.hT + k * HS + r0);  // h_{t-1} of steps r0..r0+3
+        const float av[4] = {a.x, a.y, a.z, a.w}, hv[4] = {h.x, h.y, h.z, h.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+#pragma unroll
+            for (int u = 0; u < 4; ++u) acc[j][u] = fmaf(av[u], hv[j], acc[j][u]);
+    }
+    float res = 0.f;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const int tr = r0 + j;
+        const bool tv = t0 + tr < A.T;
+        float Jv[4], rv[4], hcv[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int i = i0 + u;
+            const bool v = tv && i < A.n;
+            const float f = tanh_(acc[j][u]);
+            const float cur = sm.hT[i * HS + tr + 1];
+            Jv[u] = v ? (1.f - f * f) * sm.AT[i * AS + i] : 1.f;
+            rv[u] = v ? f - cur : 0.f;
+            hcv[u] = cur;
+            const float ad = fabsf(rv[u]);
+            res = (ad > res || isnan(ad)) ? ad : res;
+        }
+        *reinterpret_cast<float4 *>(sm.Js + tr * N + i0) = make_float4(Jv[0], Jv[1], Jv[2], Jv[3]);
+        *reinterpret_cast<float4 *>(sm.rs + tr * N + i0) = make_float4(rv[0], rv[1], rv[2], rv[3]);
+        *reinterpret_cast<float4 *>(sm.hc + tr * N + i0) = make_float4(hcv[0], hcv[1], hcv[2], hcv[3]);
+    }
+    return res;
+}
+
 template <int N>
 __global__ void __launch_bounds__(kThreads, 2) tanh_quasi_kernel(const TanhArgs A) {
     constexpr int C = QuasiCfg<N>::C, SUB = QuasiCfg<N>::SUB, L = QuasiCfg<N>::L, TCH = QuasiCfg<N>::TCH;
-    constexpr int AS = TanhSmem<N, TCH>::AS;
+    static_assert(N % 4 == 0 && (N / 4) * (TCH / 4) == kThreads, "one 4 x 4 block per thread");
     extern __shared__ __align__(16) unsigned char smraw[];
-    TanhSmem<N, TCH> &sm = *reinterpret_cast<TanhSmem<N, TCH> *>(smraw);
+    QuasiSmem<N> &sm = *reinterpret_cast<QuasiSmem<N> *>(smraw);
     __shared__ ScanSmem<1, (C <= 32 ? C : 32)> ss;
     __shared__ Scan64Smem s64;
     __shared__ unsigned s_red[kThreads / 32];
@@ -356,7 +482,7 @@ __global__ void __launch_bounds__(kThreads, 2) tanh_quasi_kernel(const TanhArgs 
     const long ntiles = nseq * nchunk;
     LookBack<1> lb{A.agg, A.inc};
     if (tid == 0) s_fail = 0;
-    tanh_stage_params<N, TCH>(A, sm);
+    quasi_stage_params<N>(A, sm);
     int iters = 0;
     float last_delta = 0.f;
     bool stop_all = false;
@@ -372,25 +498,17 @@ __global__ void __launch_bounds__(kThreads, 2) tanh_quasi_kernel(const TanhArgs 
             const int b = tw.seq;
             const int t0 = chunk * TCH;
             __syncthreads();
-            tanh_stage_tile<N, TCH>(A, sm, b, t0, k, (k > 0 && chunk > 0) ? side_in + (tile - nseq) * C : nullptr,
-                                    false);
+            quasi_stage_tile<N>(A, sm, b, t0, k > 0, (k > 0 && chunk > 0) ? side_in + (tile - nseq) * C : nullptr);
+            __syncthreads();
+            quasi_phase_a<N>(A, sm, b, t0);
             __syncthreads();
             const bool cv = c < A.n;
-            const float aii = sm.AT[c * AS + c];
-            float Jr[L], rr[L], hc[L];
-#pragma unroll
-            for (int i = 0; i < L; ++i) {
-                const int tr = s * L + i, t = t0 + tr;
-                const bool v = cv && t < A.T;
-                const float f = cv ? tanh_(tanh_preact<N, TCH>(A, sm, b, v ? t : t0, tr, c)) : 0.f;
-                const float cur = sm.hs[(tr + 1) * N + c];
-                Jr[i] = v ? (1.f - f * f) * aii : 1.f;
-                rr[i] = v ? f - cur : 0.f;
-                hc[i] = cur;
-            }
             Aff<1> e = Aff<1>::ident();
 #pragma unroll
-            for (int i = 0; i < L; ++i) e = compose(e, Aff<1>{Jr[i], rr[i]});
+            for (int i = 0; i < L; ++i) {
+                const int tr = s * L + i;
+                e = compose(e, Aff<1>{sm.Js[tr * N + c], sm.rs[tr * N + c]});
+            }
             Aff<1> excl, total;
             const float zero[1] = {0.f};
             float carry_c;
@@ -427,8 +545,8 @@ __global__ void __launch_bounds__(kThreads, 2) tanh_quasi_kernel(const TanhArgs 
 #pragma unroll
             for (int i = 0; i < L; ++i) {
                 const int tr = s * L + i, t = t0 + tr;
-                d = fmaf(Jr[i], d, rr[i]);
-                const float hn = hc[i] + d;
+                d = fmaf(sm.Js[tr * N + c], d, sm.rs[tr * N + c]);
+                const float hn = sm.hc[tr * N + c] + d;
                 if (cv && t < A.T) {
                     const float ad = fabsf(d);
                     my_max = (ad > my_max || isnan(d)) ? ad : my_max;
@@ -452,23 +570,18 @@ __global__ void __launch_bounds__(kThreads, 2) tanh_quasi_kernel(const TanhArgs 
         if (last_delta < A.tol) break;
     }
     if (A.residual_out && !stop_all) {
+        // max |h_t - f(h_{t-1}, x_t)| at the result: phase A's max |r| with the result
+        // staged as the iterate
         float my_res = 0.f;
         TileWalk tw(nseq);
         for (long tile = blockIdx.x; tile < ntiles; tile += gridDim.x, tw.next()) {
-            const int chunk = tw.chunk;
             const int b = tw.seq;
-            const int t0 = chunk * TCH;
+            const int t0 = tw.chunk * TCH;
             __syncthreads();
-            tanh_stage_tile<N, TCH>(A, sm, b, t0, 1, nullptr, true);
+            quasi_stage_tile<N>(A, sm, b, t0, true, nullptr);
             __syncthreads();
-            for (int e = tid; e < TCH * N; e += kThreads) {
-                const int tr = e / N, i = e % N;
-                if (t0 + tr < A.T && i < A.n) {
-                    const float f = tanh_(tanh_preact<N, TCH>(A, sm, b, t0 + tr, tr, i));
-                    const float ad = fabsf(sm.hs[(tr + 1) * N + i] - f);
-                    my_res = (ad > my_res || isnan(ad)) ? ad : my_res;
-                }
-            }
+            const float r = quasi_phase_a<N>(A, sm, b, t0);
+            my_res = (r > my_res || isnan(r)) ? r : my_res;
         }
         const unsigned bits = block_max_bits(my_res, s_red);
         if (tid == 0) atomicMax(&A.ctl->res_bits, bits);
@@ -656,7 +769,7 @@ template <class K> int set_smem(K kern, size_t bytes) {
 template <int N> size_t deer_smem() {
     return ((sizeof(TanhSmem<N, DeerCfg<N>::TCH>) + 15) & ~size_t(15)) + sizeof(DeerExtra<N>);
 }
-template <int N> size_t quasi_smem() { return sizeof(TanhSmem<N, QuasiCfg<N>::TCH>); }
+template <int N> size_t quasi_smem() { return sizeof(QuasiSmem<N>); }
 
 template <int N> int tanh_plan_n(const NewtonTanhReq &r, int num_sms, Plan *plan) {
     if (r.quasi) {

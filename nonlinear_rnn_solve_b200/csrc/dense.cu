@@ -351,9 +351,11 @@ template <int N> struct QuasiSmem {
     float AT[N * AS];                   // AT[k][i] = A[i][k]
     float Wt[8 * AS];                   // Wt[q][i] = W[i][q]
     float bz[N];
+    float diag[N];                      // A_ii
     float hT[N * HS];                   // hT[k][r] = h^(k) of unit k at step t0 - 1 + r
+    float hr[(TCH + 1) * N];            // the same states by row: hr[r][k] (conflict-free row reads)
     float xT[8 * HS];                   // xT[q][tr] = x of input q at step t0 + tr
-    float Js[TCH * N], rs[TCH * N], hc[TCH * N];  // per (step row, unit)
+    float Js[TCH * N], rs[TCH * N];     // per (step row, unit)
 };
 
 template <int N> __device__ void quasi_stage_params(const TanhArgs &A, QuasiSmem<N> &sm) {
@@ -367,6 +369,7 @@ template <int N> __device__ void quasi_stage_params(const TanhArgs &A, QuasiSmem
         sm.Wt[q * AS + i] = (!A.xproj && q < A.in && i < A.n) ? A.W[(size_t)i * A.in + q] : 0.f;
     }
     for (int i = threadIdx.x; i < N; i += kThreads) sm.bz[i] = (!A.xproj && A.bias && i < A.n) ? A.bias[i] : 0.f;
+    for (int i = threadIdx.x; i < N; i += kThreads) sm.diag[i] = i < A.n ? A.A[(size_t)i * A.n + i] : 0.f;
 }
 
 // Stage the tile's states (h^(k) rows t0-1 .. t0+TCH-1: h0 before t = 0, the side
@@ -386,6 +389,7 @@ __device__ void quasi_stage_tile(const TanhArgs &A, QuasiSmem<N> &sm, int b, int
                 v = (r == 0 && prev_side) ? prev_side[i] : A.h[((size_t)b * A.T + t) * A.n + i];
         }
         sm.hT[i * HS + r] = v;
+        sm.hr[e] = v;
     }
     if (!A.xproj) {
         for (int e = threadIdx.x; e < TCH * 8; e += kThreads) {
@@ -394,6 +398,53 @@ __device__ void quasi_stage_tile(const TanhArgs &A, QuasiSmem<N> &sm, int b, int
         }
     }
 }
+
+// The next tile's states and inputs, loaded into registers while the current tile
+// computes, and written to shared memory (as quasi_stage_tile does) when it starts.
+template <int N> struct QuasiPrefetch {
+    static constexpr int TCH = QuasiSmem<N>::TCH, HS = QuasiSmem<N>::HS;
+    static constexpr int HPT = ((TCH + 1) * N + kThreads - 1) / kThreads;
+    static constexpr int XPT = TCH * 8 / kThreads;
+    float hv[HPT], xv[XPT];
+    __device__ __forceinline__ void load(const TanhArgs &A, int b, int t0, bool have_h, const float *prev_side) {
+#pragma unroll
+        for (int j = 0; j < HPT; ++j) {
+            const int e = threadIdx.x + j * kThreads, r = e / N, i = e % N, t = t0 + r - 1;
+            float v = 0.f;
+            if (e < (TCH + 1) * N && i < A.n) {
+                if (t < 0)
+                    v = A.h0 ? A.h0[(size_t)b * A.n + i] : 0.f;
+                else if (t < A.T && have_h)
+                    v = (r == 0 && prev_side) ? prev_side[i] : A.h[((size_t)b * A.T + t) * A.n + i];
+            }
+            hv[j] = v;
+        }
+        if (!A.xproj) {
+#pragma unroll
+            for (int j = 0; j < XPT; ++j) {
+                const int e = threadIdx.x + j * kThreads, r = e / 8, q = e % 8, t = t0 + r;
+                xv[j] = (q < A.in && t < A.T) ? A.x[((size_t)b * A.T + t) * A.in + q] : 0.f;
+            }
+        }
+    }
+    __device__ __forceinline__ void store(const TanhArgs &A, QuasiSmem<N> &sm) const {
+#pragma unroll
+        for (int j = 0; j < HPT; ++j) {
+            const int e = threadIdx.x + j * kThreads;
+            if (e < (TCH + 1) * N) {
+                sm.hT[(e % N) * HS + e / N] = hv[j];
+                sm.hr[e] = hv[j];
+            }
+        }
+        if (!A.xproj) {
+#pragma unroll
+            for (int j = 0; j < XPT; ++j) {
+                const int e = threadIdx.x + j * kThreads;
+                sm.xT[(e % 8) * HS + e / 8] = xv[j];
+            }
+        }
+    }
+};
 
 // Phase A: f = tanh(A h_{t-1} + p_t) for the thread's 4 x 4 block; J = (1 - f^2) A_ii
 // (identity outside the sequence), r = f - h^(k)_t; returns max |r| over valid entries.
@@ -442,26 +493,26 @@ __device__ float quasi_phase_a(const TanhArgs &A, QuasiSmem<N> &sm, int b, int t
             for (int u = 0; u < 4; ++u) acc[j][u] = fmaf(av[u], hv[j], acc[j][u]);
     }
     float res = 0.f;
+    const float4 dg4 = *reinterpret_cast<const float4 *>(sm.diag + i0);
+    const float dg[4] = {dg4.x, dg4.y, dg4.z, dg4.w};
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
         const int tr = r0 + j;
         const bool tv = t0 + tr < A.T;
-        float Jv[4], rv[4], hcv[4];
+        const float4 c4 = *reinterpret_cast<const float4 *>(sm.hr + (tr + 1) * N + i0);  // h^(k)_t
+        const float cur[4] = {c4.x, c4.y, c4.z, c4.w};
+        float Jv[4], rv[4];
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-            const int i = i0 + u;
-            const bool v = tv && i < A.n;
+            const bool v = tv && i0 + u < A.n;
             const float f = tanh_(acc[j][u]);
-            const float cur = sm.hT[i * HS + tr + 1];
-            Jv[u] = v ? (1.f - f * f) * sm.AT[i * AS + i] : 1.f;
-            rv[u] = v ? f - cur : 0.f;
-            hcv[u] = cur;
+            Jv[u] = v ? (1.f - f * f) * dg[u] : 1.f;
+            rv[u] = v ? f - cur[u] : 0.f;
             const float ad = fabsf(rv[u]);
             res = (ad > res || isnan(ad)) ? ad : res;
         }
         *reinterpret_cast<float4 *>(sm.Js + tr * N + i0) = make_float4(Jv[0], Jv[1], Jv[2], Jv[3]);
         *reinterpret_cast<float4 *>(sm.rs + tr * N + i0) = make_float4(rv[0], rv[1], rv[2], rv[3]);
-        *reinterpret_cast<float4 *>(sm.hc + tr * N + i0) = make_float4(hcv[0], hcv[1], hcv[2], hcv[3]);
     }
     return res;
 }
@@ -483,6 +534,7 @@ __global__ void __launch_bounds__(kThreads, 2) tanh_quasi_kernel(const TanhArgs 
     LookBack<1> lb{A.agg, A.inc};
     if (tid == 0) s_fail = 0;
     quasi_stage_params<N>(A, sm);
+    QuasiPrefetch<N> pf;
     int iters = 0;
     float last_delta = 0.f;
     bool stop_all = false;
@@ -493,13 +545,29 @@ __global__ void __launch_bounds__(kThreads, 2) tanh_quasi_kernel(const TanhArgs 
         float *side_out = A.side + (size_t)((k + 1) & 1) * ntiles * C;
         float my_max = 0.f;
         TileWalk tw(nseq);
+        bool staged = false;  // pf holds this tile's data
         for (long tile = blockIdx.x; tile < ntiles; tile += gridDim.x, tw.next()) {
             const int chunk = tw.chunk;
             const int b = tw.seq;
             const int t0 = chunk * TCH;
             __syncthreads();
-            quasi_stage_tile<N>(A, sm, b, t0, k > 0, (k > 0 && chunk > 0) ? side_in + (tile - nseq) * C : nullptr);
+            if (staged)
+                pf.store(A, sm);
+            else
+                quasi_stage_tile<N>(A, sm, b, t0, k > 0, (k > 0 && chunk > 0) ? side_in + (tile - nseq) * C : nullptr);
             __syncthreads();
+            // the next tile of this iteration (its states are the previous iteration's:
+            // nothing this iteration writes) is loaded while this one computes
+            staged = tile + gridDim.x < ntiles;
+            if (staged) {
+                int nch = chunk + tw.step_ch, nsq = b + tw.step_sq;
+                if (nsq >= nseq) {
+                    nsq -= (int)nseq;
+                    ++nch;
+                }
+                const long nt = tile + gridDim.x;
+                pf.load(A, nsq, nch * TCH, k > 0, (k > 0 && nch > 0) ? side_in + (nt - nseq) * C : nullptr);
+            }
             quasi_phase_a<N>(A, sm, b, t0);
             __syncthreads();
             const bool cv = c < A.n;
@@ -546,7 +614,7 @@ __global__ void __launch_bounds__(kThreads, 2) tanh_quasi_kernel(const TanhArgs 
             for (int i = 0; i < L; ++i) {
                 const int tr = s * L + i, t = t0 + tr;
                 d = fmaf(sm.Js[tr * N + c], d, sm.rs[tr * N + c]);
-                const float hn = sm.hc[tr * N + c] + d;
+                const float hn = sm.hr[(tr + 1) * N + c] + d;
                 if (cv && t < A.T) {
                     const float ad = fabsf(d);
                     my_max = (ad > my_max || isnan(d)) ? ad : my_max;

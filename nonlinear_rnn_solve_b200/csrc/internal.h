@@ -35,6 +35,7 @@ struct Plan {
     int S = 1;                     // state components per unit
     int threads = 256;             // threads per CTA
     int halo_w = 1;                // side-buffer values per tile boundary and channel
+    int tab = 0;                   // adjoint: shared-memory gradient table variant
 };
 
 struct DbgHost {

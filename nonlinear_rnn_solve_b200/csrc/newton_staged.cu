@@ -442,22 +442,30 @@ __global__ void __launch_bounds__(NT, MINB)
                 tile_compute<Cell, Lay, IN, true>(A, smem, cell, s, c, t0, k, hp, wz, bz, Jr, rr, hc);
             else
                 tile_compute<Cell, Lay, IN, false>(A, smem, cell, s, c, t0, k, hp, wz, bz, Jr, rr, hc);
+            const long next = tile + gridDim.x;
+            auto refill = [&]() {
+                if (next < ntiles) {
+                    int nch = chunk, nsq = seq;
+                    advance(nch, nsq);
+                    issue(nch, nsq, k > 0);
+                }
+            };
+            if (!Lay::kTma) {
+                // cp.async layouts: refill as soon as every thread is done with the stage
+                __syncthreads();
+                refill();
+            }
             Aff<S> e = Aff<S>::ident();
 #pragma unroll
             for (int i = 0; i < L; ++i) e = compose(e, make_aff<S>(Jr[i], rr[i]));
             Aff<S> excl, total;
-            cta_scan<S, C, NT>(e, sm, excl, total);  // the one CTA barrier of the common path
+            cta_scan<S, C, NT>(e, sm, excl, total);  // the one CTA barrier of the TMA path
             if (s_fail) {
                 drain();
                 return;  // a bounded wait ran out; the status says so
             }
-            // past the barrier every thread is done reading the stage: refill it
-            const long next = tile + gridDim.x;
-            if (next < ntiles) {
-                int nch = chunk, nsq = seq;
-                advance(nch, nsq);
-                issue(nch, nsq, k > 0);
-            }
+            // TMA: past the barrier every thread is done reading the stage: refill it
+            if (Lay::kTma) refill();
             // the previous tile's staged results (written before the barrier) leave now
             if (fl_b >= 0) Lay::flush(A, smem + (par ^ 1) * Lay::OUT_STRIDE, fl_b, fl_ct, fl_t);
             // carry entering the tile: from the halo when its composed map is constant

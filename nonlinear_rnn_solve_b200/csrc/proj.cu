@@ -3,10 +3,10 @@
 // is computed once per forward pass; "Para-Seq" README, Main features: GRU/LSTM layers
 // with input projections).
 //
-// bf16 path: a tcgen05 GEMM.  Each CTA computes one 128 x 256 fp32 tile of xproj:
+// bf16 path: a tcgen05 GEMM.  Persistent CTAs compute 128 x 256 fp32 tiles of xproj:
 //   warp 0  (one elected thread) streams 128x64 tiles of x and 256x64 tiles of W into a
 //           4-stage shared-memory ring with TMA (128-byte swizzle, no multicast);
-//   warp 1  allocates 256 TMEM columns and (one elected thread) issues
+//   warp 1  allocates 2 x 256 TMEM columns and (one elected thread) issues
 //           tcgen05.mma.cta_group::1.kind::f16 (M = 128, N = 256, K = 16, bf16 x bf16 ->
 //           fp32 in TMEM), releasing each stage with tcgen05.commit;
 //   warps 2-5 read the accumulator with tcgen05.ld (32 lanes x 16 columns per load), add
@@ -15,6 +15,8 @@
 // status bit, frees its TMEM and returns.
 // fp32 path: a CUDA-core tiled GEMM (x and W both fp32).
 #include <cuda.h>
+
+#include <algorithm>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -76,18 +78,25 @@ __device__ __forceinline__ unsigned long long smem_desc(unsigned addr) {
 // Instruction descriptor: D fp32, A and B bf16, both K-major, N = 256, M = 128.
 constexpr unsigned IDESC = (1u << 4) | (1u << 7) | (1u << 10) | ((unsigned)(BN >> 3) << 17) | ((unsigned)(BM >> 4) << 24);
 
+// Persistent CTAs (one per SM) walk the output tiles n-fastest, so the CTAs that run
+// at the same time share rows of x in L2 (W stays resident).  The accumulator is
+// double-buffered in TMEM (2 x 256 columns): the epilogue warps drain tile i while the
+// MMA thread accumulates tile i + 1, and the TMA producer runs ahead across tiles.
 __global__ void __launch_bounds__(THREADS, 1)
     proj_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const float *__restrict__ bias, float *__restrict__ y, int M, int N, int K, int *sticky) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     // 1024-byte alignment for the swizzled tiles
     unsigned char *smem = reinterpret_cast<unsigned char *>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-    __shared__ __align__(8) unsigned long long bar_full[STAGES], bar_empty[STAGES], bar_acc;
+    __shared__ __align__(8) unsigned long long bar_full[STAGES], bar_empty[STAGES], acc_full[2], acc_empty[2];
     __shared__ unsigned tmem_base_sh;
     __shared__ volatile int abort_flag;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int m0 = blockIdx.x * BM, n0 = blockIdx.y * BN;
     const int kblocks = (K + BK - 1) / BK;
+    const int mtiles = (M + BM - 1) / BM, ntiles_n = (N + BN - 1) / BN;
+    const int ntiles = mtiles * ntiles_n;
+    // 32-byte vector stores need 32-byte aligned rows
+    const bool vec8 = (N & 7) == 0 && ((uintptr_t)y & 31) == 0;
 
     if (threadIdx.x == 0) {
         abort_flag = 0;
@@ -95,12 +104,15 @@ __global__ void __launch_bounds__(THREADS, 1)
             mbar_init(smem_u32(&bar_full[s]), 1);
             mbar_init(smem_u32(&bar_empty[s]), 1);
         }
-        mbar_init(smem_u32(&bar_acc), 1);
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(smem_u32(&acc_full[a]), 1);
+            mbar_init(smem_u32(&acc_empty[a]), 4);  // one arrival per epilogue warp
+        }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&tmem_base_sh)),
-                     "r"(TMEM_COLS)
+                     "r"(2 * TMEM_COLS)
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
@@ -110,57 +122,79 @@ __global__ void __launch_bounds__(THREADS, 1)
     const unsigned tmem = tmem_base_sh;
 
     if (warp == 0) {
-        if (lane == 0) {  // TMA producer
-            for (int kb = 0; kb < kblocks; ++kb) {
-                const int s = kb % STAGES;
-                const unsigned ph = (unsigned)(kb / STAGES) & 1u;
-                if (!mbar_wait(smem_u32(&bar_empty[s]), ph ^ 1u, &abort_flag)) { abort_flag = 1; break; }
-                unsigned char *sa = smem + s * STAGE_BYTES;
-                const unsigned fb = smem_u32(&bar_full[s]);
-                mbar_expect_tx(fb, STAGE_BYTES);
-                tma_load_2d(smem_u32(sa), &tmA, kb * BK, m0, fb);
-                tma_load_2d(smem_u32(sa + A_BYTES), &tmB, kb * BK, n0, fb);
+        if (lane == 0) {  // TMA producer, continuous over this CTA's tiles
+            int it = 0;
+            for (int tile = blockIdx.x; tile < ntiles && !abort_flag; tile += gridDim.x) {
+                const int m0 = (tile / ntiles_n) * BM, n0 = (tile % ntiles_n) * BN;
+                for (int kb = 0; kb < kblocks; ++kb, ++it) {
+                    const int s = it % STAGES;
+                    const unsigned ph = (unsigned)(it / STAGES) & 1u;
+                    if (!mbar_wait(smem_u32(&bar_empty[s]), ph ^ 1u, &abort_flag)) { abort_flag = 1; break; }
+                    unsigned char *sa = smem + s * STAGE_BYTES;
+                    const unsigned fb = smem_u32(&bar_full[s]);
+                    mbar_expect_tx(fb, STAGE_BYTES);
+                    tma_load_2d(smem_u32(sa), &tmA, kb * BK, m0, fb);
+                    tma_load_2d(smem_u32(sa + A_BYTES), &tmB, kb * BK, n0, fb);
+                }
             }
         }
     } else if (warp == 1) {
         if (lane == 0) {  // MMA issuer
-            for (int kb = 0; kb < kblocks; ++kb) {
-                const int s = kb % STAGES;
-                const unsigned ph = (unsigned)(kb / STAGES) & 1u;
-                if (!mbar_wait(smem_u32(&bar_full[s]), ph, &abort_flag)) { abort_flag = 1; break; }
+            int it = 0, ti = 0;
+            for (int tile = blockIdx.x; tile < ntiles && !abort_flag; tile += gridDim.x, ++ti) {
+                const int a = ti & 1;
+                const unsigned acc = tmem + (unsigned)(a * TMEM_COLS);
+                // the epilogue has drained this accumulator (its previous tile)
+                if (!mbar_wait(smem_u32(&acc_empty[a]), ((unsigned)(ti >> 1) & 1u) ^ 1u, &abort_flag)) {
+                    abort_flag = 1;
+                    break;
+                }
                 asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-                const unsigned a0 = smem_u32(smem + s * STAGE_BYTES), b0 = a0 + A_BYTES;
+                for (int kb = 0; kb < kblocks; ++kb, ++it) {
+                    const int s = it % STAGES;
+                    const unsigned ph = (unsigned)(it / STAGES) & 1u;
+                    if (!mbar_wait(smem_u32(&bar_full[s]), ph, &abort_flag)) { abort_flag = 1; break; }
+                    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+                    const unsigned a0 = smem_u32(smem + s * STAGE_BYTES), b0 = a0 + A_BYTES;
 #pragma unroll
-                for (int k = 0; k < BK / 16; ++k) {
-                    const unsigned long long ad = smem_desc(a0 + k * 32), bd = smem_desc(b0 + k * 32);
-                    const unsigned accum = (kb > 0 || k > 0) ? 1u : 0u;
-                    asm volatile(
-                        "{\n\t.reg .pred p;\n\t"
-                        "setp.ne.b32 p, %4, 0;\n\t"
-                        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem),
-                        "l"(ad), "l"(bd), "r"(IDESC), "r"(accum)
-                        : "memory");
+                    for (int k = 0; k < BK / 16; ++k) {
+                        const unsigned long long ad = smem_desc(a0 + k * 32), bd = smem_desc(b0 + k * 32);
+                        const unsigned accum = (kb > 0 || k > 0) ? 1u : 0u;
+                        asm volatile(
+                            "{\n\t.reg .pred p;\n\t"
+                            "setp.ne.b32 p, %4, 0;\n\t"
+                            "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(acc),
+                            "l"(ad), "l"(bd), "r"(IDESC), "r"(accum)
+                            : "memory");
+                    }
+                    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                                     smem_u32(&bar_empty[s]))
+                                 : "memory");
                 }
                 asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                                 smem_u32(&bar_empty[s]))
+                                 smem_u32(&acc_full[a]))
                              : "memory");
             }
-            asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                             smem_u32(&bar_acc))
-                         : "memory");
         }
     } else {
         // epilogue: warps 2..5 own TMEM lanes 32*(warp % 4) .. +31, i.e. tile rows
         const int q = warp & 3;
-        const int row = m0 + q * 32 + lane;
-        const bool ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bar_acc), 0u, &abort_flag));
-        if (!ok) abort_flag = 1;
-        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-        if (ok) {
+        int ti = 0;
+        for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++ti) {
+            const int a = ti & 1;
+            const int m0 = (tile / ntiles_n) * BM, n0 = (tile % ntiles_n) * BN;
+            const int row = m0 + q * 32 + lane;
+            const bool ok =
+                __all_sync(0xffffffffu, mbar_wait(smem_u32(&acc_full[a]), (unsigned)(ti >> 1) & 1u, &abort_flag));
+            if (!ok) {
+                abort_flag = 1;
+                break;
+            }
+            asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 #pragma unroll 1
             for (int c = 0; c < BN; c += 16) {
                 unsigned r[16];
-                const unsigned taddr = tmem + ((unsigned)(q * 32) << 16) + (unsigned)c;
+                const unsigned taddr = tmem + ((unsigned)(q * 32) << 16) + (unsigned)(a * TMEM_COLS + c);
                 asm volatile(
                     "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, "
                     "%13, %14, %15}, [%16];"
@@ -169,23 +203,51 @@ __global__ void __launch_bounds__(THREADS, 1)
                       "=r"(r[15])
                     : "r"(taddr));
                 asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+                if (c + 16 >= BN) {
+                    // every column of this accumulator is in registers: hand it back
+                    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+                    __syncwarp();
+                    if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&acc_empty[a])) : "memory");
+                }
                 const int col = n0 + c;
                 if (row < M) {
-                    float *yr = y + (size_t)row * N + col;
-                    if (col + 16 <= N && (N & 3) == 0) {
+                    float v[16];
 #pragma unroll
-                        for (int j = 0; j < 16; j += 4) {
-                            float4 v;
-                            v.x = __uint_as_float(r[j]) + (bias ? __ldg(bias + col + j) : 0.f);
-                            v.y = __uint_as_float(r[j + 1]) + (bias ? __ldg(bias + col + j + 1) : 0.f);
-                            v.z = __uint_as_float(r[j + 2]) + (bias ? __ldg(bias + col + j + 2) : 0.f);
-                            v.w = __uint_as_float(r[j + 3]) + (bias ? __ldg(bias + col + j + 3) : 0.f);
-                            *reinterpret_cast<float4 *>(yr + j) = v;
+                    for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(r[j]);
+                    const bool full = col + 16 <= N;
+                    if (bias) {
+                        if (full) {
+#pragma unroll
+                            for (int j = 0; j < 16; j += 4) {
+                                const float4 bv = __ldg(reinterpret_cast<const float4 *>(bias + col + j));
+                                v[j] += bv.x;
+                                v[j + 1] += bv.y;
+                                v[j + 2] += bv.z;
+                                v[j + 3] += bv.w;
+                            }
+                        } else {
+#pragma unroll
+                            for (int j = 0; j < 16; ++j)
+                                if (col + j < N) v[j] += __ldg(bias + col + j);
                         }
+                    }
+                    float *yr = y + (size_t)row * N + col;
+                    if (full && vec8) {
+                        // whole 32-byte sectors per lane
+#pragma unroll
+                        for (int j = 0; j < 16; j += 8)
+                            asm volatile("st.global.v8.f32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(yr + j),
+                                         "f"(v[j]), "f"(v[j + 1]), "f"(v[j + 2]), "f"(v[j + 3]), "f"(v[j + 4]),
+                                         "f"(v[j + 5]), "f"(v[j + 6]), "f"(v[j + 7])
+                                         : "memory");
+                    } else if (full && (N & 3) == 0) {
+#pragma unroll
+                        for (int j = 0; j < 16; j += 4)
+                            *reinterpret_cast<float4 *>(yr + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
                     } else {
 #pragma unroll
                         for (int j = 0; j < 16; ++j)
-                            if (col + j < N) yr[j] = __uint_as_float(r[j]) + (bias ? __ldg(bias + col + j) : 0.f);
+                            if (col + j < N) yr[j] = v[j];
                     }
                 }
             }
@@ -196,7 +258,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (abort_flag && threadIdx.x == 0) atomicOr(sticky, kStTimeout);
     if (warp == 1) {
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS) : "memory");
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(2 * TMEM_COLS) : "memory");
     }
 }
 
@@ -301,7 +363,11 @@ cudaError_t proj_launch(int x_dtype, const void *x, const void *W, const float *
     const int smem = gemm::STAGES * gemm::STAGE_BYTES + 1024;
     cudaError_t e = cudaFuncSetAttribute(gemm::proj_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    dim3 grid((M + gemm::BM - 1) / gemm::BM, (N + gemm::BN - 1) / gemm::BN);
+    int dev = 0, sms = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    const long tiles = (long)((M + gemm::BM - 1) / gemm::BM) * ((N + gemm::BN - 1) / gemm::BN);
+    const int grid = (int)std::min<long>(tiles, sms);  // persistent: one CTA per SM
     gemm::proj_bf16_kernel<<<grid, gemm::THREADS, smem, st>>>(ta, tb, bias, y, M, N, K, sticky);
     *launches = 1;
     return cudaGetLastError();

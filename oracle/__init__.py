@@ -175,6 +175,23 @@ def input_proj(x, W, bias=None):
     return y.reshape(*x64.shape[:-1], W64.shape[0])
 
 
+def input_proj_backward(grad_xproj, x, W):
+    """Gradients of L = <grad_xproj, x W^T + bias> (float64 library matmuls).
+
+    The projection is linear in x, W and bias, so its reverse pass is three plain
+    contractions ("Para-Seq" README, Main features: trainable GRU/LSTM layers whose
+    input projection precedes the parallel solve):
+      grad_x    [M, K] = grad_xproj [M, N] @ W [N, K]
+      grad_W    [N, K] = grad_xproj^T @ x [M, K]
+      grad_bias [N]    = column sums of grad_xproj
+    Leading dimensions of grad_xproj and x are flattened to M.
+    """
+    g64, x64, W64 = _f64(grad_xproj), _f64(x), _f64(W)
+    g2 = g64.reshape(-1, g64.shape[-1])
+    x2 = x64.reshape(-1, x64.shape[-1])
+    return g2 @ W64, g2.T @ x2, g2.sum(axis=0)
+
+
 def model_from_inputs(cell, inputs, quasi=False):
     """Build a Model from the arrays of ``workloads.generate`` (projection in fp64)."""
     x = inputs["x"]

@@ -378,6 +378,48 @@ def test_input_proj_matches_brute_force():
                 assert abs(y[b, t, n] - ref) < 1e-12
 
 
+def test_input_proj_backward_matches_brute_force_sums():
+    rng = np.random.default_rng(92)
+    M, K, N = 5, 4, 3
+    g = rng.standard_normal((M, N))
+    x = rng.standard_normal((M, K))
+    W = rng.standard_normal((N, K))
+    gx, gW, gb = oracle.input_proj_backward(g, x, W)
+    for m in range(M):
+        for k in range(K):
+            assert abs(gx[m, k] - sum(g[m, n] * W[n, k] for n in range(N))) < 1e-12
+    for n in range(N):
+        for k in range(K):
+            assert abs(gW[n, k] - sum(g[m, n] * x[m, k] for m in range(M))) < 1e-12
+        assert abs(gb[n] - sum(g[m, n] for m in range(M))) < 1e-12
+
+
+def test_input_proj_backward_matches_autograd_of_library_linear():
+    """The gradients of torch.nn.functional.linear (a library layer, autograd)."""
+    rng = np.random.default_rng(93)
+    x = torch.tensor(rng.standard_normal((2, 3, 6)), dtype=f64, requires_grad=True)
+    W = torch.tensor(rng.standard_normal((4, 6)), dtype=f64, requires_grad=True)
+    bias = torch.tensor(rng.standard_normal(4), dtype=f64, requires_grad=True)
+    g = rng.standard_normal((2, 3, 4))
+    (torch.nn.functional.linear(x, W, bias) * torch.tensor(g)).sum().backward()
+    gx, gW, gb = oracle.input_proj_backward(g, x.detach().numpy(), W.detach().numpy())
+    assert np.abs(gx.reshape(2, 3, 6) - x.grad.numpy()).max() < 1e-12
+    assert np.abs(gW - W.grad.numpy()).max() < 1e-12
+    assert np.abs(gb - bias.grad.numpy()).max() < 1e-12
+
+
+def test_input_proj_backward_adjoint_identity():
+    """<g, x W^T> = <grad_W, W> = <grad_x, x> (the projection is bilinear)."""
+    rng = np.random.default_rng(94)
+    g = rng.standard_normal((7, 5))
+    x = rng.standard_normal((7, 3))
+    W = rng.standard_normal((5, 3))
+    gx, gW, _ = oracle.input_proj_backward(g, x, W)
+    lhs = float((g * oracle.input_proj(x, W)).sum())
+    assert abs(lhs - float((gW * W).sum())) < 1e-10
+    assert abs(lhs - float((gx * x).sum())) < 1e-10
+
+
 def test_model_from_inputs_layout_gate_major():
     """xproj[b, t, g, u] uses W row g*H + u (gate-major), as the layout promises."""
     w = wl.WORKLOADS["gru_b1_t1024_in4_h8"].resized(T=3)

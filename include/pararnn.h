@@ -107,6 +107,25 @@ int pararnn_set_stream(pararnn_ctx *ctx, void *cuda_stream);
 int pararnn_input_proj(pararnn_ctx *ctx, const void *x, int x_dtype, const void *W,
                        const float *bias, float *xproj, int M, int K, int N);
 
+/* Reverse pass of the input projection, for L = <grad_xproj, x W^T + bias>:
+ *   grad_x [M, K] = grad_xproj [M, N] W,   grad_W [N, K] = grad_xproj^T x,
+ *   grad_bias [N] = column sums of grad_xproj
+ * (the projection is linear, so these are its exact gradients; with
+ * pararnn_adjoint_backward they complete the gradient of a trainable layer:
+ * "Para-Seq" README, Main features).  grad_xproj fp32 [M, N].  x and W as for
+ * pararnn_input_proj: both bf16 (x_dtype PARARNN_BF16: grad_xproj is rounded to bf16,
+ * nearest-even, for the tensor-core products, fp32 accumulation; the bias gradient
+ * sums the fp32 values) or both fp32 (CUDA cores).  Each of grad_x, grad_W, grad_bias
+ * may be NULL (not computed); outputs are overwritten, not accumulated.
+ * Shapes: M, K, N >= 1; bf16 needs M, K, N multiples of 8 (16-byte rows of every
+ * operand, including the transposed copies); M * N and M * K <= 2^40.  All pointers
+ * 16-byte aligned.  The context keeps a scratch buffer of the bf16 copies
+ * (4 M N + 2 M K + 2 N K bytes) for later calls.
+ * Returns EINVAL, EALIGN, ENOMEM or ECUDA. */
+int pararnn_input_proj_backward(pararnn_ctx *ctx, const float *grad_xproj, const void *x, int x_dtype,
+                                const void *W, float *grad_x, float *grad_W, float *grad_bias, int M, int K,
+                                int N);
+
 /* Newton (DEER) / quasi-Newton forward solve of the whole sequence
  * ("Parallelizing non-linear sequential models over the sequence length", Approach;
  * quasi: "Towards Scalable and Stable Parallelization of Nonlinear RNNs", Abstract).

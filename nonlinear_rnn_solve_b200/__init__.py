@@ -42,7 +42,7 @@ EXPORTED = [
     "pararnn_create", "pararnn_destroy", "pararnn_set_stream", "pararnn_input_proj",
     "pararnn_newton_forward", "pararnn_linear_scan", "pararnn_adjoint_backward",
     "pararnn_get_status", "pararnn_strerror", "pararnn_debug_set", "pararnn_last_launch_count",
-    "pararnn_linear_scan_noalloc",
+    "pararnn_linear_scan_noalloc", "pararnn_input_proj_backward",
 ]
 
 
@@ -86,6 +86,7 @@ def lib() -> ctypes.CDLL:
         L.pararnn_debug_set.argtypes = [vp, i, ctypes.c_longlong]
         L.pararnn_last_launch_count.argtypes = [vp]
         L.pararnn_linear_scan_noalloc.argtypes = [i, vp, vp, vp, vp, i, i, i, i, vp, vp]
+        L.pararnn_input_proj_backward.argtypes = [vp, vp, vp, i, vp, vp, vp, vp, i, i, i]
         for name in EXPORTED:
             if getattr(L, name).restype is None and name != "pararnn_strerror":
                 getattr(L, name).restype = i
@@ -155,6 +156,21 @@ def pararnn_input_proj(ctx, x, W, bias, xproj) -> None:
     N = W.shape[0]
     _check(lib().pararnn_input_proj(ctx, _p(x), dt, _p(W), _p(bias, torch.float32),
                                     _p(xproj, torch.float32), M, K, N), "pararnn_input_proj")
+
+
+def pararnn_input_proj_backward(ctx, grad_xproj, x, W, grad_x, grad_W, grad_bias) -> None:
+    """grad_x = grad_xproj @ W, grad_W = grad_xproj^T @ x, grad_bias = column sums
+    (x, W both bf16 or both fp32; any output may be None)."""
+    if x.dtype != W.dtype or x.dtype not in (torch.bfloat16, torch.float32):
+        raise TypeError("x and W must both be bf16 or both fp32")
+    dt = PARARNN_BF16 if x.dtype == torch.bfloat16 else PARARNN_F32
+    K = x.shape[-1]
+    M = x.numel() // K
+    N = W.shape[0]
+    f32 = torch.float32
+    _check(lib().pararnn_input_proj_backward(ctx, _p(grad_xproj, f32), _p(x), dt, _p(W), _p(grad_x, f32),
+                                             _p(grad_W, f32), _p(grad_bias, f32), M, K, N),
+           "pararnn_input_proj_backward")
 
 
 def pararnn_newton_forward(ctx, xproj, params, h0, h_out, max_iters, tol, iters_out,

@@ -17,6 +17,8 @@ struct pararnn_ctx {
     int num_sms = 0;
     void *ws = nullptr;        // workspace: control block, flags, aggregates, side buffers
     size_t ws_bytes = 0;
+    void *scratch = nullptr;   // plain scratch of the projection backward (bf16 copies)
+    size_t scratch_bytes = 0;
     int *sticky = nullptr;     // sticky device status word
     prn::DbgHost dbg;
     int last_launches = 0;
@@ -126,6 +128,7 @@ int pararnn_destroy(pararnn_ctx *ctx) {
     DeviceGuard g(ctx->device);
     cudaStreamSynchronize(ctx->stream);
     if (ctx->ws) cudaFree(ctx->ws);
+    if (ctx->scratch) cudaFree(ctx->scratch);
     if (ctx->sticky) cudaFree(ctx->sticky);
     delete ctx;
     return PARARNN_OK;
@@ -255,6 +258,40 @@ int pararnn_input_proj(pararnn_ctx *ctx, const void *x, int x_dtype, const void 
     ctx->last_launches = 0;
     int launches = 0;
     int rc = cuda_rc(prn::proj_launch(x_dtype, x, W, bias, xproj, M, K, N, ctx->num_sms, ctx->stream, &launches, ctx->sticky));
+    if (rc == PARARNN_OK) ctx->last_launches = launches;
+    return rc;
+}
+
+int pararnn_input_proj_backward(pararnn_ctx *ctx, const float *grad_xproj, const void *x, int x_dtype, const void *W,
+                                float *grad_x, float *grad_W, float *grad_bias, int M, int K, int N) {
+    if (!ctx || !grad_xproj || !x || !W || M < 1 || K < 1 || N < 1) return PARARNN_EINVAL;
+    if (x_dtype != PARARNN_F32 && x_dtype != PARARNN_BF16) return PARARNN_EINVAL;
+    if (misaligned(grad_xproj) || misaligned(x) || misaligned(W) || misaligned(grad_x) || misaligned(grad_W) ||
+        misaligned(grad_bias))
+        return PARARNN_EALIGN;
+    int chk = prn::proj_bwd_check(x_dtype, M, K, N);
+    if (chk) return chk;
+    DeviceGuard g(ctx->device);
+    if (!g.ok) return PARARNN_ECUDA;
+    ctx->last_launches = 0;
+    // a buffer of its own: the look-back workspace must only ever hold epoch-tagged words
+    const size_t need = prn::proj_bwd_scratch_bytes(x_dtype, M, K, N);
+    if (ctx->scratch_bytes < need) {
+        if (ctx->scratch) {
+            if (cudaStreamSynchronize(ctx->stream) != cudaSuccess) return PARARNN_ECUDA;
+            cudaFree(ctx->scratch);
+            ctx->scratch = nullptr;
+            ctx->scratch_bytes = 0;
+        }
+        if (cudaMalloc(&ctx->scratch, need) != cudaSuccess) {
+            cudaGetLastError();
+            return PARARNN_ENOMEM;
+        }
+        ctx->scratch_bytes = need;
+    }
+    int launches = 0;
+    int rc = cuda_rc(prn::proj_bwd_launch(x_dtype, grad_xproj, x, W, grad_x, grad_W, grad_bias, M, K, N, ctx->scratch,
+                                          ctx->num_sms, ctx->stream, &launches, ctx->sticky));
     if (rc == PARARNN_OK) ctx->last_launches = launches;
     return rc;
 }

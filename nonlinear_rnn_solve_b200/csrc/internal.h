@@ -107,6 +107,13 @@ int proj_check(int x_dtype, int M, int K, int N);
 cudaError_t proj_launch(int x_dtype, const void *x, const void *W, const float *bias, float *y, int M,
                         int K, int N, int num_sms, cudaStream_t st, int *launches, int *sticky);
 
+// ---- input projection backward ------------------------------------------------------
+int proj_bwd_check(int x_dtype, int M, int K, int N);
+size_t proj_bwd_scratch_bytes(int x_dtype, int M, int K, int N);
+cudaError_t proj_bwd_launch(int x_dtype, const float *gx, const void *x, const void *W, float *grad_x, float *grad_W,
+                            float *grad_bias, int M, int K, int N, void *scratch, int num_sms, cudaStream_t st,
+                            int *launches, int *sticky);
+
 // Helpers.
 int occupancy_grid(const void *kernel, int threads, size_t smem, int num_sms, long ntiles);
 

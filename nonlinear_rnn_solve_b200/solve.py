@@ -46,6 +46,19 @@ def input_proj(ctx, x, W, bias=None):
     return out
 
 
+def input_proj_backward(ctx, grad_xproj, x, W, need_x=True, need_W=True, need_bias=True):
+    """Gradients of the projection: (grad_x [..., K], grad_W [N, K], grad_bias [N]);
+    entries not requested are None."""
+    from . import pararnn_input_proj_backward
+    dev = x.device
+    K, N = x.shape[-1], W.shape[0]
+    gx = torch.empty(*x.shape[:-1], K, device=dev, dtype=torch.float32) if need_x else None
+    gW = torch.empty(N, K, device=dev, dtype=torch.float32) if need_W else None
+    gb = torch.empty(N, device=dev, dtype=torch.float32) if need_bias else None
+    pararnn_input_proj_backward(ctx, grad_xproj, x, W, gx, gW, gb)
+    return gx, gW, gb
+
+
 def linear_scan(ctx, kind, J, b, h0=None, reverse=False):
     from . import PARARNN_SCAN_BLOCK2, PARARNN_SCAN_DENSE, PARARNN_SCAN_DIAG
     k = {"diag": PARARNN_SCAN_DIAG, "block2": PARARNN_SCAN_BLOCK2, "dense": PARARNN_SCAN_DENSE}[kind]

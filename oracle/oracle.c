@@ -43,7 +43,9 @@ enum { ORC_SCAN_DIAG = 0, ORC_SCAN_BLOCK2 = 1, ORC_SCAN_DENSE = 2 };
 
 typedef struct {
     int cell;            /* ORC_GRU / ORC_LSTM / ORC_TANH */
-    int quasi;           /* tanh only: keep only the diagonal of the Jacobian [ELK] */
+    int quasi;           /* keep only the diagonal of the Jacobian in the Newton iteration
+                          * [ELK]: tanh (n x n -> diagonal) and LSTM (each 2x2 block -> its
+                          * diagonal, the ParaLSTM diagonal scan backend [SEQ]) */
     long B, T, H;        /* H = units (GRU, LSTM) or state size n (tanh) */
     const double *xproj; /* [B][T][G][H]: W x_t + bias per gate (tanh: U x_t + b) */
     const double *a;     /* [3][H] recurrent diagonals: GRU (z,r,c), LSTM (f,g,o) */
@@ -312,6 +314,10 @@ int orc_newton(const orc_model *m, const double *h0, int max_iters, double tol, 
                 double dloc = 0.0;
                 for (long t = 0; t < T; ++t) {
                     unit_eval(m, b, t, u, pk, f, J, NULL, NULL);
+                    if (m->quasi && S == 2) { /* diagonal of the 2x2 block: c and h decouple */
+                        J[1] = 0.0;
+                        J[2] = 0.0;
+                    }
                     long idx = ((b * T + t) * H + u) * S;
                     for (long i = 0; i < S; ++i) {
                         double s = f[i];

@@ -201,7 +201,7 @@ def test_reverse_scan_is_transpose_of_forward(kind):
 
 # ------------------------------------------------------------------------- Newton
 @pytest.mark.parametrize("cell,quasi", [("gru", False), ("lstm", False), ("tanh", False),
-                                        ("tanh", True)])
+                                        ("tanh", True), ("lstm", True)])
 def test_newton_iterates_match_stacked_system_solve(cell, quasi):
     H = 3
     m, xp, prm, h0 = _rand_model(cell, B=2, T=7, H=H, seed=21, quasi=quasi)
@@ -215,7 +215,7 @@ def test_newton_iterates_match_stacked_system_solve(cell, quasi):
 
 
 @pytest.mark.parametrize("cell,quasi", [("gru", False), ("lstm", False), ("tanh", False),
-                                        ("tanh", True)])
+                                        ("tanh", True), ("lstm", True)])
 def test_newton_exact_prefix_and_fixed_point(cell, quasi):
     """After k updates h_1..h_k equal the rollout; the fixed point is the rollout."""
     T = 14
@@ -276,6 +276,17 @@ def test_quasi_needs_at_least_as_many_iterations_as_deer():
     _, i_full, _ = oracle.model_from_inputs("tanh", inp).newton(max_iters=512, tol=1e-5)
     _, i_quasi, _ = oracle.model_from_inputs("tanh", inp, quasi=True).newton(max_iters=512, tol=1e-5)
     assert i_quasi >= i_full
+
+
+def test_quasi_lstm_needs_at_least_as_many_iterations_as_block_newton():
+    """The diagonal (quasi) backend drops the c-h coupling of each 2x2 block: same
+    fixed point, no faster convergence."""
+    w = wl.WORKLOADS["lstm_b4_t8192_h1024_bf16"].resized(B=2, T=256, H=16, inp=16, bf16=False)
+    inp = wl.generate(w)
+    h_b, i_b, _ = oracle.model_from_inputs("lstm", inp).newton(max_iters=256, tol=1e-9)
+    h_q, i_q, _ = oracle.model_from_inputs("lstm", inp, quasi=True).newton(max_iters=256, tol=1e-9)
+    assert i_q >= i_b
+    np.testing.assert_allclose(h_q, h_b, atol=1e-8)
 
 
 def test_newton_zero_iterations_returns_initial_guess():

@@ -62,7 +62,11 @@ typedef enum {
     PARARNN_GRU_DIAG = 0,        /* diagonal ParaGRU, diagonal Jacobian */
     PARARNN_LSTM_CIFG_PEEP = 1,  /* CIFG + peephole ParaLSTM, 2x2 Jacobian per unit */
     PARARNN_RNN_TANH_DENSE = 2,  /* vanilla tanh RNN, full n x n Jacobian (DEER) */
-    PARARNN_RNN_TANH_QUASI = 3   /* vanilla tanh RNN, diagonal of the Jacobian (quasi-DEER) */
+    PARARNN_RNN_TANH_QUASI = 3,  /* vanilla tanh RNN, diagonal of the Jacobian (quasi-DEER) */
+    PARARNN_LSTM_CIFG_PEEP_QUASI = 4 /* ParaLSTM with the diagonal scan backend: each 2x2 block
+                                        replaced by its diagonal in the Newton iteration ("Para-Seq"
+                                        README, Main features: structured block and diagonal scan
+                                        backends); same fixed point, same adjoint */
 } pararnn_cell;
 
 typedef enum { PARARNN_SCAN_DIAG = 0, PARARNN_SCAN_BLOCK2 = 1, PARARNN_SCAN_DENSE = 2 } pararnn_scan_kind;

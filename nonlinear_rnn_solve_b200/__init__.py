@@ -30,6 +30,7 @@ PARARNN_GRU_DIAG = 0
 PARARNN_LSTM_CIFG_PEEP = 1
 PARARNN_RNN_TANH_DENSE = 2
 PARARNN_RNN_TANH_QUASI = 3
+PARARNN_LSTM_CIFG_PEEP_QUASI = 4
 
 PARARNN_SCAN_DIAG = 0
 PARARNN_SCAN_BLOCK2 = 1

@@ -156,10 +156,11 @@ int pararnn_newton_forward(pararnn_ctx *ctx, const float *xproj, const pararnn_p
     prn::Plan plan;
     prn::Work w;
     int rc;
-    if (p->cell == PARARNN_GRU_DIAG || p->cell == PARARNN_LSTM_CIFG_PEEP) {
-        const int lstm = p->cell == PARARNN_LSTM_CIFG_PEEP;
+    if (p->cell == PARARNN_GRU_DIAG || p->cell == PARARNN_LSTM_CIFG_PEEP || p->cell == PARARNN_LSTM_CIFG_PEEP_QUASI) {
+        const int lstm = p->cell != PARARNN_GRU_DIAG;
+        const int quasi = p->cell == PARARNN_LSTM_CIFG_PEEP_QUASI;
         if (!p->a || (lstm && !p->peep)) return PARARNN_EINVAL;
-        prn::NewtonDiagReq r{lstm, p->B, p->T, p->H, p->in, xproj, p->x, p->W, p->bias, p->a, p->peep, h0, h_out,
+        prn::NewtonDiagReq r{lstm, quasi, p->B, p->T, p->H, p->in, xproj, p->x, p->W, p->bias, p->a, p->peep, h0, h_out,
                              max_iters, tol, iters_out, final_delta_out, residual_out};
         if (prn::newton_diag_plan(r, ctx->num_sms, &plan)) return PARARNN_ECUDA;
         if ((rc = prepare(ctx, plan, &w))) return rc;
@@ -224,8 +225,11 @@ int pararnn_adjoint_backward(pararnn_ctx *ctx, const float *xproj, const pararnn
                              float *grad_h0) {
     if (!ctx || !p || !xproj || !h || !grad_h || !grad_xproj || !grad_params) return PARARNN_EINVAL;
     if (p->B < 1 || p->T < 1 || p->H < 1) return PARARNN_EINVAL;
-    if (p->cell != PARARNN_GRU_DIAG && p->cell != PARARNN_LSTM_CIFG_PEEP) return PARARNN_EUNSUPPORTED;
-    const int lstm = p->cell == PARARNN_LSTM_CIFG_PEEP;
+    // the quasi backend changes the iteration only: the adjoint at the solution is the
+    // exact-Jacobian one for both LSTM cells
+    if (p->cell != PARARNN_GRU_DIAG && p->cell != PARARNN_LSTM_CIFG_PEEP && p->cell != PARARNN_LSTM_CIFG_PEEP_QUASI)
+        return PARARNN_EUNSUPPORTED;
+    const int lstm = p->cell != PARARNN_GRU_DIAG;
     if (!p->a || (lstm && !p->peep)) return PARARNN_EINVAL;
     if (misaligned(xproj) || misaligned(h) || misaligned(grad_h) || misaligned(grad_xproj) || misaligned(h0) ||
         misaligned(grad_h0))

@@ -49,6 +49,7 @@ struct DbgHost {
 // ---- Newton forward, diagonal / 2x2-block cells (GRU, LSTM) -----------------------
 struct NewtonDiagReq {
     int cell;  // 0 GRU, 1 LSTM
+    int quasi; // LSTM: keep only the diagonal of each 2x2 Jacobian block
     int B, T, H, in;
     const float *xproj, *x, *W, *bias, *a, *peep, *h0;
     float *h;

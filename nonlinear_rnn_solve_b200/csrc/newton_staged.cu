@@ -207,6 +207,10 @@ __device__ __forceinline__ void tile_compute(const NewtonDiagArgs &A, float *sme
                 cell.eval_pre(p, hp, f, J);  // p was formed with the prescaled weights
             else
                 cell.eval(p, hp, f, J);
+            if (S == 2 && A.quasi) {  // diagonal scan backend: c and h decouple
+                J[1 % (S * S)] = 0.f;
+                J[2 % (S * S)] = 0.f;
+            }
 #pragma unroll
             for (int q = 0; q < S; ++q) {
                 rr[i][q] = v ? f[q] - cur[q] : 0.f;

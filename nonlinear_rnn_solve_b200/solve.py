@@ -8,15 +8,16 @@ from __future__ import annotations
 import torch
 
 from . import (PARARNN_GRU_DIAG, PARARNN_LSTM_CIFG_PEEP, PARARNN_RNN_TANH_DENSE,
-               PARARNN_RNN_TANH_QUASI, make_params, pararnn_adjoint_backward,
+               PARARNN_RNN_TANH_QUASI, PARARNN_LSTM_CIFG_PEEP_QUASI, make_params, pararnn_adjoint_backward,
                pararnn_input_proj, pararnn_linear_scan, pararnn_newton_forward)
 
 CELLS = {"gru": PARARNN_GRU_DIAG, "lstm": PARARNN_LSTM_CIFG_PEEP,
-         "tanh": PARARNN_RNN_TANH_DENSE, "tanh_quasi": PARARNN_RNN_TANH_QUASI}
+         "tanh": PARARNN_RNN_TANH_DENSE, "tanh_quasi": PARARNN_RNN_TANH_QUASI,
+         "lstm_quasi": PARARNN_LSTM_CIFG_PEEP_QUASI}
 
 
 def state_shape(cell, B, T, H):
-    return (B, T, H, 2) if cell == "lstm" else (B, T, H)
+    return (B, T, H, 2) if cell in ("lstm", "lstm_quasi") else (B, T, H)
 
 
 def newton_forward(ctx, cell, B, T, H, *, xproj=None, x=None, W=None, bias=None, a=None,
@@ -73,7 +74,8 @@ def adjoint_backward(ctx, cell, B, T, H, *, xproj, a, peep=None, h0=None, h, gra
     dev = xproj.device
     prm = make_params(CELLS[cell], B, T, H, 0, a=a, peep=peep)
     gx = torch.empty(B, T, 3, H, device=dev, dtype=torch.float32)
-    gp = torch.empty(5 if cell == "lstm" else 3, H, device=dev, dtype=torch.float32)
-    gh0 = torch.empty((B, H, 2) if cell == "lstm" else (B, H), device=dev, dtype=torch.float32)
+    lstm = cell in ("lstm", "lstm_quasi")
+    gp = torch.empty(5 if lstm else 3, H, device=dev, dtype=torch.float32)
+    gh0 = torch.empty((B, H, 2) if lstm else (B, H), device=dev, dtype=torch.float32)
     pararnn_adjoint_backward(ctx, xproj, prm, h0, h, grad_h, gx, gp, gh0)
     return gx, gp, gh0

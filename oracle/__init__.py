@@ -44,7 +44,7 @@ class _Model(ctypes.Structure):
     _fields_ = [("cell", ctypes.c_int), ("quasi", ctypes.c_int),
                 ("B", ctypes.c_long), ("T", ctypes.c_long), ("H", ctypes.c_long),
                 ("xproj", ctypes.c_void_p), ("a", ctypes.c_void_p),
-                ("peep", ctypes.c_void_p), ("A", ctypes.c_void_p)]
+                ("peep", ctypes.c_void_p), ("A", ctypes.c_void_p), ("solver", ctypes.c_int)]
 
 
 _lib = None
@@ -83,7 +83,9 @@ class Model:
     xproj: [B, T, G, H] (G = 3 GRU/LSTM, 1 tanh), a: [3, H], peep: [2, H], A: [n, n].
     """
 
-    def __init__(self, cell, xproj, a=None, peep=None, A=None, quasi=False):
+    SOLVERS = {"newton": 0, "jacobi": 1, "picard": 2}
+
+    def __init__(self, cell, xproj, a=None, peep=None, A=None, quasi=False, solver="newton"):
         self.cell = cell
         self.xproj = _f64(xproj)
         B, T, G, H = self.xproj.shape
@@ -92,8 +94,9 @@ class Model:
         self.a, self.peep, self.A = _f64(a), _f64(peep), _f64(A)
         self.quasi = bool(quasi)
         self.S = 2 if cell == "lstm" else 1
+        self.solver = solver
         self._m = _Model(CELL_IDS[cell], int(self.quasi), B, T, H, _ptr(self.xproj),
-                         _ptr(self.a), _ptr(self.peep), _ptr(self.A))
+                         _ptr(self.a), _ptr(self.peep), _ptr(self.A), self.SOLVERS[solver])
 
     @property
     def state_shape(self):
@@ -192,7 +195,7 @@ def input_proj_backward(grad_xproj, x, W):
     return g2 @ W64, g2.T @ x2, g2.sum(axis=0)
 
 
-def model_from_inputs(cell, inputs, quasi=False):
+def model_from_inputs(cell, inputs, quasi=False, solver="newton"):
     """Build a Model from the arrays of ``workloads.generate`` (projection in fp64)."""
     x = inputs["x"]
     B, T, _ = x.shape
@@ -201,7 +204,7 @@ def model_from_inputs(cell, inputs, quasi=False):
     H = xp.shape[-1] // G
     xp = xp.reshape(B, T, G, H)
     return Model(cell, xp, a=inputs.get("a"), peep=inputs.get("peep"), A=inputs.get("A"),
-                 quasi=quasi)
+                 quasi=quasi, solver=solver)
 
 
 def linear_scan(kind, J, b, h0=None, reverse=False):

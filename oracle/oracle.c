@@ -51,7 +51,23 @@ typedef struct {
     const double *a;     /* [3][H] recurrent diagonals: GRU (z,r,c), LSTM (f,g,o) */
     const double *peep;  /* [2][H] LSTM peepholes (w_f, w_o) */
     const double *A;     /* [n][n] tanh recurrent matrix */
+    int solver;          /* linearisation used by orc_newton: ORC_NEWTON (the cell's
+                          * Jacobian, or its diagonal with quasi), ORC_JACOBI (J = 0),
+                          * ORC_PICARD (J = I) ["Para-Seq" README, Main features] */
 } orc_model;
+
+enum { ORC_NEWTON = 0, ORC_JACOBI = 1, ORC_PICARD = 2 };
+
+/* The fixed-point schemes share the Newton loop and differ only in the matrix the step
+ * map is linearised with: Jacobi keeps none of it (every step is re-evaluated from
+ * the previous iterate), Picard the identity (the update accumulates the increments
+ * f(h^(k)_{t-1}) - h^(k)_{t-1} along t). */
+static void solver_jacobian(const orc_model *m, long D, double *J)
+{
+    if (m->solver == ORC_NEWTON) return;
+    for (long i = 0; i < D; ++i)
+        for (long j = 0; j < D; ++j) J[i * D + j] = (m->solver == ORC_PICARD && i == j) ? 1.0 : 0.0;
+}
 
 void orc_set_threads(int n)
 {
@@ -281,6 +297,7 @@ int orc_newton(const orc_model *m, const double *h0, int max_iters, double tol, 
                 double dloc = 0.0;
                 for (long t = 0; t < T; ++t) {
                     tanh_step(m, m->xproj + (b * T + t) * n, pk, f, J);
+                    solver_jacobian(m, n, J);
                     for (long i = 0; i < n; ++i) { /* b_t = f_t - J_t h^(k)_{t-1} */
                         double s = f[i];
                         for (long j = 0; j < n; ++j) s -= J[i * n + j] * pk[j];
@@ -318,6 +335,7 @@ int orc_newton(const orc_model *m, const double *h0, int max_iters, double tol, 
                         J[1] = 0.0;
                         J[2] = 0.0;
                     }
+                    solver_jacobian(m, S, J);
                     long idx = ((b * T + t) * H + u) * S;
                     for (long i = 0; i < S; ++i) {
                         double s = f[i];

@@ -289,6 +289,46 @@ def test_quasi_lstm_needs_at_least_as_many_iterations_as_block_newton():
     np.testing.assert_allclose(h_q, h_b, atol=1e-8)
 
 
+def _fixed_point_sweeps(lib, xp, h0, iters, solver):
+    """Jacobi: h^(k+1)_t = f(h^(k)_{t-1}); Picard: h^(k+1)_t = h^(k+1)_{t-1} +
+    f(h^(k)_{t-1}) - h^(k)_{t-1}; both from h^(0) = 0, with the library cell."""
+    xpt, h0t = torch.tensor(xp), torch.tensor(h0)
+    B, T = xp.shape[:2]
+    hs = torch.zeros((B, T) + tuple(h0t.shape[1:]), dtype=f64)
+    for _ in range(iters):
+        prev = torch.cat([h0t[:, None], hs[:, :-1]], 1)
+        f = torch.stack([lib.step(xpt[:, t], prev[:, t]) for t in range(T)], 1)
+        if solver == "jacobi":
+            hs = f
+        else:
+            inc = f - prev
+            new, acc = [], h0t
+            for t in range(T):
+                acc = acc + inc[:, t]
+                new.append(acc)
+            hs = torch.stack(new, 1)
+    return hs.numpy()
+
+
+@pytest.mark.parametrize("cell", CELLS)
+@pytest.mark.parametrize("solver", ["jacobi", "picard"])
+def test_fixed_point_sweeps_match_their_definition(cell, solver):
+    """The Jacobi (J = 0) and Picard (J = I) linearisations in the Newton loop equal the
+    sweeps written out with the library cell, and keep the exact-prefix property."""
+    H, T = 3, 9
+    m, xp, prm, h0 = _rand_model(cell, B=2, T=T, H=H, seed=61)
+    m = oracle.Model(cell, xp, solver=solver, **prm)
+    lib = _lib(cell, H, prm)
+    R = m.rollout(h0)
+    for k in (1, 2, 5):
+        h, iters, _ = m.newton(h0, max_iters=k, tol=0.0)
+        assert iters == k
+        np.testing.assert_allclose(h, _fixed_point_sweeps(lib, xp, h0, k, solver), atol=1e-12)
+        np.testing.assert_allclose(h[:, :k], R[:, :k], atol=1e-12)
+    h, iters, _ = m.newton(h0, max_iters=T + 1, tol=1e-13)
+    np.testing.assert_allclose(h, R, atol=1e-12)
+
+
 def test_newton_zero_iterations_returns_initial_guess():
     m, xp, prm, h0 = _rand_model("gru", B=1, T=5, H=2, seed=3)
     h, iters, d = m.newton(h0, max_iters=0, tol=1e-6)

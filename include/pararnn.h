@@ -89,7 +89,17 @@ typedef struct {
     const float *x;        /* [B, T, in] fp32 (fused projection) */
     const float *W;        /* [G*H, in] fp32 (fused projection) */
     const float *bias;     /* [G*H] fp32 or NULL (fused projection) */
+    int solver;            /* pararnn_solver (0 = Newton) */
 } pararnn_params;
+
+/* Fixed-point scheme of pararnn_newton_forward ("Para-Seq" README, Main features:
+ * sequential, Jacobi, Picard, DEER and quasi-DEER modes).  All share the loop
+ * "linearise at h^(k), solve h^(k+1)_t = J_t h^(k+1)_{t-1} + f_t - J_t h^(k)_{t-1} by
+ * scan" and differ in J_t: the cell's Jacobian (NEWTON; its diagonal for the *_QUASI
+ * cells), zero (JACOBI: h^(k+1)_t = f(h^(k)_{t-1}), every step in parallel), or the
+ * identity (PICARD: the increments f(h^(k)_{t-1}) - h^(k)_{t-1} are summed along t).
+ * Every scheme reaches the rollout; after k iterations the first k states are exact. */
+typedef enum { PARARNN_SOLVER_NEWTON = 0, PARARNN_SOLVER_JACOBI = 1, PARARNN_SOLVER_PICARD = 2 } pararnn_solver;
 
 /* Create a context on `device` that enqueues on `cuda_stream` (a cudaStream_t, or
  * NULL for the legacy default stream).  *ctx is NULL on failure. */

@@ -31,6 +31,9 @@ PARARNN_LSTM_CIFG_PEEP = 1
 PARARNN_RNN_TANH_DENSE = 2
 PARARNN_RNN_TANH_QUASI = 3
 PARARNN_LSTM_CIFG_PEEP_QUASI = 4
+PARARNN_SOLVER_NEWTON = 0
+PARARNN_SOLVER_JACOBI = 1
+PARARNN_SOLVER_PICARD = 2
 
 PARARNN_SCAN_DIAG = 0
 PARARNN_SCAN_BLOCK2 = 1
@@ -57,7 +60,8 @@ class pararnn_params(ctypes.Structure):
     _fields_ = [("cell", ctypes.c_int), ("B", ctypes.c_int), ("T", ctypes.c_int),
                 ("H", ctypes.c_int), ("in_", ctypes.c_int),
                 ("a", ctypes.c_void_p), ("peep", ctypes.c_void_p), ("A", ctypes.c_void_p),
-                ("x", ctypes.c_void_p), ("W", ctypes.c_void_p), ("bias", ctypes.c_void_p)]
+                ("x", ctypes.c_void_p), ("W", ctypes.c_void_p), ("bias", ctypes.c_void_p),
+                ("solver", ctypes.c_int)]
 
 
 _lib = None
@@ -141,10 +145,10 @@ def pararnn_set_stream(ctx, stream=None) -> None:
     _check(lib().pararnn_set_stream(ctx, _stream_handle(stream)), "pararnn_set_stream")
 
 
-def make_params(cell, B, T, H, inp=0, a=None, peep=None, A=None, x=None, W=None, bias=None):
+def make_params(cell, B, T, H, inp=0, a=None, peep=None, A=None, x=None, W=None, bias=None, solver=0):
     f32 = torch.float32
     return pararnn_params(int(cell), int(B), int(T), int(H), int(inp), _p(a, f32), _p(peep, f32),
-                          _p(A, f32), _p(x, f32), _p(W, f32), _p(bias, f32))
+                          _p(A, f32), _p(x, f32), _p(W, f32), _p(bias, f32), int(solver))
 
 
 def pararnn_input_proj(ctx, x, W, bias, xproj) -> None:

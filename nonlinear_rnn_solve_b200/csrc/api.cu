@@ -146,6 +146,9 @@ int pararnn_newton_forward(pararnn_ctx *ctx, const float *xproj, const pararnn_p
     if (!ctx || !p || !h_out || !iters_out) return PARARNN_EINVAL;
     if (p->B < 1 || p->T < 1 || p->H < 1 || max_iters < 0 || max_iters > (1 << 30)) return PARARNN_EINVAL;
     if (!(tol == tol)) return PARARNN_EINVAL;
+    if (p->solver < PARARNN_SOLVER_NEWTON || p->solver > PARARNN_SOLVER_PICARD) return PARARNN_EINVAL;
+    // linearisation of the fixed-point scheme: zero (Jacobi), identity (Picard), else the cell's
+    const int jm_solver = p->solver == PARARNN_SOLVER_JACOBI ? 2 : p->solver == PARARNN_SOLVER_PICARD ? 3 : 0;
     const bool fused = xproj == nullptr;
     if (fused && (!p->x || !p->W || p->in < 1 || p->in > 8)) return PARARNN_EINVAL;
     if (misaligned(xproj) || misaligned(h_out) || misaligned(h0) || (fused && misaligned(p->x)))
@@ -158,9 +161,9 @@ int pararnn_newton_forward(pararnn_ctx *ctx, const float *xproj, const pararnn_p
     int rc;
     if (p->cell == PARARNN_GRU_DIAG || p->cell == PARARNN_LSTM_CIFG_PEEP || p->cell == PARARNN_LSTM_CIFG_PEEP_QUASI) {
         const int lstm = p->cell != PARARNN_GRU_DIAG;
-        const int quasi = p->cell == PARARNN_LSTM_CIFG_PEEP_QUASI;
+        const int jmode = jm_solver ? jm_solver : (p->cell == PARARNN_LSTM_CIFG_PEEP_QUASI ? 1 : 0);
         if (!p->a || (lstm && !p->peep)) return PARARNN_EINVAL;
-        prn::NewtonDiagReq r{lstm, quasi, p->B, p->T, p->H, p->in, xproj, p->x, p->W, p->bias, p->a, p->peep, h0, h_out,
+        prn::NewtonDiagReq r{lstm, jmode, p->B, p->T, p->H, p->in, xproj, p->x, p->W, p->bias, p->a, p->peep, h0, h_out,
                              max_iters, tol, iters_out, final_delta_out, residual_out};
         if (prn::newton_diag_plan(r, ctx->num_sms, &plan)) return PARARNN_ECUDA;
         if ((rc = prepare(ctx, plan, &w))) return rc;
@@ -172,7 +175,9 @@ int pararnn_newton_forward(pararnn_ctx *ctx, const float *xproj, const pararnn_p
     } else if (p->cell == PARARNN_RNN_TANH_DENSE || p->cell == PARARNN_RNN_TANH_QUASI) {
         if (!p->A) return PARARNN_EINVAL;
         if (p->H > 64) return PARARNN_EUNSUPPORTED;
-        prn::NewtonTanhReq r{p->cell == PARARNN_RNN_TANH_QUASI, p->B, p->T, p->H, p->in, xproj, p->x, p->W,
+        // Jacobi and Picard have diagonal linearisations: they run on the quasi (diagonal) kernel
+        const int quasi = p->cell == PARARNN_RNN_TANH_QUASI || jm_solver != 0;
+        prn::NewtonTanhReq r{quasi, jm_solver, p->B, p->T, p->H, p->in, xproj, p->x, p->W,
                              p->bias, p->A, h0, h_out, max_iters, tol, iters_out, final_delta_out, residual_out};
         int prc = prn::newton_tanh_plan(r, ctx->num_sms, &plan);
         if (prc == 1) return PARARNN_EUNSUPPORTED;

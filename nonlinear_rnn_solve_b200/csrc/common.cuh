@@ -121,6 +121,21 @@ __device__ __forceinline__ float rcp_hw(float y) {
 }
 constexpr float kLog2e = 1.4426950408889634f;
 
+// The matrix the step map is linearised with (see jmode): the Jacobian as evaluated
+// (0), the diagonal of a 2x2 block (1), zero (2, Jacobi) or the identity (3, Picard).
+template <int S> __device__ __forceinline__ void apply_jmode(int jmode, float *J) {
+    if (jmode == 0) return;
+    if (jmode == 1) {
+        if (S == 2) {
+            J[1 % (S * S)] = 0.f;
+            J[2 % (S * S)] = 0.f;
+        }
+        return;
+    }
+#pragma unroll
+    for (int q = 0; q < S * S; ++q) J[q] = (jmode == 3 && q % (S + 1) == 0) ? 1.f : 0.f;
+}
+
 __device__ __forceinline__ bool finitef(float v) { return fabsf(v) <= 3.402823466e38f; }
 
 // ------------------------------------------------------------------ affine elements

@@ -26,6 +26,7 @@ namespace prn {
 
 struct TanhArgs {
     int B, T, n, in;
+    int jmode;  // quasi kernel: 0 the diagonal of the Jacobian, 2 zero (Jacobi), 3 identity (Picard)
     const float *xproj, *x, *W, *bias, *A, *h0;
     float *h;
     int max_iters;
@@ -506,7 +507,7 @@ __device__ float quasi_phase_a(const TanhArgs &A, QuasiSmem<N> &sm, int b, int t
         for (int u = 0; u < 4; ++u) {
             const bool v = tv && i0 + u < A.n;
             const float f = tanh_(acc[j][u]);
-            Jv[u] = v ? (1.f - f * f) * dg[u] : 1.f;
+            Jv[u] = !v ? 1.f : A.jmode == 2 ? 0.f : A.jmode == 3 ? 1.f : (1.f - f * f) * dg[u];
             rv[u] = v ? f - cur[u] : 0.f;
             const float ad = fabsf(rv[u]);
             res = (ad > res || isnan(ad)) ? ad : res;
@@ -889,6 +890,7 @@ cudaError_t newton_tanh_launch(const NewtonTanhReq &r, const Plan &plan, const W
     A.B = r.B;
     A.T = r.T;
     A.n = r.n;
+    A.jmode = r.jmode;
     A.in = r.in;
     A.xproj = r.xproj;
     A.x = r.x;

@@ -48,8 +48,8 @@ struct DbgHost {
 
 // ---- Newton forward, diagonal / 2x2-block cells (GRU, LSTM) -----------------------
 struct NewtonDiagReq {
-    int cell;  // 0 GRU, 1 LSTM
-    int quasi; // LSTM: keep only the diagonal of each 2x2 Jacobian block
+    int cell;   // 0 GRU, 1 LSTM
+    int jmode;  // linearisation: 0 Jacobian, 1 LSTM block diagonal, 2 zero (Jacobi), 3 identity (Picard)
     int B, T, H, in;
     const float *xproj, *x, *W, *bias, *a, *peep, *h0;
     float *h;
@@ -66,6 +66,7 @@ cudaError_t newton_diag_launch(const NewtonDiagReq &r, const Plan &plan, const W
 // ---- Newton forward, tanh RNN (dense DEER and quasi-DEER) -------------------------
 struct NewtonTanhReq {
     int quasi;
+    int jmode;  // 0: the cell's (quasi) Jacobian, 2 zero (Jacobi), 3 identity (Picard)
     int B, T, n, in;
     const float *xproj, *x, *W, *bias, *A, *h0;
     float *h;

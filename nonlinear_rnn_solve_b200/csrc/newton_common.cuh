@@ -11,7 +11,7 @@ namespace prn {
 
 struct NewtonDiagArgs {
     int B, T, H, in;
-    int quasi;  // LSTM: the diagonal of each 2x2 Jacobian block only
+    int jmode;  // linearisation (apply_jmode)
     const float *xproj, *x, *W, *bias, *a, *peep, *h0;
     float *h;
     int max_iters;

@@ -99,10 +99,7 @@ __global__ void __launch_bounds__(kThreads, 2) newton_diag_kernel(const NewtonDi
                 if (k > 0 && v) load_state<S>(A.h, ((size_t)b * A.T + t) * A.H + hh, cur);
                 float f[S], J[S * S];
                 cell.eval(p, hp, f, J);
-                if (S == 2 && A.quasi) {  // diagonal scan backend: c and h decouple
-                    J[1] = 0.f;
-                    J[2 % (S * S)] = 0.f;
-                }
+                apply_jmode<S>(A.jmode, J);
 #pragma unroll
                 for (int q = 0; q < S; ++q) {
                     rr[i][q] = v ? f[q] - cur[q] : 0.f;
@@ -243,7 +240,7 @@ cudaError_t newton_diag_launch(const NewtonDiagReq &r, const Plan &plan, const W
     A.T = r.T;
     A.H = r.H;
     A.in = r.in;
-    A.quasi = r.quasi;
+    A.jmode = r.jmode;
     A.xproj = r.xproj;
     A.x = r.x;
     A.W = r.W;

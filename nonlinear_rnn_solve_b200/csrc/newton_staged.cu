@@ -207,10 +207,7 @@ __device__ __forceinline__ void tile_compute(const NewtonDiagArgs &A, float *sme
                 cell.eval_pre(p, hp, f, J);  // p was formed with the prescaled weights
             else
                 cell.eval(p, hp, f, J);
-            if (S == 2 && A.quasi) {  // diagonal scan backend: c and h decouple
-                J[1 % (S * S)] = 0.f;
-                J[2 % (S * S)] = 0.f;
-            }
+            apply_jmode<S>(A.jmode, J);
 #pragma unroll
             for (int q = 0; q < S; ++q) {
                 rr[i][q] = v ? f[q] - cur[q] : 0.f;
@@ -416,6 +413,7 @@ __global__ void __launch_bounds__(NT, MINB)
                         p[g] = acc;
                     }
                     cell.eval_pre(p, hprv, f, J);
+                    apply_jmode<S>(A.jmode, J);  // the halo linearises like the tile
 #pragma unroll
                     for (int q = 0; q < S; ++q) r[q] = f[q] - hcur[q];
                     he = make_aff<S>(J, r);

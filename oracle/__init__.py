@@ -44,7 +44,8 @@ class _Model(ctypes.Structure):
     _fields_ = [("cell", ctypes.c_int), ("quasi", ctypes.c_int),
                 ("B", ctypes.c_long), ("T", ctypes.c_long), ("H", ctypes.c_long),
                 ("xproj", ctypes.c_void_p), ("a", ctypes.c_void_p),
-                ("peep", ctypes.c_void_p), ("A", ctypes.c_void_p), ("solver", ctypes.c_int)]
+                ("peep", ctypes.c_void_p), ("A", ctypes.c_void_p), ("solver", ctypes.c_int),
+                ("lambda_", ctypes.c_double)]
 
 
 _lib = None
@@ -83,9 +84,10 @@ class Model:
     xproj: [B, T, G, H] (G = 3 GRU/LSTM, 1 tanh), a: [3, H], peep: [2, H], A: [n, n].
     """
 
-    SOLVERS = {"newton": 0, "jacobi": 1, "picard": 2}
+    SOLVERS = {"newton": 0, "jacobi": 1, "picard": 2, "elk": 3}
 
-    def __init__(self, cell, xproj, a=None, peep=None, A=None, quasi=False, solver="newton"):
+    def __init__(self, cell, xproj, a=None, peep=None, A=None, quasi=False, solver="newton",
+                 damping=0.0):
         self.cell = cell
         self.xproj = _f64(xproj)
         B, T, G, H = self.xproj.shape
@@ -95,8 +97,11 @@ class Model:
         self.quasi = bool(quasi)
         self.S = 2 if cell == "lstm" else 1
         self.solver = solver
+        assert solver != "elk" or cell in ("gru", "lstm"), "ELK here: diagonal linearisations of GRU/LSTM"
+        self.damping = float(damping)
         self._m = _Model(CELL_IDS[cell], int(self.quasi), B, T, H, _ptr(self.xproj),
-                         _ptr(self.a), _ptr(self.peep), _ptr(self.A), self.SOLVERS[solver])
+                         _ptr(self.a), _ptr(self.peep), _ptr(self.A), self.SOLVERS[solver],
+                         self.damping)
 
     @property
     def state_shape(self):
@@ -195,7 +200,7 @@ def input_proj_backward(grad_xproj, x, W):
     return g2 @ W64, g2.T @ x2, g2.sum(axis=0)
 
 
-def model_from_inputs(cell, inputs, quasi=False, solver="newton"):
+def model_from_inputs(cell, inputs, quasi=False, solver="newton", damping=0.0):
     """Build a Model from the arrays of ``workloads.generate`` (projection in fp64)."""
     x = inputs["x"]
     B, T, _ = x.shape
@@ -204,7 +209,7 @@ def model_from_inputs(cell, inputs, quasi=False, solver="newton"):
     H = xp.shape[-1] // G
     xp = xp.reshape(B, T, G, H)
     return Model(cell, xp, a=inputs.get("a"), peep=inputs.get("peep"), A=inputs.get("A"),
-                 quasi=quasi, solver=solver)
+                 quasi=quasi, solver=solver, damping=damping)
 
 
 def linear_scan(kind, J, b, h0=None, reverse=False):

@@ -53,10 +53,12 @@ typedef struct {
     const double *A;     /* [n][n] tanh recurrent matrix */
     int solver;          /* linearisation used by orc_newton: ORC_NEWTON (the cell's
                           * Jacobian, or its diagonal with quasi), ORC_JACOBI (J = 0),
-                          * ORC_PICARD (J = I) ["Para-Seq" README, Main features] */
+                          * ORC_PICARD (J = I) ["Para-Seq" README, Main features], or
+                          * ORC_ELK (diagonal Jacobian, damped step, see orc_newton) */
+    double lambda;       /* ELK damping (>= 0; 0 gives the quasi-Newton step) */
 } orc_model;
 
-enum { ORC_NEWTON = 0, ORC_JACOBI = 1, ORC_PICARD = 2 };
+enum { ORC_NEWTON = 0, ORC_JACOBI = 1, ORC_PICARD = 2, ORC_ELK = 3 };
 
 /* The fixed-point schemes share the Newton loop and differ only in the matrix the step
  * map is linearised with: Jacobi keeps none of it (every step is re-evaluated from
@@ -64,7 +66,7 @@ enum { ORC_NEWTON = 0, ORC_JACOBI = 1, ORC_PICARD = 2 };
  * f(h^(k)_{t-1}) - h^(k)_{t-1} along t). */
 static void solver_jacobian(const orc_model *m, long D, double *J)
 {
-    if (m->solver == ORC_NEWTON) return;
+    if (m->solver == ORC_NEWTON || m->solver == ORC_ELK) return;
     for (long i = 0; i < D; ++i)
         for (long j = 0; j < D; ++j) J[i * D + j] = (m->solver == ORC_PICARD && i == j) ? 1.0 : 0.0;
 }
@@ -273,6 +275,36 @@ static double absmax_update(double cur, double v)
     return v > cur ? v : cur;
 }
 
+/* ELK ["Towards Scalable and Stable Parallelization of Nonlinear RNNs", Abstract: the
+ * Levenberg-Marquardt step computed by Kalman smoothing], for a diagonal linearisation.
+ * With x = h^(k+1) - h^(k), a_t the diagonal of J_t and r_t = f_t - h^(k)_t, the damped
+ * step minimises
+ *     sum_t (x_t - a_t x_{t-1} - r_t)^2 + lambda sum_t x_t^2,    x_0 = 0 (h_0 is given),
+ * the Levenberg-Marquardt objective of the stacked residual.  That is the MAP path of
+ * the state-space model x_t = a_t x_{t-1} + r_t + w_t, w_t ~ N(0, 1), observed as
+ * y_t = 0 = x_t + v_t, v_t ~ N(0, 1/lambda): a Kalman filter forward, then a
+ * Rauch-Tung-Striebel smoother backward, one scalar component at a time.  lambda = 0
+ * (no observations) returns the quasi-Newton step.  Scratch: 5 T doubles. */
+static void elk_component(long T, const double *a, const double *r, double lambda, double *xs, double *work)
+{
+    double *Pm = work, *mm = work + T, *P = work + 2 * T, *mf = work + 3 * T;
+    double Pp = 0.0, mp = 0.0; /* filtered variance and mean before t = 0 (known) */
+    for (long t = 0; t < T; ++t) {
+        Pm[t] = a[t] * a[t] * Pp + 1.0;           /* predicted variance */
+        mm[t] = a[t] * mp + r[t];                 /* predicted mean */
+        const double K = lambda * Pm[t] / (1.0 + lambda * Pm[t]); /* gain, Pm / (Pm + 1/lambda) */
+        P[t] = (1.0 - K) * Pm[t];
+        mf[t] = (1.0 - K) * mm[t];                /* update with the observation 0 */
+        Pp = P[t];
+        mp = mf[t];
+    }
+    xs[T - 1] = mf[T - 1];
+    for (long t = T - 2; t >= 0; --t) {
+        const double G = P[t] * a[t + 1] / Pm[t + 1];
+        xs[t] = mf[t] + G * (xs[t + 1] - mm[t + 1]);
+    }
+}
+
 int orc_newton(const orc_model *m, const double *h0, int max_iters, double tol, double *h_out,
                int *iters_out, double *delta_log, int log_len)
 {
@@ -318,6 +350,39 @@ int orc_newton(const orc_model *m, const double *h0, int max_iters, double tol, 
                 free(f);
                 free(bt);
                 free(z0);
+            }
+        } else if (m->solver == ORC_ELK) {
+#pragma omp parallel for schedule(static) reduction(max : delta)
+            for (long bu = 0; bu < B * H; ++bu) {
+                long b = bu / H, u = bu % H;
+                double *a = malloc(sizeof(double) * T * S), *r = malloc(sizeof(double) * T * S);
+                double *xs = malloc(sizeof(double) * T), *work = malloc(sizeof(double) * 5 * T);
+                double pk[2] = {0.0, 0.0}, f[2], J[4];
+                if (h0)
+                    for (long s = 0; s < S; ++s) pk[s] = h0[(b * H + u) * S + s];
+                for (long t = 0; t < T; ++t) { /* linearise at h^(k): diagonal of J, residual */
+                    unit_eval(m, b, t, u, pk, f, J, NULL, NULL);
+                    long idx = ((b * T + t) * H + u) * S;
+                    for (long s = 0; s < S; ++s) {
+                        a[s * T + t] = J[s * S + s];
+                        r[s * T + t] = f[s] - hk[idx + s];
+                        pk[s] = hk[idx + s];
+                    }
+                }
+                double dloc = 0.0;
+                for (long s = 0; s < S; ++s) {
+                    elk_component(T, a + s * T, r + s * T, m->lambda, xs, work);
+                    for (long t = 0; t < T; ++t) {
+                        long idx = ((b * T + t) * H + u) * S + s;
+                        hn[idx] = hk[idx] + xs[t];
+                        dloc = absmax_update(dloc, xs[t]);
+                    }
+                }
+                if (dloc > delta) delta = dloc;
+                free(a);
+                free(r);
+                free(xs);
+                free(work);
             }
         } else {
 #pragma omp parallel for schedule(static) reduction(max : delta)

@@ -329,6 +329,67 @@ def test_fixed_point_sweeps_match_their_definition(cell, solver):
     np.testing.assert_allclose(h, R, atol=1e-12)
 
 
+def _lm_stacked(lib, xp, h0, iters, lam, state_shape):
+    """Levenberg-Marquardt on the stacked residual F(h) = 0 with a dense solve:
+    h <- h - (Jd^T Jd + lam I)^{-1} Jd^T F, where Jd is dF/dh (autograd) with only the
+    diagonal of each sub-diagonal block kept (the diagonal linearisation)."""
+    xpt, h0t = torch.tensor(xp), torch.tensor(h0)
+    hs = torch.zeros(state_shape, dtype=f64)
+    B, T = hs.shape[:2]
+    D = hs[0, 0].numel()
+    out = []
+    for _ in range(iters):
+        F = tc.stacked_residual(lib, xpt, h0t, hs).reshape(-1)
+        Jf = torch.autograd.functional.jacobian(
+            lambda v: tc.stacked_residual(lib, xpt, h0t, v.reshape(hs.shape)).reshape(-1), hs.reshape(-1))
+        Jm = Jf.reshape(B, T, D, B, T, D).clone()
+        off = ~torch.eye(D, dtype=torch.bool)
+        for b in range(B):
+            for t in range(1, T):
+                blk = Jm[b, t, :, b, t - 1, :]
+                blk[off] = 0.0
+        Jd = Jm.reshape(B * T * D, B * T * D)
+        step = torch.linalg.solve(Jd.T @ Jd + lam * torch.eye(Jd.shape[0], dtype=f64), Jd.T @ F)
+        hs = hs - step.reshape(hs.shape)
+        out.append(hs.clone())
+    return out
+
+
+@pytest.mark.parametrize("cell", ["gru", "lstm"])
+@pytest.mark.parametrize("lam", [0.3, 2.0])
+def test_elk_step_is_levenberg_marquardt_on_stacked_system(cell, lam):
+    """The Kalman-smoother step equals the dense Levenberg-Marquardt step."""
+    H = 3
+    m, xp, prm, h0 = _rand_model(cell, B=2, T=8, H=H, seed=71)
+    m = oracle.Model(cell, xp, solver="elk", damping=lam, **prm)
+    refs = _lm_stacked(_lib(cell, H, prm), xp, h0, 3, lam, m.state_shape)
+    for k, ref in enumerate(refs, start=1):
+        h, iters, _ = m.newton(h0, max_iters=k, tol=0.0)
+        assert iters == k
+        np.testing.assert_allclose(h, ref.numpy(), atol=1e-11)
+
+
+@pytest.mark.parametrize("cell", ["gru", "lstm"])
+def test_elk_without_damping_is_the_diagonal_newton_step(cell):
+    m, xp, prm, h0 = _rand_model(cell, B=2, T=30, H=4, seed=72)
+    e = oracle.Model(cell, xp, solver="elk", damping=0.0, **prm)
+    q = oracle.Model(cell, xp, quasi=True, **prm)  # GRU: its Jacobian is already diagonal
+    for k in (1, 2, 4):
+        np.testing.assert_allclose(e.newton(h0, max_iters=k, tol=0.0)[0], q.newton(h0, max_iters=k, tol=0.0)[0],
+                                   atol=1e-12)
+
+
+@pytest.mark.parametrize("cell", ["gru", "lstm"])
+def test_elk_converges_to_rollout_and_damping_shortens_steps(cell):
+    m, xp, prm, h0 = _rand_model(cell, B=2, T=40, H=4, seed=73, scale=1.5)
+    R = m.rollout(h0)
+    h, iters, d = oracle.Model(cell, xp, solver="elk", damping=0.5, **prm).newton(h0, max_iters=400, tol=1e-12)
+    np.testing.assert_allclose(h, R, atol=1e-10)
+    first = [oracle.Model(cell, xp, solver="elk", damping=lam, **prm).newton(h0, max_iters=1, tol=0.0)[2][0]
+             for lam in (0.0, 0.5, 5.0)]
+    assert first[0] > first[1] > first[2]
+
+
 def test_newton_zero_iterations_returns_initial_guess():
     m, xp, prm, h0 = _rand_model("gru", B=1, T=5, H=2, seed=3)
     h, iters, d = m.newton(h0, max_iters=0, tol=1e-6)

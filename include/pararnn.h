@@ -90,6 +90,7 @@ typedef struct {
     const float *W;        /* [G*H, in] fp32 (fused projection) */
     const float *bias;     /* [G*H] fp32 or NULL (fused projection) */
     int solver;            /* pararnn_solver (0 = Newton) */
+    float damping;         /* ELK: Levenberg-Marquardt damping lambda >= 0 */
 } pararnn_params;
 
 /* Fixed-point scheme of pararnn_newton_forward ("Para-Seq" README, Main features:
@@ -99,7 +100,18 @@ typedef struct {
  * cells), zero (JACOBI: h^(k+1)_t = f(h^(k)_{t-1}), every step in parallel), or the
  * identity (PICARD: the increments f(h^(k)_{t-1}) - h^(k)_{t-1} are summed along t).
  * Every scheme reaches the rollout; after k iterations the first k states are exact. */
-typedef enum { PARARNN_SOLVER_NEWTON = 0, PARARNN_SOLVER_JACOBI = 1, PARARNN_SOLVER_PICARD = 2 } pararnn_solver;
+typedef enum {
+    PARARNN_SOLVER_NEWTON = 0,
+    PARARNN_SOLVER_JACOBI = 1,
+    PARARNN_SOLVER_PICARD = 2,
+    /* ELK ("Towards Scalable and Stable Parallelization of Nonlinear RNNs", Abstract):
+     * the Levenberg-Marquardt step of the stacked system, i.e. the minimiser of
+     * sum_t |x_t - J_t x_{t-1} - r_t|^2 + damping sum_t |x_t|^2 (x = h^(k+1) - h^(k),
+     * r_t = f_t - h^(k)_t), computed by a parallel Kalman filter and smoother; J_t is
+     * diagonal: ParaGRU (ELK) and ParaLSTM with each block's diagonal (quasi-ELK).
+     * damping = 0 gives the quasi-Newton step; larger damping shortens the steps. */
+    PARARNN_SOLVER_ELK = 3
+} pararnn_solver;
 
 /* Create a context on `device` that enqueues on `cuda_stream` (a cudaStream_t, or
  * NULL for the legacy default stream).  *ctx is NULL on failure. */

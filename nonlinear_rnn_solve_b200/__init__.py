@@ -34,6 +34,7 @@ PARARNN_LSTM_CIFG_PEEP_QUASI = 4
 PARARNN_SOLVER_NEWTON = 0
 PARARNN_SOLVER_JACOBI = 1
 PARARNN_SOLVER_PICARD = 2
+PARARNN_SOLVER_ELK = 3
 
 PARARNN_SCAN_DIAG = 0
 PARARNN_SCAN_BLOCK2 = 1
@@ -61,7 +62,7 @@ class pararnn_params(ctypes.Structure):
                 ("H", ctypes.c_int), ("in_", ctypes.c_int),
                 ("a", ctypes.c_void_p), ("peep", ctypes.c_void_p), ("A", ctypes.c_void_p),
                 ("x", ctypes.c_void_p), ("W", ctypes.c_void_p), ("bias", ctypes.c_void_p),
-                ("solver", ctypes.c_int)]
+                ("solver", ctypes.c_int), ("damping", ctypes.c_float)]
 
 
 _lib = None
@@ -145,10 +146,11 @@ def pararnn_set_stream(ctx, stream=None) -> None:
     _check(lib().pararnn_set_stream(ctx, _stream_handle(stream)), "pararnn_set_stream")
 
 
-def make_params(cell, B, T, H, inp=0, a=None, peep=None, A=None, x=None, W=None, bias=None, solver=0):
+def make_params(cell, B, T, H, inp=0, a=None, peep=None, A=None, x=None, W=None, bias=None, solver=0,
+                damping=0.0):
     f32 = torch.float32
     return pararnn_params(int(cell), int(B), int(T), int(H), int(inp), _p(a, f32), _p(peep, f32),
-                          _p(A, f32), _p(x, f32), _p(W, f32), _p(bias, f32), int(solver))
+                          _p(A, f32), _p(x, f32), _p(W, f32), _p(bias, f32), int(solver), float(damping))
 
 
 def pararnn_input_proj(ctx, x, W, bias, xproj) -> None:

@@ -146,7 +146,8 @@ int pararnn_newton_forward(pararnn_ctx *ctx, const float *xproj, const pararnn_p
     if (!ctx || !p || !h_out || !iters_out) return PARARNN_EINVAL;
     if (p->B < 1 || p->T < 1 || p->H < 1 || max_iters < 0 || max_iters > (1 << 30)) return PARARNN_EINVAL;
     if (!(tol == tol)) return PARARNN_EINVAL;
-    if (p->solver < PARARNN_SOLVER_NEWTON || p->solver > PARARNN_SOLVER_PICARD) return PARARNN_EINVAL;
+    if (p->solver < PARARNN_SOLVER_NEWTON || p->solver > PARARNN_SOLVER_ELK) return PARARNN_EINVAL;
+    if (p->solver == PARARNN_SOLVER_ELK && !(p->damping >= 0.f && p->damping < 3.0e38f)) return PARARNN_EINVAL;
     // linearisation of the fixed-point scheme: zero (Jacobi), identity (Picard), else the cell's
     const int jm_solver = p->solver == PARARNN_SOLVER_JACOBI ? 2 : p->solver == PARARNN_SOLVER_PICARD ? 3 : 0;
     const bool fused = xproj == nullptr;
@@ -165,15 +166,19 @@ int pararnn_newton_forward(pararnn_ctx *ctx, const float *xproj, const pararnn_p
         if (!p->a || (lstm && !p->peep)) return PARARNN_EINVAL;
         prn::NewtonDiagReq r{lstm, jmode, p->B, p->T, p->H, p->in, xproj, p->x, p->W, p->bias, p->a, p->peep, h0, h_out,
                              max_iters, tol, iters_out, final_delta_out, residual_out};
-        if (prn::newton_diag_plan(r, ctx->num_sms, &plan)) return PARARNN_ECUDA;
+        const bool elk = p->solver == PARARNN_SOLVER_ELK;
+        if ((elk ? prn::elk_plan(r, ctx->num_sms, &plan) : prn::newton_diag_plan(r, ctx->num_sms, &plan)))
+            return PARARNN_ECUDA;
         if ((rc = prepare(ctx, plan, &w))) return rc;
         if (max_iters == 0) {
             const size_t n = (size_t)p->B * p->T * p->H * (lstm ? 2 : 1);
             if (cudaMemsetAsync(h_out, 0, n * sizeof(float), ctx->stream) != cudaSuccess) return PARARNN_ECUDA;
         }
-        rc = cuda_rc(prn::newton_diag_launch(r, plan, w, ctx->dbg, ctx->stream));
+        rc = cuda_rc(elk ? prn::elk_launch(r, p->damping, plan, w, ctx->dbg, ctx->stream)
+                         : prn::newton_diag_launch(r, plan, w, ctx->dbg, ctx->stream));
     } else if (p->cell == PARARNN_RNN_TANH_DENSE || p->cell == PARARNN_RNN_TANH_QUASI) {
         if (!p->A) return PARARNN_EINVAL;
+        if (p->solver == PARARNN_SOLVER_ELK) return PARARNN_EUNSUPPORTED;
         if (p->H > 64) return PARARNN_EUNSUPPORTED;
         // Jacobi and Picard have diagonal linearisations: they run on the quasi (diagonal) kernel
         const int quasi = p->cell == PARARNN_RNN_TANH_QUASI || jm_solver != 0;

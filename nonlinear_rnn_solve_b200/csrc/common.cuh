@@ -252,9 +252,9 @@ __device__ __forceinline__ unsigned long long ld_relaxed_u64(const unsigned long
     return v;
 }
 
-template <int S, int C, int NT = kThreads> struct ScanSmem {
+template <int S, int C, int NT = kThreads, class E = Aff<S>> struct ScanSmem {
     static constexpr int NW = NT / 32;
-    Aff<S> wtot[NW][C];  // per-warp totals (scan order)
+    E wtot[NW][C];  // per-warp totals (scan order)
     float carry[C][S];   // carry entering the tile, per channel
 };
 
@@ -263,28 +263,28 @@ template <int S, int C, int NT = kThreads> struct ScanSmem {
 // On return: `excl` is the composition of the elements before this thread's
 // position (identity for s = 0) and `total` (valid in warp 0, lanes c < C) is the
 // tile's aggregate for channel c.
-template <int S, int C, int NT = kThreads>
-__device__ __forceinline__ void cta_scan(const Aff<S> &e, ScanSmem<S, C, NT> &sm, Aff<S> &excl, Aff<S> &total) {
+template <int S, int C, int NT = kThreads, class E = Aff<S>>
+__device__ __forceinline__ void cta_scan(const E &e, ScanSmem<S, C, NT, E> &sm, E &excl, E &total) {
     static_assert(32 % C == 0, "C must divide 32");
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    Aff<S> inc = e;
+    E inc = e;
 #pragma unroll
     for (int off = C; off < 32; off <<= 1) {
-        Aff<S> o = inc.shfl_up(off);
+        E o = inc.shfl_up(off);
         if (lane >= off) inc = compose(o, inc);
     }
-    Aff<S> wex = inc.shfl_up(C);
-    if (lane < C) wex = Aff<S>::ident();
+    E wex = inc.shfl_up(C);
+    if (lane < C) wex = E::ident();
     if (lane >= 32 - C) sm.wtot[warp][lane - (32 - C)] = inc;
     __syncthreads();
     const int c = lane % C;
-    Aff<S> pre = Aff<S>::ident();
+    E pre = E::ident();
     for (int w = 0; w < warp; ++w) pre = compose(pre, sm.wtot[w][c]);
     excl = compose(pre, wex);
     if (warp == 0 && lane < C) {
-        Aff<S> t = Aff<S>::ident();
+        E t = E::ident();
 #pragma unroll
-        for (int w = 0; w < ScanSmem<S, C, NT>::NW; ++w) t = compose(t, sm.wtot[w][lane]);
+        for (int w = 0; w < ScanSmem<S, C, NT, E>::NW; ++w) t = compose(t, sm.wtot[w][lane]);
         total = t;
     }
 }
@@ -293,10 +293,10 @@ __device__ __forceinline__ void cta_scan(const Aff<S> &e, ScanSmem<S, C, NT> &sm
 // slot i, channel c).  Every wait is bounded (abort flag, dbg.wait_ns).
 //
 // publish_agg: lanes c < C publish the tile aggregate (tiles with chunk > 0).
-template <int S, int C>
-__device__ __forceinline__ void publish_agg(const LookBack<S> &lb, const Aff<S> &total, long tile, int chunk,
+template <int S, int C, class E = Aff<S>>
+__device__ __forceinline__ void publish_agg(const LookBack<S> &lb, const E &total, long tile, int chunk,
                                             unsigned epoch, const Dbg &dbg) {
-    constexpr int KF = Aff<S>::kFloats;
+    constexpr int KF = E::kFloats;
     const int lane = threadIdx.x & 31;
     if (chunk == 0 || lane >= C || dbg.skip_tile == tile) return;
     float tv[KF];
@@ -319,18 +319,18 @@ template <int S> __device__ __forceinline__ bool aff_is_const(const float *v) {
     return true;
 }
 
-template <int S, int C>
+template <int S, int C, class E = Aff<S>>
 __device__ bool resolve_carry(const LookBack<S> &lb, long tile, int chunk, long nseq, unsigned epoch,
                               const float *base, float *carry, Ctl *ctl, int *sticky, const Dbg &dbg) {
     constexpr int WIN = 32 / C;
-    constexpr int KF = Aff<S>::kFloats;
+    constexpr int KF = E::kFloats;
     const int lane = threadIdx.x & 31, i = lane / C, c = lane % C;
     if (chunk == 0) {
 #pragma unroll
         for (int q = 0; q < S; ++q) carry[q] = base[q];
         return true;
     }
-    Aff<S> acc = Aff<S>::ident();  // composition of everything between here and the window
+    E acc = E::ident();  // composition of everything between here and the window
     long pred = tile - nseq;
     int pchunk = chunk - 1;
     for (;;) {
@@ -338,12 +338,12 @@ __device__ bool resolve_carry(const LookBack<S> &lb, long tile, int chunk, long 
         const long my_tile = pred - (long)i * nseq;
         unsigned long long t0 = 0;
         int polls = 0;
-        Aff<S> v;
+        E v;
         unsigned st;  // 0 not ready, 1 aggregate, 2 known value
         for (;;) {
             st = 2u;
             if (my_chunk < 0) {
-                v = Aff<S>::cst(base);
+                v = E::cst(base);
             } else {
                 unsigned long long wi[S], wa[KF];
 #pragma unroll
@@ -363,9 +363,9 @@ __device__ bool resolve_carry(const LookBack<S> &lb, long tile, int chunk, long 
                     av[q] = __uint_as_float((unsigned)(wa[q] >> 32));
                 }
                 if (inc_ok) {
-                    v = Aff<S>::cst(iv);
+                    v = E::cst(iv);
                 } else if (agg_ok) {
-                    v = Aff<S>::from_floats(av);
+                    v = E::from_floats(av);
                     st = aff_is_const<S>(av) ? 2u : 1u;
                 } else {
                     st = 0u;
@@ -388,10 +388,10 @@ __device__ bool resolve_carry(const LookBack<S> &lb, long tile, int chunk, long 
             if ((slot_ready & need_w) == need_w) {
                 // reduce the window up to the first known slot; slot 0 is the nearest
                 // predecessor (applied last)
-                if (i > first) v = Aff<S>::ident();
+                if (i > first) v = E::ident();
 #pragma unroll
                 for (int off = C; off < 32; off <<= 1) {
-                    Aff<S> o = v.shfl_down(off);
+                    E o = v.shfl_down(off);
                     if (lane + off < 32) v = compose(o, v);
                 }
                 acc = compose(v, acc);
@@ -423,8 +423,8 @@ __device__ bool resolve_carry(const LookBack<S> &lb, long tile, int chunk, long 
 }
 
 // publish_inc: lanes c < C publish the tile's inclusive value total(carry).
-template <int S, int C>
-__device__ __forceinline__ void publish_inc(const LookBack<S> &lb, const Aff<S> &total, const float *carry, long tile,
+template <int S, int C, class E = Aff<S>>
+__device__ __forceinline__ void publish_inc(const LookBack<S> &lb, const E &total, const float *carry, long tile,
                                             unsigned epoch, const Dbg &dbg) {
     const int lane = threadIdx.x & 31;
     if (lane >= C || dbg.skip_tile == tile) return;
@@ -439,16 +439,16 @@ __device__ __forceinline__ void publish_inc(const LookBack<S> &lb, const Aff<S> 
 // `halo` (optional, channel c): the composed map of the steps just before the tile,
 // evaluated by the tile itself; when its matrix part is exactly zero it is a constant
 // whose value is the carry, and no predecessor is read.
-template <int S, int C, int NT = kThreads>
-__device__ bool look_back(const LookBack<S> &lb, ScanSmem<S, C, NT> &sm, const Aff<S> &total, long tile,
+template <int S, int C, int NT = kThreads, class E = Aff<S>>
+__device__ bool look_back(const LookBack<S> &lb, ScanSmem<S, C, NT, E> &sm, const E &total, long tile,
                           int chunk, long nseq, unsigned epoch, const float *base /* [S], channel c */,
-                          Ctl *ctl, int *sticky, const Dbg &dbg, const Aff<S> *halo = nullptr) {
+                          Ctl *ctl, int *sticky, const Dbg &dbg, const E *halo = nullptr) {
     const int lane = threadIdx.x & 31;
-    publish_agg<S, C>(lb, total, tile, chunk, epoch, dbg);
+    publish_agg<S, C, E>(lb, total, tile, chunk, epoch, dbg);
     float carry[S];
     bool known = false;
     if (halo != nullptr && chunk > 0) {
-        float hv[Aff<S>::kFloats];
+        float hv[E::kFloats];
         halo->to_floats(hv);
         known = __all_sync(0xffffffffu, lane >= C || aff_is_const<S>(hv));
         if (known) {
@@ -456,8 +456,8 @@ __device__ bool look_back(const LookBack<S> &lb, ScanSmem<S, C, NT> &sm, const A
             for (int q = 0; q < S; ++q) carry[q] = hv[S * S + q];
         }
     }
-    if (!known && !resolve_carry<S, C>(lb, tile, chunk, nseq, epoch, base, carry, ctl, sticky, dbg)) return false;
-    publish_inc<S, C>(lb, total, carry, tile, epoch, dbg);
+    if (!known && !resolve_carry<S, C, E>(lb, tile, chunk, nseq, epoch, base, carry, ctl, sticky, dbg)) return false;
+    publish_inc<S, C, E>(lb, total, carry, tile, epoch, dbg);
     if (lane < C) {
 #pragma unroll
         for (int q = 0; q < S; ++q) sm.carry[lane][q] = carry[q];

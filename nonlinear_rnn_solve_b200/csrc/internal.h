@@ -63,6 +63,11 @@ int newton_staged_plan(const NewtonDiagReq &r, int num_sms, Plan *plan);  // 1: 
 cudaError_t newton_diag_launch(const NewtonDiagReq &r, const Plan &plan, const Work &w,
                                const DbgHost &dbg, cudaStream_t st);
 
+// ELK (damped Newton by Kalman smoothing) for the diagonal linearisations (elk.cu).
+int elk_plan(const NewtonDiagReq &r, int num_sms, Plan *plan);
+cudaError_t elk_launch(const NewtonDiagReq &r, float lambda, const Plan &plan, const Work &w, const DbgHost &dbg,
+                       cudaStream_t st);
+
 // ---- Newton forward, tanh RNN (dense DEER and quasi-DEER) -------------------------
 struct NewtonTanhReq {
     int quasi;

@@ -20,19 +20,19 @@ def state_shape(cell, B, T, H):
     return (B, T, H, 2) if cell in ("lstm", "lstm_quasi") else (B, T, H)
 
 
-SOLVERS = {"newton": 0, "jacobi": 1, "picard": 2}
+SOLVERS = {"newton": 0, "jacobi": 1, "picard": 2, "elk": 3}
 
 
 def newton_forward(ctx, cell, B, T, H, *, xproj=None, x=None, W=None, bias=None, a=None,
                    peep=None, A=None, h0=None, max_iters=None, tol=1e-6, residual=False,
-                   h_out=None, solver="newton"):
+                   h_out=None, solver="newton", damping=0.0):
     """Newton / quasi-Newton (or Jacobi / Picard) solve.  Returns dict(h, iters, delta,
     residual) (device tensors)."""
     dev = (xproj if xproj is not None else x).device
     inp = 0 if x is None else x.shape[-1]
     prm = make_params(CELLS[cell], B, T, H, inp, a=a, peep=peep, A=A,
                       x=x if xproj is None else None, W=W if xproj is None else None,
-                      bias=bias if xproj is None else None, solver=SOLVERS[solver])
+                      bias=bias if xproj is None else None, solver=SOLVERS[solver], damping=damping)
     if h_out is None:
         h_out = torch.empty(state_shape(cell, B, T, H), device=dev, dtype=torch.float32)
     iters = torch.zeros(1, device=dev, dtype=torch.int32)

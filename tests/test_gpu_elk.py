@@ -1,0 +1,96 @@
+"""GPU parity: ELK (Levenberg-Marquardt damped Newton by parallel Kalman smoothing) for
+ParaGRU and the ParaLSTM block diagonal (quasi-ELK).
+
+The kernel runs three scans per iteration (filter variance as a 2x2 projective scan,
+filter mean, reverse smoother).  Bars: with tol = 0 and k iterations, the iterate
+within 1e-4 x max(1, |h|_max) of the oracle's (Kalman filter + RTS smoother in fp64,
+pinned to a dense Levenberg-Marquardt solve); with a tolerance, the oracle's iteration
+count and the converged states within 1e-4.  Shapes: a single channel over many tiles
+(look-back across 32 chunks), unit counts below and above the 32-channel tile, raw
+inputs and projected inputs; two damping values.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gpu_util import gpu, host, max_abs, need_gpu
+
+from nonlinear_rnn_solve_b200 import Context, PararnnError, solve
+from nonlinear_rnn_solve_b200 import workloads as wl
+
+pytestmark = pytest.mark.gpu
+TOL = 1e-4
+
+
+@pytest.fixture(scope="module")
+def ctx():
+    need_gpu()
+    c = Context(0)
+    yield c
+    c.close()
+
+
+def _workload(cell, B, T, H, inp, seed):
+    base = "gru_b1_t1024_in4_h8" if cell == "gru" else "lstm_b4_t8192_h1024_bf16"
+    return wl.WORKLOADS[base].resized(B=B, T=T, H=H, inp=inp, seed=seed, bf16=False, tol=1e-5,
+                                      max_iters=T + 1, w_dist="uniform_fan_in")
+
+
+def _run(ctx, cell, w, inp, lam, max_iters, tol, m=None, use_xproj=False):
+    t = {k: gpu(v) for k, v in inp.items() if v is not None}
+    kw = dict(a=t["a"], peep=t.get("peep"), h0=t["h0"], max_iters=max_iters, tol=tol, solver="elk", damping=lam)
+    if use_xproj:
+        out = solve.newton_forward(ctx.ctx, cell, w.B, w.T, w.H, xproj=gpu(m.xproj.astype(np.float32)), **kw)
+    else:
+        out = solve.newton_forward(ctx.ctx, cell, w.B, w.T, w.H, x=t["x"], W=t["W"], bias=t["bias"], **kw)
+    torch.cuda.synchronize()
+    assert ctx.status() == 0
+    return out
+
+
+CASES = [  # (cell, B, T, H, in, xproj)
+    ("gru", 2, 300, 5, 3, False),
+    ("gru", 4, 65536, 1, 2, False),
+    ("gru", 2, 500, 64, 4, True),
+    ("lstm", 2, 300, 33, 4, False),
+    ("lstm", 2, 400, 64, 4, True),
+]
+
+
+@pytest.mark.parametrize("lam", [0.5, 3.0])
+@pytest.mark.parametrize("case", CASES)
+def test_elk_iterates_match_oracle(ctx, lam, case):
+    cell, B, T, H, inp_w, use_xproj = case
+    w = _workload(cell, B, T, H, inp_w, seed=B * 13 + T + H)
+    inp = wl.generate(w)
+    m = oracle.model_from_inputs(cell, inp, solver="elk", damping=lam)
+    for k in (1, 2, 5):
+        out = _run(ctx, cell, w, inp, lam, k, 0.0, m, use_xproj)
+        assert int(out["iters"].item()) == k
+        h_ref, _, _ = m.newton(inp["h0"], max_iters=k, tol=0.0)
+        scale = max(1.0, float(np.abs(h_ref).max()))
+        assert max_abs(host(out["h"]), h_ref) <= TOL * scale, (lam, k)
+
+
+@pytest.mark.parametrize("cell", ["gru", "lstm"])
+def test_elk_converges_with_oracle_iteration_count(ctx, cell):
+    w = _workload(cell, 2, 700, 8, 3, seed=3)
+    inp = wl.generate(w)
+    m = oracle.model_from_inputs(cell, inp, solver="elk", damping=1.0)
+    h_ref, it_ref, d_ref = m.newton(inp["h0"], max_iters=w.max_iters, tol=w.tol)
+    out = _run(ctx, cell, w, inp, 1.0, w.max_iters, w.tol)
+    assert int(out["iters"].item()) == it_ref, (int(out["iters"].item()), it_ref, d_ref)
+    assert max_abs(host(out["h"]), h_ref) <= TOL
+
+
+def test_elk_rejects_negative_damping_and_the_dense_cell(ctx):
+    w = _workload("gru", 1, 32, 2, 2, seed=1)
+    inp = wl.generate(w)
+    with pytest.raises(PararnnError):
+        _run(ctx, "gru", w, inp, -1.0, 3, 0.0)
+    tw = wl.WORKLOADS["tanh_b16_t65536_in4_n8_quasi"].resized(B=1, T=32)
+    ti = {k: gpu(v) for k, v in wl.generate(tw).items() if v is not None}
+    with pytest.raises(PararnnError):
+        solve.newton_forward(ctx.ctx, "tanh_quasi", 1, 32, tw.H, x=ti["x"], W=ti["W"], bias=ti["bias"], A=ti["A"],
+                             h0=ti["h0"], max_iters=3, tol=0.0, solver="elk", damping=1.0)

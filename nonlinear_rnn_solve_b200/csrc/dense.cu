@@ -819,6 +819,159 @@ __global__ void __launch_bounds__(kThreads, 1) dense_scan_kernel(const DScanArgs
     }
 }
 
+// Small states (n <= 8): one warp per tile, so the sequential walks synchronise with
+// warp shuffles instead of CTA barriers.  Lane l holds P[r][c], P[r][c + 1] of the
+// chunk map (r = l / 4, c = 2 (l % 4)) and D[r]; a step needs row r of M_t and the
+// column entries P[k][c] from lane 4 k + l % 4.  The warp stages blocks of 32 steps
+// of J and b in shared memory with cp.async, one block ahead of its walk.  Tiles are
+// taken in increasing order by the warps of a cooperative grid, so a tile's
+// predecessor is always resident or done; the carry chain across tiles is the
+// inclusive chain of the kernel above.
+constexpr int kDsw = 1024;            // steps per warp tile
+constexpr int kDswBlk = 32;           // steps per staged block
+constexpr int kDswWarps = 4;          // warps per CTA
+constexpr int kDswBuf = kDswBlk * 72;  // floats per staging buffer: 32 (n^2 + n), n <= 8
+
+__device__ __forceinline__ void cp_async4(float *dst, const float *src, bool valid) {
+    const unsigned d = (unsigned)__cvta_generic_to_shared(dst);
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(d), "l"(src), "r"(valid ? 4 : 0) : "memory");
+}
+
+// Stage J for times jt0 .. jt0 + 31 and b for times bt0 .. bt0 + 31 (zero beyond T).
+__device__ __forceinline__ void dsw_stage(const DScanArgs &A, float *buf, int b, int jt0, int bt0) {
+    const int lane = threadIdx.x & 31, n = A.n, nn = n * n;
+    const size_t row = (size_t)b * A.T;
+    for (int e = lane; e < kDswBlk * nn; e += 32) {
+        const int tt = jt0 + e / nn;
+        cp_async4(buf + e, A.J + (row + min(tt, A.T - 1)) * nn + e % nn, tt < A.T);
+    }
+    for (int e = lane; e < kDswBlk * n; e += 32) {
+        const int tt = bt0 + e / n;
+        cp_async4(buf + kDswBlk * nn + e, A.b + (row + min(tt, A.T - 1)) * n + e % n, tt < A.T);
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+
+__global__ void __launch_bounds__(kDswWarps * 32) dense_scan_warp_kernel(const DScanArgs A) {
+    extern __shared__ __align__(16) float dsw_smem[];
+    const int lane = threadIdx.x & 31, r = lane >> 2, c = (lane & 3) * 2, n = A.n, nn = n * n;
+    float *const buf0 = dsw_smem + (threadIdx.x >> 5) * 2 * kDswBuf;
+    const long gw = (long)blockIdx.x * kDswWarps + (threadIdx.x >> 5);
+    const long nwarps = (long)gridDim.x * kDswWarps;
+    const int nchunk = (A.T + kDsw - 1) / kDsw;
+    const long nseq = A.B;
+    const long ntiles = nseq * nchunk;
+    const unsigned epoch = A.epoch0 + 1u;
+    for (long tile = gw; tile < ntiles; tile += nwarps) {
+        const int chunk = (int)(tile / nseq), b = (int)(tile % nseq);  // scan order
+        const int tch = A.reverse ? nchunk - 1 - chunk : chunk;
+        const int tbeg = tch * kDsw;
+        const int steps = min(kDsw, A.T - tbeg);
+        const int nblk = (steps + kDswBlk - 1) / kDswBlk;
+        // block j covers scan steps 32 j .. 32 j + 31; their times form one run
+        auto blk_t0 = [&](int j) {  // smallest time of block j
+            return A.reverse ? tbeg + steps - min(steps, kDswBlk * (j + 1)) : tbeg + kDswBlk * j;
+        };
+        auto stage = [&](int j) {
+            const int t0 = blk_t0(j);
+            dsw_stage(A, buf0 + (j & 1) * kDswBuf, b, A.reverse ? t0 + 1 : t0, t0);
+        };
+        // M_t row r (entries k < n) and b_t[r] of scan step i, from the staged block
+        auto row_of = [&](int i, float *m, float &bt) {
+            const int j = i / kDswBlk, t = A.reverse ? tbeg + steps - 1 - i : tbeg + i;
+            const int t0 = blk_t0(j);
+            const float *bf = buf0 + (j & 1) * kDswBuf;
+#pragma unroll
+            for (int k = 0; k < 8; ++k) m[k] = 0.f;
+            bt = 0.f;
+            if (r >= n) return;
+            bt = bf[kDswBlk * nn + (t - t0) * n + r];
+            if (!A.reverse) {
+                const float *J = bf + (t - t0) * nn + r * n;
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    if (k < n) m[k] = J[k];
+            } else if (t + 1 < A.T) {  // row r of J_{t+1}^T
+                const float *J = bf + (t + 1 - (t0 + 1)) * nn + r;
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    if (k < n) m[k] = J[k * n];
+            } else {
+                m[r] = 1.f;
+            }
+        };
+        // walk 1: the chunk map x -> P x + D
+        float p0 = (r == c) ? 1.f : 0.f, p1 = (r == c + 1) ? 1.f : 0.f, d = 0.f;
+        stage(0);
+        for (int j = 0; j < nblk; ++j) {
+            if (j + 1 < nblk) {
+                stage(j + 1);
+                asm volatile("cp.async.wait_group 1;" ::: "memory");
+            } else {
+                asm volatile("cp.async.wait_group 0;" ::: "memory");
+            }
+            __syncwarp();
+            const int iend = min(steps, kDswBlk * (j + 1));
+            for (int i = kDswBlk * j; i < iend; ++i) {
+                float m[8], bt;
+                row_of(i, m, bt);
+                float q0 = 0.f, q1 = 0.f, qd = bt;
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    q0 = fmaf(m[k], __shfl_sync(0xffffffffu, p0, 4 * k + (lane & 3)), q0);
+                    q1 = fmaf(m[k], __shfl_sync(0xffffffffu, p1, 4 * k + (lane & 3)), q1);
+                    qd = fmaf(m[k], __shfl_sync(0xffffffffu, d, 4 * k), qd);
+                }
+                p0 = q0;
+                p1 = q1;
+                d = qd;
+            }
+            __syncwarp();  // the buffer of block j is refilled by stage(j + 2)
+        }
+        // carry entering the tile, then publish this tile's inclusive value
+        float cv = 0.f;
+        int bad = 0;
+        if (lane < 8) {
+            if (chunk == 0) {
+                cv = (A.h0 && lane < n) ? A.h0[(size_t)b * n + lane] : 0.f;
+            } else if (!wait_word(A.inc + (tile - nseq) * 8 + lane, epoch, &cv, A.ctl, A.sticky, A.dbg)) {
+                bad = 1;
+            }
+        }
+        if (__any_sync(0xffffffffu, bad)) return;  // a bounded wait ran out; the status says so
+        const float c0 = __shfl_sync(0xffffffffu, cv, c), c1 = __shfl_sync(0xffffffffu, cv, c + 1);
+        float inc = fmaf(p0, c0, p1 * c1);
+        inc += __shfl_xor_sync(0xffffffffu, inc, 1);
+        inc += __shfl_xor_sync(0xffffffffu, inc, 2);
+        inc += d;
+        if ((lane & 3) == 0 && A.dbg.skip_tile != tile) st_relaxed_u64(A.inc + tile * 8 + r, pack_tag(inc, epoch));
+        // walk 2: the outputs from the carry
+        float v = __shfl_sync(0xffffffffu, cv, r);  // v[r], replicated over the row's lanes
+        stage(0);
+        for (int j = 0; j < nblk; ++j) {
+            if (j + 1 < nblk) {
+                stage(j + 1);
+                asm volatile("cp.async.wait_group 1;" ::: "memory");
+            } else {
+                asm volatile("cp.async.wait_group 0;" ::: "memory");
+            }
+            __syncwarp();
+            const int iend = min(steps, kDswBlk * (j + 1));
+            for (int i = kDswBlk * j; i < iend; ++i) {
+                const int t = A.reverse ? tbeg + steps - 1 - i : tbeg + i;
+                float m[8], bt;
+                row_of(i, m, bt);
+                float q = bt;
+#pragma unroll
+                for (int k = 0; k < 8; ++k) q = fmaf(m[k], __shfl_sync(0xffffffffu, v, 4 * k), q);
+                v = q;
+                if ((lane & 3) == 0 && r < n) A.out[((size_t)b * A.T + t) * n + r] = v;
+            }
+            __syncwarp();
+        }
+    }
+}
+
 // ------------------------------------------------------------------ host side
 namespace {
 
@@ -922,6 +1075,24 @@ cudaError_t newton_tanh_launch(const NewtonTanhReq &r, const Plan &plan, const W
 int scan_dense_plan(const ScanReq &r, int num_sms, Plan *plan) {
     if (r.N > 64) return 1;
     const int N = pad_n(r.N);
+    if (N == 8) {  // one warp per tile
+        plan->kernel = reinterpret_cast<const void *>(&dense_scan_warp_kernel);
+        plan->dyn_smem = kDswWarps * 2 * kDswBuf * (int)sizeof(float);
+        if (cudaFuncSetAttribute(plan->kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, plan->dyn_smem) !=
+            cudaSuccess)
+            return -1;
+        plan->ntiles = (long)r.B * ((r.T + kDsw - 1) / kDsw);
+        plan->C = N;
+        plan->agg_words = 0;
+        plan->inc_words = (size_t)plan->ntiles * 8;
+        plan->side_bytes = 0;
+        plan->epochs = 2;
+        plan->variant = 1008;
+        plan->threads = kDswWarps * 32;
+        const long ctas = (plan->ntiles + kDswWarps - 1) / kDswWarps;
+        plan->grid = occupancy_grid(plan->kernel, plan->threads, plan->dyn_smem, num_sms, ctas);
+        return plan->grid > 0 ? 0 : -1;
+    }
     size_t sm = 0;
     const void *kern = nullptr;
     int TCH = 0;
@@ -965,7 +1136,7 @@ cudaError_t scan_dense_launch(const ScanReq &r, const Plan &plan, const Work &w,
     A.dbg.delta_log_cap = 0;
     A.dbg.no_halo = 1;
     void *args[] = {&A};
-    return cudaLaunchCooperativeKernel(plan.kernel, dim3(plan.grid), dim3(kThreads), args, plan.dyn_smem, st);
+    return cudaLaunchCooperativeKernel(plan.kernel, dim3(plan.grid), dim3(plan.threads), args, plan.dyn_smem, st);
 }
 
 }  // namespace prn

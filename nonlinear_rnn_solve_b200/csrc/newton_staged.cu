@@ -174,7 +174,7 @@ template <class Cell, int LL, int NT> struct Wide {
 
 // One tile's compute phase: f, J and the residual for the thread's L steps, read from
 // the staged slab.  FULL: every step lies inside the sequence (no guards).
-template <class Cell, class Lay, int IN, bool FULL>
+template <class Cell, class Lay, int IN, bool FULL, bool JM>
 __device__ __forceinline__ void tile_compute(const NewtonDiagArgs &A, float *smem, const Cell &cell, int s, int c,
                                              int t0, int k, float *hp, const float (&wz)[3][IN > 0 ? IN : 1],
                                              const float (&bz)[3], float (&Jr)[Lay::L][Cell::S * Cell::S],
@@ -207,7 +207,7 @@ __device__ __forceinline__ void tile_compute(const NewtonDiagArgs &A, float *sme
                 cell.eval_pre(p, hp, f, J);  // p was formed with the prescaled weights
             else
                 cell.eval(p, hp, f, J);
-            apply_jmode<S>(A.jmode, J);
+            if (JM) apply_jmode<S>(A.jmode, J);  // JM: a linearisation other than the Jacobian
 #pragma unroll
             for (int q = 0; q < S; ++q) {
                 rr[i][q] = v ? f[q] - cur[q] : 0.f;
@@ -353,7 +353,7 @@ __global__ void __launch_bounds__(NT, MINB)
         int par = 0;                    // tile parity within the iteration
         int fl_b = -1, fl_ct = 0, fl_t = 0;  // staged results still to be written (previous tile)
         for (long tile = blockIdx.x; tile < ntiles; tile += gridDim.x, advance(chunk, seq), par ^= 1) {
-            ScanSmem<S, C, NT> &sm = sm2[par];
+            ScanSmem<S, C, NT> &sm = sm2[Lay::kTma ? par : 0];  // cp.async layouts keep a barrier after the scan
             const int b = C == 1 ? seq : seq / nct;
             const int ct = C == 1 ? 0 : seq % nct;
             const int h = ct * C + c;
@@ -440,10 +440,20 @@ __global__ void __launch_bounds__(NT, MINB)
                 }
             }
             float Jr[L][S * S], rr[L][S], hc[L][S];
-            if (tch0 + TCH <= A.T)
-                tile_compute<Cell, Lay, IN, true>(A, smem, cell, s, c, t0, k, hp, wz, bz, Jr, rr, hc);
-            else
-                tile_compute<Cell, Lay, IN, false>(A, smem, cell, s, c, t0, k, hp, wz, bz, Jr, rr, hc);
+            // the tile-uniform choices (whole tile inside the sequence, linearisation)
+            // select code paths here, not per step
+            const bool full = tch0 + TCH <= A.T;
+            if (A.jmode == 0) {
+                if (full)
+                    tile_compute<Cell, Lay, IN, true, false>(A, smem, cell, s, c, t0, k, hp, wz, bz, Jr, rr, hc);
+                else
+                    tile_compute<Cell, Lay, IN, false, false>(A, smem, cell, s, c, t0, k, hp, wz, bz, Jr, rr, hc);
+            } else {
+                if (full)
+                    tile_compute<Cell, Lay, IN, true, true>(A, smem, cell, s, c, t0, k, hp, wz, bz, Jr, rr, hc);
+                else
+                    tile_compute<Cell, Lay, IN, false, true>(A, smem, cell, s, c, t0, k, hp, wz, bz, Jr, rr, hc);
+            }
             const long next = tile + gridDim.x;
             auto refill = [&]() {
                 if (next < ntiles) {
@@ -452,11 +462,6 @@ __global__ void __launch_bounds__(NT, MINB)
                     issue(nch, nsq, k > 0);
                 }
             };
-            if (!Lay::kTma) {
-                // cp.async layouts: refill as soon as every thread is done with the stage
-                __syncthreads();
-                refill();
-            }
             Aff<S> e = Aff<S>::ident();
 #pragma unroll
             for (int i = 0; i < L; ++i) e = compose(e, make_aff<S>(Jr[i], rr[i]));
@@ -466,8 +471,8 @@ __global__ void __launch_bounds__(NT, MINB)
                 drain();
                 return;  // a bounded wait ran out; the status says so
             }
-            // TMA: past the barrier every thread is done reading the stage: refill it
-            if (Lay::kTma) refill();
+            // past the barrier every thread is done reading the stage: refill it
+            refill();
             // the previous tile's staged results (written before the barrier) leave now
             if (fl_b >= 0) Lay::flush(A, smem + (par ^ 1) * Lay::OUT_STRIDE, fl_b, fl_ct, fl_t);
             // carry entering the tile: from the halo when its composed map is constant
@@ -547,6 +552,12 @@ __global__ void __launch_bounds__(NT, MINB)
             fl_b = b;
             fl_ct = ct;
             fl_t = tch0;
+            if (!Lay::kTma && next >= ntiles) {
+                // cp.async layouts: prefetch this CTA's first tile for the next iteration
+                // (their stores went straight to h; the barrier orders them before the copies)
+                __syncthreads();
+                issue(first_ch, first_sq, true);
+            }
         }
         // the last tile's staged results
         __syncthreads();
@@ -555,7 +566,7 @@ __global__ void __launch_bounds__(NT, MINB)
         if (tid == 0) atomicMax(&A.ctl->delta_bits[k % 3], bits);
         // prefetch this CTA's first tile for the next iteration: past the barriers of the
         // block max, all of this CTA's stores to it are done (no other CTA writes it)
-        issue(first_ch, first_sq, true);
+        if (Lay::kTma) issue(first_ch, first_sq, true);
         if (!grid_sync(A.ctl, A.sticky, A.dbg)) {
             drain();
             return;

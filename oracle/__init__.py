@@ -7,8 +7,9 @@ the CUDA library: the two share only the seeded input generator.
 
 The arithmetic lives in ``oracle.c`` (plain C, fp64, sequential in time, OpenMP
 only over independent sequences).  This module marshals numpy arrays into it
-and holds the one step that is a library primitive: the input projection
-``x W^T + bias`` as a float64 numpy matmul.
+and holds the two steps that are library primitives: the input projection
+``x W^T + bias`` as a float64 numpy matmul, and the matrix exponential that
+discretises a linear ODE over one step (``scipy.linalg.expm``).
 
 Every function here is pinned by the CPU tests against something other than
 itself (PyTorch's reference GRU/LSTM/RNN cells, autograd Jacobians, dense
@@ -228,3 +229,66 @@ def linear_scan(kind, J, b, h0=None, reverse=False):
                               ctypes.c_int(int(bool(reverse))))
     assert rc == 0
     return out
+
+
+LSIM_INTERP = {"zoh": 0, "foh": 1}
+
+
+def lsim_discretize(A, B, h, interp="zoh"):
+    """One step of the linear ODE dx/dt = A x + B u, exact for an input held constant
+    over the step ("zoh") or varying linearly between samples ("foh"): returns
+    (Ad, G0, G1) with x_{k+1} = Ad x_k + G0 u_k + G1 u_{k+1}.
+
+    ("Para-Seq" README, Quick example: ``lsim(A, B, C, D, U, t)`` on a fixed-step time
+    grid; the pages name no hold rule, and these are the two exact ones.)  Both come
+    from one exponential of a block upper-triangular matrix (Van Loan's construction):
+      zoh: expm([[A h, B h], [0, 0]])            = [[Ad, P0], [0, I]]
+      foh: expm([[A h, B h, 0], [0, 0, I], [0, 0, 0]]) = [[Ad, P0, P1], [0, I, I], [0, 0, I]]
+    with P0 = int_0^h e^{A s} ds B and P1 = int_0^h e^{A s} (h - s)/h ds B.  A held
+    input gives G0 = P0, G1 = 0; a linear one u(t_k + s) = u_k + (s/h)(u_{k+1} - u_k)
+    gives G0 = P0 - P1, G1 = P1.
+    """
+    import scipy.linalg
+
+    A, B = _f64(A), _f64(B)
+    n, m = B.shape
+    if LSIM_INTERP[interp] == 0:
+        M = np.zeros((n + m, n + m))
+        M[:n, :n] = A * h
+        M[:n, n:] = B * h
+        E = scipy.linalg.expm(M)
+        return E[:n, :n].copy(), E[:n, n:].copy(), np.zeros((n, m))
+    M = np.zeros((n + 2 * m, n + 2 * m))
+    M[:n, :n] = A * h
+    M[:n, n:n + m] = B * h
+    M[n:n + m, n + m:] = np.eye(m)
+    E = scipy.linalg.expm(M)
+    P0, P1 = E[:n, n:n + m], E[:n, n + m:]
+    return E[:n, :n].copy(), (P0 - P1).copy(), P1.copy()
+
+
+def lsim(A, B, C, D, U, h, x0=None, interp="zoh"):
+    """Fixed-step linear simulation ("Para-Seq" README, Quick example): the system
+    discretised by ``lsim_discretize`` and stepped sequentially in fp64 (oracle.c).
+
+    U [T, m] or [batch, T, m]; x0 [n] or [batch, n] (zero when None).  Returns
+    (y [.., T, p], x [.., T, n]): x_0 = x0, x_k = Ad x_{k-1} + G0 u_{k-1} + G1 u_k,
+    y_k = C x_k + D u_k (D None: no feedthrough).
+    """
+    U = _f64(U)
+    single = U.ndim == 2
+    if single:
+        U = U[None]
+    Bt, T, m = U.shape
+    Ad, G0, G1 = lsim_discretize(A, B, h, interp)
+    n = Ad.shape[0]
+    C = _f64(C)
+    p = C.shape[0]
+    D = None if D is None else _f64(D)
+    if x0 is not None:
+        x0 = np.ascontiguousarray(np.broadcast_to(_f64(x0), (Bt, n)))
+    y = np.zeros((Bt, T, p))
+    x = np.zeros((Bt, T, n))
+    _L().orc_lti_sim(ctypes.c_long(Bt), ctypes.c_long(T), ctypes.c_int(n), ctypes.c_int(m), ctypes.c_int(p),
+                     _ptr(Ad), _ptr(G0), _ptr(G1), _ptr(C), _ptr(D), _ptr(U), _ptr(x0), _ptr(y), _ptr(x))
+    return (y[0], x[0]) if single else (y, x)

@@ -620,3 +620,52 @@ double orc_residual(const orc_model *m, const double *h0, const double *h)
     }
     return res;
 }
+
+/* ------------------------------------------------------------------ lsim
+ * Fixed-step simulation of a linear time-invariant system, dx/dt = A x + B u,
+ * y = C x + D u ("Para-Seq" README, Quick example and the `src.ode_solvers` row of
+ * Main features: scan-based fixed-step linear simulation).  The continuous system
+ * arrives already discretised over one step (Ad, G0, G1; see oracle/__init__.py):
+ *   x_0 = x0 (zero when absent),
+ *   x_k = Ad x_{k-1} + G0 u_{k-1} + G1 u_k      for k = 1 .. T-1,
+ *   y_k = C x_k + D u_k                          for k = 0 .. T-1.
+ * Plain sequential loop in time, OpenMP over the independent input sequences.
+ * Layouts (row-major): Ad [n,n], G0 and G1 [n,m], C [p,n], D [p,m] or NULL,
+ * U [B,T,m], x0 [B,n] or NULL, y [B,T,p], x [B,T,n] or NULL. */
+void orc_lti_sim(long B, long T, int n, int m, int p, const double *Ad, const double *G0, const double *G1,
+                 const double *C, const double *D, const double *U, const double *x0, double *y, double *x)
+{
+#pragma omp parallel for schedule(static)
+    for (long b = 0; b < B; ++b) {
+        double *cur = calloc((size_t)n, sizeof(double)), *nxt = calloc((size_t)n, sizeof(double));
+        const double *ub = U + (size_t)b * T * m;
+        if (x0)
+            for (int i = 0; i < n; ++i) cur[i] = x0[(size_t)b * n + i];
+        for (long k = 0; k < T; ++k) {
+            const double *uk = ub + (size_t)k * m;
+            if (k > 0) {
+                const double *up = uk - m;
+                for (int i = 0; i < n; ++i) {
+                    double acc = 0.0;
+                    for (int j = 0; j < n; ++j) acc += Ad[i * n + j] * cur[j];
+                    for (int q = 0; q < m; ++q) acc += G0[i * m + q] * up[q] + G1[i * m + q] * uk[q];
+                    nxt[i] = acc;
+                }
+                double *t = cur;
+                cur = nxt;
+                nxt = t;
+            }
+            for (int r = 0; r < p; ++r) {
+                double acc = 0.0;
+                for (int j = 0; j < n; ++j) acc += C[r * n + j] * cur[j];
+                if (D)
+                    for (int q = 0; q < m; ++q) acc += D[r * m + q] * uk[q];
+                y[((size_t)b * T + k) * p + r] = acc;
+            }
+            if (x)
+                for (int i = 0; i < n; ++i) x[((size_t)b * T + k) * n + i] = cur[i];
+        }
+        free(cur);
+        free(nxt);
+    }
+}

@@ -2,7 +2,8 @@
 
 Tolerance: max abs error <= 1e-5 for the fp32 linear scan.  Inputs: J ~ U(-1, 1),
 b ~ N(0, 1) (seeded), shapes spanning several tiles and a ragged tail, T = 1,
-N not a multiple of the channel tile.
+N not a multiple of the channel tile; N a multiple of 32 (the shared-memory staged
+kernel) with T ragged against its 128- and 64-step tiles and below one tile.
 """
 import numpy as np
 import pytest
@@ -37,7 +38,7 @@ def _draw(kind, B, T, N, seed, with_h0):
 
 
 SHAPES = [(1, 1, 1), (2, 5, 3), (3, 4097, 1), (2, 8193, 1), (2, 300, 33), (1, 1000, 8), (4, 1025, 2),
-          (2, 129, 64), (1, 3000, 17)]
+          (2, 129, 64), (1, 3000, 17), (2, 1000, 32), (1, 5000, 96), (3, 70, 32)]
 
 
 @pytest.mark.parametrize("kind", ["diag", "block2"])

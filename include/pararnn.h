@@ -183,6 +183,27 @@ int pararnn_newton_forward(pararnn_ctx *ctx, const float *xproj, const pararnn_p
 int pararnn_linear_scan(pararnn_ctx *ctx, int kind, const float *J, const float *b,
                         const float *h0, float *h_out, int B, int T, int N, int reverse);
 
+/* Fixed-step simulation of the linear time-invariant system dx/dt = A x + B u,
+ * y = C x + D u, by a chunked parallel scan ("Para-Seq" README, Quick example
+ * `lsim(A, B, C, D, U, t)`, and the `src.ode_solvers` row of Main features; Notes and
+ * limitations: fixed-step time grids only).  Samples t_k = t_0 + k dt, k = 0 .. T-1:
+ *   x_0 = x0 (or 0),  x_k = Ad x_{k-1} + G0 u_{k-1} + G1 u_k,  y_k = C x_k + D u_k,
+ * where one step of the ODE is solved exactly for an input held over the step
+ * (interp = 0: Ad = e^{A dt}, G0 = int_0^dt e^{A s} ds B, G1 = 0) or varying linearly
+ * between samples (interp = 1).  The discretisation runs on the device in fp64; the
+ * recurrence in fp32.
+ *   A [n, n], Bm [n, m], C [p, n], D [p, m] or NULL (no feedthrough): row-major, device
+ *   U [batch, T, m];  x0 [batch, n] or NULL;  y_out [batch, T, p];  x_out [batch, T, n]
+ *   or NULL (states not written).  All fp32 device pointers, caller-owned.
+ * 1 <= n <= 32, 1 <= m <= 16, 1 <= p <= 32, batch >= 1, T >= 1, 0 < dt finite,
+ * interp 0 or 1.  The context keeps a scratch buffer (the discretised matrices and
+ * about batch * T * n' / 31 floats of chunk states, n' = n rounded up to a power of
+ * two) for later calls.
+ * Returns EINVAL, ENOMEM or ECUDA. */
+int pararnn_lsim(pararnn_ctx *ctx, const float *A, const float *Bm, const float *C, const float *D, int n, int m,
+                 int p, const float *U, const float *x0, double dt, int interp, int batch, int T, float *y_out,
+                 float *x_out);
+
 /* Adjoint backward at the states h returned by pararnn_newton_forward, for
  * L = sum_t <grad_h_t, h_t> ("Para-Seq" README, Main features: adjoint backward with
  * reverse adjoint scans; DEER summary, Surprising findings: the backward pass is one

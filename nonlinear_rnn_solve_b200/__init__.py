@@ -47,7 +47,7 @@ EXPORTED = [
     "pararnn_create", "pararnn_destroy", "pararnn_set_stream", "pararnn_input_proj",
     "pararnn_newton_forward", "pararnn_linear_scan", "pararnn_adjoint_backward",
     "pararnn_get_status", "pararnn_strerror", "pararnn_debug_set", "pararnn_last_launch_count",
-    "pararnn_linear_scan_noalloc", "pararnn_input_proj_backward",
+    "pararnn_linear_scan_noalloc", "pararnn_input_proj_backward", "pararnn_lsim",
 ]
 
 
@@ -93,6 +93,7 @@ def lib() -> ctypes.CDLL:
         L.pararnn_last_launch_count.argtypes = [vp]
         L.pararnn_linear_scan_noalloc.argtypes = [i, vp, vp, vp, vp, i, i, i, i, vp, vp]
         L.pararnn_input_proj_backward.argtypes = [vp, vp, vp, i, vp, vp, vp, vp, i, i, i]
+        L.pararnn_lsim.argtypes = [vp, vp, vp, vp, vp, i, i, i, vp, vp, ctypes.c_double, i, i, i, vp, vp]
         for name in EXPORTED:
             if getattr(L, name).restype is None and name != "pararnn_strerror":
                 getattr(L, name).restype = i
@@ -163,6 +164,18 @@ def pararnn_input_proj(ctx, x, W, bias, xproj) -> None:
     N = W.shape[0]
     _check(lib().pararnn_input_proj(ctx, _p(x), dt, _p(W), _p(bias, torch.float32),
                                     _p(xproj, torch.float32), M, K, N), "pararnn_input_proj")
+
+
+def pararnn_lsim(ctx, A, Bm, C, D, U, x0, dt, interp, y_out, x_out) -> None:
+    """Fixed-step linear simulation: A [n,n], Bm [n,m], C [p,n], D [p,m] or None,
+    U [batch,T,m], x0 [batch,n] or None, y_out [batch,T,p], x_out [batch,T,n] or None."""
+    f32 = torch.float32
+    n, m = Bm.shape
+    p = C.shape[0]
+    batch, T = U.shape[0], U.shape[1]
+    _check(lib().pararnn_lsim(ctx, _p(A, f32), _p(Bm, f32), _p(C, f32), _p(D, f32), n, m, p, _p(U, f32),
+                              _p(x0, f32), float(dt), int(interp), batch, T, _p(y_out, f32), _p(x_out, f32)),
+           "pararnn_lsim")
 
 
 def pararnn_input_proj_backward(ctx, grad_xproj, x, W, grad_x, grad_W, grad_bias) -> None:

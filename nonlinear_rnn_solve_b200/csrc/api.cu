@@ -89,6 +89,23 @@ int prepare(pararnn_ctx *ctx, const prn::Plan &plan, prn::Work *w) {
     return PARARNN_OK;
 }
 
+// Make the plain scratch buffer at least `need` bytes (grows, never shrinks).
+int ensure_scratch(pararnn_ctx *ctx, size_t need) {
+    if (ctx->scratch_bytes >= need) return PARARNN_OK;
+    if (ctx->scratch) {
+        if (cudaStreamSynchronize(ctx->stream) != cudaSuccess) return PARARNN_ECUDA;
+        cudaFree(ctx->scratch);
+        ctx->scratch = nullptr;
+        ctx->scratch_bytes = 0;
+    }
+    if (cudaMalloc(&ctx->scratch, need) != cudaSuccess) {
+        cudaGetLastError();
+        return PARARNN_ENOMEM;
+    }
+    ctx->scratch_bytes = need;
+    return PARARNN_OK;
+}
+
 int cuda_rc(cudaError_t e) {
     if (e == cudaSuccess) return PARARNN_OK;
     cudaGetLastError();
@@ -289,23 +306,28 @@ int pararnn_input_proj_backward(pararnn_ctx *ctx, const float *grad_xproj, const
     if (!g.ok) return PARARNN_ECUDA;
     ctx->last_launches = 0;
     // a buffer of its own: the look-back workspace must only ever hold epoch-tagged words
-    const size_t need = prn::proj_bwd_scratch_bytes(x_dtype, M, K, N);
-    if (ctx->scratch_bytes < need) {
-        if (ctx->scratch) {
-            if (cudaStreamSynchronize(ctx->stream) != cudaSuccess) return PARARNN_ECUDA;
-            cudaFree(ctx->scratch);
-            ctx->scratch = nullptr;
-            ctx->scratch_bytes = 0;
-        }
-        if (cudaMalloc(&ctx->scratch, need) != cudaSuccess) {
-            cudaGetLastError();
-            return PARARNN_ENOMEM;
-        }
-        ctx->scratch_bytes = need;
-    }
+    int rc0 = ensure_scratch(ctx, prn::proj_bwd_scratch_bytes(x_dtype, M, K, N));
+    if (rc0) return rc0;
     int launches = 0;
     int rc = cuda_rc(prn::proj_bwd_launch(x_dtype, grad_xproj, x, W, grad_x, grad_W, grad_bias, M, K, N, ctx->scratch,
                                           ctx->num_sms, ctx->stream, &launches, ctx->sticky));
+    if (rc == PARARNN_OK) ctx->last_launches = launches;
+    return rc;
+}
+
+int pararnn_lsim(pararnn_ctx *ctx, const float *A, const float *Bm, const float *C, const float *D, int n, int m, int p,
+                 const float *U, const float *x0, double dt, int interp, int batch, int T, float *y_out,
+                 float *x_out) {
+    if (!ctx || !A || !Bm || !C || !U || !y_out) return PARARNN_EINVAL;
+    prn::LsimReq r{A, Bm, C, D, n, m, p, U, x0, dt, interp, batch, T, y_out, x_out};
+    if (prn::lsim_check(r)) return PARARNN_EINVAL;
+    DeviceGuard g(ctx->device);
+    if (!g.ok) return PARARNN_ECUDA;
+    ctx->last_launches = 0;
+    int rc = ensure_scratch(ctx, prn::lsim_scratch_bytes(r));
+    if (rc) return rc;
+    int launches = 0;
+    rc = cuda_rc(prn::lsim_launch(r, static_cast<float *>(ctx->scratch), ctx->stream, &launches));
     if (rc == PARARNN_OK) ctx->last_launches = launches;
     return rc;
 }

@@ -122,6 +122,21 @@ cudaError_t proj_bwd_launch(int x_dtype, const float *gx, const void *x, const v
                             int *launches, int *sticky);
 
 // Helpers.
+// Fixed-step linear simulation (lsim.cu).
+constexpr int kLsimMaxN = 32, kLsimMaxM = 16, kLsimMaxP = 32;
+struct LsimReq {
+    const float *A, *Bm, *C, *D;  // [n,n], [n,m], [p,n], [p,m] or NULL
+    int n, m, p;
+    const float *U, *x0;  // [batch,T,m], [batch,n] or NULL
+    double h;             // time step
+    int interp;           // 0 held input, 1 linear between samples
+    long batch, T;
+    float *y, *x;         // [batch,T,p], [batch,T,n] or NULL
+};
+int lsim_check(const LsimReq &r);
+size_t lsim_scratch_bytes(const LsimReq &r);
+cudaError_t lsim_launch(const LsimReq &r, float *scratch, cudaStream_t st, int *launches);
+
 int occupancy_grid(const void *kernel, int threads, size_t smem, int num_sms, long ntiles);
 
 }  // namespace prn

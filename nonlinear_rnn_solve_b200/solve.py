@@ -64,6 +64,35 @@ def input_proj_backward(ctx, grad_xproj, x, W, need_x=True, need_W=True, need_bi
     return gx, gW, gb
 
 
+def lsim(ctx, A, B, C, D, U, t, x0=None, interp="zoh", return_states=True):
+    """Fixed-step simulation of dx/dt = A x + B u, y = C x + D u on the time grid t
+    (1-D, evenly spaced; its first point is x0's time).  U [T, m] or [batch, T, m];
+    x0 [n] or [batch, n].  interp: "zoh" (input held over each step) or "foh" (linear
+    between samples).  Returns (y, x) shaped like U with m replaced by p and n (x None
+    when return_states is False)."""
+    from . import pararnn_lsim
+    single = U.dim() == 2
+    U3 = U.unsqueeze(0) if single else U
+    batch, T, _ = U3.shape
+    n, p = A.shape[0], C.shape[0]
+    tt = torch.as_tensor(t, dtype=torch.float64).cpu().reshape(-1)
+    if tt.numel() != T:
+        raise ValueError("t must have one point per input sample")
+    dt = float(tt[1] - tt[0]) if T > 1 else 1.0
+    if T > 2 and float((tt.diff() - dt).abs().max()) > 1e-6 * max(abs(dt), 1e-30) + 1e-12:
+        raise ValueError("lsim needs a fixed-step time grid")
+    if x0 is not None:
+        x0 = x0.reshape(1, n).expand(batch, n).contiguous() if x0.dim() == 1 else x0.contiguous()
+    dev = U.device
+    y = torch.empty(batch, T, p, device=dev, dtype=torch.float32)
+    x = torch.empty(batch, T, n, device=dev, dtype=torch.float32) if return_states else None
+    pararnn_lsim(ctx, A.contiguous(), B.contiguous(), C.contiguous(), None if D is None else D.contiguous(),
+                 U3.contiguous(), x0, dt, {"zoh": 0, "foh": 1}[interp], y, x)
+    if single:
+        return y[0], (None if x is None else x[0])
+    return y, x
+
+
 def linear_scan(ctx, kind, J, b, h0=None, reverse=False):
     from . import PARARNN_SCAN_BLOCK2, PARARNN_SCAN_DENSE, PARARNN_SCAN_DIAG
     k = {"diag": PARARNN_SCAN_DIAG, "block2": PARARNN_SCAN_BLOCK2, "dense": PARARNN_SCAN_DENSE}[kind]

@@ -204,6 +204,23 @@ template <> __device__ __forceinline__ Aff<2> make_aff<2>(const float *J, const 
     return {J[0], J[1], J[2], J[3], d[0], d[1]};
 }
 
+// ------------------------------------------------------------------ cp.async
+// Asynchronous copies global -> shared, 16 or 4 bytes; src_bytes 0 / valid false
+// zero-fills the destination without reading the source.
+__device__ __forceinline__ void cp_async16(float *dst, const float *src, int src_bytes) {
+    const unsigned d = (unsigned)__cvta_generic_to_shared(dst);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(d), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async4(float *dst, const float *src, bool valid) {
+    const unsigned d = (unsigned)__cvta_generic_to_shared(dst);
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(d), "l"(src), "r"(valid ? 4 : 0) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+template <int N> __device__ __forceinline__ void cp_async_wait_group() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
 // ------------------------------------------------------------------ tile walk
 // Grid-stride walk over tiles numbered tile = chunk * nseq + seq (seq fastest): the
 // coordinates advance by gridDim.x tiles per step without dividing (plans keep tile

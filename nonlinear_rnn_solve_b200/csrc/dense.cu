@@ -832,11 +832,6 @@ constexpr int kDswBlk = 32;           // steps per staged block
 constexpr int kDswWarps = 4;          // warps per CTA
 constexpr int kDswBuf = kDswBlk * 72;  // floats per staging buffer: 32 (n^2 + n), n <= 8
 
-__device__ __forceinline__ void cp_async4(float *dst, const float *src, bool valid) {
-    const unsigned d = (unsigned)__cvta_generic_to_shared(dst);
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(d), "l"(src), "r"(valid ? 4 : 0) : "memory");
-}
-
 // Stage J for times jt0 .. jt0 + 31 and b for times bt0 .. bt0 + 31 (zero beyond T).
 __device__ __forceinline__ void dsw_stage(const DScanArgs &A, float *buf, int b, int jt0, int bt0) {
     const int lane = threadIdx.x & 31, n = A.n, nn = n * n;

@@ -28,9 +28,10 @@ namespace prn {
 namespace {
 
 constexpr int kChunk = 32;     // steps per thread, every level
-constexpr int kThreadsL = 128;  // threads per CTA of the chunk passes
+constexpr int kThreadsL = 128;  // threads per CTA of the input-level passes
+constexpr int kThreadsLv = 32;  // of the upper-level passes (few threads: spread over the SMs)
 constexpr int kDiscThreads = 1024;
-constexpr int kTaylor = 14;  // degree; the scaled matrix has 1-norm <= 1/2
+constexpr int kTaylor = 10;  // degree; the scaled matrix has 1-norm <= 1/4
 
 __host__ __device__ constexpr long up4(long x) { return (x + 3) & ~3L; }
 
@@ -53,20 +54,34 @@ struct MatLayout {
 };
 
 // ------------------------------------------------------------------ discretisation (fp64)
-// Product of q x q row-major matrices in shared memory, by the whole CTA.
+// Product of q x q row-major matrices in shared memory, by the whole CTA: a 2 x 2
+// block of Z per thread (one shared load per multiply-add).
 __device__ void smem_matmul(const double *X, const double *Y, double *Z, int q) {
-    for (int idx = threadIdx.x; idx < q * q; idx += blockDim.x) {
-        const int i = idx / q, j = idx % q;
-        double acc = 0.0;
-        for (int k = 0; k < q; ++k) acc = fma(X[i * q + k], Y[k * q + j], acc);
-        Z[idx] = acc;
+    const int qb = (q + 1) / 2;
+    for (int idx = threadIdx.x; idx < qb * qb; idx += blockDim.x) {
+        const int i0 = 2 * (idx / qb), j0 = 2 * (idx % qb);
+        const int i1 = min(i0 + 1, q - 1), j1 = min(j0 + 1, q - 1);
+        double a00 = 0.0, a01 = 0.0, a10 = 0.0, a11 = 0.0;
+        for (int k = 0; k < q; ++k) {
+            const double x0 = X[i0 * q + k], x1 = X[i1 * q + k], y0 = Y[k * q + j0], y1 = Y[k * q + j1];
+            a00 = fma(x0, y0, a00);
+            a01 = fma(x0, y1, a01);
+            a10 = fma(x1, y0, a10);
+            a11 = fma(x1, y1, a11);
+        }
+        Z[i0 * q + j0] = a00;
+        if (j0 + 1 < q) Z[i0 * q + j0 + 1] = a01;
+        if (i0 + 1 < q) {
+            Z[(i0 + 1) * q + j0] = a10;
+            if (j0 + 1 < q) Z[(i0 + 1) * q + j0 + 1] = a11;
+        }
     }
     __syncthreads();
 }
 
 // One CTA: e^M for M = [[A h, B h, 0], [0, 0, I], [0, 0, 0]] (the last block row and
-// column only with the linear hold), by scaling M to 1-norm <= 1/2, a degree-14
-// Taylor polynomial in Horner form (truncation below 1e-21 relative), and squaring
+// column only with the linear hold), by scaling M to 1-norm <= 1/4, a degree-10
+// Taylor polynomial in Horner form (truncation below 1e-14 relative), and squaring
 // back (Moler and Van Loan, "Nineteen dubious ways to compute the exponential of a
 // matrix", method 3).  Then the chunk powers Ad^(32^l) by five squarings per level.
 __global__ void __launch_bounds__(kDiscThreads) lsim_discretize_kernel(const float *A, const float *Bm, const float *C,
@@ -96,7 +111,7 @@ __global__ void __launch_bounds__(kDiscThreads) lsim_discretize_kernel(const flo
         }
         int s = 0;
         double scale = 1.0;
-        while (!(nrm * scale <= 0.5) && s < 1100) {  // NaN stops at the bound
+        while (!(nrm * scale <= 0.25) && s < 1100) {  // NaN stops at the bound
             scale *= 0.5;
             ++s;
         }
@@ -202,6 +217,32 @@ __device__ __forceinline__ void mv_acc(const float *MT, const float (&x)[NP], fl
     }
 }
 
+// NP floats of a level element (16-byte aligned when NP is a multiple of 4).
+template <int NP> __device__ __forceinline__ void load_vec(const float *p, float (&v)[NP]) {
+    if constexpr (NP % 4 == 0) {
+#pragma unroll
+        for (int i = 0; i < NP; i += 4) {
+            const float4 t = *reinterpret_cast<const float4 *>(p + i);
+            v[i] = t.x;
+            v[i + 1] = t.y;
+            v[i + 2] = t.z;
+            v[i + 3] = t.w;
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < NP; ++i) v[i] = p[i];
+    }
+}
+template <int NP> __device__ __forceinline__ void store_vec(float *p, const float (&v)[NP]) {
+    if constexpr (NP % 4 == 0) {
+#pragma unroll
+        for (int i = 0; i < NP; i += 4) *reinterpret_cast<float4 *>(p + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+    } else {
+#pragma unroll
+        for (int i = 0; i < NP; ++i) p[i] = v[i];
+    }
+}
+
 struct LsimArgs {
     long B, T;      // sequences and steps of the input level
     int n, m, p, interp;
@@ -221,26 +262,76 @@ __device__ __forceinline__ void stage_mats(float *dst, const float *src, long co
     __syncthreads();
 }
 
-// One step of the input level: x <- Ad x + G0 u_{k-1} + G1 u_k (x <- x0 at k = 0).
+// The input-level passes read and write the samples through shared memory.  A CTA's
+// threads own consecutive chunks, whose steps are consecutive in the flattened
+// [batch, T] order, and the CTA walks them in sub-blocks of SB steps: per sub-block
+// it copies every chunk's SB + 1 input rows (from the step before the sub-block on;
+// consecutive threads read consecutive floats of a chunk's rows) and, in the last
+// pass, writes the SB output rows back the same way.  Row strides are odd, so threads
+// reading their own chunk's rows hit distinct banks.
+struct IoPlan {
+    int SB;          // steps per sub-block: 1, 2, 4 or 8 (divides the chunk)
+    int ustr, ystr;  // floats per chunk: input rows, output rows
+};
+
+// Per-CTA chunk table: the flattened index of each chunk's first step (b T + 32 j)
+// and its step within the sequence (32 j; -1 for a thread past the last chunk).
+struct ChunkTab {
+    long flat[kThreadsL];
+    long k0[kThreadsL];
+};
+
+__device__ __forceinline__ void fill_tab(ChunkTab &tab, bool valid, long b, long j, long T) {
+    tab.flat[threadIdx.x] = b * T + j * kChunk;
+    tab.k0[threadIdx.x] = valid ? j * kChunk : -1;
+}
+
+// Issue the copies of rows k0 + s SB - 1 .. k0 + s SB + SB - 1 of every chunk (zero
+// outside 0 <= k < T) as one commit group; consecutive threads take consecutive
+// floats of a chunk's rows.
+__device__ __forceinline__ void stage_u(const LsimArgs &A, const IoPlan &io, const ChunkTab &tab, float *su, int s) {
+    const int rows = (io.SB + 1) * A.m;
+    const float inv = 1.0f / (float)rows;  // exact quotient below: e < 2^15, rows <= 144
+    for (int e = threadIdx.x; e < kThreadsL * rows; e += kThreadsL) {
+        const int c = __float2int_rd(((float)e + 0.5f) * inv), w = e - c * rows;
+        const long k0 = tab.k0[c];
+        const long kb = k0 + (long)s * io.SB - 1;
+        const bool ok = k0 >= 0 && (long)w >= max(0L, -kb) * A.m && (long)w < (A.T - kb) * A.m;
+        const long src = (tab.flat[c] + (long)s * io.SB - 1) * A.m + w;
+        cp_async4(su + c * io.ustr + w, A.U + (ok ? src : 0), ok);
+    }
+    cp_async_commit();
+}
+
+// Write the SB output rows of every chunk's sub-block s (steps below T); consecutive
+// threads take consecutive floats of a chunk's rows.
+__device__ __forceinline__ void store_y(const LsimArgs &A, const IoPlan &io, const ChunkTab &tab, const float *sy,
+                                        int s) {
+    const int rows = io.SB * A.p;
+    const float inv = 1.0f / (float)rows;
+    for (int e = threadIdx.x; e < kThreadsL * rows; e += kThreadsL) {
+        const int c = __float2int_rd(((float)e + 0.5f) * inv), w = e - c * rows;
+        const long k0 = tab.k0[c];
+        const long kb = k0 + (long)s * io.SB;
+        if (k0 >= 0 && (long)w < (A.T - kb) * A.p) A.y[(tab.flat[c] + (long)s * io.SB) * A.p + w] = sy[c * io.ystr + w];
+    }
+}
+
+// One step of the input level, k >= 1: x <- Ad x + G0 u_{k-1} + G1 u_k (up, uk: the
+// staged rows of steps k - 1 and k).
 template <int NP>
 __device__ __forceinline__ void input_step(const LsimArgs &A, const float *sAd, const float *sG0, const float *sG1,
-                                           long b, long k, float (&x)[NP]) {
-    if (k == 0) {
-#pragma unroll
-        for (int i = 0; i < NP; ++i) x[i] = (A.x0 && i < A.n) ? A.x0[b * A.n + i] : 0.f;
-        return;
-    }
+                                           const float *up, const float *uk, float (&x)[NP]) {
     float y[NP];
 #pragma unroll
     for (int i = 0; i < NP; ++i) y[i] = 0.f;
     mv_acc<NP>(sAd, x, y);
-    const float *uk = A.U + (b * A.T + k) * A.m;
     for (int q = 0; q < A.m; ++q) {
-        const float u0 = __ldg(uk - A.m + q);
+        const float u0 = up[q];
 #pragma unroll
         for (int i = 0; i < NP; ++i) y[i] = fmaf(sG0[q * NP + i], u0, y[i]);
         if (A.interp) {
-            const float u1 = __ldg(uk + q);
+            const float u1 = uk[q];
 #pragma unroll
             for (int i = 0; i < NP; ++i) y[i] = fmaf(sG1[q * NP + i], u1, y[i]);
         }
@@ -249,30 +340,54 @@ __device__ __forceinline__ void input_step(const LsimArgs &A, const float *sAd, 
     for (int i = 0; i < NP; ++i) x[i] = y[i];
 }
 
+template <int NP>
+__device__ __forceinline__ void load_x0(const LsimArgs &A, long b, float (&x)[NP]) {
+#pragma unroll
+    for (int i = 0; i < NP; ++i) x[i] = (A.x0 && i < A.n) ? A.x0[b * A.n + i] : 0.f;
+}
+
 // Input level, first pass: each thread's chunk from a zero state (chunk 0 from x0);
 // writes the chunk's end state.
 template <int NP>
-__global__ void __launch_bounds__(kThreadsL) lsim_local0_kernel(const LsimArgs A) {
+__global__ void __launch_bounds__(kThreadsL) lsim_local0_kernel(const LsimArgs A, const IoPlan io) {
     extern __shared__ __align__(16) float sm[];
     const MatLayout Lm(NP, A.m, A.p, 0);
     stage_mats(sm, A.mats, Lm.c);
+    float *su = sm + Lm.c;
     const long nch = (A.T + kChunk - 1) / kChunk;
-    const long g = (long)blockIdx.x * blockDim.x + threadIdx.x;
-    if (g >= A.B * nch) return;
-    const long b = g / nch, j = g % nch;
+    const long g0 = (long)blockIdx.x * kThreadsL, g = g0 + threadIdx.x;
+    const bool valid = g < A.B * nch;
+    const long b = valid ? g / nch : 0, j = valid ? g % nch : 0;
+    const long k1 = valid ? min(A.T, (j + 1) * kChunk) : 0;
+    __shared__ ChunkTab tab;
+    fill_tab(tab, valid, b, j, A.T);
     float x[NP];
 #pragma unroll
     for (int i = 0; i < NP; ++i) x[i] = 0.f;
-    const long k1 = min(A.T, (j + 1) * kChunk);
-    for (long k = j * kChunk; k < k1; ++k) input_step<NP>(A, sm + Lm.ad, sm + Lm.g0, sm + Lm.g1, b, k, x);
-    float4 *o = reinterpret_cast<float4 *>(A.agg_out + g * NP);
-    if constexpr (NP % 4 == 0) {
-#pragma unroll
-        for (int i = 0; i < NP; i += 4) o[i / 4] = make_float4(x[i], x[i + 1], x[i + 2], x[i + 3]);
-    } else {
-#pragma unroll
-        for (int i = 0; i < NP; ++i) A.agg_out[g * NP + i] = x[i];
+    __syncthreads();
+    const int nsb = kChunk / io.SB;
+    stage_u(A, io, tab, su, 0);
+    for (int s = 0; s < nsb; ++s) {
+        // two input buffers: the next sub-block's copies fly during this one's steps
+        if (s + 1 < nsb) {
+            stage_u(A, io, tab, su + ((s + 1) & 1) * kThreadsL * io.ustr, s + 1);
+            cp_async_wait_group<1>();
+        } else {
+            cp_async_wait_all();
+        }
+        __syncthreads();
+        const float *row = su + (s & 1) * kThreadsL * io.ustr + threadIdx.x * io.ustr;
+        for (int i = 0; i < io.SB; ++i) {
+            const long k = j * kChunk + (long)s * io.SB + i;
+            if (k >= k1) break;
+            if (k == 0)
+                load_x0<NP>(A, b, x);
+            else
+                input_step<NP>(A, sm + Lm.ad, sm + Lm.g0, sm + Lm.g1, row + i * A.m, row + (i + 1) * A.m, x);
+        }
+        __syncthreads();
     }
+    if (valid) store_vec<NP>(A.agg_out + g * NP, x);
 }
 
 // Upper levels: elements e_k (NP floats each) with matrix P = Ad^(32^l):
@@ -281,7 +396,7 @@ __global__ void __launch_bounds__(kThreadsL) lsim_local0_kernel(const LsimArgs A
 //                      inclusive end state of the previous chunk, one level up),
 //                      written over e_k.
 template <int NP, bool FIX>
-__global__ void __launch_bounds__(kThreadsL) lsim_level_kernel(const LsimArgs A) {
+__global__ void __launch_bounds__(kThreadsLv) lsim_level_kernel(const LsimArgs A) {
     extern __shared__ __align__(16) float sm[];
     stage_mats(sm, A.mats + A.mat_pw, up4((long)NP * NP));
     const long nch = (A.T + kChunk - 1) / kChunk;
@@ -292,58 +407,99 @@ __global__ void __launch_bounds__(kThreadsL) lsim_level_kernel(const LsimArgs A)
 #pragma unroll
     for (int i = 0; i < NP; ++i) x[i] = (FIX && j > 0 && A.carry) ? A.carry[(g - 1) * NP + i] : 0.f;
     const long k1 = min(A.T, (j + 1) * kChunk);
-    for (long k = j * kChunk; k < k1; ++k) {
-        float *e = A.agg_in + (b * A.T + k) * NP;
+    float *e = A.agg_in + (b * A.T + j * kChunk) * NP;
+    float en[NP];  // the next element, loaded one step ahead
+    load_vec<NP>(e, en);
+    for (long k = j * kChunk; k < k1; ++k, e += NP) {
         float y[NP];
 #pragma unroll
-        for (int i = 0; i < NP; ++i) y[i] = e[i];
+        for (int i = 0; i < NP; ++i) y[i] = en[i];
+        if (k + 1 < k1) load_vec<NP>(e + NP, en);
         mv_acc<NP>(sm, x, y);
 #pragma unroll
         for (int i = 0; i < NP; ++i) x[i] = y[i];
-        if (FIX) {
-#pragma unroll
-            for (int i = 0; i < NP; ++i) e[i] = x[i];
-        }
+        if (FIX) store_vec<NP>(e, x);
     }
-    if (!FIX) {
-#pragma unroll
-        for (int i = 0; i < NP; ++i) A.agg_out[g * NP + i] = x[i];
-    }
+    if (!FIX) store_vec<NP>(A.agg_out + g * NP, x);
 }
 
 // Input level, last pass: each chunk from its entering state; writes y and x.
 template <int NP>
-__global__ void __launch_bounds__(kThreadsL) lsim_out_kernel(const LsimArgs A) {
+__global__ void __launch_bounds__(kThreadsL) lsim_out_kernel(const LsimArgs A, const IoPlan io) {
     extern __shared__ __align__(16) float sm[];
     const MatLayout Lm(NP, A.m, A.p, 0);
     stage_mats(sm, A.mats, Lm.pw);
+    float *su = sm + Lm.pw, *sy = su + 2 * kThreadsL * io.ustr;
     const long nch = (A.T + kChunk - 1) / kChunk;
-    const long g = (long)blockIdx.x * blockDim.x + threadIdx.x;
-    if (g >= A.B * nch) return;
-    const long b = g / nch, j = g % nch;
+    const long g0 = (long)blockIdx.x * kThreadsL, g = g0 + threadIdx.x;
+    const bool valid = g < A.B * nch;
+    const long b = valid ? g / nch : 0, j = valid ? g % nch : 0;
+    const long k1 = valid ? min(A.T, (j + 1) * kChunk) : 0;
+    float *yrow = sy + threadIdx.x * io.ystr;
+    const float *sC = sm + Lm.c, *sD = sm + Lm.d;
+    __shared__ ChunkTab tab;
+    fill_tab(tab, valid, b, j, A.T);
     float x[NP];
 #pragma unroll
-    for (int i = 0; i < NP; ++i) x[i] = (j > 0 && A.carry) ? A.carry[(g - 1) * NP + i] : 0.f;
-    const long k1 = min(A.T, (j + 1) * kChunk);
-    const float *sC = sm + Lm.c, *sD = sm + Lm.d;
-    for (long k = j * kChunk; k < k1; ++k) {
-        input_step<NP>(A, sm + Lm.ad, sm + Lm.g0, sm + Lm.g1, b, k, x);
-        const float *uk = A.U + (b * A.T + k) * A.m;
-        float *yk = A.y + (b * A.T + k) * A.p;
-        for (int r = 0; r < A.p; ++r) {
-            float acc = 0.f;
-#pragma unroll
-            for (int i = 0; i < NP; ++i) acc = fmaf(sC[r * NP + i], x[i], acc);
-            for (int q = 0; q < A.m; ++q) acc = fmaf(sD[r * A.m + q], __ldg(uk + q), acc);
-            yk[r] = acc;
+    for (int i = 0; i < NP; ++i) x[i] = (valid && j > 0 && A.carry) ? A.carry[(g - 1) * NP + i] : 0.f;
+    __syncthreads();
+    const int nsb = kChunk / io.SB;
+    stage_u(A, io, tab, su, 0);
+    for (int s = 0; s < nsb; ++s) {
+        if (s + 1 < nsb) {
+            stage_u(A, io, tab, su + ((s + 1) & 1) * kThreadsL * io.ustr, s + 1);
+            cp_async_wait_group<1>();
+        } else {
+            cp_async_wait_all();
         }
-        if (A.x) {
-            float *xk = A.x + (b * A.T + k) * A.n;
+        __syncthreads();
+        const float *row = su + (s & 1) * kThreadsL * io.ustr + threadIdx.x * io.ustr;
+        for (int i = 0; i < io.SB; ++i) {
+            const long k = j * kChunk + (long)s * io.SB + i;
+            if (k >= k1) break;
+            const float *uk = row + (i + 1) * A.m;
+            if (k == 0)
+                load_x0<NP>(A, b, x);
+            else
+                input_step<NP>(A, sm + Lm.ad, sm + Lm.g0, sm + Lm.g1, row + i * A.m, uk, x);
+            for (int r = 0; r < A.p; ++r) {
+                float acc = 0.f;
+                if constexpr (NP % 4 == 0) {
 #pragma unroll
-            for (int i = 0; i < NP; ++i)
-                if (i < A.n) xk[i] = x[i];
+                    for (int c = 0; c < NP; c += 4) {
+                        const float4 cv = lds4(sC + r * NP + c);
+                        acc = fmaf(cv.x, x[c], fmaf(cv.y, x[c + 1], fmaf(cv.z, x[c + 2], fmaf(cv.w, x[c + 3], acc))));
+                    }
+                } else {
+#pragma unroll
+                    for (int c = 0; c < NP; ++c) acc = fmaf(sC[r * NP + c], x[c], acc);
+                }
+                for (int q = 0; q < A.m; ++q) acc = fmaf(sD[r * A.m + q], uk[q], acc);
+                yrow[i * A.p + r] = acc;
+            }
+            if (A.x) {
+                float *xk = A.x + (b * A.T + k) * A.n;
+#pragma unroll
+                for (int c = 0; c < NP; ++c)
+                    if (c < A.n) xk[c] = x[c];
+            }
         }
+        __syncthreads();
+        store_y(A, io, tab, sy, s);
     }
+}
+
+// Sub-block length: the largest of 8, 4, 2, 1 steps whose staged rows (two input
+// buffers, one output buffer) fit 128 floats per chunk: 64 KB for the CTA.
+IoPlan io_plan(int m, int p) {
+    IoPlan io{1, 0, 0};
+    for (int sb = 8; sb >= 1; sb >>= 1) {
+        io.SB = sb;
+        io.ustr = ((sb + 1) * m) | 1;
+        io.ystr = (sb * p) | 1;
+        if (2 * io.ustr + io.ystr <= 128) break;
+    }
+    return io;
 }
 
 int pad_state(int n) {
@@ -397,20 +553,27 @@ cudaError_t launch_np(const LsimReq &r, float *scratch, cudaStream_t st, int *la
     A.x = r.x;
     A.mats = mats;
     A.carry = nullptr;
-    auto grid = [&](long T) { return (unsigned)((r.batch * ((T + kChunk - 1) / kChunk) + kThreadsL - 1) / kThreadsL); };
-    const size_t sm_in = (size_t)Lm.c * sizeof(float), sm_out = (size_t)Lm.pw * sizeof(float);
+    auto grid = [&](long T, int nt) { return (unsigned)((r.batch * ((T + kChunk - 1) / kChunk) + nt - 1) / nt); };
+    const IoPlan io = io_plan(r.m, r.p);
+    const size_t sm_in = (size_t)(Lm.c + 2 * kThreadsL * io.ustr) * sizeof(float);
+    const size_t sm_out = (size_t)(Lm.pw + kThreadsL * (2 * io.ustr + io.ystr)) * sizeof(float);
+    if ((e = cudaFuncSetAttribute(lsim_local0_kernel<NP>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_in)) !=
+            cudaSuccess ||
+        (e = cudaFuncSetAttribute(lsim_out_kernel<NP>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_out)) !=
+            cudaSuccess)
+        return e;
     const size_t sm_lv = (size_t)Lm.ps * sizeof(float);
     if (L > 0) {
         A.T = r.T;
         A.agg_out = agg[1];
-        lsim_local0_kernel<NP><<<grid(r.T), kThreadsL, sm_in, st>>>(A);
+        lsim_local0_kernel<NP><<<grid(r.T, kThreadsL), kThreadsL, sm_in, st>>>(A, io);
         ++nl;
         for (int l = 1; l < L; ++l) {
             A.T = Tl[l];
             A.agg_in = agg[l];
             A.agg_out = agg[l + 1];
             A.mat_pw = Lm.pw + (l - 1) * Lm.ps;
-            lsim_level_kernel<NP, false><<<grid(Tl[l]), kThreadsL, sm_lv, st>>>(A);
+            lsim_level_kernel<NP, false><<<grid(Tl[l], kThreadsLv), kThreadsLv, sm_lv, st>>>(A);
             ++nl;
         }
         for (int l = L; l >= 1; --l) {
@@ -419,13 +582,13 @@ cudaError_t launch_np(const LsimReq &r, float *scratch, cudaStream_t st, int *la
             A.agg_out = nullptr;
             A.carry = l < L ? agg[l + 1] : nullptr;
             A.mat_pw = Lm.pw + (l - 1) * Lm.ps;
-            lsim_level_kernel<NP, true><<<grid(Tl[l]), kThreadsL, sm_lv, st>>>(A);
+            lsim_level_kernel<NP, true><<<grid(Tl[l], kThreadsLv), kThreadsLv, sm_lv, st>>>(A);
             ++nl;
         }
         A.carry = agg[1];
     }
     A.T = r.T;
-    lsim_out_kernel<NP><<<grid(r.T), kThreadsL, sm_out, st>>>(A);
+    lsim_out_kernel<NP><<<grid(r.T, kThreadsL), kThreadsL, sm_out, st>>>(A, io);
     *launches = nl + 1;
     return cudaGetLastError();
 }

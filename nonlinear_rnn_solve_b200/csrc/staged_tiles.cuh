@@ -1,6 +1,5 @@
 // staged_tiles.cuh -- shared-memory staging for the long-sequence Newton kernels:
-// cp.async and TMA (cp.async.bulk.tensor, no multicast) copies with mbarrier
-// completion, the 128-byte swizzle of TMA rows, and the TmaLong tile layout (H = 1).
+// TMA (cp.async.bulk.tensor, no multicast) copies with mbarrier completion, the 128-byte swizzle of TMA rows, and the TmaLong tile layout (H = 1).
 #pragma once
 #include <cuda.h>
 
@@ -10,15 +9,6 @@
 
 namespace prn {
 
-__device__ __forceinline__ void cp_async16(float *dst, const float *src, int src_bytes) {
-    const unsigned d = (unsigned)__cvta_generic_to_shared(dst);
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(d), "l"(src), "r"(src_bytes) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
-template <int N> __device__ __forceinline__ void cp_async_wait_group() {
-    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
 
 __device__ __forceinline__ unsigned smem_addr(const void *p) { return (unsigned)__cvta_generic_to_shared(p); }
 __device__ __forceinline__ void mbar_init(unsigned long long *bar, unsigned count) {

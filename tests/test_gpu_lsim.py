@@ -3,7 +3,7 @@
 The device discretises the ODE in fp64 and runs the recurrence in fp32.  With the
 contraction rate rho = |e^{A h}| < 1, each step's rounding (about (n + m) 2^-24 of the
 state) is damped geometrically, so the accumulated error stays below
-(n + m) 2^-24 max|x| / (1 - rho); the systems here have 1 - rho >= 0.04, which bounds
+(n + m) 2^-24 max|x| / (1 - rho); the systems here have 1 - rho >= 0.03, which bounds
 it by 1e-4 x max(1, max|y|), the bar used (an integrator, rho = 1, grows T 2^-24 and
 stays inside it at T = 1025).  Shapes: T = 1 and T against the 32-step chunk (31, 33,
 1025; 40000 = three chunk levels), state sizes padded 1 -> 32, the largest m and p,

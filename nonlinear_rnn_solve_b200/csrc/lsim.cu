@@ -489,15 +489,18 @@ __global__ void __launch_bounds__(kThreadsL) lsim_out_kernel(const LsimArgs A, c
     }
 }
 
+#ifndef PRN_LSIM_IO_FLOATS
+#define PRN_LSIM_IO_FLOATS 64
+#endif
 // Sub-block length: the largest of 8, 4, 2, 1 steps whose staged rows (two input
-// buffers, one output buffer) fit 128 floats per chunk: 64 KB for the CTA.
+// buffers, one output buffer) fit PRN_LSIM_IO_FLOATS floats per chunk.
 IoPlan io_plan(int m, int p) {
     IoPlan io{1, 0, 0};
     for (int sb = 8; sb >= 1; sb >>= 1) {
         io.SB = sb;
         io.ustr = ((sb + 1) * m) | 1;
         io.ystr = (sb * p) | 1;
-        if (2 * io.ustr + io.ystr <= 128) break;
+        if (2 * io.ustr + io.ystr <= PRN_LSIM_IO_FLOATS) break;
     }
     return io;
 }

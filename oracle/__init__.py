@@ -98,7 +98,6 @@ class Model:
         self.quasi = bool(quasi)
         self.S = 2 if cell == "lstm" else 1
         self.solver = solver
-        assert solver != "elk" or cell in ("gru", "lstm"), "ELK here: diagonal linearisations of GRU/LSTM"
         self.damping = float(damping)
         self._m = _Model(CELL_IDS[cell], int(self.quasi), B, T, H, _ptr(self.xproj),
                          _ptr(self.a), _ptr(self.peep), _ptr(self.A), self.SOLVERS[solver],

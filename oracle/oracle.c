@@ -54,7 +54,8 @@ typedef struct {
     int solver;          /* linearisation used by orc_newton: ORC_NEWTON (the cell's
                           * Jacobian, or its diagonal with quasi), ORC_JACOBI (J = 0),
                           * ORC_PICARD (J = I) ["Para-Seq" README, Main features], or
-                          * ORC_ELK (diagonal Jacobian, damped step, see orc_newton) */
+                          * ORC_ELK (diagonal Jacobian, damped step, see orc_newton;
+                          * for the tanh RNN the diagonal of its dense Jacobian) */
     double lambda;       /* ELK damping (>= 0; 0 gives the quasi-Newton step) */
 } orc_model;
 
@@ -317,7 +318,44 @@ int orc_newton(const orc_model *m, const double *h0, int max_iters, double tol, 
     int iters = 0;
     for (int k = 0; k < max_iters; ++k) {
         double delta = 0.0;
-        if (m->cell == ORC_TANH) {
+        if (m->cell == ORC_TANH && m->solver == ORC_ELK) {
+            /* quasi-ELK for the dense tanh RNN: the diagonal of its Jacobian at h^(k),
+             * then the same per-unit Kalman smoother as the diagonal cells below */
+            long n = H;
+#pragma omp parallel for schedule(dynamic, 1) reduction(max : delta)
+            for (long b = 0; b < B; ++b) {
+                double *J = malloc(sizeof(double) * n * n), *f = malloc(sizeof(double) * n);
+                double *a = malloc(sizeof(double) * n * T), *r = malloc(sizeof(double) * n * T);
+                double *xs = malloc(sizeof(double) * T), *work = malloc(sizeof(double) * 5 * T);
+                double *z0 = calloc(n, sizeof(double));
+                const double *pk = h0 ? h0 + b * n : z0; /* h^(k)_{t-1} */
+                for (long t = 0; t < T; ++t) {
+                    tanh_step(m, m->xproj + (b * T + t) * n, pk, f, J);
+                    for (long i = 0; i < n; ++i) {
+                        a[i * T + t] = J[i * n + i];
+                        r[i * T + t] = f[i] - hk[(b * T + t) * n + i];
+                    }
+                    pk = hk + (b * T + t) * n;
+                }
+                double dloc = 0.0;
+                for (long i = 0; i < n; ++i) {
+                    elk_component(T, a + i * T, r + i * T, m->lambda, xs, work);
+                    for (long t = 0; t < T; ++t) {
+                        long idx = (b * T + t) * n + i;
+                        hn[idx] = hk[idx] + xs[t];
+                        dloc = absmax_update(dloc, xs[t]);
+                    }
+                }
+                if (dloc > delta) delta = dloc;
+                free(J);
+                free(f);
+                free(a);
+                free(r);
+                free(xs);
+                free(work);
+                free(z0);
+            }
+        } else if (m->cell == ORC_TANH) {
             long n = H;
 #pragma omp parallel for schedule(dynamic, 1) reduction(max : delta)
             for (long b = 0; b < B; ++b) {

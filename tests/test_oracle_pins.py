@@ -355,7 +355,7 @@ def _lm_stacked(lib, xp, h0, iters, lam, state_shape):
     return out
 
 
-@pytest.mark.parametrize("cell", ["gru", "lstm"])
+@pytest.mark.parametrize("cell", ["gru", "lstm", "tanh"])
 @pytest.mark.parametrize("lam", [0.3, 2.0])
 def test_elk_step_is_levenberg_marquardt_on_stacked_system(cell, lam):
     """The Kalman-smoother step equals the dense Levenberg-Marquardt step."""
@@ -369,7 +369,7 @@ def test_elk_step_is_levenberg_marquardt_on_stacked_system(cell, lam):
         np.testing.assert_allclose(h, ref.numpy(), atol=1e-11)
 
 
-@pytest.mark.parametrize("cell", ["gru", "lstm"])
+@pytest.mark.parametrize("cell", ["gru", "lstm", "tanh"])
 def test_elk_without_damping_is_the_diagonal_newton_step(cell):
     m, xp, prm, h0 = _rand_model(cell, B=2, T=30, H=4, seed=72)
     e = oracle.Model(cell, xp, solver="elk", damping=0.0, **prm)
@@ -379,7 +379,7 @@ def test_elk_without_damping_is_the_diagonal_newton_step(cell):
                                    atol=1e-12)
 
 
-@pytest.mark.parametrize("cell", ["gru", "lstm"])
+@pytest.mark.parametrize("cell", ["gru", "lstm", "tanh"])
 def test_elk_converges_to_rollout_and_damping_shortens_steps(cell):
     m, xp, prm, h0 = _rand_model(cell, B=2, T=40, H=4, seed=73, scale=1.5)
     R = m.rollout(h0)

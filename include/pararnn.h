@@ -108,7 +108,8 @@ typedef enum {
      * the Levenberg-Marquardt step of the stacked system, i.e. the minimiser of
      * sum_t |x_t - J_t x_{t-1} - r_t|^2 + damping sum_t |x_t|^2 (x = h^(k+1) - h^(k),
      * r_t = f_t - h^(k)_t), computed by a parallel Kalman filter and smoother; J_t is
-     * diagonal: ParaGRU (ELK) and ParaLSTM with each block's diagonal (quasi-ELK).
+     * diagonal: ParaGRU (ELK), ParaLSTM with each block's diagonal and the tanh RNN
+     * (either tanh cell id, n <= 64) with the diagonal of its Jacobian (quasi-ELK).
      * damping = 0 gives the quasi-Newton step; larger damping shortens the steps. */
     PARARNN_SOLVER_ELK = 3
 } pararnn_solver;

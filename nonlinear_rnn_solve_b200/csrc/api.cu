@@ -195,13 +195,14 @@ int pararnn_newton_forward(pararnn_ctx *ctx, const float *xproj, const pararnn_p
                          : prn::newton_diag_launch(r, plan, w, ctx->dbg, ctx->stream));
     } else if (p->cell == PARARNN_RNN_TANH_DENSE || p->cell == PARARNN_RNN_TANH_QUASI) {
         if (!p->A) return PARARNN_EINVAL;
-        if (p->solver == PARARNN_SOLVER_ELK) return PARARNN_EUNSUPPORTED;
         if (p->H > 64) return PARARNN_EUNSUPPORTED;
-        // Jacobi and Picard have diagonal linearisations: they run on the quasi (diagonal) kernel
+        // Jacobi and Picard have diagonal linearisations: they run on the quasi (diagonal)
+        // kernel; ELK takes the diagonal of the Jacobian for either cell (quasi-ELK)
+        const bool elk = p->solver == PARARNN_SOLVER_ELK;
         const int quasi = p->cell == PARARNN_RNN_TANH_QUASI || jm_solver != 0;
         prn::NewtonTanhReq r{quasi, jm_solver, p->B, p->T, p->H, p->in, xproj, p->x, p->W,
                              p->bias, p->A, h0, h_out, max_iters, tol, iters_out, final_delta_out, residual_out};
-        int prc = prn::newton_tanh_plan(r, ctx->num_sms, &plan);
+        int prc = elk ? prn::elk_tanh_plan(r, ctx->num_sms, &plan) : prn::newton_tanh_plan(r, ctx->num_sms, &plan);
         if (prc == 1) return PARARNN_EUNSUPPORTED;
         if (prc) return PARARNN_ECUDA;
         if ((rc = prepare(ctx, plan, &w))) return rc;
@@ -209,7 +210,8 @@ int pararnn_newton_forward(pararnn_ctx *ctx, const float *xproj, const pararnn_p
             const size_t n = (size_t)p->B * p->T * p->H;
             if (cudaMemsetAsync(h_out, 0, n * sizeof(float), ctx->stream) != cudaSuccess) return PARARNN_ECUDA;
         }
-        rc = cuda_rc(prn::newton_tanh_launch(r, plan, w, ctx->dbg, ctx->stream));
+        rc = cuda_rc(elk ? prn::elk_tanh_launch(r, p->damping, plan, w, ctx->dbg, ctx->stream)
+                         : prn::newton_tanh_launch(r, plan, w, ctx->dbg, ctx->stream));
     } else {
         return PARARNN_EINVAL;
     }

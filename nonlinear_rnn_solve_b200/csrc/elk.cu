@@ -2,7 +2,8 @@
 // the damped step computed by parallel Kalman smoothing ("Towards Scalable and Stable
 // Parallelization of Nonlinear RNNs", Abstract; "Para-Seq" README, Main features: ELK
 // and quasi-ELK), for the diagonal linearisations: ParaGRU (its Jacobian is diagonal)
-// and the ParaLSTM with each 2x2 block reduced to its diagonal (quasi-ELK).
+// the ParaLSTM with each 2x2 block reduced to its diagonal, and the dense tanh RNN with
+// the diagonal of its Jacobian (quasi-ELK).
 //
 // Every state component is a scalar channel (LSTM: c and h of a unit are two channels).
 // With a_t the diagonal Jacobian entry, r_t = f_t - h^(k)_t and x = h^(k+1) - h^(k), the
@@ -24,6 +25,7 @@
 #include <string.h>
 
 #include <algorithm>
+#include <type_traits>
 
 #include "cells.cuh"
 #include "common.cuh"
@@ -95,13 +97,62 @@ struct ElkArgs {
     NewtonDiagArgs A;
     float lambda;
     float *sa, *sr, *sP, *sm;  // [B, T, D] scratch, D = H * S
+    const float *Amat;         // tanh RNN: recurrent matrix [n, n] (A.H = n)
 };
+
+// Cell tag of the dense tanh RNN, h_t = tanh(A h_{t-1} + p_t): its linearisation (the
+// Jacobian's diagonal (1 - f^2) A_ii and r = f - h^(k)) needs the whole state row, so
+// a pass over rows writes a and r to the scratch before the scans read them.
+struct TanhLin {
+    static constexpr int S = 1;
+};
+constexpr int kElkMaxN = 64;
+
+// The tanh RNN at the iterate in h (k = 0: h^(0) = 0): per row (b, t) and unit i,
+// f = tanh(p_t + sum_j A_ij h_{t-1,j}); writes a = (1 - f^2) A_ii and r = f - h_t, or
+// (residual) folds |h_t - f| into my_max.  sAt: A transposed in shared memory.
+// IN = 0: p from xproj [B, T, n]; IN = -1: p = bias + W x_t (W [n, in], in <= 8).
+template <int IN>
+__device__ void tanh_lin_pass(const ElkArgs &E, const float *sAt, int k, bool residual, float &my_max) {
+    const NewtonDiagArgs &A = E.A;
+    const int n = A.H;
+    const int rpc = kThreads / n;  // rows per CTA and pass
+    const int lr = threadIdx.x / n, i = threadIdx.x - lr * n;
+    const long nrows = (long)A.B * A.T;
+    const bool have_h = k > 0 || residual;
+    for (long row0 = (long)blockIdx.x * rpc; row0 < nrows; row0 += (long)gridDim.x * rpc) {
+        const long row = row0 + lr;
+        if (lr >= rpc || row >= nrows) continue;
+        const long b = row / A.T, t = row - b * A.T;
+        const float *hp = t == 0 ? (A.h0 ? A.h0 + b * n : nullptr) : (have_h ? A.h + (row - 1) * n : nullptr);
+        float z;
+        if (IN == 0) {
+            z = A.xproj[row * n + i];
+        } else {
+            z = A.bias ? A.bias[i] : 0.f;
+            for (int q = 0; q < A.in; ++q) z = fmaf(A.W[(size_t)i * A.in + q], A.x[row * A.in + q], z);
+        }
+        if (hp)
+            for (int j = 0; j < n; ++j) z = fmaf(sAt[j * n + i], hp[j], z);
+        const float f = tanhf(z);
+        const float cur = have_h ? A.h[row * n + i] : 0.f;
+        if (residual) {
+            const float ad = fabsf(cur - f);
+            my_max = (ad > my_max || isnan(ad)) ? ad : my_max;
+        } else {
+            E.sa[row * n + i] = (1.f - f * f) * sAt[i * n + i];
+            E.sr[row * n + i] = f - cur;
+        }
+    }
+}
 
 template <class Cell, int C, int L, int IN>
 __global__ void __launch_bounds__(kThreads, 2) elk_kernel(const ElkArgs E) {
     const NewtonDiagArgs &A = E.A;
     constexpr int S = Cell::S;
     constexpr int SUB = kThreads / C, TCH = SUB * L;
+    constexpr bool kTanh = std::is_same<Cell, TanhLin>::value;
+    __shared__ float s_At[kTanh ? kElkMaxN * kElkMaxN : 1];
     __shared__ ScanSmem<2, C, kThreads, PAff2> sm2;
     __shared__ ScanSmem<1, C> sm1;
     __shared__ unsigned s_red[kThreads / 32];
@@ -116,6 +167,8 @@ __global__ void __launch_bounds__(kThreads, 2) elk_kernel(const ElkArgs E) {
     LookBack<2> lb2{A.agg, A.inc};
     LookBack<1> lb1{A.agg, A.inc};
     if (tid == 0) s_fail = 0;
+    if (kTanh)
+        for (int e = tid; e < A.H * A.H; e += kThreads) s_At[(e % A.H) * A.H + e / A.H] = E.Amat[e];
     __syncthreads();
 
     int iters = 0;
@@ -124,6 +177,11 @@ __global__ void __launch_bounds__(kThreads, 2) elk_kernel(const ElkArgs E) {
     for (int k = 0; k < A.max_iters; ++k) {
         const unsigned ep = A.epoch0 + 3u * (unsigned)k;
         if (blockIdx.x == 0 && tid == 0) A.ctl->delta_bits[(k + 1) % 3] = 0u;
+        if constexpr (kTanh) {  // linearise the whole iterate first
+            float unused = 0.f;
+            tanh_lin_pass<IN>(E, s_At, k, false, unused);
+            if (!grid_sync(A.ctl, A.sticky, A.dbg)) return;
+        }
 
         // ---------------- phase A: linearise, filter variance
         {
@@ -134,49 +192,61 @@ __global__ void __launch_bounds__(kThreads, 2) elk_kernel(const ElkArgs E) {
                 const bool cv = ch < D;
                 const int u = cv ? ch / S : 0, q = cv ? ch % S : 0;
                 const int t0 = chunk * TCH + s * L;
-                Cell cell;
-                cell.load(A.a, A.peep, A.H, u);
-                Proj<IN> pj;
-                pj.load(A, u);
-                float hp[S];
-#pragma unroll
-                for (int j = 0; j < S; ++j) hp[j] = 0.f;
-                if (t0 == 0) {
-                    if (A.h0) load_state<S>(A.h0, (size_t)b * A.H + u, hp);
-                } else if (k > 0 && t0 - 1 < A.T) {
-                    load_state<S>(A.h, ((size_t)b * A.T + (t0 - 1)) * A.H + u, hp);
-                }
                 float av[L];
                 PAff2 e = PAff2::ident();
+                if constexpr (kTanh) {  // a_t from the linearisation pass
 #pragma unroll
-                for (int i = 0; i < L; ++i) {
-                    const int t = t0 + i;
-                    const bool v = cv && t < A.T;
-                    float p[3], cur[S], f[S], J[S * S];
-                    pj.get(b, v ? t : 0, u, p);
-#pragma unroll
-                    for (int j = 0; j < S; ++j) cur[j] = 0.f;
-                    if (k > 0 && v) load_state<S>(A.h, ((size_t)b * A.T + t) * A.H + u, cur);
-                    cell.eval(p, hp, f, J);
-                    float fq = f[0], cq = cur[0], aq = J[0];
-#pragma unroll
-                    for (int j = 1; j < S; ++j)
-                        if (q == j) {
-                            fq = f[j];
-                            cq = cur[j];
-                            aq = J[j * S + j];
-                        }
-#pragma unroll
-                    for (int j = 0; j < S; ++j) hp[j] = cur[j];
-                    av[i] = v ? aq : 0.f;
-                    if (v) {
-                        const size_t o = ((size_t)b * A.T + t) * D + ch;
-                        E.sa[o] = aq;
-                        E.sr[o] = fq - cq;
+                    for (int i = 0; i < L; ++i) {
+                        const int t = t0 + i;
+                        const bool v = cv && t < A.T;
+                        const float aq = v ? E.sa[((size_t)b * A.T + t) * D + ch] : 0.f;
+                        av[i] = aq;
+                        const float a2 = aq * aq;
+                        e = compose(e, v ? PAff2{a2, 1.f, lam * a2, lam + 1.f, 0.f, 0.f} : PAff2::ident());
                     }
-                    // M_t (identity outside the sequence)
-                    const float a2 = aq * aq;
-                    e = compose(e, v ? PAff2{a2, 1.f, lam * a2, lam + 1.f, 0.f, 0.f} : PAff2::ident());
+                } else {
+                    Cell cell;
+                    cell.load(A.a, A.peep, A.H, u);
+                    Proj<IN> pj;
+                    pj.load(A, u);
+                    float hp[S];
+#pragma unroll
+                    for (int j = 0; j < S; ++j) hp[j] = 0.f;
+                    if (t0 == 0) {
+                        if (A.h0) load_state<S>(A.h0, (size_t)b * A.H + u, hp);
+                    } else if (k > 0 && t0 - 1 < A.T) {
+                        load_state<S>(A.h, ((size_t)b * A.T + (t0 - 1)) * A.H + u, hp);
+                    }
+#pragma unroll
+                    for (int i = 0; i < L; ++i) {
+                        const int t = t0 + i;
+                        const bool v = cv && t < A.T;
+                        float p[3], cur[S], f[S], J[S * S];
+                        pj.get(b, v ? t : 0, u, p);
+#pragma unroll
+                        for (int j = 0; j < S; ++j) cur[j] = 0.f;
+                        if (k > 0 && v) load_state<S>(A.h, ((size_t)b * A.T + t) * A.H + u, cur);
+                        cell.eval(p, hp, f, J);
+                        float fq = f[0], cq = cur[0], aq = J[0];
+#pragma unroll
+                        for (int j = 1; j < S; ++j)
+                            if (q == j) {
+                                fq = f[j];
+                                cq = cur[j];
+                                aq = J[j * S + j];
+                            }
+#pragma unroll
+                        for (int j = 0; j < S; ++j) hp[j] = cur[j];
+                        av[i] = v ? aq : 0.f;
+                        if (v) {
+                            const size_t o = ((size_t)b * A.T + t) * D + ch;
+                            E.sa[o] = aq;
+                            E.sr[o] = fq - cq;
+                        }
+                        // M_t (identity outside the sequence)
+                        const float a2 = aq * aq;
+                        e = compose(e, v ? PAff2{a2, 1.f, lam * a2, lam + 1.f, 0.f, 0.f} : PAff2::ident());
+                    }
                 }
                 PAff2 excl, total;
                 cta_scan<2, C, kThreads, PAff2>(e, sm2, excl, total);
@@ -331,8 +401,22 @@ __global__ void __launch_bounds__(kThreads, 2) elk_kernel(const ElkArgs E) {
         }
         if (last_delta < A.tol) break;
     }
-    if (A.residual_out && !stop_all)
-        if (!residual_pass<Cell, C, L, IN>(A, s_red)) return;
+    if (A.residual_out && !stop_all) {
+        if constexpr (kTanh) {
+            float my_res = 0.f;
+            tanh_lin_pass<IN>(E, s_At, 1, true, my_res);
+            const unsigned bits = block_max_bits(my_res, s_red);
+            if (tid == 0) atomicMax(&A.ctl->res_bits, bits);
+            if (!grid_sync(A.ctl, A.sticky, A.dbg)) return;
+            if (blockIdx.x == 0 && tid == 0) {
+                const unsigned rb = ld_acquire(&A.ctl->res_bits);
+                *A.residual_out = __uint_as_float(rb);
+                if (rb >= 0x7f800000u) atomicOr(A.sticky, kStNonfinite);
+            }
+        } else {
+            if (!residual_pass<Cell, C, L, IN>(A, s_red)) return;
+        }
+    }
     if (blockIdx.x == 0 && tid == 0) {
         *A.iters_out = iters;
         if (A.delta_out) *A.delta_out = last_delta;
@@ -365,25 +449,90 @@ template <class Cell, int IN> const void *elk_by_C(int C) {
 
 }  // namespace
 
-int elk_plan(const NewtonDiagReq &r, int num_sms, Plan *plan) {
-    const int S = r.cell == 1 ? 2 : 1;
-    const int D = r.H * S;
-    const int C = pick_C(D);
+namespace {
+
+// Tiles, workspace and grid of an ELK solve over D scalar channels per sequence.
+int elk_plan_common(const void *kernel, long B, long T, int D, int C, int max_iters, int num_sms, Plan *plan) {
     const int TCH = (kThreads / C) * kElkL;
-    const long nseq = (long)r.B * ((D + C - 1) / C);
-    plan->ntiles = nseq * ((r.T + TCH - 1) / TCH);
-    const bool fused = r.xproj == nullptr;
-    plan->kernel = S == 1 ? (fused ? elk_by_C<GruCell, -1>(C) : elk_by_C<GruCell, 0>(C))
-                          : (fused ? elk_by_C<LstmCell, -1>(C) : elk_by_C<LstmCell, 0>(C));
+    const long nseq = B * ((D + C - 1) / C);
+    plan->ntiles = nseq * ((T + TCH - 1) / TCH);
+    plan->kernel = kernel;
     plan->variant = C;
     plan->C = C;
     plan->dyn_smem = 0;
     plan->agg_words = (size_t)plan->ntiles * C * 6;  // phase A: 2x2 blocks; B, C reuse them
     plan->inc_words = (size_t)plan->ntiles * C * 2;
-    plan->side_bytes = 4 * (size_t)r.B * r.T * D * sizeof(float);  // a, r, P, m
-    plan->epochs = 3u * (unsigned)r.max_iters + 1u;
+    plan->side_bytes = 4 * (size_t)B * T * D * sizeof(float);  // a, r, P, m
+    plan->epochs = 3u * (unsigned)max_iters + 1u;
     plan->grid = occupancy_grid(plan->kernel, kThreads, 0, num_sms, plan->ntiles);
     return plan->grid > 0 ? 0 : -1;
+}
+
+cudaError_t elk_launch_common(ElkArgs &E, long D, float lambda, const Plan &plan, const Work &w, const DbgHost &dbg,
+                              cudaStream_t st) {
+    NewtonDiagArgs &A = E.A;
+    A.ctl = w.ctl;
+    A.sticky = w.sticky;
+    A.agg = w.agg;
+    A.inc = w.inc;
+    A.side = w.side;
+    A.epoch0 = w.epoch0;
+    A.dbg.wait_ns = dbg.wait_ns;
+    A.dbg.skip_tile = dbg.skip_tile;
+    A.dbg.delta_log = dbg.delta_log;
+    A.dbg.delta_log_cap = dbg.delta_log_cap;
+    A.dbg.no_halo = 1;
+    const size_t n = (size_t)A.B * A.T * D;
+    E.lambda = lambda;
+    E.sa = w.side;
+    E.sr = w.side + n;
+    E.sP = w.side + 2 * n;
+    E.sm = w.side + 3 * n;
+    void *args[] = {&E};
+    return cudaLaunchCooperativeKernel(plan.kernel, dim3(plan.grid), dim3(kThreads), args, 0, st);
+}
+
+}  // namespace
+
+int elk_plan(const NewtonDiagReq &r, int num_sms, Plan *plan) {
+    const int S = r.cell == 1 ? 2 : 1;
+    const int D = r.H * S;
+    const int C = pick_C(D);
+    const bool fused = r.xproj == nullptr;
+    const void *k = S == 1 ? (fused ? elk_by_C<GruCell, -1>(C) : elk_by_C<GruCell, 0>(C))
+                           : (fused ? elk_by_C<LstmCell, -1>(C) : elk_by_C<LstmCell, 0>(C));
+    return elk_plan_common(k, r.B, r.T, D, C, r.max_iters, num_sms, plan);
+}
+
+int elk_tanh_plan(const NewtonTanhReq &r, int num_sms, Plan *plan) {
+    if (r.n > kElkMaxN) return 1;
+    const int C = pick_C(r.n);
+    const void *k = r.xproj ? elk_by_C<TanhLin, 0>(C) : elk_by_C<TanhLin, -1>(C);
+    return elk_plan_common(k, r.B, r.T, r.n, C, r.max_iters, num_sms, plan);
+}
+
+cudaError_t elk_tanh_launch(const NewtonTanhReq &r, float lambda, const Plan &plan, const Work &w,
+                            const DbgHost &dbg, cudaStream_t st) {
+    ElkArgs E;
+    memset(&E, 0, sizeof(E));
+    NewtonDiagArgs &A = E.A;
+    A.B = r.B;
+    A.T = r.T;
+    A.H = r.n;
+    A.in = r.in;
+    A.xproj = r.xproj;
+    A.x = r.x;
+    A.W = r.W;
+    A.bias = r.bias;
+    A.h0 = r.h0;
+    A.h = r.h;
+    A.max_iters = r.max_iters;
+    A.tol = r.tol;
+    A.iters_out = r.iters_out;
+    A.delta_out = r.delta_out;
+    A.residual_out = r.residual_out;
+    E.Amat = r.A;
+    return elk_launch_common(E, r.n, lambda, plan, w, dbg, st);
 }
 
 cudaError_t elk_launch(const NewtonDiagReq &r, float lambda, const Plan &plan, const Work &w, const DbgHost &dbg,
@@ -409,25 +558,7 @@ cudaError_t elk_launch(const NewtonDiagReq &r, float lambda, const Plan &plan, c
     A.iters_out = r.iters_out;
     A.delta_out = r.delta_out;
     A.residual_out = r.residual_out;
-    A.ctl = w.ctl;
-    A.sticky = w.sticky;
-    A.agg = w.agg;
-    A.inc = w.inc;
-    A.side = w.side;
-    A.epoch0 = w.epoch0;
-    A.dbg.wait_ns = dbg.wait_ns;
-    A.dbg.skip_tile = dbg.skip_tile;
-    A.dbg.delta_log = dbg.delta_log;
-    A.dbg.delta_log_cap = dbg.delta_log_cap;
-    A.dbg.no_halo = 1;
-    const size_t n = (size_t)r.B * r.T * r.H * (r.cell == 1 ? 2 : 1);
-    E.lambda = lambda;
-    E.sa = w.side;
-    E.sr = w.side + n;
-    E.sP = w.side + 2 * n;
-    E.sm = w.side + 3 * n;
-    void *args[] = {&E};
-    return cudaLaunchCooperativeKernel(plan.kernel, dim3(plan.grid), dim3(kThreads), args, 0, st);
+    return elk_launch_common(E, (long)r.H * (r.cell == 1 ? 2 : 1), lambda, plan, w, dbg, st);
 }
 
 }  // namespace prn

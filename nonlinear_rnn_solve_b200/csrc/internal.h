@@ -81,6 +81,10 @@ struct NewtonTanhReq {
     float *delta_out, *residual_out;
 };
 int newton_tanh_plan(const NewtonTanhReq &r, int num_sms, Plan *plan);
+// ELK for the tanh RNN (quasi-ELK: the diagonal of its Jacobian), n <= 64; 1: unsupported
+int elk_tanh_plan(const NewtonTanhReq &r, int num_sms, Plan *plan);
+cudaError_t elk_tanh_launch(const NewtonTanhReq &r, float lambda, const Plan &plan, const Work &w,
+                            const DbgHost &dbg, cudaStream_t st);
 cudaError_t newton_tanh_launch(const NewtonTanhReq &r, const Plan &plan, const Work &w,
                                const DbgHost &dbg, cudaStream_t st);
 

@@ -1,5 +1,5 @@
 """GPU parity: ELK (Levenberg-Marquardt damped Newton by parallel Kalman smoothing) for
-ParaGRU and the ParaLSTM block diagonal (quasi-ELK).
+ParaGRU, the ParaLSTM block diagonal and the tanh RNN's Jacobian diagonal (quasi-ELK).
 
 The kernel runs three scans per iteration (filter variance as a 2x2 projective scan,
 filter mean, reverse smoother).  Bars: with tol = 0 and k iterations, the iterate
@@ -7,7 +7,7 @@ within 1e-4 x max(1, |h|_max) of the oracle's (Kalman filter + RTS smoother in f
 pinned to a dense Levenberg-Marquardt solve); with a tolerance, the oracle's iteration
 count and the converged states within 1e-4.  Shapes: a single channel over many tiles
 (look-back across 32 chunks), unit counts below and above the 32-channel tile, raw
-inputs and projected inputs; two damping values.
+inputs and projected inputs, tanh state sizes 5, 8 and 64; two damping values.
 """
 import numpy as np
 import pytest
@@ -32,14 +32,16 @@ def ctx():
 
 
 def _workload(cell, B, T, H, inp, seed):
-    base = "gru_b1_t1024_in4_h8" if cell == "gru" else "lstm_b4_t8192_h1024_bf16"
+    base = {"gru": "gru_b1_t1024_in4_h8", "lstm": "lstm_b4_t8192_h1024_bf16",
+            "tanh": "tanh_b16_t65536_in4_n8_deer"}[cell]
     return wl.WORKLOADS[base].resized(B=B, T=T, H=H, inp=inp, seed=seed, bf16=False, tol=1e-5,
                                       max_iters=T + 1, w_dist="uniform_fan_in")
 
 
 def _run(ctx, cell, w, inp, lam, max_iters, tol, m=None, use_xproj=False):
     t = {k: gpu(v) for k, v in inp.items() if v is not None}
-    kw = dict(a=t["a"], peep=t.get("peep"), h0=t["h0"], max_iters=max_iters, tol=tol, solver="elk", damping=lam)
+    kw = dict(a=t.get("a"), peep=t.get("peep"), A=t.get("A"), h0=t["h0"], max_iters=max_iters, tol=tol,
+              solver="elk", damping=lam)
     if use_xproj:
         out = solve.newton_forward(ctx.ctx, cell, w.B, w.T, w.H, xproj=gpu(m.xproj.astype(np.float32)), **kw)
     else:
@@ -55,6 +57,9 @@ CASES = [  # (cell, B, T, H, in, xproj)
     ("gru", 2, 500, 64, 4, True),
     ("lstm", 2, 300, 33, 4, False),
     ("lstm", 2, 400, 64, 4, True),
+    ("tanh", 3, 700, 8, 4, False),
+    ("tanh", 2, 4096 + 33, 5, 4, False),
+    ("tanh", 2, 300, 64, 4, True),
 ]
 
 
@@ -73,7 +78,7 @@ def test_elk_iterates_match_oracle(ctx, lam, case):
         assert max_abs(host(out["h"]), h_ref) <= TOL * scale, (lam, k)
 
 
-@pytest.mark.parametrize("cell", ["gru", "lstm"])
+@pytest.mark.parametrize("cell", ["gru", "lstm", "tanh"])
 def test_elk_converges_with_oracle_iteration_count(ctx, cell):
     w = _workload(cell, 2, 700, 8, 3, seed=3)
     inp = wl.generate(w)
@@ -84,13 +89,35 @@ def test_elk_converges_with_oracle_iteration_count(ctx, cell):
     assert max_abs(host(out["h"]), h_ref) <= TOL
 
 
-def test_elk_rejects_negative_damping_and_the_dense_cell(ctx):
+def test_elk_rejects_negative_damping_and_wide_dense_cells(ctx):
     w = _workload("gru", 1, 32, 2, 2, seed=1)
     inp = wl.generate(w)
     with pytest.raises(PararnnError):
         _run(ctx, "gru", w, inp, -1.0, 3, 0.0)
-    tw = wl.WORKLOADS["tanh_b16_t65536_in4_n8_quasi"].resized(B=1, T=32)
+    tw = wl.WORKLOADS["tanh_b16_t65536_in4_n64_quasi"].resized(B=1, T=32, H=65)
     ti = {k: gpu(v) for k, v in wl.generate(tw).items() if v is not None}
     with pytest.raises(PararnnError):
         solve.newton_forward(ctx.ctx, "tanh_quasi", 1, 32, tw.H, x=ti["x"], W=ti["W"], bias=ti["bias"], A=ti["A"],
                              h0=ti["h0"], max_iters=3, tol=0.0, solver="elk", damping=1.0)
+
+
+def test_tanh_elk_residual_and_both_cell_ids(ctx):
+    """Either tanh cell id runs quasi-ELK; the residual output is max |h_t - f(h_{t-1})|
+    at the result, as the oracle computes it."""
+    w = _workload("tanh", 2, 500, 8, 4, seed=12)
+    inp = wl.generate(w)
+    m = oracle.model_from_inputs("tanh", inp, solver="elk", damping=0.7)
+    t = {k: gpu(v) for k, v in inp.items() if v is not None}
+    outs = []
+    for cell in ("tanh", "tanh_quasi"):
+        o = solve.newton_forward(ctx.ctx, cell, w.B, w.T, w.H, x=t["x"], W=t["W"], bias=t["bias"], A=t["A"],
+                                 h0=t["h0"], max_iters=4, tol=0.0, solver="elk", damping=0.7, residual=True)
+        torch.cuda.synchronize()
+        assert ctx.status() == 0
+        outs.append(o)
+    h_ref, _, _ = m.newton(inp["h0"], max_iters=4, tol=0.0)
+    for o in outs:
+        assert max_abs(host(o["h"]), h_ref) <= TOL * max(1.0, float(np.abs(h_ref).max()))
+        res = float(o["residual"].item())
+        # |residual difference| <= (1 + max_i sum_j |A_ij|) x the state difference
+        assert abs(res - m.residual(h_ref, inp["h0"])) <= 3e-4

@@ -289,15 +289,16 @@ __device__ __forceinline__ void fill_tab(ChunkTab &tab, bool valid, long b, long
 // Issue the copies of rows k0 + s SB - 1 .. k0 + s SB + SB - 1 of every chunk (zero
 // outside 0 <= k < T) as one commit group; consecutive threads take consecutive
 // floats of a chunk's rows.
-__device__ __forceinline__ void stage_u(const LsimArgs &A, const IoPlan &io, const ChunkTab &tab, float *su, int s) {
-    const int rows = (io.SB + 1) * A.m;
+__device__ __forceinline__ void stage_u(const LsimArgs &A, int m, const IoPlan &io, const ChunkTab &tab, float *su,
+                                        int s) {
+    const int rows = (io.SB + 1) * m;
     const float inv = 1.0f / (float)rows;  // exact quotient below: e < 2^15, rows <= 144
     for (int e = threadIdx.x; e < kThreadsL * rows; e += kThreadsL) {
         const int c = __float2int_rd(((float)e + 0.5f) * inv), w = e - c * rows;
         const long k0 = tab.k0[c];
         const long kb = k0 + (long)s * io.SB - 1;
-        const bool ok = k0 >= 0 && (long)w >= max(0L, -kb) * A.m && (long)w < (A.T - kb) * A.m;
-        const long src = (tab.flat[c] + (long)s * io.SB - 1) * A.m + w;
+        const bool ok = k0 >= 0 && (long)w >= max(0L, -kb) * m && (long)w < (A.T - kb) * m;
+        const long src = (tab.flat[c] + (long)s * io.SB - 1) * m + w;
         cp_async4(su + c * io.ustr + w, A.U + (ok ? src : 0), ok);
     }
     cp_async_commit();
@@ -305,32 +306,37 @@ __device__ __forceinline__ void stage_u(const LsimArgs &A, const IoPlan &io, con
 
 // Write the SB output rows of every chunk's sub-block s (steps below T); consecutive
 // threads take consecutive floats of a chunk's rows.
-__device__ __forceinline__ void store_y(const LsimArgs &A, const IoPlan &io, const ChunkTab &tab, const float *sy,
-                                        int s) {
-    const int rows = io.SB * A.p;
+__device__ __forceinline__ void store_y(const LsimArgs &A, int p, const IoPlan &io, const ChunkTab &tab,
+                                        const float *sy, int s) {
+    const int rows = io.SB * p;
     const float inv = 1.0f / (float)rows;
     for (int e = threadIdx.x; e < kThreadsL * rows; e += kThreadsL) {
         const int c = __float2int_rd(((float)e + 0.5f) * inv), w = e - c * rows;
         const long k0 = tab.k0[c];
         const long kb = k0 + (long)s * io.SB;
-        if (k0 >= 0 && (long)w < (A.T - kb) * A.p) A.y[(tab.flat[c] + (long)s * io.SB) * A.p + w] = sy[c * io.ystr + w];
+        if (k0 >= 0 && (long)w < (A.T - kb) * p) A.y[(tab.flat[c] + (long)s * io.SB) * p + w] = sy[c * io.ystr + w];
     }
 }
 
 // One step of the input level, k >= 1: x <- Ad x + G0 u_{k-1} + G1 u_k (up, uk: the
-// staged rows of steps k - 1 and k).
-template <int NP>
+// staged rows of steps k - 1 and k).  MM > 0: the input width m as a constant.
+template <int NP, int MM>
 __device__ __forceinline__ void input_step(const LsimArgs &A, const float *sAd, const float *sG0, const float *sG1,
                                            const float *up, const float *uk, float (&x)[NP]) {
+    const int m = MM > 0 ? MM : A.m;
     float y[NP];
 #pragma unroll
     for (int i = 0; i < NP; ++i) y[i] = 0.f;
     mv_acc<NP>(sAd, x, y);
-    for (int q = 0; q < A.m; ++q) {
+#pragma unroll 4
+    for (int q = 0; q < m; ++q) {
         const float u0 = up[q];
 #pragma unroll
         for (int i = 0; i < NP; ++i) y[i] = fmaf(sG0[q * NP + i], u0, y[i]);
-        if (A.interp) {
+    }
+    if (A.interp) {
+#pragma unroll 4
+        for (int q = 0; q < m; ++q) {
             const float u1 = uk[q];
 #pragma unroll
             for (int i = 0; i < NP; ++i) y[i] = fmaf(sG1[q * NP + i], u1, y[i]);
@@ -348,8 +354,9 @@ __device__ __forceinline__ void load_x0(const LsimArgs &A, long b, float (&x)[NP
 
 // Input level, first pass: each thread's chunk from a zero state (chunk 0 from x0);
 // writes the chunk's end state.
-template <int NP>
+template <int NP, int MM>
 __global__ void __launch_bounds__(kThreadsL) lsim_local0_kernel(const LsimArgs A, const IoPlan io) {
+    const int m = MM > 0 ? MM : A.m;
     extern __shared__ __align__(16) float sm[];
     const MatLayout Lm(NP, A.m, A.p, 0);
     stage_mats(sm, A.mats, Lm.c);
@@ -366,11 +373,11 @@ __global__ void __launch_bounds__(kThreadsL) lsim_local0_kernel(const LsimArgs A
     for (int i = 0; i < NP; ++i) x[i] = 0.f;
     __syncthreads();
     const int nsb = kChunk / io.SB;
-    stage_u(A, io, tab, su, 0);
+    stage_u(A, m, io, tab, su, 0);
     for (int s = 0; s < nsb; ++s) {
         // two input buffers: the next sub-block's copies fly during this one's steps
         if (s + 1 < nsb) {
-            stage_u(A, io, tab, su + ((s + 1) & 1) * kThreadsL * io.ustr, s + 1);
+            stage_u(A, m, io, tab, su + ((s + 1) & 1) * kThreadsL * io.ustr, s + 1);
             cp_async_wait_group<1>();
         } else {
             cp_async_wait_all();
@@ -383,7 +390,7 @@ __global__ void __launch_bounds__(kThreadsL) lsim_local0_kernel(const LsimArgs A
             if (k == 0)
                 load_x0<NP>(A, b, x);
             else
-                input_step<NP>(A, sm + Lm.ad, sm + Lm.g0, sm + Lm.g1, row + i * A.m, row + (i + 1) * A.m, x);
+                input_step<NP, MM>(A, sm + Lm.ad, sm + Lm.g0, sm + Lm.g1, row + i * m, row + (i + 1) * m, x);
         }
         __syncthreads();
     }
@@ -424,8 +431,9 @@ __global__ void __launch_bounds__(kThreadsLv) lsim_level_kernel(const LsimArgs A
 }
 
 // Input level, last pass: each chunk from its entering state; writes y and x.
-template <int NP>
+template <int NP, int MM, int PP>
 __global__ void __launch_bounds__(kThreadsL) lsim_out_kernel(const LsimArgs A, const IoPlan io) {
+    const int m = MM > 0 ? MM : A.m, p = PP > 0 ? PP : A.p;
     extern __shared__ __align__(16) float sm[];
     const MatLayout Lm(NP, A.m, A.p, 0);
     stage_mats(sm, A.mats, Lm.pw);
@@ -444,10 +452,10 @@ __global__ void __launch_bounds__(kThreadsL) lsim_out_kernel(const LsimArgs A, c
     for (int i = 0; i < NP; ++i) x[i] = (valid && j > 0 && A.carry) ? A.carry[(g - 1) * NP + i] : 0.f;
     __syncthreads();
     const int nsb = kChunk / io.SB;
-    stage_u(A, io, tab, su, 0);
+    stage_u(A, m, io, tab, su, 0);
     for (int s = 0; s < nsb; ++s) {
         if (s + 1 < nsb) {
-            stage_u(A, io, tab, su + ((s + 1) & 1) * kThreadsL * io.ustr, s + 1);
+            stage_u(A, m, io, tab, su + ((s + 1) & 1) * kThreadsL * io.ustr, s + 1);
             cp_async_wait_group<1>();
         } else {
             cp_async_wait_all();
@@ -457,12 +465,13 @@ __global__ void __launch_bounds__(kThreadsL) lsim_out_kernel(const LsimArgs A, c
         for (int i = 0; i < io.SB; ++i) {
             const long k = j * kChunk + (long)s * io.SB + i;
             if (k >= k1) break;
-            const float *uk = row + (i + 1) * A.m;
+            const float *uk = row + (i + 1) * m;
             if (k == 0)
                 load_x0<NP>(A, b, x);
             else
-                input_step<NP>(A, sm + Lm.ad, sm + Lm.g0, sm + Lm.g1, row + i * A.m, uk, x);
-            for (int r = 0; r < A.p; ++r) {
+                input_step<NP, MM>(A, sm + Lm.ad, sm + Lm.g0, sm + Lm.g1, row + i * m, uk, x);
+#pragma unroll 4
+            for (int r = 0; r < p; ++r) {
                 float acc = 0.f;
                 if constexpr (NP % 4 == 0) {
 #pragma unroll
@@ -474,8 +483,9 @@ __global__ void __launch_bounds__(kThreadsL) lsim_out_kernel(const LsimArgs A, c
 #pragma unroll
                     for (int c = 0; c < NP; ++c) acc = fmaf(sC[r * NP + c], x[c], acc);
                 }
-                for (int q = 0; q < A.m; ++q) acc = fmaf(sD[r * A.m + q], uk[q], acc);
-                yrow[i * A.p + r] = acc;
+#pragma unroll 4
+                for (int q = 0; q < m; ++q) acc = fmaf(sD[r * m + q], uk[q], acc);
+                yrow[i * p + r] = acc;
             }
             if (A.x) {
                 float *xk = A.x + (b * A.T + k) * A.n;
@@ -485,7 +495,7 @@ __global__ void __launch_bounds__(kThreadsL) lsim_out_kernel(const LsimArgs A, c
             }
         }
         __syncthreads();
-        store_y(A, io, tab, sy, s);
+        store_y(A, p, io, tab, sy, s);
     }
 }
 
@@ -560,16 +570,28 @@ cudaError_t launch_np(const LsimReq &r, float *scratch, cudaStream_t st, int *la
     const IoPlan io = io_plan(r.m, r.p);
     const size_t sm_in = (size_t)(Lm.c + 2 * kThreadsL * io.ustr) * sizeof(float);
     const size_t sm_out = (size_t)(Lm.pw + kThreadsL * (2 * io.ustr + io.ystr)) * sizeof(float);
-    if ((e = cudaFuncSetAttribute(lsim_local0_kernel<NP>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_in)) !=
-            cudaSuccess ||
-        (e = cudaFuncSetAttribute(lsim_out_kernel<NP>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_out)) !=
-            cudaSuccess)
+    // m = p in {1, 2, 4}: input and output widths as constants; otherwise run-time widths
+    const int w = r.m == r.p && (r.m == 1 || r.m == 2 || r.m == 4) ? r.m : 0;
+    const void *k_local0 = w == 1   ? (const void *)&lsim_local0_kernel<NP, 1>
+                           : w == 2 ? (const void *)&lsim_local0_kernel<NP, 2>
+                           : w == 4 ? (const void *)&lsim_local0_kernel<NP, 4>
+                                    : (const void *)&lsim_local0_kernel<NP, 0>;
+    const void *k_out = w == 1   ? (const void *)&lsim_out_kernel<NP, 1, 1>
+                        : w == 2 ? (const void *)&lsim_out_kernel<NP, 2, 2>
+                        : w == 4 ? (const void *)&lsim_out_kernel<NP, 4, 4>
+                                 : (const void *)&lsim_out_kernel<NP, 0, 0>;
+    if ((e = cudaFuncSetAttribute(k_local0, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_in)) != cudaSuccess ||
+        (e = cudaFuncSetAttribute(k_out, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_out)) != cudaSuccess)
         return e;
+    IoPlan io_arg = io;
+    void *io_args[] = {&A, &io_arg};
     const size_t sm_lv = (size_t)Lm.ps * sizeof(float);
     if (L > 0) {
         A.T = r.T;
         A.agg_out = agg[1];
-        lsim_local0_kernel<NP><<<grid(r.T, kThreadsL), kThreadsL, sm_in, st>>>(A, io);
+        if ((e = cudaLaunchKernel(k_local0, dim3(grid(r.T, kThreadsL)), dim3(kThreadsL), io_args, sm_in, st)) !=
+            cudaSuccess)
+            return e;
         ++nl;
         for (int l = 1; l < L; ++l) {
             A.T = Tl[l];
@@ -591,7 +613,8 @@ cudaError_t launch_np(const LsimReq &r, float *scratch, cudaStream_t st, int *la
         A.carry = agg[1];
     }
     A.T = r.T;
-    lsim_out_kernel<NP><<<grid(r.T, kThreadsL), kThreadsL, sm_out, st>>>(A, io);
+    if ((e = cudaLaunchKernel(k_out, dim3(grid(r.T, kThreadsL)), dim3(kThreadsL), io_args, sm_out, st)) != cudaSuccess)
+        return e;
     *launches = nl + 1;
     return cudaGetLastError();
 }

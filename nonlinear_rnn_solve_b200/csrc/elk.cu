@@ -110,14 +110,17 @@ constexpr int kElkMaxN = 64;
 
 // The tanh RNN at the iterate in h (k = 0: h^(0) = 0): per row (b, t) and unit i,
 // f = tanh(p_t + sum_j A_ij h_{t-1,j}); writes a = (1 - f^2) A_ii and r = f - h_t, or
-// (residual) folds |h_t - f| into my_max.  sAt: A transposed in shared memory.
+// (residual) folds |h_t - f| into my_max.  sAt: A transposed in shared memory with
+// rows padded to n4 = n rounded up to a multiple of 4 (zeros beyond n).  A thread
+// takes four consecutive units of one row: per j one 16-byte load of A's column
+// entries and one (four-j) state load feed four multiply-adds.
 // IN = 0: p from xproj [B, T, n]; IN = -1: p = bias + W x_t (W [n, in], in <= 8).
 template <int IN>
-__device__ void tanh_lin_pass(const ElkArgs &E, const float *sAt, int k, bool residual, float &my_max) {
+__device__ void tanh_lin_pass(const ElkArgs &E, const float *sAt, int n4, int k, bool residual, float &my_max) {
     const NewtonDiagArgs &A = E.A;
     const int n = A.H;
-    const int rpc = kThreads / n;  // rows per CTA and pass
-    const int lr = threadIdx.x / n, i = threadIdx.x - lr * n;
+    const int tpr = n4 / 4, rpc = kThreads / tpr;  // threads per row, rows per CTA and pass
+    const int lr = threadIdx.x / tpr, i0 = (threadIdx.x - lr * tpr) * 4;
     const long nrows = (long)A.B * A.T;
     const bool have_h = k > 0 || residual;
     for (long row0 = (long)blockIdx.x * rpc; row0 < nrows; row0 += (long)gridDim.x * rpc) {
@@ -125,23 +128,53 @@ __device__ void tanh_lin_pass(const ElkArgs &E, const float *sAt, int k, bool re
         if (lr >= rpc || row >= nrows) continue;
         const long b = row / A.T, t = row - b * A.T;
         const float *hp = t == 0 ? (A.h0 ? A.h0 + b * n : nullptr) : (have_h ? A.h + (row - 1) * n : nullptr);
-        float z;
-        if (IN == 0) {
-            z = A.xproj[row * n + i];
-        } else {
-            z = A.bias ? A.bias[i] : 0.f;
-            for (int q = 0; q < A.in; ++q) z = fmaf(A.W[(size_t)i * A.in + q], A.x[row * A.in + q], z);
+        float z[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int i = i0 + u;
+            z[u] = 0.f;
+            if (i < n) {
+                if (IN == 0) {
+                    z[u] = A.xproj[row * n + i];
+                } else {
+                    z[u] = A.bias ? A.bias[i] : 0.f;
+                    for (int q = 0; q < A.in; ++q) z[u] = fmaf(A.W[(size_t)i * A.in + q], A.x[row * A.in + q], z[u]);
+                }
+            }
         }
-        if (hp)
-            for (int j = 0; j < n; ++j) z = fmaf(sAt[j * n + i], hp[j], z);
-        const float f = tanhf(z);
-        const float cur = have_h ? A.h[row * n + i] : 0.f;
-        if (residual) {
-            const float ad = fabsf(cur - f);
-            my_max = (ad > my_max || isnan(ad)) ? ad : my_max;
-        } else {
-            E.sa[row * n + i] = (1.f - f * f) * sAt[i * n + i];
-            E.sr[row * n + i] = f - cur;
+        if (hp) {
+            auto col = [&](int j, float hj) {
+                const float4 a4 = *reinterpret_cast<const float4 *>(sAt + j * n4 + i0);
+                z[0] = fmaf(a4.x, hj, z[0]);
+                z[1] = fmaf(a4.y, hj, z[1]);
+                z[2] = fmaf(a4.z, hj, z[2]);
+                z[3] = fmaf(a4.w, hj, z[3]);
+            };
+            if (n % 4 == 0) {  // rows of h start on 16 bytes (h, h0 16-byte aligned)
+                for (int j = 0; j < n; j += 4) {
+                    const float4 h4 = *reinterpret_cast<const float4 *>(hp + j);
+                    col(j, h4.x);
+                    col(j + 1, h4.y);
+                    col(j + 2, h4.z);
+                    col(j + 3, h4.w);
+                }
+            } else {
+                for (int j = 0; j < n; ++j) col(j, hp[j]);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int i = i0 + u;
+            if (i >= n) break;
+            const float f = tanhf(z[u]);
+            const float cur = have_h ? A.h[row * n + i] : 0.f;
+            if (residual) {
+                const float ad = fabsf(cur - f);
+                my_max = (ad > my_max || isnan(ad)) ? ad : my_max;
+            } else {
+                E.sa[row * n + i] = (1.f - f * f) * sAt[i * n4 + i];
+                E.sr[row * n + i] = f - cur;
+            }
         }
     }
 }
@@ -152,7 +185,8 @@ __global__ void __launch_bounds__(kThreads, 2) elk_kernel(const ElkArgs E) {
     constexpr int S = Cell::S;
     constexpr int SUB = kThreads / C, TCH = SUB * L;
     constexpr bool kTanh = std::is_same<Cell, TanhLin>::value;
-    __shared__ float s_At[kTanh ? kElkMaxN * kElkMaxN : 1];
+    __shared__ __align__(16) float s_At[kTanh ? kElkMaxN * kElkMaxN : 4];
+    const int n4 = (A.H + 3) & ~3;  // tanh: padded row length of s_At
     __shared__ ScanSmem<2, C, kThreads, PAff2> sm2;
     __shared__ ScanSmem<1, C> sm1;
     __shared__ unsigned s_red[kThreads / 32];
@@ -168,7 +202,10 @@ __global__ void __launch_bounds__(kThreads, 2) elk_kernel(const ElkArgs E) {
     LookBack<1> lb1{A.agg, A.inc};
     if (tid == 0) s_fail = 0;
     if (kTanh)
-        for (int e = tid; e < A.H * A.H; e += kThreads) s_At[(e % A.H) * A.H + e / A.H] = E.Amat[e];
+        for (int e = tid; e < n4 * n4; e += kThreads) {
+            const int j = e / n4, i = e % n4;  // s_At[j][i] = A[i][j]
+            s_At[e] = (i < A.H && j < A.H) ? E.Amat[i * A.H + j] : 0.f;
+        }
     __syncthreads();
 
     int iters = 0;
@@ -179,7 +216,7 @@ __global__ void __launch_bounds__(kThreads, 2) elk_kernel(const ElkArgs E) {
         if (blockIdx.x == 0 && tid == 0) A.ctl->delta_bits[(k + 1) % 3] = 0u;
         if constexpr (kTanh) {  // linearise the whole iterate first
             float unused = 0.f;
-            tanh_lin_pass<IN>(E, s_At, k, false, unused);
+            tanh_lin_pass<IN>(E, s_At, n4, k, false, unused);
             if (!grid_sync(A.ctl, A.sticky, A.dbg)) return;
         }
 
@@ -404,7 +441,7 @@ __global__ void __launch_bounds__(kThreads, 2) elk_kernel(const ElkArgs E) {
     if (A.residual_out && !stop_all) {
         if constexpr (kTanh) {
             float my_res = 0.f;
-            tanh_lin_pass<IN>(E, s_At, 1, true, my_res);
+            tanh_lin_pass<IN>(E, s_At, n4, 1, true, my_res);
             const unsigned bits = block_max_bits(my_res, s_red);
             if (tid == 0) atomicMax(&A.ctl->res_bits, bits);
             if (!grid_sync(A.ctl, A.sticky, A.dbg)) return;

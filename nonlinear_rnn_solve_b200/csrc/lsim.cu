@@ -36,11 +36,12 @@ constexpr int kTaylor = 10;  // degree; the scaled matrix has 1-norm <= 1/4
 __host__ __device__ constexpr long up4(long x) { return (x + 3) & ~3L; }
 
 // Offsets (floats) of the fp32 matrices the discretisation writes, padded to NP:
-// AdT [NP][NP] (AdT[j][i] = Ad[i][j]), G0T, G1T [m][NP], Cp [p][NP], Dm [p][m], then
-// the transposed chunk powers Ad^(32^l), l = 1 .. levels, [NP][NP] each at a stride of
-// ps floats.  Every offset is a multiple of 4 floats (16-byte copies).
+// AdT [NP][NP] (AdT[j][i] = Ad[i][j]), G0T, G1T [m][NP], Cp [p][NP], Dm [p][m], the
+// chunk kernels KT [33][m][NP] (below), then the transposed chunk powers Ad^(32^l),
+// l = 1 .. levels, [NP][NP] each at a stride of ps floats.  Every offset is a multiple
+// of 4 floats (16-byte copies).
 struct MatLayout {
-    long ad, g0, g1, c, d, pw, ps, total;
+    long ad, g0, g1, c, d, kk, pw, ps, total;
     __host__ __device__ MatLayout(int NP, int m, int p, int levels) {
         ps = up4((long)NP * NP);
         ad = 0;
@@ -48,12 +49,36 @@ struct MatLayout {
         g1 = up4(g0 + (long)m * NP);
         c = up4(g1 + (long)m * NP);
         d = up4(c + (long)p * NP);
-        pw = up4(d + (long)p * m);
+        kk = up4(d + (long)p * m);
+        pw = up4(kk + (long)(kChunk + 1) * m * NP);
         total = pw + levels * ps;
     }
 };
 
+// The end state of a 32-step chunk k0 .. k0 + 31 (k0 >= 1) run from a zero state is
+// linear in its inputs u_{k0-1} .. u_{k0+31}:
+//   x_{k0+31} = sum_{l=-1}^{31} K_l u_{k0+l},
+//   K_l = Ad^(30-l) (G0 + Ad G1) (0 <= l <= 30),  K_31 = G1,  K_{-1} = Ad^31 G0,
+// so the first pass contracts each chunk's inputs with these 33 n x m matrices (n m
+// multiply-adds per step) instead of stepping the recurrence (n^2 + n m), where they
+// fit in shared memory.
+constexpr long kMaxChunkKernelFloats = 8192;
+__host__ __device__ inline bool use_chunk_kernels(int NP, int m) {
+    return (long)(kChunk + 1) * m * NP <= kMaxChunkKernelFloats;
+}
+
 // ------------------------------------------------------------------ discretisation (fp64)
+// Z [n x m] = X [n x n] Y [n x m], row-major in shared memory, by the whole CTA.
+__device__ void smem_matmul_rect(const double *X, const double *Y, double *Z, int n, int m) {
+    for (int idx = threadIdx.x; idx < n * m; idx += blockDim.x) {
+        const int i = idx / m, j = idx % m;
+        double acc = 0.0;
+        for (int k = 0; k < n; ++k) acc = fma(X[i * n + k], Y[k * m + j], acc);
+        Z[idx] = acc;
+    }
+    __syncthreads();
+}
+
 // Product of q x q row-major matrices in shared memory, by the whole CTA: a 2 x 2
 // block of Z per thread (one shared load per multiply-add).
 __device__ void smem_matmul(const double *X, const double *Y, double *Z, int q) {
@@ -164,6 +189,43 @@ __global__ void __launch_bounds__(kDiscThreads) lsim_discretize_kernel(const flo
         mats[Lm.c + idx] = j < n ? C[r * n + j] : 0.f;
     }
     for (int idx = tid; idx < p * m; idx += blockDim.x) mats[Lm.d + idx] = D ? D[idx] : 0.f;
+    if (use_chunk_kernels(NP, m)) {
+        // chunk kernels K_l; X holds Ad [n n] | V [n m] | W [n m] (q^2 >= n^2 + 2 n m)
+        double *Ad = X, *V = X + n * n, *W = V + n * m;
+        __syncthreads();
+        for (int idx = tid; idx < n * n; idx += blockDim.x) Ad[idx] = E[(idx / n) * q + idx % n];
+        auto g0 = [&](int i, int qq) { return E[i * q + n + qq] - (interp ? E[i * q + n + m + qq] : 0.0); };
+        auto g1 = [&](int i, int qq) { return interp ? E[i * q + n + m + qq] : 0.0; };
+        auto put = [&](int l, const double *M) {  // K_l (l = -1 .. 31) from M [n m] (NULL: G1)
+            for (int idx = tid; idx < m * NP; idx += blockDim.x) {
+                const int qq = idx / NP, i = idx % NP;
+                const double v = i < n ? (M ? M[i * m + qq] : g1(i, qq)) : 0.0;
+                mats[Lm.kk + (long)(l + 1) * m * NP + idx] = (float)v;
+            }
+        };
+        for (int idx = tid; idx < n * m; idx += blockDim.x) W[idx] = g1(idx / m, idx % m);
+        __syncthreads();
+        smem_matmul_rect(Ad, W, V, n, m);  // V = Ad G1
+        for (int idx = tid; idx < n * m; idx += blockDim.x) V[idx] += g0(idx / m, idx % m);
+        __syncthreads();
+        for (int l = 30; l >= 0; --l) {  // K_l = Ad^(30-l) (G0 + Ad G1)
+            put(l, V);
+            if (l > 0) {
+                smem_matmul_rect(Ad, V, W, n, m);
+                for (int idx = tid; idx < n * m; idx += blockDim.x) V[idx] = W[idx];
+                __syncthreads();
+            }
+        }
+        put(31, nullptr);  // K_31 = G1
+        for (int idx = tid; idx < n * m; idx += blockDim.x) V[idx] = g0(idx / m, idx % m);
+        __syncthreads();
+        for (int r = 0; r < kChunk - 1; ++r) {  // K_{-1} = Ad^31 G0
+            smem_matmul_rect(Ad, V, W, n, m);
+            for (int idx = tid; idx < n * m; idx += blockDim.x) V[idx] = W[idx];
+            __syncthreads();
+        }
+        put(-1, V);
+    }
     // chunk powers: X <- Ad (n x n), then five squarings per level
     __syncthreads();
     for (int idx = tid; idx < n * n; idx += blockDim.x) X[idx] = E[(idx / n) * q + idx % n];
@@ -274,16 +336,23 @@ struct IoPlan {
     int ustr, ystr;  // floats per chunk: input rows, output rows
 };
 
-// Per-CTA chunk table: the flattened index of each chunk's first step (b T + 32 j)
-// and its step within the sequence (32 j; -1 for a thread past the last chunk).
+// Per-CTA chunk table, filled by each thread for its own chunk: the flattened index
+// of the chunk's first step (b T + 32 j), the steps left in its sequence from there
+// (T - 32 j; a large negative number for a thread past the last chunk, so no row of
+// it is ever in range) and whether it is a sequence's first chunk (whose row before
+// the first step does not exist), so the copy loops need no per-element division or
+// 64-bit bounds arithmetic.
 struct ChunkTab {
     long flat[kThreadsL];
-    long k0[kThreadsL];
+    int rem[kThreadsL];
+    int first[kThreadsL];
 };
+constexpr int kNoRows = -(1 << 24);
 
 __device__ __forceinline__ void fill_tab(ChunkTab &tab, bool valid, long b, long j, long T) {
-    tab.flat[threadIdx.x] = b * T + j * kChunk;
-    tab.k0[threadIdx.x] = valid ? j * kChunk : -1;
+    tab.flat[threadIdx.x] = valid ? b * T + j * kChunk : 0;
+    tab.rem[threadIdx.x] = valid ? (int)(T - j * kChunk) : kNoRows;
+    tab.first[threadIdx.x] = j == 0;
 }
 
 // Issue the copies of rows k0 + s SB - 1 .. k0 + s SB + SB - 1 of every chunk (zero
@@ -293,12 +362,13 @@ __device__ __forceinline__ void stage_u(const LsimArgs &A, int m, const IoPlan &
                                         int s) {
     const int rows = (io.SB + 1) * m;
     const float inv = 1.0f / (float)rows;  // exact quotient below: e < 2^15, rows <= 144
+    const int sb = s * io.SB;
     for (int e = threadIdx.x; e < kThreadsL * rows; e += kThreadsL) {
         const int c = __float2int_rd(((float)e + 0.5f) * inv), w = e - c * rows;
-        const long k0 = tab.k0[c];
-        const long kb = k0 + (long)s * io.SB - 1;
-        const bool ok = k0 >= 0 && (long)w >= max(0L, -kb) * m && (long)w < (A.T - kb) * m;
-        const long src = (tab.flat[c] + (long)s * io.SB - 1) * m + w;
+        // row r = w / m is step k0 + sb - 1 + r: inside the sequence when
+        // sb - 1 + r < rem, and r > 0 for the first chunk's first sub-block
+        const bool ok = w < (tab.rem[c] - sb + 1) * m && (w >= m || sb > 0 || !tab.first[c]);
+        const long src = (tab.flat[c] + sb - 1) * m + w;
         cp_async4(su + c * io.ustr + w, A.U + (ok ? src : 0), ok);
     }
     cp_async_commit();
@@ -310,11 +380,10 @@ __device__ __forceinline__ void store_y(const LsimArgs &A, int p, const IoPlan &
                                         const float *sy, int s) {
     const int rows = io.SB * p;
     const float inv = 1.0f / (float)rows;
+    const int sb = s * io.SB;
     for (int e = threadIdx.x; e < kThreadsL * rows; e += kThreadsL) {
         const int c = __float2int_rd(((float)e + 0.5f) * inv), w = e - c * rows;
-        const long k0 = tab.k0[c];
-        const long kb = k0 + (long)s * io.SB;
-        if (k0 >= 0 && (long)w < (A.T - kb) * p) A.y[(tab.flat[c] + (long)s * io.SB) * p + w] = sy[c * io.ystr + w];
+        if (w < (tab.rem[c] - sb) * p) A.y[(tab.flat[c] + sb) * p + w] = sy[c * io.ystr + w];
     }
 }
 
@@ -359,8 +428,10 @@ __global__ void __launch_bounds__(kThreadsL) lsim_local0_kernel(const LsimArgs A
     const int m = MM > 0 ? MM : A.m;
     extern __shared__ __align__(16) float sm[];
     const MatLayout Lm(NP, A.m, A.p, 0);
-    stage_mats(sm, A.mats, Lm.c);
-    float *su = sm + Lm.c;
+    const bool kern = use_chunk_kernels(NP, m);
+    const long staged = kern ? Lm.pw : Lm.c;  // with the chunk kernels KT
+    stage_mats(sm, A.mats, staged);
+    float *su = sm + staged;
     const long nch = (A.T + kChunk - 1) / kChunk;
     const long g0 = (long)blockIdx.x * kThreadsL, g = g0 + threadIdx.x;
     const bool valid = g < A.B * nch;
@@ -384,13 +455,39 @@ __global__ void __launch_bounds__(kThreadsL) lsim_local0_kernel(const LsimArgs A
         }
         __syncthreads();
         const float *row = su + (s & 1) * kThreadsL * io.ustr + threadIdx.x * io.ustr;
-        for (int i = 0; i < io.SB; ++i) {
-            const long k = j * kChunk + (long)s * io.SB + i;
-            if (k >= k1) break;
-            if (k == 0)
-                load_x0<NP>(A, b, x);
-            else
-                input_step<NP, MM>(A, sm + Lm.ad, sm + Lm.g0, sm + Lm.g1, row + i * m, row + (i + 1) * m, x);
+        if (kern && j > 0) {
+            // x += K_l u_l for the sub-block's rows l = s SB - 1 (first sub-block only:
+            // later ones start at the row the previous one ended with) .. s SB + SB - 1;
+            // rows past T were staged as zeros
+            for (int r = s == 0 ? 0 : 1; r <= io.SB; ++r) {
+                const float *KT = sm + Lm.kk + (long)(s * io.SB + r) * m * NP;
+#pragma unroll 4
+                for (int q = 0; q < m; ++q) {
+                    const float uq = row[r * m + q];
+                    if constexpr (NP % 4 == 0) {
+#pragma unroll
+                        for (int i = 0; i < NP; i += 4) {
+                            const float4 kv = lds4(KT + q * NP + i);
+                            x[i] = fmaf(kv.x, uq, x[i]);
+                            x[i + 1] = fmaf(kv.y, uq, x[i + 1]);
+                            x[i + 2] = fmaf(kv.z, uq, x[i + 2]);
+                            x[i + 3] = fmaf(kv.w, uq, x[i + 3]);
+                        }
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < NP; ++i) x[i] = fmaf(KT[q * NP + i], uq, x[i]);
+                    }
+                }
+            }
+        } else {
+            for (int i = 0; i < io.SB; ++i) {
+                const long k = j * kChunk + (long)s * io.SB + i;
+                if (k >= k1) break;
+                if (k == 0)
+                    load_x0<NP>(A, b, x);
+                else
+                    input_step<NP, MM>(A, sm + Lm.ad, sm + Lm.g0, sm + Lm.g1, row + i * m, row + (i + 1) * m, x);
+            }
         }
         __syncthreads();
     }
@@ -568,7 +665,8 @@ cudaError_t launch_np(const LsimReq &r, float *scratch, cudaStream_t st, int *la
     A.carry = nullptr;
     auto grid = [&](long T, int nt) { return (unsigned)((r.batch * ((T + kChunk - 1) / kChunk) + nt - 1) / nt); };
     const IoPlan io = io_plan(r.m, r.p);
-    const size_t sm_in = (size_t)(Lm.c + 2 * kThreadsL * io.ustr) * sizeof(float);
+    const size_t sm_in =
+        (size_t)((use_chunk_kernels(NP, r.m) ? Lm.pw : Lm.c) + 2 * kThreadsL * io.ustr) * sizeof(float);
     const size_t sm_out = (size_t)(Lm.pw + kThreadsL * (2 * io.ustr + io.ystr)) * sizeof(float);
     // m = p in {1, 2, 4}: input and output widths as constants; otherwise run-time widths
     const int w = r.m == r.p && (r.m == 1 || r.m == 2 || r.m == 4) ? r.m : 0;

@@ -12,12 +12,13 @@
 // squaring of a Taylor polynomial.
 //
 // The matrix of the recurrence is the same at every step, so the scan carries states
-// only: a thread runs 32 consecutive steps from a zero state and emits the chunk's end
-// state; those end states form a sequence of the same kind with matrix Ad^32, chunked
-// again until one chunk covers a level; a fix-up pass turns every level's end states
-// into the states entering the next chunk, top down; the last pass re-runs each
-// 32-step chunk from its entering state and writes y (and x).  Every pass is
-// independent per thread: no CTA waits on another.
+// only: a thread takes 32 consecutive steps and emits the chunk's end state from a
+// zero state (a contraction of the chunk's inputs with 33 precomputed matrices, or the
+// recurrence stepped); those end states form a sequence of the same kind with matrix
+// Ad^32, chunked again until one chunk covers a level; a fix-up pass turns every
+// level's end states into the states entering the next chunk, top down; the last pass
+// re-runs each 32-step chunk from its entering state and writes y (and x).  Every pass
+// is independent per thread: no CTA waits on another.
 #include <cuda_runtime.h>
 
 #include "common.cuh"

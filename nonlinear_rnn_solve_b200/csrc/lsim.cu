@@ -339,10 +339,11 @@ struct IoPlan {
 
 // Per-CTA chunk table, filled by each thread for its own chunk: the flattened index
 // of the chunk's first step (b T + 32 j), the steps left in its sequence from there
-// (T - 32 j; a large negative number for a thread past the last chunk, so no row of
-// it is ever in range) and whether it is a sequence's first chunk (whose row before
-// the first step does not exist), so the copy loops need no per-element division or
-// 64-bit bounds arithmetic.
+// (T - 32 j, capped at 33, beyond which no row of a chunk reaches, so the products
+// with m or p below stay small; a large negative number for a thread past the last
+// chunk, so no row of it is ever in range) and whether it is a sequence's first chunk
+// (whose row before the first step does not exist), so the copy loops need no
+// per-element division or 64-bit bounds arithmetic.
 struct ChunkTab {
     long flat[kThreadsL];
     int rem[kThreadsL];
@@ -352,7 +353,7 @@ constexpr int kNoRows = -(1 << 24);
 
 __device__ __forceinline__ void fill_tab(ChunkTab &tab, bool valid, long b, long j, long T) {
     tab.flat[threadIdx.x] = valid ? b * T + j * kChunk : 0;
-    tab.rem[threadIdx.x] = valid ? (int)(T - j * kChunk) : kNoRows;
+    tab.rem[threadIdx.x] = valid ? (int)min(T - j * kChunk, (long)kChunk + 1) : kNoRows;
     tab.first[threadIdx.x] = j == 0;
 }
 

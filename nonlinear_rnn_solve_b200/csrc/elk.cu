@@ -471,7 +471,10 @@ int pick_C(int D) {
     return c;
 }
 
-constexpr int kElkL = 8;
+#ifndef PRN_ELK_L
+#define PRN_ELK_L 8
+#endif
+constexpr int kElkL = PRN_ELK_L;  // steps per thread
 
 template <class Cell, int IN> const void *elk_by_C(int C) {
     switch (C) {

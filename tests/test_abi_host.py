@@ -58,6 +58,8 @@ def test_null_context_and_pointers_are_rejected():
     assert L.pararnn_linear_scan(None, 0, None, None, None, None, 1, 1, 1, 0) == EINVAL
     assert L.pararnn_adjoint_backward(None, None, ctypes.byref(p), None, None, None, None, None, None) == EINVAL
     assert L.pararnn_input_proj(None, None, 0, None, None, None, 1, 1, 1) == EINVAL
+    assert L.pararnn_input_proj_backward(None, None, None, 0, None, None, None, None, 1, 1, 1) == EINVAL
+    assert L.pararnn_lsim(None, None, None, None, None, 1, 1, 1, None, None, 0.1, 0, 1, 1, None, None) == EINVAL
     st = ctypes.c_int()
     assert L.pararnn_get_status(None, ctypes.byref(st)) == EINVAL
     assert L.pararnn_debug_set(None, 1, 5) == EINVAL
@@ -75,3 +77,18 @@ def test_binding_refuses_cpu_tensors():
     import torch
     with pytest.raises(TypeError):
         prn._p(torch.zeros(4))
+
+
+def test_lsim_binding_checks_the_time_grid_on_the_host():
+    """The fixed-step grid and its length are checked before any device call."""
+    import numpy as np
+    import torch
+    from nonlinear_rnn_solve_b200 import solve
+    A, B, C = torch.zeros(2, 2), torch.zeros(2, 1), torch.zeros(1, 2)
+    U = torch.zeros(6, 1)
+    with pytest.raises(ValueError):  # uneven steps
+        solve.lsim(None, A, B, C, None, U, np.array([0.0, 1.0, 2.0, 3.5, 4.0, 5.0]))
+    with pytest.raises(ValueError):  # one time per sample
+        solve.lsim(None, A, B, C, None, U, np.arange(5) * 0.1)
+    with pytest.raises(TypeError):  # even grid: reaches the binding, which takes CUDA tensors only
+        solve.lsim(None, A, B, C, None, U, np.arange(6) * 0.1)

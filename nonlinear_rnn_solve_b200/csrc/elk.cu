@@ -471,10 +471,11 @@ int pick_C(int D) {
     return c;
 }
 
-#ifndef PRN_ELK_L
-#define PRN_ELK_L 8
-#endif
-constexpr int kElkL = PRN_ELK_L;  // steps per thread
+// Steps per thread: 16 for tiles of 32 channels (wide states: a 64-step tile would
+// spend most of its time in the look-back), 8 for narrower ones (long sequences of
+// few channels, where 8 measured faster).
+constexpr int kElkL = 8, kElkLWide = 16;
+int elk_L(int C) { return C == 32 ? kElkLWide : kElkL; }
 
 template <class Cell, int IN> const void *elk_by_C(int C) {
     switch (C) {
@@ -483,7 +484,7 @@ template <class Cell, int IN> const void *elk_by_C(int C) {
         case 4: return reinterpret_cast<const void *>(&elk_kernel<Cell, 4, kElkL, IN>);
         case 8: return reinterpret_cast<const void *>(&elk_kernel<Cell, 8, kElkL, IN>);
         case 16: return reinterpret_cast<const void *>(&elk_kernel<Cell, 16, kElkL, IN>);
-        default: return reinterpret_cast<const void *>(&elk_kernel<Cell, 32, kElkL, IN>);
+        default: return reinterpret_cast<const void *>(&elk_kernel<Cell, 32, kElkLWide, IN>);
     }
 }
 
@@ -493,7 +494,7 @@ namespace {
 
 // Tiles, workspace and grid of an ELK solve over D scalar channels per sequence.
 int elk_plan_common(const void *kernel, long B, long T, int D, int C, int max_iters, int num_sms, Plan *plan) {
-    const int TCH = (kThreads / C) * kElkL;
+    const int TCH = (kThreads / C) * elk_L(C);
     const long nseq = B * ((D + C - 1) / C);
     plan->ntiles = nseq * ((T + TCH - 1) / TCH);
     plan->kernel = kernel;

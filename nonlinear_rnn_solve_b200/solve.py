@@ -73,8 +73,16 @@ def lsim(ctx, A, B, C, D, U, t, x0=None, interp="zoh", return_states=True):
     from . import pararnn_lsim
     single = U.dim() == 2
     U3 = U.unsqueeze(0) if single else U
-    batch, T, _ = U3.shape
+    if U3.dim() != 3:
+        raise ValueError("U must be [T, m] or [batch, T, m]")
+    batch, T, m = U3.shape
     n, p = A.shape[0], C.shape[0]
+    # the C ABI takes bare pointers: every operand's shape is checked here
+    if A.shape != (n, n) or B.shape != (n, m) or C.shape != (p, n) or (D is not None and D.shape != (p, m)):
+        raise ValueError(f"shapes: A {tuple(A.shape)}, B {tuple(B.shape)}, C {tuple(C.shape)}, "
+                         f"D {None if D is None else tuple(D.shape)} do not fit n = {n}, m = {m}, p = {p}")
+    if x0 is not None and x0.shape not in ((n,), (batch, n)):
+        raise ValueError(f"x0 must be [{n}] or [{batch}, {n}]")
     tt = torch.as_tensor(t, dtype=torch.float64).cpu().reshape(-1)
     if tt.numel() != T:
         raise ValueError("t must have one point per input sample")

@@ -92,3 +92,12 @@ def test_lsim_binding_checks_the_time_grid_on_the_host():
         solve.lsim(None, A, B, C, None, U, np.arange(5) * 0.1)
     with pytest.raises(TypeError):  # even grid: reaches the binding, which takes CUDA tensors only
         solve.lsim(None, A, B, C, None, U, np.arange(6) * 0.1)
+    t = np.arange(6) * 0.1
+    with pytest.raises(ValueError):  # B with 2 inputs, U with 1
+        solve.lsim(None, A, torch.zeros(2, 2), C, None, U, t)
+    with pytest.raises(ValueError):  # C not [p, n]
+        solve.lsim(None, A, B, torch.zeros(1, 3), None, U, t)
+    with pytest.raises(ValueError):  # D not [p, m]
+        solve.lsim(None, A, B, C, torch.zeros(2, 1), U, t)
+    with pytest.raises(ValueError):  # x0 not [n]
+        solve.lsim(None, A, B, C, None, U, t, x0=torch.zeros(3))

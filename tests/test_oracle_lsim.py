@@ -132,3 +132,24 @@ def test_batch_rows_are_independent_runs():
     for i in range(3):
         yi, xi = oracle.lsim(A, B, C, np.zeros((p, m)), U[i], h, x0=x0[i], interp="foh")
         assert np.array_equal(y[i], yi) and np.array_equal(x[i], xi)
+
+
+@pytest.mark.parametrize("interp", ["zoh", "foh"])
+def test_chunk_end_state_is_a_fixed_linear_map_of_its_inputs(interp):
+    """From a zero state before step k0, the state after 32 steps is
+    sum_{l=-1}^{31} K_l u_{k0+l} with K_l = Ad^(30-l) (G0 + Ad G1) for 0 <= l <= 30,
+    K_31 = G1 and K_{-1} = Ad^31 G0: the identity the first scan pass contracts with."""
+    rng = np.random.default_rng(17)
+    n, m, h = 4, 3, 0.07
+    A = rng.standard_normal((n, n)) * 0.4 - np.eye(n)
+    B = rng.standard_normal((n, m))
+    Ad, G0, G1 = oracle.lsim_discretize(A, B, h, interp)
+    u = rng.standard_normal((33, m))  # u_{k0-1} .. u_{k0+31}
+    x = np.zeros(n)
+    for i in range(32):  # steps k0 .. k0 + 31, each from u_{k-1} and u_k
+        x = Ad @ x + G0 @ u[i] + G1 @ u[i + 1]
+    P = np.linalg.matrix_power
+    K = {l: P(Ad, 30 - l) @ (G0 + Ad @ G1) for l in range(31)}
+    K[31], K[-1] = G1, P(Ad, 31) @ G0
+    y = sum(K[l] @ u[l + 1] for l in range(-1, 32))
+    assert np.abs(x - y).max() < 1e-12

@@ -23,6 +23,12 @@ def state_shape(cell, B, T, H):
 SOLVERS = {"newton": 0, "jacobi": 1, "picard": 2, "elk": 3}
 
 
+def _need(t, count, name):
+    """The C ABI takes bare pointers: check each operand's element count first."""
+    if t is not None and t.numel() != count:
+        raise ValueError(f"{name} has {t.numel()} elements, expected {count}")
+
+
 def newton_forward(ctx, cell, B, T, H, *, xproj=None, x=None, W=None, bias=None, a=None,
                    peep=None, A=None, h0=None, max_iters=None, tol=1e-6, residual=False,
                    h_out=None, solver="newton", damping=0.0):
@@ -30,6 +36,21 @@ def newton_forward(ctx, cell, B, T, H, *, xproj=None, x=None, W=None, bias=None,
     residual) (device tensors)."""
     dev = (xproj if xproj is not None else x).device
     inp = 0 if x is None else x.shape[-1]
+    G = 1 if cell in ("tanh", "tanh_quasi") else 3
+    S = 2 if cell in ("lstm", "lstm_quasi") else 1
+    if xproj is not None:
+        _need(xproj, B * T * G * H, "xproj [B, T, G, H]")
+    else:
+        _need(x, B * T * inp, "x [B, T, in]")
+        _need(W, G * H * inp, "W [G*H, in]")
+        _need(bias, G * H, "bias [G*H]")
+    if G == 3:
+        _need(a, 3 * H, "a [3, H]")
+        _need(peep, 2 * H, "peep [2, H]")
+    else:
+        _need(A, H * H, "A [n, n]")
+    _need(h0, B * H * S, "h0")
+    _need(h_out, B * T * H * S, "h_out")
     prm = make_params(CELLS[cell], B, T, H, inp, a=a, peep=peep, A=A,
                       x=x if xproj is None else None, W=W if xproj is None else None,
                       bias=bias if xproj is None else None, solver=SOLVERS[solver], damping=damping)
@@ -46,6 +67,8 @@ def newton_forward(ctx, cell, B, T, H, *, xproj=None, x=None, W=None, bias=None,
 def input_proj(ctx, x, W, bias=None):
     """xproj = x W^T + bias with x [..., K] and W [N, K] (both bf16 or both fp32)."""
     N = W.shape[0]
+    _need(W, N * x.shape[-1], "W [N, K]")
+    _need(bias, N, "bias [N]")
     out = torch.empty(*x.shape[:-1], N, device=x.device, dtype=torch.float32)
     pararnn_input_proj(ctx, x, W, bias, out)
     return out
@@ -57,6 +80,8 @@ def input_proj_backward(ctx, grad_xproj, x, W, need_x=True, need_W=True, need_bi
     from . import pararnn_input_proj_backward
     dev = x.device
     K, N = x.shape[-1], W.shape[0]
+    _need(W, N * K, "W [N, K]")
+    _need(grad_xproj, (x.numel() // K) * N, "grad_xproj [M, N]")
     gx = torch.empty(*x.shape[:-1], K, device=dev, dtype=torch.float32) if need_x else None
     gW = torch.empty(N, K, device=dev, dtype=torch.float32) if need_W else None
     gb = torch.empty(N, device=dev, dtype=torch.float32) if need_bias else None
@@ -105,6 +130,10 @@ def linear_scan(ctx, kind, J, b, h0=None, reverse=False):
     from . import PARARNN_SCAN_BLOCK2, PARARNN_SCAN_DENSE, PARARNN_SCAN_DIAG
     k = {"diag": PARARNN_SCAN_DIAG, "block2": PARARNN_SCAN_BLOCK2, "dense": PARARNN_SCAN_DENSE}[kind]
     B, T, N = b.shape[:3]
+    S = 2 if kind == "block2" else 1
+    _need(b, B * T * N * S, "b")
+    _need(J, B * T * N * (N if kind == "dense" else S * S), "J")
+    _need(h0, B * N * S, "h0")
     out = torch.empty_like(b)
     pararnn_linear_scan(ctx, k, J, b, h0, out, B, T, N, reverse)
     return out
@@ -113,6 +142,13 @@ def linear_scan(ctx, kind, J, b, h0=None, reverse=False):
 def adjoint_backward(ctx, cell, B, T, H, *, xproj, a, peep=None, h0=None, h, grad_h):
     """Adjoint gradients at states h.  Returns (grad_xproj, grad_params, grad_h0)."""
     dev = xproj.device
+    S = 2 if cell in ("lstm", "lstm_quasi") else 1
+    _need(xproj, B * T * 3 * H, "xproj [B, T, 3, H]")
+    _need(a, 3 * H, "a [3, H]")
+    _need(peep, 2 * H, "peep [2, H]")
+    _need(h0, B * H * S, "h0")
+    _need(h, B * T * H * S, "h")
+    _need(grad_h, B * T * H * S, "grad_h")
     prm = make_params(CELLS[cell], B, T, H, 0, a=a, peep=peep)
     gx = torch.empty(B, T, 3, H, device=dev, dtype=torch.float32)
     lstm = cell in ("lstm", "lstm_quasi")

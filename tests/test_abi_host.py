@@ -101,3 +101,27 @@ def test_lsim_binding_checks_the_time_grid_on_the_host():
         solve.lsim(None, A, B, C, torch.zeros(2, 1), U, t)
     with pytest.raises(ValueError):  # x0 not [n]
         solve.lsim(None, A, B, C, None, U, t, x0=torch.zeros(3))
+
+
+def test_wrappers_check_operand_sizes_before_the_pointer_only_calls():
+    """A wrong-sized operand raises ValueError on the host (the C calls take bare
+    pointers and would read or write past it)."""
+    import torch
+    from nonlinear_rnn_solve_b200 import solve
+    z = torch.zeros
+    with pytest.raises(ValueError):  # block2 J must be [B, T, N, 2, 2]
+        solve.linear_scan(None, "block2", z(2, 5, 3), z(2, 5, 3, 2))
+    with pytest.raises(ValueError):  # h0 [B, N]
+        solve.linear_scan(None, "diag", z(2, 5, 3), z(2, 5, 3), z(3))
+    with pytest.raises(ValueError):  # xproj [B, T, 3, H]
+        solve.newton_forward(None, "gru", 2, 5, 4, xproj=z(2, 5, 4), a=z(3, 4))
+    with pytest.raises(ValueError):  # LSTM h0 holds (c, h) pairs
+        solve.newton_forward(None, "lstm", 2, 5, 4, xproj=z(2, 5, 3, 4), a=z(3, 4), peep=z(2, 4), h0=z(2, 4))
+    with pytest.raises(ValueError):  # tanh A [n, n]
+        solve.newton_forward(None, "tanh", 2, 5, 4, xproj=z(2, 5, 4), A=z(4, 3))
+    with pytest.raises(ValueError):  # grad_h like h
+        solve.adjoint_backward(None, "gru", 2, 5, 4, xproj=z(2, 5, 3, 4), a=z(3, 4), h=z(2, 5, 4), grad_h=z(2, 4, 4))
+    with pytest.raises(ValueError):  # W [N, K]
+        solve.input_proj(None, z(6, 8), z(16, 7))
+    with pytest.raises(ValueError):  # grad_xproj [M, N]
+        solve.input_proj_backward(None, z(6, 15), z(6, 8), z(16, 8))

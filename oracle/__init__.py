@@ -1,4 +1,6 @@
-"""fp64 CPU oracle for the Newton (DEER) / quasi-Newton evaluation of nonlinear RNNs.
+"""fp64 CPU oracle for the Newton (DEER) / quasi-Newton evaluation of nonlinear RNNs,
+its fixed-point variants, the linear scans, the adjoint and the fixed-step simulation of
+linear ODEs (lsim).
 
 TEST INFRASTRUCTURE.  Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU
 baseline / reference leg of ``bench.py`` may import this package.  The CUDA
@@ -13,7 +15,8 @@ discretises a linear ODE over one step (``scipy.linalg.expm``).
 
 Every function here is pinned by the CPU tests against something other than
 itself (PyTorch's reference GRU/LSTM/RNN cells, autograd Jacobians, dense
-linear solves of the stacked system, closed forms and invariants).
+linear solves of the stacked system, closed forms and invariants; for lsim, closed
+forms, exact quadrature sums, an RK4 integration and scipy's own lsim).
 """
 from __future__ import annotations
 

@@ -1,6 +1,8 @@
 /*
  * oracle.c -- plain, slow fp64 CPU reference for the Newton (DEER) and quasi-Newton
- * evaluation of nonlinear RNNs over the whole sequence.
+ * evaluation of nonlinear RNNs over the whole sequence, its fixed-point variants
+ * (Jacobi, Picard, ELK), the linear scans, the adjoint, and the fixed-step simulation
+ * of linear ODEs (lsim).
  *
  * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may call, link or load
  * this file; only the tests, the smoke check and the CPU-baseline leg of the
@@ -16,7 +18,8 @@
  *           Models", abstract  (one system of equations solved by Newton iterations).
  *   [SEQ]   "Para-Seq" README, sections "Main features" (diagonal ParaGRU,
  *           CIFG/peephole ParaLSTM with 2x2 blocks, vanilla tanh RNN, adjoint
- *           backward) and "Background" (linearise, then solve the linear recurrence).
+ *           backward, scan-based fixed-step ODE solvers), "Quick example" (lsim) and
+ *           "Background" (linearise, then solve the linear recurrence).
  *
  * Readings taken where the pages are silent (each is also listed in the design notes):
  *   - Newton update in the b-form: J_t and f_t are evaluated at the previous iterate,

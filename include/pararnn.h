@@ -168,7 +168,8 @@ int pararnn_input_proj_backward(pararnn_ctx *ctx, const float *grad_xproj, const
  *              delta fell below tol); max_iters = 0 leaves h_out = 0 and writes 0
  *   final_delta_out  device float or NULL: delta of the last iteration
  *   residual_out     device float or NULL: max |h_t - f(h_{t-1}, x_t)| at the result
- * Supported: GRU and LSTM any H; tanh RNN with n <= 64.  B, T >= 1. */
+ * Supported: GRU and LSTM any H; tanh RNN with n <= 64 (EUNSUPPORTED above), every
+ * solver for every cell.  B, T >= 1. */
 int pararnn_newton_forward(pararnn_ctx *ctx, const float *xproj, const pararnn_params *p,
                            const float *h0, float *h_out, int max_iters, float tol,
                            int *iters_out, float *final_delta_out, float *residual_out);

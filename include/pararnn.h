@@ -56,7 +56,7 @@ extern "C" {
 #define PARARNN_ENOMEM (-4)      /* workspace allocation failed */
 #define PARARNN_ENONFINITE (-5)  /* device: an iterate or residual became NaN or Inf */
 #define PARARNN_ETIMEOUT (-6)    /* device: a bounded wait (look-back, grid barrier) ran out */
-#define PARARNN_EUNSUPPORTED (-7) /* valid request outside what this build implements */
+#define PARARNN_EUNSUPPORTED (-7) /* valid request outside what the library implements */
 
 typedef enum {
     PARARNN_GRU_DIAG = 0,        /* diagonal ParaGRU, diagonal Jacobian */

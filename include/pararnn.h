@@ -255,14 +255,16 @@ int pararnn_last_launch_count(pararnn_ctx *ctx);
  *   - Runs on the calling thread's current device, on `cuda_stream` (NULL = legacy
  *     default stream).  Inputs and outputs are caller-owned device memory as for
  *     pararnn_linear_scan.
- *   - The first call on a device resolves the array's device address
- *     (cudaGetSymbolAddress) and clears it; make that first call before any stream
- *     capture.
+ *   - Every call looks up the array's device address (cudaGetSymbolAddress, which
+ *     allocates nothing).  The first call on a device, and the first call after the
+ *     device's primary context was re-created (cudaDeviceReset), clears the array;
+ *     make that first call before any stream capture.
  *   - All calls share the one array and it keeps the last call's contents: calls that
  *     overlap on the GPU (other streams, other host threads on the same device) race
  *     and must be serialised by the caller.
- *   - status_out: optional device int, set to 0 by the call; non-zero afterwards means a
- *     bounded wait of the scan ran out (the output is then not valid).
+ *   - status_out: required device int (PARARNN_EINVAL when NULL), set to 0 by the
+ *     call; non-zero afterwards means a bounded wait of the scan ran out (the output
+ *     is then not valid).  It is the only place such a timeout is reported.
  *   - Returns PARARNN_ESCRATCH, before enqueuing anything, when the problem's scratch
  *     exceeds the array: diag needs about 24 bytes per tile channel, i.e. roughly
  *     B*N*T/128*24 bytes for N >= 32 (B*N*T up to ~89 million) and B*T/4096*24 bytes for

@@ -139,6 +139,29 @@ def linear_scan(ctx, kind, J, b, h0=None, reverse=False):
     return out
 
 
+def linear_scan_noalloc(kind, J, b, h0=None, reverse=False, status_out=None, h_out=None, stream=None):
+    """The allocation-free scan (diag or block2) on the current device and stream.
+
+    Checks every operand's element count before the pointer-only C call.  Returns
+    (h_out, status_out); status_out (one int32 on the device) is non-zero after the
+    call when a bounded wait ran out."""
+    from . import PARARNN_SCAN_BLOCK2, PARARNN_SCAN_DIAG, pararnn_linear_scan_noalloc
+    k = {"diag": PARARNN_SCAN_DIAG, "block2": PARARNN_SCAN_BLOCK2}[kind]
+    B, T, N = b.shape[:3]
+    S = 2 if kind == "block2" else 1
+    _need(b, B * T * N * S, "b")
+    _need(J, B * T * N * S * S, "J")
+    _need(h0, B * N * S, "h0")
+    _need(h_out, B * T * N * S, "h_out")
+    _need(status_out, 1, "status_out")
+    if h_out is None:
+        h_out = torch.empty_like(b)
+    if status_out is None:
+        status_out = torch.zeros(1, device=b.device, dtype=torch.int32)
+    pararnn_linear_scan_noalloc(k, J, b, h0, h_out, B, T, N, reverse, status_out=status_out, stream=stream)
+    return h_out, status_out
+
+
 def adjoint_backward(ctx, cell, B, T, H, *, xproj, a, peep=None, h0=None, h, grad_h):
     """Adjoint gradients at states h.  Returns (grad_xproj, grad_params, grad_h0)."""
     dev = xproj.device

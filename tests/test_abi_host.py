@@ -125,3 +125,17 @@ def test_wrappers_check_operand_sizes_before_the_pointer_only_calls():
         solve.input_proj(None, z(6, 8), z(16, 7))
     with pytest.raises(ValueError):  # grad_xproj [M, N]
         solve.input_proj_backward(None, z(6, 15), z(6, 8), z(16, 8))
+    with pytest.raises(ValueError):  # allocation-free scan: block2 J [B, T, N, 2, 2]
+        solve.linear_scan_noalloc("block2", z(2, 5, 3, 2), z(2, 5, 3, 2))
+    with pytest.raises(ValueError):  # allocation-free scan: h_out like b
+        solve.linear_scan_noalloc("diag", z(2, 5, 3), z(2, 5, 3), h_out=z(2, 5, 2))
+    with pytest.raises(ValueError):  # allocation-free scan: one status word
+        solve.linear_scan_noalloc("diag", z(2, 5, 3), z(2, 5, 3), status_out=z(2, dtype=torch.int32))
+
+
+def test_noalloc_scan_rejects_a_missing_status_word_on_the_host():
+    """A NULL status word is refused before any device call (a timeout would otherwise go
+    unreported)."""
+    L = prn.lib()
+    x = ctypes.c_void_p(256)
+    assert L.pararnn_linear_scan_noalloc(0, x, x, None, x, 1, 4, 1, 0, None, None) == prn.PARARNN_EINVAL

@@ -36,7 +36,6 @@ def _inputs(kind, B, T, N, seed):
 def test_noalloc_scan_matches_context_scan_twice(kind, shape, reverse):
     need_gpu()
     B, T, N = shape
-    code = prn.PARARNN_SCAN_DIAG if kind == "diag" else prn.PARARNN_SCAN_BLOCK2
     status = torch.full((1,), 7, dtype=torch.int32, device="cuda")
     for call in range(2):  # two calls in a row: the shared scratch is reused
         J, b, h0 = _inputs(kind, B, T, N, seed=1000 * call + B * 7 + T + N)
@@ -45,7 +44,7 @@ def test_noalloc_scan_matches_context_scan_twice(kind, shape, reverse):
             torch.cuda.synchronize()
             assert ctx.status() == 0
         out = torch.full_like(b, float("nan"))
-        prn.pararnn_linear_scan_noalloc(code, J, b, h0, out, B, T, N, reverse, status_out=status)
+        solve.linear_scan_noalloc(kind, J, b, h0, reverse=reverse, status_out=status, h_out=out)
         torch.cuda.synchronize()
         assert int(status.item()) == 0
         assert float(np.max(np.abs(host(out) - host(ref)))) <= TOL
@@ -55,6 +54,16 @@ def test_noalloc_rejects_problems_beyond_the_scratch():
     need_gpu()
     B, T, N = 64, 65536, 2048  # about 1.2 GB of scratch as a diag scan: far beyond 16 MiB
     J = torch.empty(16, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    # the raw mirror on purpose: the call returns before enqueuing anything
     with pytest.raises(prn.PararnnError) as e:
-        prn.pararnn_linear_scan_noalloc(prn.PARARNN_SCAN_DIAG, J, J, None, J, B, T, N)
+        prn.pararnn_linear_scan_noalloc(prn.PARARNN_SCAN_DIAG, J, J, None, J, B, T, N, status_out=status)
     assert e.value.code == prn.PARARNN_ESCRATCH
+
+
+def test_noalloc_requires_a_status_word():
+    need_gpu()
+    J = torch.zeros(4, device="cuda")
+    with pytest.raises(prn.PararnnError) as e:
+        prn.pararnn_linear_scan_noalloc(prn.PARARNN_SCAN_DIAG, J, J, None, J, 1, 4, 1)
+    assert e.value.code == prn.PARARNN_EINVAL

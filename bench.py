@@ -1,19 +1,30 @@
 """Benchmark: Newton-solved state elements per second on B200 (one JSON line).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload NAME]
+                    [--workload NAME] [--leg WORKLOAD:PART] [--skip-extras]
 
 A step is one Newton (DEER) forward solve of the whole workload to convergence:
 the fused cell + Jacobian + scan kernel iterating on the device until
 max|delta| < tol.  Default workload: the DEER GRU benchmark shape (batch 16,
 2^20 steps, state size 1, input width 2), synthetic seeded inputs.
 
+Besides the headline, the line carries ``per_config``: every other workload of the
+path timed on the device (CUDA events, L2 flushed between repeats, median), leg by
+leg -- the projection GEMM, the Newton forward, the adjoint backward and the
+projection backward of the LLM-width ParaGRU / ParaLSTM layers; the tanh RNN with
+full DEER and quasi-DEER at n = 8 and 64 -- each with its algorithmic bytes or flops
+and its fraction of the bound it sits on, next to the fp64 oracle's sequential
+rollout (the "naive sequential application") on all host cores and on one core.
+
+``--leg WORKLOAD:PART`` times one leg alone and prints its line (profiling runs).
+
 Multi-GPU (torchrun, one process per GPU): every rank solves its own batch of the
 same shape (independent sequences, seed offset by rank); no collective on the
 data path ("scaling": "weak"); the step time is the max over ranks.
 
---impl reference times the fp64 CPU oracle (the sequential-in-time Newton solve
-as the pages describe it) on the host cores, on rank 0 only.
+--impl reference times the fp64 CPU oracle on the host cores, on rank 0 only: the
+sequential rollout h_t = f(h_{t-1}, x_t) of the whole workload per step (the states
+the Newton solve converges to), with the oracle's own Newton solve timed beside it.
 """
 from __future__ import annotations
 
@@ -156,27 +167,353 @@ def max_over_ranks(values, device=None):
     return [float(v) for v in t.tolist()]
 
 
-def _cpu_oracle_sample(w, inp, max_seconds=20.0):
-    """Time the fp64 oracle Newton solve on a bounded sample of the workload."""
+def _oracle_threads():
+    return len(os.sched_getaffinity(0))
+
+
+def _oracle_sample_model(w, inp, nb, units):
+    """fp64 oracle model of a sample of the workload: the first ``nb`` sequences and, for
+    the layers, the first ``units`` units (every sequence of the method is independent
+    of the others, so a sample is a set of whole sequences)."""
     import oracle
-    threads = len(os.sched_getaffinity(0))
-    oracle.set_threads(threads)
-    # sample: whole sequences of the workload (every one has the same length)
-    nb = w.B
-    sub = {k: (v[:nb] if k in ("x", "h0", "g") else v) for k, v in inp.items()}
-    m = oracle.model_from_inputs(w.cell, sub, quasi=w.quasi)
+    x = inp["x"][:nb]
+    h0 = inp["h0"][:nb]
+    if w.cell == wl.TANH or units >= w.H:
+        sub = dict(inp, x=x, h0=h0)
+        return oracle.model_from_inputs(w.cell, sub, quasi=w.quasi), h0, nb * (1 if w.cell == wl.TANH else w.H)
+    H = w.H
+    rows = np.concatenate([np.arange(g * H, g * H + units) for g in range(3)])
+    xp = oracle.input_proj(x, inp["W"][rows], inp["bias"][rows]).reshape(nb, w.T, 3, units)
+    m = oracle.Model(w.cell, xp, a=inp["a"][:, :units],
+                     peep=inp["peep"][:, :units] if w.cell == wl.LSTM else None)
+    return m, np.ascontiguousarray(h0[:, :units]), nb * units
+
+
+def _time_cpu(fn, budget_s):
+    """Mean wall time of fn() over as many runs as fit in about budget_s (at least one)."""
+    fn()  # first touch of the sample's memory, page faults, thread start-up
     t0 = time.perf_counter()
     reps = 0
     while True:
-        _, iters, _ = m.newton(sub["h0"], max_iters=min(w.max_iters, 10_000), tol=w.tol)
+        fn()
         reps += 1
-        if time.perf_counter() - t0 > max_seconds / 4 or reps >= 3:
-            break
-    dt = (time.perf_counter() - t0) / reps
-    elems = nb * w.T * w.H
+        el = time.perf_counter() - t0
+        if el > budget_s or reps >= 20:
+            return el / reps, reps
+
+
+def cpu_rollout(w, inp, nb, units, threads, budget_s=1.0):
+    """The fp64 oracle's sequential rollout h_t = f(h_{t-1}, x_t) (the "naive
+    sequential application" the pages' speedups are quoted against) on a sample of
+    whole sequences, with ``threads`` OpenMP threads over independent sequences."""
+    import oracle
+    m, h0, _ = _oracle_sample_model(w, inp, nb, units)
+    oracle.set_threads(threads)
+    dt, reps = _time_cpu(lambda: m.rollout(h0), budget_s)
+    if w.cell == wl.TANH:
+        elems, what = nb * w.T * w.H, f"{nb} sequence(s) of {w.T} steps at state size {w.H}"
+    else:
+        elems, what = nb * w.T * units, f"{nb * units} unit sequence(s) of {w.T} steps ({nb} batch x {units} unit(s))"
     return {"value": elems / dt, "unit": "state elements/s", "cores": threads, "kind": "oracle",
-            "sample": f"fp64 oracle Newton solve of {nb} x {w.T} x {w.H} states ({iters} iterations), "
+            "sample": f"fp64 oracle sequential rollout of {what}, mean of {reps} run(s)"}
+
+
+def _rollout_sample(w, steps, min_seq=1):
+    """(batch rows, units) of a sample of whole sequences, about ``steps`` sequence steps
+    (scaled by the n^2 cost of a dense step for the tanh RNN), at least ``min_seq``
+    sequences where the workload has that many."""
+    if w.cell == wl.TANH:
+        return min(w.B, max(min_seq, steps * 64 // (w.H * w.H) // w.T)), w.H
+    nseq = max(min_seq, steps // w.T)
+    if nseq >= w.B:
+        return w.B, min(w.H, nseq // w.B)
+    return nseq, 1
+
+
+def cpu_baselines(w, inp):
+    """Rollout on all cores and on one core, each on a bounded sample."""
+    threads = _oracle_threads()
+    nb, units = _rollout_sample(w, 1 << 22, min_seq=threads)
+    allc = cpu_rollout(w, inp, nb, units, threads)
+    nb1, units1 = _rollout_sample(w, 1 << 20)
+    one = cpu_rollout(w, inp, nb1, units1, 1, budget_s=0.5)
+    return allc, one
+
+
+def cpu_newton(w, inp, threads, budget_s=3.0):
+    """The fp64 oracle's own Newton solve of the whole workload (for information)."""
+    import oracle
+    oracle.set_threads(threads)
+    m = oracle.model_from_inputs(w.cell, inp, quasi=w.quasi)
+    res = {}
+
+    def run():
+        res["it"] = m.newton(inp["h0"], max_iters=min(w.max_iters, 10_000), tol=w.tol)[1]
+
+    dt, reps = _time_cpu(run, budget_s)
+    return {"value": w.elems / dt, "unit": "state elements/s", "cores": threads, "kind": "oracle",
+            "sample": f"fp64 oracle Newton solve of the whole workload ({res['it']} iterations), "
                       f"mean of {reps} run(s)"}
+
+
+# ---------------------------------------------------------------- per-config legs
+PER_CONFIG = ["gru_b1_t1024_in4_h8", "gru_b8_t4096_h2048_bf16", "lstm_b4_t8192_h1024_bf16",
+              "tanh_b16_t65536_in4_n8_quasi", "tanh_b16_t65536_in4_n8_deer",
+              "tanh_b16_t65536_in4_n64_deer", "tanh_b16_t65536_in4_n64_quasi"]
+LAYER_PARTS = ["proj", "forward", "backward", "proj_backward"]
+
+
+def _fp32_peak_tflops():
+    """FP32 FMA peak from the unit counts and the clock: 148 SMs x 128 FMA lanes x 2 flops
+    x the maximum SM clock (MEASURED_PEAKS.json's sm_max_mhz, else 1965 MHz)."""
+    mhz = 1965.0
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            mhz = float(json.load(f).get("sm_max_mhz", mhz))
+    except Exception:
+        pass
+    return 148 * 128 * 2 * mhz * 1e6 / 1e12
+
+
+def _bf16_peak_tflops():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured (burst)"
+    except Exception:
+        return 1590.0, "fallback"
+
+
+def forward_bytes(w, iters, residual):
+    """Algorithmic HBM bytes of one Newton forward solve: each iteration reads the inputs
+    and the previous iterate once and writes the new one (the first reads no iterate, it
+    is zero); the residual pass reads the inputs and the result once."""
+    S, n = w.state_per_unit, w.H
+    elems = w.B * w.T * w.H
+    if w.cell == wl.TANH or (w.inp <= 8 and w.H <= 8):
+        # raw inputs, projection recomputed in the kernel: x once per step per iteration
+        xb = 4 * w.B * w.T * w.inp
+        sb = 4 * elems * S
+        per_first, per_next = xb + sb, xb + 2 * sb
+        res = xb + sb
+    else:
+        pb = 4 * w.G * elems  # projected inputs, fp32
+        sb = 4 * elems * S
+        per_first, per_next = pb + sb, pb + 2 * sb
+        res = pb + sb
+    if iters <= 0:
+        return 0
+    return per_first + (iters - 1) * per_next + (res if residual else 0)
+
+
+def tanh_flops(w, iters, quasi):
+    """Algorithmic fp32 flops of the tanh RNN forward: per step and iteration
+    f = tanh(A h + U x + b) (2 n^2 + 2 n in), the Jacobian's scaling and the scan update
+    (4 n); full DEER adds the chain products of the n x n Jacobians, n^3 multiply-adds
+    per step, and the dense update n^2 (matrix-vector) instead of the diagonal one."""
+    n = w.H
+    per = 2 * n * n + 2 * n * w.inp + 4 * n
+    if not quasi:
+        per += 2 * n ** 3 + 2 * n * n
+    return per * w.B * w.T * iters
+
+
+class _Legs:
+    """Device timing of the legs of one workload through the C ABI (inputs resident)."""
+
+    def __init__(self, ctx, dev, stream, flush, reps, warmup):
+        self.ctx, self.dev, self.stream, self.flush = ctx, dev, stream, flush
+        self.reps, self.warmup = reps, warmup
+
+    def time(self, fn):
+        import torch
+        for _ in range(self.warmup):
+            fn()
+        torch.cuda.synchronize(self.dev)
+        ts = []
+        for _ in range(self.reps):
+            self.flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(self.stream)
+            fn()
+            b.record(self.stream)
+            torch.cuda.synchronize(self.dev)
+            ts.append(a.elapsed_time(b))
+        return float(statistics.median(ts))
+
+
+def _hbm_entry(ms, nbytes, peak):
+    ach = nbytes / (ms / 1e3) / 1e9
+    return {"bound": "hbm", "alg_bytes": int(nbytes), "achieved": ach, "peak": peak, "unit": "GB/s",
+            "frac": ach / peak}
+
+
+def _tensor_entry(ms, flops, peak, kind):
+    ach = flops / (ms / 1e3) / 1e12
+    return {"bound": "tensor", "alg_flops": int(flops), "achieved": ach, "peak": peak, "unit": "TFLOP/s",
+            "frac": ach / peak, "peak_kind": kind}
+
+
+def _alu_entry(ms, flops, peak):
+    ach = flops / (ms / 1e3) / 1e12
+    return {"bound": "alu", "alg_flops": int(flops), "achieved": ach, "peak": peak, "unit": "TFLOP/s",
+            "frac": ach / peak, "peak_kind": "fp32 FMA: 148 SMs x 128 lanes x 2 flops x max SM clock"}
+
+
+def measure_workload(L, w, inp, parts=None):
+    """Time the legs of workload ``w``; returns {part: entry}."""
+    import torch
+
+    from nonlinear_rnn_solve_b200 import solve
+
+    ctx, dev = L.ctx, L.dev
+    hbm, _ = _peaks()
+    out = {}
+    f32 = lambda k: torch.from_numpy(inp[k]).to(dev)  # noqa: E731
+    sc = {"iters": torch.zeros(1, dtype=torch.int32, device=dev), "delta": torch.zeros(1, device=dev),
+          "residual": torch.zeros(1, device=dev)}
+    elems = w.elems
+    if w.cell == wl.TANH or (w.inp <= 8 and w.H <= 8):
+        t = {k: f32(k) for k in inp if k != "g"}
+        cell = ("tanh_quasi" if w.quasi else "tanh") if w.cell == wl.TANH else w.cell
+        h_out = torch.empty(solve.state_shape(cell, w.B, w.T, w.H), device=dev)
+        kw = dict(x=t["x"], W=t["W"], bias=t["bias"], A=t.get("A"), a=t.get("a"), peep=t.get("peep"))
+        if w.cell == wl.TANH and not w.quasi and w.H == 8:
+            # full DEER at n = 8 from h = 0 overflows in its first update on this input, in
+            # the fp64 oracle as on the device: record that, nothing to time
+            solve.newton_forward(ctx.ctx, cell, w.B, w.T, w.H, h0=t["h0"], max_iters=4, tol=w.tol,
+                                 h_out=h_out, scalars=sc, **kw)
+            torch.cuda.synchronize(dev)
+            st = _ctx_status(ctx)
+            return {"forward": {"diverges_from_zero_guess": True, "iters": int(sc["iters"].item()),
+                                "device_status": st}}
+        fn = lambda: solve.newton_forward(ctx.ctx, cell, w.B, w.T, w.H, h0=t["h0"],  # noqa: E731
+                                          max_iters=w.max_iters, tol=w.tol, h_out=h_out, scalars=sc, **kw)
+        ms = L.time(fn)
+        it = int(sc["iters"].item())
+        e = {"ms": ms, "iters": it, "elems_per_s": elems / (ms / 1e3), "device_status": _ctx_status(ctx)}
+        nb = forward_bytes(w, it, False)
+        if w.cell == wl.TANH:
+            fl = tanh_flops(w, it, w.quasi)
+            e["roofline"] = _alu_entry(ms, fl, _fp32_peak_tflops()) if not w.quasi else _hbm_entry(ms, nb, hbm)
+            e["roofline_other"] = _hbm_entry(ms, nb, hbm) if not w.quasi else _alu_entry(ms, fl, _fp32_peak_tflops())
+        else:
+            e["roofline"] = dict(_hbm_entry(ms, nb, hbm), bound="latency",
+                                 note="8,192 state elements: launch and iteration latency, no bandwidth claim")
+        out["forward"] = e
+        return out
+    # the LLM-width layers: projection GEMM, forward on xproj, adjoint, projection backward
+    parts = parts or LAYER_PARTS
+    B, T, H, K = w.B, w.T, w.H, w.inp
+    M, N = B * T, 3 * H
+    bf = lambda a: torch.from_numpy(wl.bf16_bits(a).view(np.int16)).to(dev).view(torch.bfloat16)  # noqa: E731
+    x = bf(inp["x"].reshape(M, K))
+    W = bf(inp["W"])
+    bias = f32("bias")
+    a = f32("a")
+    peep = f32("peep") if w.cell == wl.LSTM else None
+    h0 = f32("h0")
+    xp = torch.empty(M, N, device=dev)
+    from nonlinear_rnn_solve_b200 import pararnn_input_proj
+    pararnn_input_proj(ctx.ctx, x, W, bias, xp)
+    bf_peak, bf_kind = _bf16_peak_tflops()
+    if "proj" in parts:
+        ms = L.time(lambda: pararnn_input_proj(ctx.ctx, x, W, bias, xp))
+        out["proj"] = {"ms": ms, "shape": f"M{M} K{K} N{N} bf16 -> fp32",
+                       "roofline": _tensor_entry(ms, 2 * M * N * K, bf_peak, bf_kind)}
+    xp4 = xp.view(B, T, 3, H)
+    h = torch.empty(solve.state_shape(w.cell, B, T, H), device=dev)
+    fwd = lambda: solve.newton_forward(ctx.ctx, w.cell, B, T, H, xproj=xp4, a=a, peep=peep,  # noqa: E731
+                                       h0=h0, max_iters=w.max_iters, tol=w.tol, residual=w.residual,
+                                       h_out=h, scalars=sc)
+    if "forward" in parts:
+        ms = L.time(fwd)
+        it = int(sc["iters"].item())
+        e = {"ms": ms, "iters": it, "elems_per_s": elems / (ms / 1e3), "device_status": _ctx_status(ctx)}
+        if w.residual:
+            e["residual"] = float(sc["residual"].item())
+        e["roofline"] = _hbm_entry(ms, forward_bytes(w, it, w.residual), hbm)
+        out["forward"] = e
+    else:
+        fwd()
+    if "backward" in parts or "proj_backward" in parts:
+        g = f32("g")
+        gx = torch.empty(B, T, 3, H, device=dev)
+        gp = torch.empty(5 if w.cell == wl.LSTM else 3, H, device=dev)
+        gh0 = torch.empty_like(h0)
+        from nonlinear_rnn_solve_b200 import make_params, pararnn_adjoint_backward
+        prm = make_params(solve.CELLS[w.cell], B, T, H, 0, a=a, peep=peep)
+        bwd = lambda: pararnn_adjoint_backward(ctx.ctx, xp4, prm, h0, h, g, gx, gp, gh0)  # noqa: E731
+        if "backward" in parts:
+            ms = L.time(bwd)
+            S = w.state_per_unit
+            nb = elems * (4 * S + 12 + 4 * S + 12)  # states, xproj, upstream grad; grad_xproj
+            out["backward"] = {"ms": ms, "elems_per_s": elems / (ms / 1e3), "device_status": _ctx_status(ctx),
+                               "roofline": _hbm_entry(ms, nb, hbm)}
+        else:
+            bwd()
+        del g
+        if "proj_backward" in parts:
+            from nonlinear_rnn_solve_b200 import pararnn_input_proj_backward
+            gxx = torch.empty(M, K, device=dev)
+            gW = torch.empty(N, K, device=dev)
+            gb = torch.empty(N, device=dev)
+            gx2 = gx.view(M, N)
+            ms = L.time(lambda: pararnn_input_proj_backward(ctx.ctx, gx2, x, W, gxx, gW, gb))
+            out["proj_backward"] = {"ms": ms, "shape": f"grad_x [M{M}, K{K}] and grad_W [N{N}, K{K}] from "
+                                                       f"fp32 grad_xproj (bf16 tensor-core products)",
+                                    "roofline": _tensor_entry(ms, 4 * M * N * K, bf_peak, bf_kind)}
+    return out
+
+
+def _ctx_status(ctx):
+    st = ctx.status()
+    return int(st)
+
+
+def per_config(ctx, dev, stream, flush, names=None, with_cpu=True):
+    """Every non-headline workload, leg by leg, with the rollout baselines."""
+    res = {}
+    L = _Legs(ctx, dev, stream, flush, reps=5, warmup=3)
+    for name in names or PER_CONFIG:
+        w = wl.WORKLOADS[name]
+        inp = wl.generate(w)
+        t0 = time.perf_counter()
+        r = {"shape": {"B": w.B, "T": w.T, "H": w.H, "in": w.inp, "tol": w.tol, "max_iters": w.max_iters}}
+        try:
+            r.update(measure_workload(L, w, inp))
+        except Exception as e:  # a failing leg is reported, the others still run
+            r["error"] = f"{type(e).__name__}: {e}"
+        if with_cpu and not (w.cell == wl.TANH and not w.quasi and w.H == 8):
+            allc, one = cpu_baselines(w, inp)
+            r["cpu_rollout"] = allc
+            r["cpu_rollout_1core"] = one
+            fw = r.get("forward", {})
+            if "elems_per_s" in fw:
+                r["speedup_vs_rollout"] = fw["elems_per_s"] / allc["value"]
+                r["speedup_vs_rollout_1core"] = fw["elems_per_s"] / one["value"]
+        r["wall_s"] = time.perf_counter() - t0
+        res[name] = r
+        del inp
+    return res
+
+
+def run_leg(args):
+    """Time one leg alone and print its line (the profiling runs use this)."""
+    import torch
+
+    from nonlinear_rnn_solve_b200 import Context
+    name, _, part = args.leg.partition(":")
+    w = wl.WORKLOADS[name]
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    ctx = Context(0, stream)
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    L = _Legs(ctx, dev, stream, flush, reps=args.steps, warmup=args.warmup)
+    inp = wl.generate(w)
+    r = measure_workload(L, w, inp, parts=[part] if part else None)
+    print(json.dumps({"leg": args.leg, "steps": args.steps, "warmup": args.warmup, "result": r}), flush=True)
+    ctx.close()
 
 
 def run_reference(args, w):
@@ -185,26 +522,26 @@ def run_reference(args, w):
         return
     inp = wl.generate(w)
     import oracle
-    threads = len(os.sched_getaffinity(0))
+    threads = _oracle_threads()
     oracle.set_threads(threads)
     m = oracle.model_from_inputs(w.cell, inp, quasi=w.quasi)
     for _ in range(args.warmup):
-        m.newton(inp["h0"], max_iters=w.max_iters, tol=w.tol)
+        m.rollout(inp["h0"])
     ts = []
-    iters = 0
     for _ in range(args.steps):
         t0 = time.perf_counter()
-        _, iters, _ = m.newton(inp["h0"], max_iters=w.max_iters, tol=w.tol)
+        m.rollout(inp["h0"])
         ts.append(time.perf_counter() - t0)
     ms = 1e3 * sum(ts) / len(ts)
     value = w.elems / (ms / 1e3)
     line = {"metric": METRIC, "value": value, "unit": "state elements/s", "n_gpus": ws, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
-            "config": {"workload": w.name, "B": w.B, "T": w.T, "H": w.H, "in": w.inp, "iters": iters,
-                       "tol": w.tol},
+            "config": {"workload": w.name, "B": w.B, "T": w.T, "H": w.H, "in": w.inp, "tol": w.tol},
             "cpu_baseline": {"value": value, "unit": "state elements/s", "cores": threads, "kind": "oracle",
-                             "sample": f"whole workload per step, fp64 oracle Newton solve ({iters} iterations)"},
+                             "sample": "whole workload per step: fp64 oracle sequential rollout "
+                                       "h_t = f(h_{t-1}, x_t), OpenMP over independent sequences"},
+            "oracle_newton": cpu_newton(w, inp, threads),
             "e2e": {"value": value, "unit": "state elements/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -279,10 +616,12 @@ def run_ours(args, w):
     stream = torch.cuda.current_stream(dev)
     ctx = Context(dev.index, stream)
 
+    sc = {"iters": torch.zeros(1, dtype=torch.int32, device=dev), "delta": torch.zeros(1, device=dev)}
+
     def step(h_out=None):
         return solve.newton_forward(ctx.ctx, w.cell, w.B, w.T, w.H, x=t["x"], W=t["W"], bias=t["bias"],
                                     a=t.get("a"), peep=t.get("peep"), h0=t["h0"], max_iters=w.max_iters,
-                                    tol=w.tol, h_out=h_out)
+                                    tol=w.tol, h_out=h_out, scalars=sc)
 
     h_out = torch.empty(solve.state_shape(w.cell, w.B, w.T, w.H), device=dev)
     for _ in range(max(args.warmup, 3)):
@@ -348,7 +687,9 @@ def run_ours(args, w):
             "wall_s_timed": wall,
         }
         if ws == 1 and not args.skip_extras:
-            line["cpu_baseline"] = _cpu_oracle_sample(w, inp)
+            allc, one = cpu_baselines(w, inp)
+            line["cpu_baseline"] = dict(allc, one_core=one, oracle_newton=cpu_newton(w, inp, allc["cores"]))
+            line["per_config"] = per_config(ctx, dev, stream, flush)
         print(json.dumps(line), flush=True)
     ctx.close()
     if ws > 1:
@@ -363,10 +704,14 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=wl.BENCH_WORKLOAD, choices=sorted(wl.WORKLOADS))
     ap.add_argument("--skip-extras", action="store_true",
-                    help="skip the e2e and CPU-baseline legs (for profiler runs)")
+                    help="skip the e2e, CPU-baseline and per-config legs (for profiler runs)")
+    ap.add_argument("--leg", default=None,
+                    help="WORKLOAD[:PART]: time one leg alone (PART: proj, forward, backward, proj_backward)")
     args = ap.parse_args()
     w = wl.WORKLOADS[args.workload]
-    if args.impl == "reference":
+    if args.leg:
+        run_leg(args)
+    elif args.impl == "reference":
         run_reference(args, w)
     else:
         run_ours(args, w)

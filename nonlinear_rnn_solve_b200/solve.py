@@ -31,9 +31,11 @@ def _need(t, count, name):
 
 def newton_forward(ctx, cell, B, T, H, *, xproj=None, x=None, W=None, bias=None, a=None,
                    peep=None, A=None, h0=None, max_iters=None, tol=1e-6, residual=False,
-                   h_out=None, solver="newton", damping=0.0):
+                   h_out=None, solver="newton", damping=0.0, scalars=None):
     """Newton / quasi-Newton (or Jacobi / Picard) solve.  Returns dict(h, iters, delta,
-    residual) (device tensors)."""
+    residual) (device tensors).  ``scalars``: optional dict with preallocated one-element
+    device tensors "iters" (int32), "delta" and "residual" (fp32), reused instead of
+    allocating new ones (no fill launches around the solve)."""
     dev = (xproj if xproj is not None else x).device
     inp = 0 if x is None else x.shape[-1]
     G = 1 if cell in ("tanh", "tanh_quasi") else 3
@@ -56,9 +58,16 @@ def newton_forward(ctx, cell, B, T, H, *, xproj=None, x=None, W=None, bias=None,
                       bias=bias if xproj is None else None, solver=SOLVERS[solver], damping=damping)
     if h_out is None:
         h_out = torch.empty(state_shape(cell, B, T, H), device=dev, dtype=torch.float32)
-    iters = torch.zeros(1, device=dev, dtype=torch.int32)
-    delta = torch.zeros(1, device=dev, dtype=torch.float32)
-    res = torch.zeros(1, device=dev, dtype=torch.float32) if residual else None
+    if scalars is not None:
+        iters, delta = scalars["iters"], scalars["delta"]
+        res = scalars["residual"] if residual else None
+        _need(iters, 1, "iters")
+        _need(delta, 1, "delta")
+        _need(res, 1, "residual")
+    else:
+        iters = torch.zeros(1, device=dev, dtype=torch.int32)
+        delta = torch.zeros(1, device=dev, dtype=torch.float32)
+        res = torch.zeros(1, device=dev, dtype=torch.float32) if residual else None
     pararnn_newton_forward(ctx, xproj, prm, h0, h_out, T if max_iters is None else max_iters, tol,
                            iters, delta, res)
     return {"h": h_out, "iters": iters, "delta": delta, "residual": res}

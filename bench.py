@@ -286,7 +286,9 @@ def _bf16_peak_tflops():
 def forward_bytes(w, iters, residual):
     """Algorithmic HBM bytes of one Newton forward solve: each iteration reads the inputs
     and the previous iterate once and writes the new one (the first reads no iterate, it
-    is zero); the residual pass reads the inputs and the result once."""
+    is zero).  The residual at the result needs one more read of the inputs and states,
+    except when the solve ran to its cap on a wide layer (H % 32 == 0, projected inputs):
+    there the last iteration forms it from the inputs it already holds."""
     S, n = w.state_per_unit, w.H
     elems = w.B * w.T * w.H
     if w.cell == wl.TANH or (w.inp <= 8 and w.H <= 8):
@@ -302,6 +304,8 @@ def forward_bytes(w, iters, residual):
         res = pb + sb
     if iters <= 0:
         return 0
+    if residual and w.H % 32 == 0 and not (w.inp <= 8 and w.H <= 8) and w.cell != wl.TANH and iters == w.max_iters:
+        res = 0
     return per_first + (iters - 1) * per_next + (res if residual else 0)
 
 

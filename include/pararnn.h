@@ -217,7 +217,12 @@ int pararnn_lsim(pararnn_ctx *ctx, const float *A, const float *Bm, const float 
  *   grad_h      like h (LSTM: (dL/dc, dL/dh) pairs)
  *   grad_xproj  [B, T, 3, H]
  *   grad_params GRU [3, H] = d/d(a_z, a_r, a_c); LSTM [5, H] = d/d(a_f, a_g, a_o, w_f, w_o)
- *               (overwritten; summed with float atomics, so the summation order varies)
+ *               (overwritten).  Summation: when NPAR * H <= 12288 each CTA accumulates
+ *               its terms in a shared-memory table with shared atomics and the per-CTA
+ *               tables are summed over CTAs in a fixed order; otherwise each tile adds
+ *               its per-unit sums with global float atomics.  Either way the order of
+ *               additions inside a CTA depends on thread timing, so the last bits can
+ *               differ between runs.
  *   grad_h0     like h0, or NULL */
 int pararnn_adjoint_backward(pararnn_ctx *ctx, const float *xproj, const pararnn_params *p,
                              const float *h0, const float *h, const float *grad_h,
@@ -237,7 +242,9 @@ const char *pararnn_strerror(int status);
  * knob 3: device pointer (float*) receiving delta_k of every Newton iteration, with
  *         knob 4 its capacity (0 disables).
  * knob 5: non-zero makes the long-sequence Newton tiles take every carry from the
- *         look-back, never from their own halo (tests of the look-back path). */
+ *         look-back, never from their own halo (tests of the look-back path).
+ * knob 6: tile shape of the wide-layer Newton kernel (H % 32 == 0, xproj given):
+ *         0 the default, 1 and 2 alternatives (measurements and tests). */
 int pararnn_debug_set(pararnn_ctx *ctx, int knob, long long value);
 
 /* Number of kernels the last call launched on the stream. */

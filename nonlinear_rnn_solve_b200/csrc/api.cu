@@ -182,7 +182,7 @@ int pararnn_newton_forward(pararnn_ctx *ctx, const float *xproj, const pararnn_p
         const int jmode = jm_solver ? jm_solver : (p->cell == PARARNN_LSTM_CIFG_PEEP_QUASI ? 1 : 0);
         if (!p->a || (lstm && !p->peep)) return PARARNN_EINVAL;
         prn::NewtonDiagReq r{lstm, jmode, p->B, p->T, p->H, p->in, xproj, p->x, p->W, p->bias, p->a, p->peep, h0, h_out,
-                             max_iters, tol, iters_out, final_delta_out, residual_out};
+                             max_iters, tol, iters_out, final_delta_out, residual_out, ctx->dbg.wide_variant};
         const bool elk = p->solver == PARARNN_SOLVER_ELK;
         if ((elk ? prn::elk_plan(r, ctx->num_sms, &plan) : prn::newton_diag_plan(r, ctx->num_sms, &plan)))
             return PARARNN_ECUDA;
@@ -383,6 +383,10 @@ int pararnn_debug_set(pararnn_ctx *ctx, int knob, long long value) {
             ctx->dbg.delta_log_cap = (int)value;
             return PARARNN_OK;
         case 5: ctx->dbg.no_halo = value != 0; return PARARNN_OK;
+        case 6:
+            if (value < 0 || value > 2) return PARARNN_EINVAL;
+            ctx->dbg.wide_variant = (int)value;
+            return PARARNN_OK;
         default: return PARARNN_EINVAL;
     }
 }

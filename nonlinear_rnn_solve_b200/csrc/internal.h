@@ -44,6 +44,7 @@ struct DbgHost {
     float *delta_log = nullptr;
     int delta_log_cap = 0;
     int no_halo = 0;
+    int wide_variant = 0;
 };
 
 // ---- Newton forward, diagonal / 2x2-block cells (GRU, LSTM) -----------------------
@@ -57,6 +58,7 @@ struct NewtonDiagReq {
     float tol;
     int *iters_out;
     float *delta_out, *residual_out;
+    int variant = 0;  // tile shape of the wide-layer kernel (0: the default)
 };
 int newton_diag_plan(const NewtonDiagReq &r, int num_sms, Plan *plan);
 int newton_staged_plan(const NewtonDiagReq &r, int num_sms, Plan *plan);  // 1: shape not covered

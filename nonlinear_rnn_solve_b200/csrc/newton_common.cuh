@@ -114,6 +114,10 @@ struct StagedMaps {
 
 // Launch of a staged plan (newton_staged.cu).
 cudaError_t newton_staged_launch(const NewtonDiagArgs &A, const Plan &plan, cudaStream_t st);
+// Wide layers, H % 32 == 0 with projected inputs (newton_wide.cu): plan (1 = shape not
+// covered) and launch.
+int newton_wide_plan(const NewtonDiagReq &r, int num_sms, Plan *plan);
+cudaError_t newton_wide_launch(const NewtonDiagArgs &A, const Plan &plan, cudaStream_t st);
 
 // Final residual r = max over every state element of |h_t - f(h_{t-1}, x_t)| at the
 // returned iterate (one read of the states and inputs), reduced over the grid.

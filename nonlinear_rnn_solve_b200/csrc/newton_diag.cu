@@ -266,6 +266,7 @@ cudaError_t newton_diag_launch(const NewtonDiagReq &r, const Plan &plan, const W
     A.dbg.delta_log_cap = dbg.delta_log_cap;
     // a withheld publication (failure-detection test) must be met by the look-back
     A.dbg.no_halo = dbg.no_halo || dbg.skip_tile >= 0;
+    if (plan.staged == 2) return newton_wide_launch(A, plan, st);
     if (plan.staged) return newton_staged_launch(A, plan, st);
     void *args[] = {&A};
     return cudaLaunchCooperativeKernel(plan.kernel, dim3(plan.grid), dim3(kThreads), args, plan.dyn_smem, st);

@@ -699,6 +699,8 @@ int newton_staged_plan(const NewtonDiagReq &r, int num_sms, Plan *plan) {
         }
         plan->staged_tma = tma ? 1 : 0;
     } else if (r.H % 32 == 0 && !fused) {
+        const int wide = newton_wide_plan(r, num_sms, plan);
+        if (wide <= 0) return wide;
         plan->variant = 132;
         rc = S == 1 ? choose<GruCell, Wide<GruCell, 16, kThreads>, 0>(plan, num_sms, r.B, r.T, r.H)
                     : choose<LstmCell, Wide<LstmCell, 8, kThreads>, 0>(plan, num_sms, r.B, r.T, r.H);

@@ -62,8 +62,30 @@ def test_withheld_publication_in_newton_times_out(ctx):
     assert max_abs(host(out["h"]), h_ref) <= 1e-4
 
 
-def test_nan_input_reports_nonfinite(ctx):
-    B, T, H = 1, 500, 4
+def test_withheld_publication_in_wide_newton_times_out(ctx):
+    """The wide-layer kernel (H % 32 == 0, xproj given): tile 1 of 3 withholds its
+    publication, tile 2's bounded wait runs out, and the context recovers."""
+    B, T, H = 1, 3 * 128, 32
+    rng = np.random.default_rng(4)
+    xp = rng.standard_normal((B, T, 3, H)).astype(np.float32)
+    a = rng.uniform(-0.5, 0.5, (3, H)).astype(np.float32)
+    pararnn_debug_set(ctx.ctx, 1, 50_000_000)
+    pararnn_debug_set(ctx.ctx, 2, 1)
+    solve.newton_forward(ctx.ctx, "gru", B, T, H, xproj=gpu(xp), a=gpu(a), max_iters=10, tol=1e-6)
+    torch.cuda.synchronize()
+    assert ctx.status() == PARARNN_ETIMEOUT
+    pararnn_debug_set(ctx.ctx, 2, -1)
+    out = solve.newton_forward(ctx.ctx, "gru", B, T, H, xproj=gpu(xp), a=gpu(a), max_iters=T, tol=1e-6)
+    torch.cuda.synchronize()
+    assert ctx.status() == 0
+    h_ref, it_ref, _ = oracle.Model("gru", xp, a=a).newton(max_iters=T, tol=1e-6)
+    assert int(out["iters"].item()) == it_ref
+    assert max_abs(host(out["h"]), h_ref) <= 1e-4
+
+
+@pytest.mark.parametrize("H", [4, 64])
+def test_nan_input_reports_nonfinite(ctx, H):
+    B, T = 1, 500
     rng = np.random.default_rng(3)
     xp = rng.standard_normal((B, T, 3, H)).astype(np.float32)
     xp[0, 123, 1, 2] = np.nan

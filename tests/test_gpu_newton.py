@@ -124,6 +124,28 @@ def test_xproj_path_fixed_iterations(ctx, cell, B, T, H):
         assert abs(float(out["residual"].item()) - m.residual(host(out["h"]), h0)) <= 1e-5 * scale
 
 
+@pytest.mark.parametrize("cell,B,T,H", [("gru", 2, 700, 64), ("lstm", 3, 333, 64)])
+def test_wide_converged_with_separate_residual(ctx, cell, B, T, H):
+    """Wide layers (H % 32 == 0, xproj given) solved to tolerance: the solve stops before
+    the cap, so the residual takes its own pass; several sequences and a ragged last
+    tile (the staged box of the last tile reaches into the next sequence's rows)."""
+    rng = np.random.default_rng(B * 11 + T + H)
+    xp = (rng.standard_normal((B, T, 3, H)) * 0.8).astype(np.float32)
+    a = rng.uniform(-0.9, 0.9, (3, H)).astype(np.float32)
+    peep = rng.uniform(-0.5, 0.5, (2, H)).astype(np.float32) if cell == "lstm" else None
+    h0 = (rng.standard_normal((B, H, 2) if cell == "lstm" else (B, H)) * 0.3).astype(np.float32)
+    m = oracle.Model(cell, xp, a=a, peep=peep)
+    h_ref, it_ref, _ = m.newton(h0, max_iters=T, tol=1e-6)
+    out = solve.newton_forward(ctx.ctx, cell, B, T, H, xproj=gpu(xp), a=gpu(a),
+                               peep=None if peep is None else gpu(peep), h0=gpu(h0), max_iters=T, tol=1e-6,
+                               residual=True)
+    torch.cuda.synchronize()
+    assert ctx.status() == 0
+    assert int(out["iters"].item()) == it_ref
+    assert max_abs(host(out["h"]), h_ref) <= TOL_STATE
+    assert abs(float(out["residual"].item()) - m.residual(host(out["h"]), h0)) <= 2e-6
+
+
 def test_zero_iterations_returns_initial_guess(ctx):
     w = _small_workload("gru", 2, 100, 4, 2, 3)
     inp = wl.generate(w)

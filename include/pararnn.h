@@ -243,8 +243,8 @@ const char *pararnn_strerror(int status);
  *         knob 4 its capacity (0 disables).
  * knob 5: non-zero makes the long-sequence Newton tiles take every carry from the
  *         look-back, never from their own halo (tests of the look-back path).
- * knob 6: tile shape of the wide-layer Newton kernel (H % 32 == 0, xproj given):
- *         0 the default, 1 and 2 alternatives (measurements and tests). */
+ * knob 6: channels per tile of the wide-layer Newton kernel (H % 32 == 0, xproj
+ *         given): 8, 16 or 32; 0 is the default (32). */
 int pararnn_debug_set(pararnn_ctx *ctx, int knob, long long value);
 
 /* Number of kernels the last call launched on the stream. */

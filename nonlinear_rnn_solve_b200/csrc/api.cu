@@ -384,7 +384,7 @@ int pararnn_debug_set(pararnn_ctx *ctx, int knob, long long value) {
             return PARARNN_OK;
         case 5: ctx->dbg.no_halo = value != 0; return PARARNN_OK;
         case 6:
-            if (value < 0 || value > 2) return PARARNN_EINVAL;
+            if (value != 0 && value != 8 && value != 16 && value != 32) return PARARNN_EINVAL;
             ctx->dbg.wide_variant = (int)value;
             return PARARNN_OK;
         default: return PARARNN_EINVAL;

@@ -14,10 +14,10 @@
 //   - every thread evaluates f, J and r = f - h^(k) for its L steps of one channel in
 //     registers (J and r never reach memory), composes them, and the CTA scans the
 //     sub-chunks (one barrier);
-//   - the carry entering the tile comes from the predecessor tile's inclusive value,
-//     which warp 0 reads before the compute phase (the predecessor normally finished a
-//     round earlier), so the common path has no look-back wait and no second barrier;
-//     otherwise the decoupled look-back of common.cuh resolves it;
+//   - the carry entering the tile is the predecessor tile's inclusive value (a chained
+//     scan across tiles): warp 0 reads it before the compute phase, when the predecessor
+//     normally finished a round earlier, and otherwise waits for it before the scan's
+//     barrier while the other warps compute -- one CTA barrier per tile either way;
 //   - h^(k+1) = h^(k) + delta is written in place (h^(k) re-read from the stage; each warp
 //     stores 128 contiguous bytes per step); the tile's last state goes to a side buffer
 //     for the successor's next iteration;
@@ -35,19 +35,26 @@
 
 namespace prn {
 
-template <class Cell, int LL, int NS> struct WideCfg {
-    static constexpr int S = Cell::S, C = 32, L = LL, SUB = kThreads / C, TCH = SUB * L, NST = NS;
+// A tile is CC channels x SUB = 256 / CC sub-chunks of L steps; a warp holds 32 / CC
+// sub-chunks.  Shared-memory rows are dense (as the TMA writes them), so the sub-chunks
+// of a warp must fall on different bank groups: for CC < 32 the row offset between
+// them, L rows of 3 CC (inputs) or CC S (states) floats, must not be a multiple of 32
+// banks (L = 7 serves CC = 16 and 8).
+template <class Cell, int CC, int LL, int NS> struct WideCfg {
+    static constexpr int S = Cell::S, C = CC, L = LL, SUB = kThreads / C, TCH = SUB * L, NST = NS;
     static constexpr int ROWP = 3 * C, ROWH = C * S;
     static constexpr int XF = TCH * ROWP, HF = TCH * ROWH;  // floats of the two boxes
     static constexpr int STAGE = XF + HF;                  // floats of one stage
     static constexpr int SMEM_FLOATS = NST * STAGE;
-    static_assert(L % 4 == 0 && TCH <= 256, "TMA box height");
-    static_assert((STAGE * 4) % 1024 == 0 && (XF * 4) % 128 == 0, "stage alignment");
+    static_assert(32 % C == 0 && TCH <= 256, "channels per tile divide a warp; TMA box height");
+    static_assert((STAGE * 4) % 128 == 0 && (XF * 4) % 128 == 0, "stage alignment");
+    static_assert(C == 32 || ((L * ROWP) % 32 != 0 && (L * ROWP * (32 / C / 2)) % 32 != 0),
+                  "sub-chunks of a warp on distinct bank groups");
 };
 
 // Per-CTA state of the wide kernel: the staging ring and the tile schedule.
-template <class Cell, int L, int NST> struct WideRun {
-    using G = WideCfg<Cell, L, NST>;
+template <class Cell, int CC, int L, int NST> struct WideRun {
+    using G = WideCfg<Cell, CC, L, NST>;
     static constexpr int S = Cell::S, C = G::C, SUB = G::SUB, TCH = G::TCH;
     const NewtonDiagArgs &A;
     const StagedMaps &M;
@@ -55,19 +62,34 @@ template <class Cell, int L, int NST> struct WideRun {
     unsigned long long *bar;  // [NST] stage-full barriers
     unsigned *done;           // [NST] warps finished with the stage (shared counters)
     ScanSmem<S, C> *sm2;      // [2] by tile parity
-    int *s_known, *s_fail;
+    int *s_fail;
     int tid, c, s, nct, nseq, nchunk;
     long ntiles, ntile_cta;
     size_t side_stride;
     LookBack<S> lb;
     unsigned phase = 0;    // bit j: parity of stage j's next completion (every thread)
     unsigned pending = 0;  // bit j: stage j has a copy in flight not yet waited for
-
-    // Tile `j` of this CTA within an iteration: its coordinates.
-    __device__ __forceinline__ void coords(long j, int &ch, int &sq) const {
-        const long tile = blockIdx.x + j * (long)gridDim.x;
-        ch = (int)(tile / nseq);
-        sq = (int)(tile - (long)ch * nseq);
+    // Coordinates (chunk, seq) of this CTA's current tile and of the tile NST places
+    // ahead, stepped by gridDim.x tiles without dividing (tile = chunk * nseq + seq).
+    struct Pos {
+        int chunk, seq;
+    };
+    Pos cur, ahead;
+    int step_ch, step_sq;
+    __device__ __forceinline__ void step(Pos &p) const {
+        p.chunk += step_ch;
+        p.seq += step_sq;
+        if (p.seq >= nseq) {
+            p.seq -= nseq;
+            ++p.chunk;
+        }
+    }
+    // Reset the walkers to this CTA's first tile (start of an iteration).
+    __device__ __forceinline__ void restart() {
+        cur.chunk = (int)(blockIdx.x / (unsigned)nseq);
+        cur.seq = (int)(blockIdx.x % (unsigned)nseq);
+        ahead = cur;
+        for (int q = 0; q < NST; ++q) step(ahead);
     }
     // Stage st <- tile (ch, sq); one thread calls it.  The proxy fences order this CTA's
     // earlier ordinary stores (h) and shared-memory reads before the TMA's accesses.
@@ -92,10 +114,10 @@ template <class Cell, int L, int NST> struct WideRun {
     // Bounded wait for stage st (each thread on the mbarrier).
     __device__ __forceinline__ bool wait(int st) {
         const unsigned par = (phase >> st) & 1u;
-        bool ok = mbar_try(bar + st, par);
+        bool ok = mbar_try_sleep(bar + st, par, 20000u);
         if (!ok) {
             const unsigned long long t0 = gtimer();
-            while (!(ok = mbar_try(bar + st, par))) {
+            while (!(ok = mbar_try_sleep(bar + st, par, 20000u))) {
                 if (ld_relaxed_int(&A.ctl->abort)) break;
                 if (gtimer() - t0 > A.dbg.wait_ns) {
                     raise_status(A.sticky, A.ctl, kStTimeout, true);
@@ -122,10 +144,10 @@ template <class Cell, int L, int NST> struct WideRun {
     // The first min(NST, tiles of this CTA) tiles of an iteration, into stages 0, 1, ..
     // (thread 0 issues; every thread records them).
     __device__ __forceinline__ void prologue(bool with_h) {
-        for (int j = 0; j < NST && j < ntile_cta; ++j) {
-            int ch, sq;
-            coords(j, ch, sq);
-            if (tid == 0) issue(j, ch, sq, with_h);
+        restart();
+        Pos w = cur;
+        for (int j = 0; j < NST && j < ntile_cta; ++j, step(w)) {
+            if (tid == 0) issue(j, w.chunk, w.seq, with_h);
             pending |= 1u << j;
         }
     }
@@ -156,8 +178,7 @@ template <class Cell, int L, int NST> struct WideRun {
         const float *shh = sx + G::XF;           // [TCH][32 * S]
         ScanSmem<S, C> &sm = sm2[par];
         const long tile = blockIdx.x + j * (long)gridDim.x;
-        int chunk, seq;
-        coords(j, chunk, seq);
+        const int chunk = cur.chunk, seq = cur.seq;
         const int b = seq / nct, ct = seq % nct;
         const int h = ct * C + c;
         const int t0 = chunk * TCH + s * L;
@@ -173,7 +194,8 @@ template <class Cell, int L, int NST> struct WideRun {
 #pragma unroll
             for (int q = 0; q < S; ++q) hp[q] = side_in[((tile - nseq) * C + c) * S + q];
         }
-        // warp 0: the predecessor's inclusive value, read early (epoch-tagged words)
+        // first row of sub-chunks (lanes c < C of warp 0): the predecessor's inclusive
+        // value, read early (epoch-tagged words)
         unsigned long long pw[S];
 #pragma unroll
         for (int q = 0; q < S; ++q) pw[q] = 0ull;
@@ -182,11 +204,7 @@ template <class Cell, int L, int NST> struct WideRun {
             for (int q = 0; q < S; ++q) pw[q] = ld_relaxed_u64(lb.inc + ((tile - nseq) * C + c) * S + q);
         }
         if (!wait(st)) *s_fail = 1;  // acted on after the scan's barrier
-        if (tid == 32 && j + NST < ntile_cta) {
-            int nch, nsq;
-            coords(j + NST, nch, nsq);
-            prefetch(nch, nsq, k > 0);
-        }
+        if (tid == 32 && j + NST < ntile_cta) prefetch(ahead.chunk, ahead.seq, k > 0);
         if (k > 0 && s > 0) {
 #pragma unroll
             for (int q = 0; q < S; ++q) hp[q] = shh[(s * L - 1) * G::ROWH + c * S + q];
@@ -216,46 +234,58 @@ template <class Cell, int L, int NST> struct WideRun {
         Aff<S> e = Aff<S>::ident();
 #pragma unroll
         for (int i = 0; i < L; ++i) e = compose(e, make_aff<S>(Jr[i], rr[i]));
-        if (s == 0) {
+        if (tid < 32) {
+            // warp 0 (its lanes c >= C belong to later sub-chunks): the carry entering the
+            // tile is the predecessor's inclusive value.  Read before the compute phase, it
+            // is normally there already; otherwise warp 0 waits for it here, before the
+            // scan's barrier, while the other warps still compute.  The predecessor has a
+            // lower tile index, so it belongs to a resident CTA (or came earlier in this
+            // one) and never waits on this tile.
             bool ok = true;
-            float cv[S];
 #pragma unroll
-            for (int q = 0; q < S; ++q) {
-                cv[q] = 0.f;  // a sequence's first tile: delta entering t = 0 is 0
-                if (chunk > 0) {
-                    ok &= (unsigned)pw[q] == epoch;
-                    cv[q] = __uint_as_float((unsigned)(pw[q] >> 32));
+            for (int q = 0; q < S; ++q)
+                if (s == 0 && chunk > 0) ok &= (unsigned)pw[q] == epoch;
+            if (!__all_sync(0xffffffffu, ok)) {
+                const unsigned long long *src = lb.inc + ((tile - nseq) * C + c) * S;
+                unsigned long long t0 = 0;
+                for (int polls = 0;; ++polls) {
+                    ok = true;
+                    if (s == 0) {
+#pragma unroll
+                        for (int q = 0; q < S; ++q) {
+                            pw[q] = ld_relaxed_u64(src + q);
+                            ok &= (unsigned)pw[q] == epoch;
+                        }
+                    }
+                    if (__all_sync(0xffffffffu, ok)) break;
+                    int bad = 0;
+                    if (tid == 0) {
+                        if (ld_relaxed_int(&A.ctl->abort)) bad = 1;
+                        if (polls == 4) t0 = gtimer();
+                        if (polls > 4 && gtimer() - t0 > A.dbg.wait_ns) {
+                            raise_status(A.sticky, A.ctl, kStTimeout, true);
+                            bad = 1;
+                        }
+                    }
+                    if (__shfl_sync(0xffffffffu, bad, 0)) {
+                        if (tid == 0) *s_fail = 1;
+                        break;
+                    }
+                    if (polls > 4) __nanosleep(32);
                 }
             }
-            const bool known = __all_sync(0xffffffffu, ok) && A.dbg.skip_tile < 0;
-            if (known) {
+            if (s == 0) {
 #pragma unroll
-                for (int q = 0; q < S; ++q) sm.carry[c][q] = cv[q];
+                for (int q = 0; q < S; ++q) sm.carry[c][q] = chunk > 0 ? __uint_as_float((unsigned)(pw[q] >> 32)) : 0.f;
             }
-            if (c == 0) s_known[par] = known ? 1 : 0;
         }
         Aff<S> excl, total;
-        cta_scan<S, C>(e, sm, excl, total);  // the one CTA barrier of the common path
+        cta_scan<S, C>(e, sm, excl, total);  // the one CTA barrier of a tile
         if (*s_fail) {
             drain();
             return false;  // a bounded wait ran out; the status says so
         }
-        if (s_known[par]) {
-            if (s == 0) publish_inc<S, C>(lb, total, sm.carry[c], tile, epoch, A.dbg);
-        } else {
-            if (s == 0) {
-                float base[S];
-#pragma unroll
-                for (int q = 0; q < S; ++q) base[q] = 0.f;
-                if (!look_back<S, C>(lb, sm, total, tile, chunk, nseq, epoch, base, A.ctl, A.sticky, A.dbg))
-                    if (c == 0) *s_fail = 1;
-            }
-            __syncthreads();
-            if (*s_fail) {
-                drain();
-                return false;
-            }
-        }
+        if (tid < 32) publish_inc<S, C>(lb, total, sm.carry[c], tile, epoch, A.dbg);
         float d[S];
         excl.apply(sm.carry[c], d);
         if (FUSE && t0 > 0) {
@@ -314,27 +344,26 @@ template <class Cell, int L, int NST> struct WideRun {
                          : "=r"(cnt)
                          : "r"(smem_addr(done + st))
                          : "memory");
-            if (cnt == SUB - 1) {
+            if (cnt == kThreads / 32 - 1) {  // every warp of the CTA is done with it
                 done[st] = 0;
-                int nch, nsq;
-                coords(j + NST, nch, nsq);
-                issue(st, nch, nsq, k > 0);
+                issue(st, ahead.chunk, ahead.seq, k > 0);
             }
         }
+        step(cur);
+        step(ahead);
         return true;
     }
 };
 
 // RES: a residual is asked for (the instantiation without it carries no residual code).
-template <class Cell, int L, int NST, int MINB, bool RES>
+template <class Cell, int CC, int L, int NST, int MINB, bool RES>
 __global__ void __launch_bounds__(kThreads, MINB)
     newton_wide_kernel(const NewtonDiagArgs A, const __grid_constant__ StagedMaps M) {
-    using R = WideRun<Cell, L, NST>;
+    using R = WideRun<Cell, CC, L, NST>;
     using G = typename R::G;
     constexpr int S = Cell::S, C = G::C, TCH = G::TCH;
     extern __shared__ __align__(1024) unsigned char smraw[];
     __shared__ ScanSmem<S, C> sm2[2];
-    __shared__ int s_known[2];
     __shared__ unsigned s_red[kThreads / 32];
     __shared__ int s_fail;
     __shared__ unsigned s_done[NST];
@@ -344,13 +373,14 @@ __global__ void __launch_bounds__(kThreads, MINB)
     r.bar = s_bar;
     r.done = s_done;
     r.sm2 = sm2;
-    r.s_known = s_known;
     r.s_fail = &s_fail;
     r.tid = threadIdx.x;
     r.c = threadIdx.x % C;
     r.s = threadIdx.x / C;
     r.nct = A.H / C;
     r.nseq = A.B * r.nct;
+    r.step_ch = (int)(gridDim.x / (unsigned)r.nseq);
+    r.step_sq = (int)(gridDim.x % (unsigned)r.nseq);
     r.nchunk = (A.T + TCH - 1) / TCH;
     r.ntiles = (long)r.nseq * r.nchunk;
     r.ntile_cta = blockIdx.x < r.ntiles ? (r.ntiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
@@ -381,8 +411,7 @@ __global__ void __launch_bounds__(kThreads, MINB)
         float my_max = 0.f, my_res = 0.f;
         bool my_bad = false;
         for (long j = 0; j < r.ntile_cta; ++j) {
-            const long tile = blockIdx.x + j * (long)gridDim.x;
-            const bool full = (tile / r.nseq + 1) * TCH <= A.T;
+            const bool full = (r.cur.chunk + 1) * TCH <= A.T;
             bool ok;
             if (RES && fuse_res)
                 ok = full ? r.template tile<true, RES>(k, j, epoch, side_in, side_out, my_max, my_res, my_bad)
@@ -459,10 +488,12 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-template <class Cell, int L, int NST, int MINB>
+template <class Cell, int CC, int L, int NST, int MINB>
 int choose_wide(Plan *plan, int num_sms, long B, long T, long H, bool res) {
-    using G = WideCfg<Cell, L, NST>;
-    auto kern = res ? &newton_wide_kernel<Cell, L, NST, MINB, true> : &newton_wide_kernel<Cell, L, NST, MINB, false>;
+    using G = WideCfg<Cell, CC, L, NST>;
+    if (H % CC) return 1;
+    auto kern = res ? &newton_wide_kernel<Cell, CC, L, NST, MINB, true>
+                    : &newton_wide_kernel<Cell, CC, L, NST, MINB, false>;
     const int smem = G::SMEM_FLOATS * (int)sizeof(float) + 1024;
     const void *f = reinterpret_cast<const void *>(kern);
     if (cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess ||
@@ -482,29 +513,29 @@ int choose_wide(Plan *plan, int num_sms, long B, long T, long H, bool res) {
 }  // namespace
 
 // Wide layers: H % 32 == 0 with projected inputs.  Returns 1 when the shape is not covered.
+// Channels per tile: 32 (128-byte rows per gate and step); 16 and 8 are selectable for
+// measurements and tests (debug knob 6) and measured slower on the layer shapes.
 int newton_wide_plan(const NewtonDiagReq &r, int num_sms, Plan *plan) {
     if (r.H % 32 || r.xproj == nullptr || !encode_fn()) return 1;
     if ((long)r.B * r.T >= (1L << 31)) return 1;  // TMA row coordinates are 32-bit
     const int S = r.cell == 1 ? 2 : 1;
     const bool res = r.residual_out != nullptr;
+    const int cc = r.variant ? r.variant : 32;
     int rc;
     if (S == 1) {
-        switch (r.variant) {
-            case 1: rc = choose_wide<GruCell, 8, 2, 3>(plan, num_sms, r.B, r.T, r.H, res); break;
-            case 2: rc = choose_wide<GruCell, 16, 2, 1>(plan, num_sms, r.B, r.T, r.H, res); break;
-            default: rc = choose_wide<GruCell, 12, 2, 2>(plan, num_sms, r.B, r.T, r.H, res); break;
-        }
+        rc = cc == 32   ? choose_wide<GruCell, 32, 12, 2, 2>(plan, num_sms, r.B, r.T, r.H, res)
+             : cc == 16 ? choose_wide<GruCell, 16, 7, 2, 2>(plan, num_sms, r.B, r.T, r.H, res)
+                        : choose_wide<GruCell, 8, 7, 2, 2>(plan, num_sms, r.B, r.T, r.H, res);
     } else {
-        switch (r.variant) {
-            case 1: rc = choose_wide<LstmCell, 4, 2, 3>(plan, num_sms, r.B, r.T, r.H, res); break;
-            default: rc = choose_wide<LstmCell, 8, 2, 2>(plan, num_sms, r.B, r.T, r.H, res); break;
-        }
+        rc = cc == 32   ? choose_wide<LstmCell, 32, 8, 2, 2>(plan, num_sms, r.B, r.T, r.H, res)
+             : cc == 16 ? choose_wide<LstmCell, 16, 7, 2, 2>(plan, num_sms, r.B, r.T, r.H, res)
+                        : choose_wide<LstmCell, 8, 7, 2, 2>(plan, num_sms, r.B, r.T, r.H, res);
     }
-    if (rc) return -1;
+    if (rc) return rc > 0 ? 1 : -1;
     if (plan->ntiles > 0x7fffffffL) return 1;
-    plan->variant = 232;
+    plan->variant = 200 + plan->C;
     plan->S = S;
-    plan->agg_words = (size_t)plan->ntiles * plan->C * (S == 1 ? 2 : 6);
+    plan->agg_words = 0;  // a chained scan: only inclusive values are published
     plan->inc_words = (size_t)plan->ntiles * plan->C * S;
     plan->side_bytes = 2 * (size_t)plan->ntiles * plan->C * S * sizeof(float);
     plan->epochs = (unsigned)r.max_iters + 1u;
@@ -513,8 +544,8 @@ int newton_wide_plan(const NewtonDiagReq &r, int num_sms, Plan *plan) {
     return 0;
 }
 
-// Launch: the tensor maps of xproj [B*T, 3, H] (boxes 32 x 3 x TCH) and of the states
-// [B*T, H*S] (boxes 32*S x TCH), passed with the arguments.
+// Launch: the tensor maps of xproj [B*T, 3, H] (boxes C x 3 x TCH) and of the states
+// [B*T, H*S] (boxes C*S x TCH), passed with the arguments.
 cudaError_t newton_wide_launch(const NewtonDiagArgs &A, const Plan &plan, cudaStream_t st) {
     StagedMaps M;
     memset(&M, 0, sizeof(M));
@@ -524,7 +555,7 @@ cudaError_t newton_wide_launch(const NewtonDiagArgs &A, const Plan &plan, cudaSt
     {
         cuuint64_t dims[3] = {(cuuint64_t)A.H, 3, (cuuint64_t)A.B * A.T};
         cuuint64_t strides[2] = {(cuuint64_t)A.H * 4, (cuuint64_t)3 * A.H * 4};
-        cuuint32_t box[3] = {32, 3, (cuuint32_t)plan.tch};
+        cuuint32_t box[3] = {(cuuint32_t)plan.C, 3, (cuuint32_t)plan.tch};
         cuuint32_t estr[3] = {1, 1, 1};
         if (fn(&M.x, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float *>(A.xproj), dims, strides, box, estr,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -534,7 +565,7 @@ cudaError_t newton_wide_launch(const NewtonDiagArgs &A, const Plan &plan, cudaSt
     {
         cuuint64_t dims[2] = {(cuuint64_t)A.H * S, (cuuint64_t)A.B * A.T};
         cuuint64_t strides[1] = {(cuuint64_t)A.H * S * 4};
-        cuuint32_t box[2] = {(cuuint32_t)(32 * S), (cuuint32_t)plan.tch};
+        cuuint32_t box[2] = {(cuuint32_t)(plan.C * S), (cuuint32_t)plan.tch};
         cuuint32_t estr[2] = {1, 1};
         if (fn(&M.h, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, A.h, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,

@@ -146,6 +146,36 @@ def test_wide_converged_with_separate_residual(ctx, cell, B, T, H):
     assert abs(float(out["residual"].item()) - m.residual(host(out["h"]), h0)) <= 2e-6
 
 
+@pytest.mark.parametrize("channels", [8, 16, 32])
+@pytest.mark.parametrize("cell,B,T,H,iters,tol", [("gru", 4, 8000, 64, 3, 0.0), ("lstm", 3, 7001, 64, 7001, 1e-6),
+                                                 ("gru", 2, 1000, 96, 2, 0.0)])
+def test_wide_tile_widths(ctx, channels, cell, B, T, H, iters, tol):
+    """Each channel width of the wide-layer tiles (8, 16, 32, forced through debug knob 6),
+    capped with the fused residual (GRU) and converged (LSTM), ragged last tiles.  The
+    first two shapes give every CTA more tiles than its staging ring holds (each stage is
+    refilled), the last one at most two."""
+    rng = np.random.default_rng(B * 13 + T + H)
+    xp = (rng.standard_normal((B, T, 3, H)) * 0.8).astype(np.float32)
+    a = rng.uniform(-0.9, 0.9, (3, H)).astype(np.float32)
+    peep = rng.uniform(-0.5, 0.5, (2, H)).astype(np.float32) if cell == "lstm" else None
+    h0 = (rng.standard_normal((B, H, 2) if cell == "lstm" else (B, H)) * 0.3).astype(np.float32)
+    m = oracle.Model(cell, xp, a=a, peep=peep)
+    h_ref, it_ref, _ = m.newton(h0, max_iters=iters, tol=tol)
+    pararnn_debug_set(ctx.ctx, 6, channels)
+    try:
+        out = solve.newton_forward(ctx.ctx, cell, B, T, H, xproj=gpu(xp), a=gpu(a),
+                                   peep=None if peep is None else gpu(peep), h0=gpu(h0), max_iters=iters, tol=tol,
+                                   residual=True)
+        torch.cuda.synchronize()
+    finally:
+        pararnn_debug_set(ctx.ctx, 6, 0)
+    assert ctx.status() == 0
+    assert int(out["iters"].item()) == it_ref
+    scale = max(1.0, float(np.abs(h_ref).max()))
+    assert max_abs(host(out["h"]), h_ref) <= TOL_STATE * scale
+    assert abs(float(out["residual"].item()) - m.residual(host(out["h"]), h0)) <= 2e-6 * scale
+
+
 def test_zero_iterations_returns_initial_guess(ctx):
     w = _small_workload("gru", 2, 100, 4, 2, 3)
     inp = wl.generate(w)

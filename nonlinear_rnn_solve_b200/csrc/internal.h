@@ -89,6 +89,10 @@ cudaError_t elk_tanh_launch(const NewtonTanhReq &r, float lambda, const Plan &pl
                             const DbgHost &dbg, cudaStream_t st);
 cudaError_t newton_tanh_launch(const NewtonTanhReq &r, const Plan &plan, const Work &w,
                                const DbgHost &dbg, cudaStream_t st);
+// quasi-DEER at n == 8 with raw inputs of width 1, 2 or 4 (tanh_quasi8.cu); 1: not covered
+int tanh_quasi8_plan(const NewtonTanhReq &r, int num_sms, Plan *plan);
+cudaError_t tanh_quasi8_launch(const NewtonTanhReq &r, const Plan &plan, const Work &w, const DbgHost &dbg,
+                               cudaStream_t st);
 
 // ---- standalone linear scan -------------------------------------------------------
 struct ScanReq {

@@ -1,0 +1,629 @@
+// tanh_quasi8.cu -- quasi-DEER for the vanilla tanh RNN h_t = tanh(A h_{t-1} + U x_t + b)
+// at state size n = 8 with raw inputs of width 4 (the projection is recomputed in the
+// kernel): the long-sequence, small-state workload of the tanh RNN.
+//
+// "Towards Scalable and Stable Parallelization of Nonlinear RNNs", Abstract: quasi-Newton
+// keeps only the diagonal of the Jacobian, J_t = diag(1 - f_t^2) diag(A), so the linear
+// recurrence of each iteration splits into n independent scalar recurrences ("Parallelizing
+// non-linear sequential models over the sequence length", Approach: the recurrence is
+// solved by a parallel scan).  f itself uses the full A h.
+//
+// Layout: a CTA of 8 warps; warp c owns unit c, lane s owns steps 16 s .. 16 s + 15 of a
+// tile of 512 steps of one sequence.  Each lane evaluates its steps (the 8-term dot
+// product reads the previous iterate's state rows from shared memory), composes them, and
+// the warp scans its 32 lanes with shuffles: no CTA barrier in the scan.  The carry
+// entering the tile comes from the tile's own evaluation of the 128 steps before it (the
+// halo): the quasi-Jacobian is contractive here, and when the composed map of those steps
+// has a matrix part that is exactly zero in fp32 it is a constant whose value is the
+// carry (the same value the scan would carry in, up to rounding order).  Otherwise the
+// warp waits (bounded) for the predecessor tile's published value of its unit.
+//
+// Data movement is by bulk copies (cp.async.bulk, no multicast), one per 16-row segment,
+// the issue shared by all warps: a tile's state and input rows arrive in padded shared-memory segments
+// (conflict-free 128-bit row reads) completing on the stage's mbarrier, two stages deep;
+// results are written to a staging tile and leave as bulk stores, together with the
+// tile's last 129 states, which the successor reads as its halo in the next iteration.
+#include <algorithm>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace prn {
+
+namespace {
+
+constexpr int kN = 8;                      // units
+constexpr int kIn = 4;                     // raw input width
+constexpr int kL = 16;                     // steps per lane
+constexpr int kT = 32 * kL;                // steps per tile
+constexpr int kHalo = 128;                 // halo steps
+constexpr int kHRows = kHalo + kT + 1;     // state rows r = 0..640: states t0 - 129 + r
+constexpr int kXRows = kHalo + kT;         // input rows r = 0..639: steps t0 - 128 + r
+constexpr int kShift = 15;                 // state row r sits at segment row r + 15, so the
+                                           // tile's own rows (129..) fill whole segments
+constexpr int kSeg = 16 * kN + 4;          // floats per 16 state (or output) rows, padded
+constexpr int kXSeg = 16 * kIn + 4;        // floats per 16 input rows, padded
+constexpr int kHSegs = (kHRows + kShift + 15) / 16;  // 41
+constexpr int kHFloats = kHSegs * kSeg;
+constexpr int kXFloats = (kXRows / 16) * kXSeg;
+constexpr int kStage = kHFloats + kXFloats;
+constexpr int kOFloats = (kT / 16) * kSeg;  // output staging
+constexpr int kSide = kHalo + 1;             // states handed to the successor
+constexpr int kSmemFloats = 2 * kStage + 2 * kOFloats;
+static_assert(kSeg % 4 == 0 && kXSeg % 4 == 0 && kStage % 4 == 0 && kHFloats % 4 == 0, "16-byte aligned segments");
+static_assert((kHalo + 1 + kShift) % 16 == 0, "the tile's own state rows start a segment");
+
+__device__ __forceinline__ int hrow(int r) { return ((r + kShift) >> 4) * kSeg + ((r + kShift) & 15) * kN; }
+__device__ __forceinline__ int xrow(int r) { return (r >> 4) * kXSeg + (r & 15) * kIn; }
+__device__ __forceinline__ int orow(int i) { return (i >> 4) * kSeg + (i & 15) * kN; }
+
+__device__ __forceinline__ unsigned saddr(const void *p) { return (unsigned)__cvta_generic_to_shared(p); }
+__device__ __forceinline__ void bulk_g2s(float *dst, const float *src, unsigned bytes, unsigned long long *bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     saddr(dst)),
+                 "l"(src), "r"(bytes), "r"(saddr(bar))
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_s2g(float *dst, const float *src, unsigned bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(saddr(src)), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void bar_init(unsigned long long *bar, unsigned count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(saddr(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void bar_expect(unsigned long long *bar, unsigned bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(saddr(bar)), "r"(bytes) : "memory");
+}
+// phase test; a thread whose phase is not complete sleeps up to ~ns nanoseconds in hardware
+__device__ __forceinline__ bool bar_try(unsigned long long *bar, unsigned parity, unsigned ns) {
+    unsigned ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(saddr(bar)), "r"(parity), "r"(ns)
+        : "memory");
+    return ok != 0;
+}
+
+struct Q8Args {
+    int B, T, jmode;
+    const float *x, *W, *bias, *A, *h0;
+    float *h;
+    int max_iters;
+    float tol;
+    int *iters_out;
+    float *delta_out, *residual_out;
+    Ctl *ctl;
+    int *sticky;
+    unsigned long long *inc;  // [ntiles][8] epoch-tagged inclusive values
+    float *side;              // two parities of [ntiles][129][8]
+    unsigned epoch0;
+    Dbg dbg;
+};
+
+// Per-warp constants of unit c: its row of A (the half holding column c first, so that
+// unit c's state is a fixed lane of the first 128-bit read), U, b -- all scaled by
+// -2 log2(e), so that exp(-2 u) is one ex2 -- and the linearisation coefficients
+// J = ja f^2 + jb: quasi-DEER (1 - f^2) A_cc, Jacobi 0, Picard 1.
+struct Q8Unit {
+    float ar[8], w[kIn], bz, ja, jb;
+    int half, sub;
+    __device__ __forceinline__ void load(const Q8Args &A, int c) {
+        constexpr float s2 = -2.f * 1.4426950408889634f;
+        half = c >> 2;
+        sub = c & 3;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            ar[k] = s2 * __ldg(A.A + c * kN + 4 * half + k);
+            ar[4 + k] = s2 * __ldg(A.A + c * kN + 4 * (1 - half) + k);
+        }
+#pragma unroll
+        for (int q = 0; q < kIn; ++q) w[q] = s2 * __ldg(A.W + c * kIn + q);
+        bz = A.bias ? s2 * __ldg(A.bias + c) : 0.f;
+        const float acc = __ldg(A.A + c * kN + c);
+        ja = A.jmode == 0 ? -acc : 0.f;
+        jb = A.jmode == 0 ? acc : A.jmode == 3 ? 1.f : 0.f;
+    }
+    __device__ __forceinline__ void row(const float *hs, int r, float4 &va, float4 &vb) const {
+        const float *p = hs + hrow(r);
+        va = *reinterpret_cast<const float4 *>(p + 4 * half);
+        vb = *reinterpret_cast<const float4 *>(p + 4 * (1 - half));
+    }
+    __device__ __forceinline__ float pick(const float4 &va) const {
+        const float lo = (sub & 1) ? va.y : va.x, hi = (sub & 1) ? va.w : va.z;
+        return (sub & 2) ? hi : lo;
+    }
+    // f = tanh(A h_{t-1} + U x_t + b) from the state row (va, vb) and input row xr
+    __device__ __forceinline__ float cell(const float *xs, int xr, const float4 &va, const float4 &vb) const {
+        const float4 xv = *reinterpret_cast<const float4 *>(xs + xrow(xr));
+        float u = fmaf(w[0], xv.x, bz), u2 = w[1] * xv.y;
+        u = fmaf(w[2], xv.z, u);
+        u2 = fmaf(w[3], xv.w, u2);
+        u = fmaf(ar[0], va.x, u);
+        u2 = fmaf(ar[1], va.y, u2);
+        u = fmaf(ar[2], va.z, u);
+        u2 = fmaf(ar[3], va.w, u2);
+        u = fmaf(ar[4], vb.x, u);
+        u2 = fmaf(ar[5], vb.y, u2);
+        u = fmaf(ar[6], vb.z, u);
+        u2 = fmaf(ar[7], vb.w, u2);
+        // tanh(x) = 2 / (1 + exp(-2 x)) - 1, with the -2 log2(e) scale already in u
+        return fmaf(2.f, rcp_hw(1.f + ex2_hw(u + u2)), -1.f);
+    }
+    __device__ __forceinline__ float jac(float f) const { return fmaf(ja * f, f, jb); }
+};
+
+class Q8Run {
+  public:
+    const Q8Args &A;
+    float *smq;
+    unsigned long long *bar;  // [2] stage-full barriers
+    int tid, lane, c, nseq, nchunk;
+    unsigned phase = 0;  // bit p: parity of stage p's next completion
+
+    __device__ __forceinline__ float *stage(int p) const { return smq + p * kStage; }
+    __device__ __forceinline__ float *outs(int p) const { return smq + 2 * kStage + p * kOFloats; }
+
+    // Every warp: its share of stage p <- tile (b, chunk) of iterate k.  State rows: the 129
+    // before the tile from the predecessor's side buffer (h0 before t = 0), the tile's own
+    // from h (none on the first iteration, whose iterate is zero); input rows.  One bulk copy
+    // per segment, only rows inside the sequence (rows past its end are never read for a
+    // valid step).  Copy ids: 0 side row 0; 1..8 side segments; 9 the row of h0; 10..41 the
+    // tile's state segments; 42..81 input segments; warp w issues ids 11 w .. 11 w + 10 and
+    // arrives once on the stage barrier (8 arrivals) with its bytes.  `first`: the first
+    // copies of an iteration, which read what other CTAs stored in the previous one.
+    __device__ void issue(int p, int b, int chunk, int k, const float *side_tile, bool first) const {
+        float *hs = stage(p), *xs = hs + kHFloats;
+        const int t0 = chunk * kT;
+        if (first) asm volatile("fence.proxy.async.global;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        const int id = lane < 11 ? 11 * c + lane : 999;
+        unsigned nb = 0;
+        float *dst = hs;
+        const float *src = A.x;
+        if (id == 0) {
+            if (k > 0 && chunk > 0) {
+                dst = hs + hrow(0);
+                src = side_tile;
+                nb = kN * 4;
+            }
+        } else if (id <= 8) {
+            if (k > 0 && chunk > 0) {
+                dst = hs + hrow(1 + 16 * (id - 1));
+                src = side_tile + (1 + 16 * (id - 1)) * kN;
+                nb = 16 * kN * 4;
+            }
+        } else if (id == 9) {
+            if (chunk == 0 && A.h0) {
+                dst = hs + hrow(kHalo);
+                src = A.h0 + (size_t)b * kN;
+                nb = kN * 4;
+            } else if (chunk == 0) {  // the state before t = 0 is zero (no h0)
+                float4 *z = reinterpret_cast<float4 *>(hs + hrow(kHalo));
+                z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+                z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+        } else if (id <= 41) {
+            const int seg = id - 10, tf = t0 + 16 * seg;
+            const int n = min(16, max(0, A.T - tf));
+            if (k > 0 && n > 0) {
+                dst = hs + hrow(kHalo + 1 + 16 * seg);
+                src = A.h + ((size_t)b * A.T + tf) * kN;
+                nb = (unsigned)n * kN * 4;
+            }
+        } else if (id <= 81) {
+            const int seg = id - 42, tf = t0 - kHalo + 16 * seg;
+            const int n = tf < 0 ? 0 : min(16, max(0, A.T - tf));
+            if (n > 0) {
+                dst = xs + xrow(16 * seg);
+                src = A.x + ((size_t)b * A.T + tf) * kIn;
+                nb = (unsigned)n * kIn * 4;
+            }
+        }
+        unsigned bytes = nb;
+#pragma unroll
+        for (int off = 16; off; off >>= 1) bytes += __shfl_xor_sync(0xffffffffu, bytes, off);
+        __syncwarp();
+        if (lane == 0) bar_expect(bar + p, bytes);
+        if (nb) bulk_g2s(dst, src, nb, bar + p);
+    }
+    // Every warp: its share of the staged results of tile (b, chunk) out to h, and of the
+    // tile's last 129 states to the side buffer (bulk stores, one group per warp).  Store
+    // ids: 0..31 state segments, 32 side row 0, 33..40 side segments; warp w stores ids
+    // 6 w .. 6 w + 5.
+    __device__ void flush(int p, int b, int chunk, float *side_tile) const {
+        const float *ob = outs(p);
+        const int t0 = chunk * kT;
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        const int id = lane < 6 ? 6 * c + lane : 999;
+        if (id < 32) {
+            const int tf = t0 + 16 * id;
+            const int n = min(16, max(0, A.T - tf));
+            if (n > 0) bulk_s2g(A.h + ((size_t)b * A.T + tf) * kN, ob + id * kSeg, (unsigned)n * kN * 4);
+        } else if (side_tile && id == 32) {
+            bulk_s2g(side_tile, ob + orow(kT - kSide), kN * 4);
+        } else if (side_tile && id <= 40) {
+            bulk_s2g(side_tile + (1 + 16 * (id - 33)) * kN, ob + orow(kT - kSide + 1 + 16 * (id - 33)), 16 * kN * 4);
+        }
+        bulk_commit();
+    }
+    // Bounded wait for stage p (every thread).
+    __device__ __forceinline__ bool wait(int p) {
+        const unsigned par = (phase >> p) & 1u;
+        bool ok = bar_try(bar + p, par, 20000u);
+        if (!ok) {
+            const unsigned long long t0 = gtimer();
+            while (!(ok = bar_try(bar + p, par, 20000u))) {
+                if (ld_relaxed_int(&A.ctl->abort)) break;
+                if (gtimer() - t0 > A.dbg.wait_ns) {
+                    raise_status(A.sticky, A.ctl, kStTimeout, true);
+                    break;
+                }
+            }
+        }
+        if (ok) phase ^= 1u << p;
+        return ok;
+    }
+};
+
+template <bool FULL, bool K0>
+__device__ __forceinline__ void q8_tile(const Q8Args &A, const Q8Unit &U, const float *hs, const float *xs, float *ob,
+                                        int lane, int c, long tile, long nseq, int chunk, int t0, unsigned epoch,
+                                        bool use_halo, float &my_max, bool &my_bad, int *s_fail) {
+    const float4 z4 = make_float4(0.f, 0.f, 0.f, 0.f);
+    // ---- halo: 32 runs of 4 steps.  Run v (steps t0 - 128 + 4 v ..) goes to lane
+    // (v >> 2) + 8 (v & 3), so that the eight lanes of a quarter-warp read eight different
+    // padded segments (conflict-free); the runs are composed in order v with shuffles
+    // from computed lanes.
+    bool known = chunk == 0;
+    float carry = 0.f;  // delta entering t = 0 is 0
+    if (chunk > 0 && use_halo) {
+        const int v = 4 * (lane & 7) + (lane >> 3);  // this lane's run
+        Aff<1> eh = Aff<1>::ident();
+        float4 va = z4, vb = z4, na = z4, nb = z4;
+        if (!K0) U.row(hs, 4 * v, va, vb);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int r = 4 * v + q;  // state row of h_{t-1}; input row of x_t
+            if (!K0) U.row(hs, r + 1, na, nb);
+            const float f = U.cell(xs, r, va, vb);
+            eh = compose(eh, Aff<1>{U.jac(f), f - U.pick(na)});
+            va = na;
+            vb = nb;
+        }
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int w = v + off < 32 ? v + off : v;  // run to compose after this one
+            const int src = (w >> 2) + 8 * (w & 3);
+            const Aff<1> o{__shfl_sync(0xffffffffu, eh.a, src), __shfl_sync(0xffffffffu, eh.d, src)};
+            if (v + off < 32) eh = compose(eh, o);
+        }
+        const float ha = __shfl_sync(0xffffffffu, eh.a, 0), hd = __shfl_sync(0xffffffffu, eh.d, 0);
+        if (ha == 0.f) {
+            known = true;
+            carry = hd;
+        }
+    }
+    // ---- the lane's 16 steps
+    float Jr[kL], rr[kL], hc[kL];
+    {
+        const int r0 = kHalo + kL * lane;
+        float4 va = z4, vb = z4, na = z4, nb = z4;
+        if (!K0 || (chunk == 0 && lane == 0)) U.row(hs, r0, va, vb);  // (K0: only h0 is not zero)
+#pragma unroll
+        for (int i = 0; i < kL; ++i) {
+            if (!K0) U.row(hs, r0 + i + 1, na, nb);
+            const float f = U.cell(xs, r0 + i, va, vb);
+            const float cur = U.pick(na);
+            const bool v = FULL || t0 + kL * lane + i < A.T;
+            Jr[i] = v ? U.jac(f) : 1.f;
+            rr[i] = v ? f - cur : 0.f;
+            hc[i] = cur;
+            va = na;
+            vb = nb;
+        }
+    }
+    Aff<1> e = Aff<1>::ident();
+#pragma unroll
+    for (int i = 0; i < kL; ++i) e = compose(e, Aff<1>{Jr[i], rr[i]});
+    Aff<1> inc = e;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const Aff<1> o = inc.shfl_up(off);
+        if (lane >= off) inc = compose(o, inc);
+    }
+    Aff<1> excl = inc.shfl_up(1);
+    if (lane == 0) excl = Aff<1>::ident();
+    const float ta = __shfl_sync(0xffffffffu, inc.a, 31), td = __shfl_sync(0xffffffffu, inc.d, 31);
+    if (!known) {
+        // the predecessor's value of this unit (chained; bounded wait)
+        const unsigned long long *src = A.inc + (size_t)(tile - nseq) * kN + c;
+        unsigned long long wv = 0, tw0 = 0;
+        int bad = 0;
+        if (lane == 0) {
+            for (int polls = 0;; ++polls) {
+                wv = ld_relaxed_u64(src);
+                if ((unsigned)wv == epoch) break;
+                if (ld_relaxed_int(&A.ctl->abort)) {
+                    bad = 1;
+                    break;
+                }
+                if (polls == 4) tw0 = gtimer();
+                if (polls > 4) {
+                    if (gtimer() - tw0 > A.dbg.wait_ns) {
+                        raise_status(A.sticky, A.ctl, kStTimeout, true);
+                        bad = 1;
+                        break;
+                    }
+                    __nanosleep(32);
+                }
+            }
+        }
+        if (__shfl_sync(0xffffffffu, bad, 0))
+            *s_fail = 1;
+        else
+            carry = __uint_as_float(__shfl_sync(0xffffffffu, (unsigned)(wv >> 32), 0));
+    }
+    if (lane == 0 && A.dbg.skip_tile != tile)
+        st_relaxed_u64(A.inc + (size_t)tile * kN + c, pack_tag(fmaf(ta, carry, td), epoch));
+    // ---- update: delta_t = J_t delta_{t-1} + r_t, h^(k+1) = h^(k) + delta
+    float d = fmaf(excl.a, carry, excl.d);
+#pragma unroll
+    for (int i = 0; i < kL; ++i) {
+        d = fmaf(Jr[i], d, rr[i]);
+        ob[orow(kL * lane + i) + c] = hc[i] + d;
+        my_max = fmaxf(my_max, fabsf(d));
+    }
+    my_bad |= !finitef(d);
+}
+
+__global__ void __launch_bounds__(kThreads, 2) tanh_quasi8_kernel(const Q8Args A) {
+    extern __shared__ __align__(16) float smq[];
+    __shared__ unsigned s_red[kThreads / 32];
+    __shared__ int s_fail;
+    __shared__ __align__(8) unsigned long long s_bar[2];
+    Q8Run R{A};
+    R.smq = smq;
+    R.bar = s_bar;
+    R.tid = threadIdx.x;
+    R.lane = threadIdx.x & 31;
+    R.c = threadIdx.x >> 5;
+    R.nseq = A.B;
+    R.nchunk = (A.T + kT - 1) / kT;
+    const int tid = threadIdx.x, lane = R.lane, c = R.c;
+    const int nseq = R.nseq, nchunk = R.nchunk;
+    const long ntiles = (long)nseq * nchunk;
+    const long ntile_cta = blockIdx.x < ntiles ? (ntiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+    const size_t side_stride = (size_t)ntiles * kSide * kN;
+    const bool use_halo = !A.dbg.no_halo;
+    if (tid == 0) {
+        s_fail = 0;
+        bar_init(s_bar, kThreads / 32);  // one arrival per warp (each issues a share of the copies)
+        bar_init(s_bar + 1, kThreads / 32);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    Q8Unit U;
+    U.load(A, c);
+    const int step_ch = (int)(gridDim.x / (unsigned)nseq), step_sq = (int)(gridDim.x % (unsigned)nseq);
+    auto stepw = [&](int &ch, int &sq) {
+        ch += step_ch;
+        sq += step_sq;
+        if (sq >= nseq) {
+            sq -= nseq;
+            ++ch;
+        }
+    };
+    __syncthreads();
+
+    unsigned pending = 0;  // bit p: stage p has copies in flight not yet waited for
+    auto drain = [&]() {
+        for (int p = 0; p < 2; ++p) {
+            if (!((pending >> p) & 1u)) continue;
+            const unsigned par = (R.phase >> p) & 1u;
+            const unsigned long long t0 = gtimer();
+            while (!bar_try(s_bar + p, par, 1000u) && gtimer() - t0 < A.dbg.wait_ns) {
+            }
+        }
+        bulk_wait_all();
+    };
+    int iters = 0;
+    float last_delta = 0.f;
+    bool stop_all = false;
+    for (int k = 0; k < A.max_iters; ++k) {
+        const unsigned epoch = A.epoch0 + (unsigned)k + 1u;
+        if (blockIdx.x == 0 && tid == 0) A.ctl->delta_bits[(k + 1) % 3] = 0u;
+        const float *side_in = A.side + (size_t)(k & 1) * side_stride;
+        float *side_out = A.side + (size_t)((k + 1) & 1) * side_stride;
+        float my_max = 0.f;
+        bool my_bad = false;
+        int ch = (int)(blockIdx.x / (unsigned)nseq), sq = (int)(blockIdx.x % (unsigned)nseq);
+        int ach = ch, asq = sq;  // two tiles ahead
+        for (int j = 0; j < 2; ++j) {  // prologue: this CTA's first two tiles
+            if (j < ntile_cta) {
+                const long tl = blockIdx.x + (long)j * gridDim.x;
+                R.issue(j, asq, ach, k, ach > 0 ? side_in + (size_t)(tl - nseq) * kSide * kN : nullptr, j == 0);
+                pending |= 1u << j;
+            }
+            stepw(ach, asq);
+        }
+        for (long j = 0; j < ntile_cta; ++j) {
+            const int par = (int)(j & 1);
+            const long tile = blockIdx.x + j * (long)gridDim.x;
+            const int b = sq, chunk = ch, t0 = chunk * kT;
+            if (!R.wait(par)) s_fail = 1;
+            pending &= ~(1u << par);
+            const float *hs = R.stage(par), *xs = hs + kHFloats;
+            float *ob = R.outs(par);
+            const bool full = t0 + kT <= A.T;
+            if (!s_fail) {
+                if (k == 0) {
+                    if (full)
+                        q8_tile<true, true>(A, U, hs, xs, ob, lane, c, tile, nseq, chunk, t0, epoch, use_halo, my_max,
+                                            my_bad, &s_fail);
+                    else
+                        q8_tile<false, true>(A, U, hs, xs, ob, lane, c, tile, nseq, chunk, t0, epoch, use_halo, my_max,
+                                             my_bad, &s_fail);
+                } else {
+                    if (full)
+                        q8_tile<true, false>(A, U, hs, xs, ob, lane, c, tile, nseq, chunk, t0, epoch, use_halo, my_max,
+                                             my_bad, &s_fail);
+                    else
+                        q8_tile<false, false>(A, U, hs, xs, ob, lane, c, tile, nseq, chunk, t0, epoch, use_halo,
+                                              my_max, my_bad, &s_fail);
+                }
+            }
+            // this warp's bulk stores of the previous tile have read their staging tile
+            bulk_wait_read_all();
+            __syncthreads();  // stage `par` consumed, staging tile `par` complete
+            if (s_fail) {
+                drain();
+                return;  // a bounded wait ran out; the status says so
+            }
+            R.flush(par, b, chunk, chunk < nchunk - 1 ? side_out + (size_t)tile * kSide * kN : nullptr);
+            if (j + 2 < ntile_cta) {
+                const long tl = tile + 2L * gridDim.x;
+                R.issue(par, asq, ach, k, ach > 0 ? side_in + (size_t)(tl - nseq) * kSide * kN : nullptr, false);
+            }
+            if (j + 2 < ntile_cta) pending |= 1u << par;
+            stepw(ach, asq);
+            stepw(ch, sq);
+        }
+        // this iteration's stores complete before any CTA reads them in the next one
+        bulk_wait_all();
+        asm volatile("fence.proxy.async.global;" ::: "memory");
+        const unsigned bits = block_max_bits(my_bad ? __int_as_float(0x7fc00000) : my_max, s_red);
+        if (tid == 0) atomicMax(&A.ctl->delta_bits[k % 3], bits);
+        if (!grid_sync(A.ctl, A.sticky, A.dbg)) return;
+        const unsigned dbits = ld_acquire(&A.ctl->delta_bits[k % 3]);
+        last_delta = __uint_as_float(dbits);
+        iters = k + 1;
+        if (blockIdx.x == 0 && tid == 0 && A.dbg.delta_log && k < A.dbg.delta_log_cap) A.dbg.delta_log[k] = last_delta;
+        if (dbits >= 0x7f800000u) {
+            if (blockIdx.x == 0 && tid == 0) atomicOr(A.sticky, kStNonfinite);
+            stop_all = true;
+            break;
+        }
+        if (last_delta < A.tol) break;
+    }
+    if (A.residual_out && !stop_all) {
+        // max |h_t - f(h_{t-1}, x_t)| at the result, one tile at a time (rows t0 - 1 ..
+        // t0 + 511 of the result and h0; plain loads, a rare pass)
+        float my_res = 0.f;
+        int ch = (int)(blockIdx.x / (unsigned)nseq), sq = (int)(blockIdx.x % (unsigned)nseq);
+        float *hs = R.stage(0), *xs = hs + kHFloats;
+        asm volatile("fence.proxy.async.global;" ::: "memory");
+        for (long j = 0; j < ntile_cta; ++j) {
+            const int t0 = ch * kT;
+            __syncthreads();
+            for (int e = tid; e < (kT + 1) * 2; e += kThreads) {
+                const int r = kHalo + (e >> 1), half = e & 1, t = t0 - 1 + (e >> 1);
+                float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (t < 0) {
+                    if (A.h0) v = *reinterpret_cast<const float4 *>(A.h0 + (size_t)sq * kN + half * 4);
+                } else if (t < A.T) {
+                    v = *reinterpret_cast<const float4 *>(A.h + ((size_t)sq * A.T + t) * kN + half * 4);
+                }
+                *reinterpret_cast<float4 *>(hs + hrow(r) + half * 4) = v;
+            }
+            for (int r = kHalo + tid; r < kXRows; r += kThreads) {
+                const int t = t0 - kHalo + r;
+                float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (t < A.T) v = *reinterpret_cast<const float4 *>(A.x + ((size_t)sq * A.T + t) * kIn);
+                *reinterpret_cast<float4 *>(xs + xrow(r)) = v;
+            }
+            __syncthreads();
+            float4 va, vb, na, nb;
+            const int r0 = kHalo + kL * lane;
+            U.row(hs, r0, va, vb);
+#pragma unroll
+            for (int i = 0; i < kL; ++i) {
+                U.row(hs, r0 + i + 1, na, nb);
+                const float f = U.cell(xs, r0 + i, va, vb);
+                if (t0 + kL * lane + i < A.T) {
+                    const float ad = fabsf(U.pick(na) - f);
+                    my_res = (ad > my_res || isnan(ad)) ? ad : my_res;
+                }
+                va = na;
+                vb = nb;
+            }
+            stepw(ch, sq);
+        }
+        const unsigned bits = block_max_bits(my_res, s_red);
+        if (tid == 0) atomicMax(&A.ctl->res_bits, bits);
+        if (!grid_sync(A.ctl, A.sticky, A.dbg)) return;
+        if (blockIdx.x == 0 && tid == 0) {
+            const unsigned rb = ld_acquire(&A.ctl->res_bits);
+            *A.residual_out = __uint_as_float(rb);
+            if (rb >= 0x7f800000u) atomicOr(A.sticky, kStNonfinite);
+        }
+    }
+    if (blockIdx.x == 0 && tid == 0) {
+        *A.iters_out = iters;
+        if (A.delta_out) *A.delta_out = last_delta;
+        if (!stop_all && A.tol > 0.f && iters == A.max_iters && !(last_delta < A.tol))
+            atomicOr(A.sticky, kStNotConverged);
+    }
+}
+
+}  // namespace
+
+// Shapes served: quasi-DEER (or Jacobi / Picard), n == 8, raw inputs of width 4.
+// Returns 1 when the shape is not covered.
+int tanh_quasi8_plan(const NewtonTanhReq &r, int num_sms, Plan *plan) {
+    if (!r.quasi || r.n != kN || r.xproj || r.in != kIn) return 1;
+    const void *kern = reinterpret_cast<const void *>(&tanh_quasi8_kernel);
+    const int smem = kSmemFloats * (int)sizeof(float);
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) return -1;
+    plan->kernel = kern;
+    plan->dyn_smem = smem;
+    plan->ntiles = (long)r.B * ((r.T + kT - 1) / kT);
+    if (plan->ntiles > 0x7fffffffL) return 1;
+    plan->C = kN;
+    plan->agg_words = 0;
+    plan->inc_words = (size_t)plan->ntiles * kN;
+    plan->side_bytes = 2 * (size_t)plan->ntiles * kSide * kN * sizeof(float);
+    plan->epochs = (unsigned)r.max_iters + 1u;
+    plan->variant = 1108;
+    plan->threads = kThreads;
+    plan->grid = occupancy_grid(plan->kernel, kThreads, smem, num_sms, plan->ntiles);
+    return plan->grid > 0 ? 0 : -1;
+}
+
+cudaError_t tanh_quasi8_launch(const NewtonTanhReq &r, const Plan &plan, const Work &w, const DbgHost &dbg,
+                               cudaStream_t st) {
+    Q8Args A;
+    A.B = r.B;
+    A.T = r.T;
+    A.jmode = r.jmode;
+    A.x = r.x;
+    A.W = r.W;
+    A.bias = r.bias;
+    A.A = r.A;
+    A.h0 = r.h0;
+    A.h = r.h;
+    A.max_iters = r.max_iters;
+    A.tol = r.tol;
+    A.iters_out = r.iters_out;
+    A.delta_out = r.delta_out;
+    A.residual_out = r.residual_out;
+    A.ctl = w.ctl;
+    A.sticky = w.sticky;
+    A.inc = w.inc;
+    A.side = w.side;
+    A.epoch0 = w.epoch0;
+    A.dbg.wait_ns = dbg.wait_ns;
+    A.dbg.skip_tile = dbg.skip_tile;
+    A.dbg.delta_log = dbg.delta_log;
+    A.dbg.delta_log_cap = dbg.delta_log_cap;
+    // a withheld publication (failure-detection test) must be met by the chained wait
+    A.dbg.no_halo = dbg.no_halo || dbg.skip_tile >= 0;
+    void *args[] = {&A};
+    return cudaLaunchCooperativeKernel(plan.kernel, dim3(plan.grid), dim3(plan.threads), args, plan.dyn_smem, st);
+}
+
+}  // namespace prn

@@ -114,6 +114,46 @@ def test_small_shapes(ctx, case):
     assert abs(float(out["residual"].item()) - m.residual(host(out["h"]), inp["h0"])) <= 2e-6
 
 
+@pytest.mark.parametrize("inp_w", [1, 2, 4])
+@pytest.mark.parametrize("halo", [True, False])
+def test_quasi_n8_tiles_halo_and_chain(ctx, inp_w, halo):
+    """The n = 8 quasi-DEER kernel (512-step tiles, a 128-step halo per tile): several
+    sequences, a ragged last tile, the carry from the halo and (debug knob 5) from the
+    predecessor's published value; residual at the result."""
+    B, T = 3, 5 * 512 + 77
+    w = wl.WORKLOADS["tanh_b16_t65536_in4_n8_quasi"].resized(B=B, T=T, inp=inp_w, seed=40 + inp_w, max_iters=T)
+    inp = wl.generate(w)
+    rng = np.random.default_rng(inp_w)
+    inp["h0"] = (rng.standard_normal(inp["h0"].shape) * 0.3).astype(np.float32)
+    pararnn_debug_set(ctx.ctx, 5, 0 if halo else 1)
+    try:
+        out = _run(ctx, w, inp, residual=True)
+    finally:
+        pararnn_debug_set(ctx.ctx, 5, 0)
+    assert ctx.status() == 0
+    m = _check(ctx, w, inp, out)
+    assert abs(float(out["residual"].item()) - m.residual(host(out["h"]), inp["h0"])) <= 2e-6
+
+
+def test_quasi_n8_withheld_publication_times_out(ctx):
+    """A tile of the n = 8 quasi-DEER kernel withholds its published values (knob 2): the
+    successor's bounded wait runs out, the status reads ETIMEOUT, the context recovers."""
+    from nonlinear_rnn_solve_b200 import PARARNN_ETIMEOUT
+    w = wl.WORKLOADS["tanh_b16_t65536_in4_n8_quasi"].resized(B=1, T=4 * 512, seed=77, max_iters=4 * 512)
+    inp = wl.generate(w)
+    pararnn_debug_set(ctx.ctx, 1, 50_000_000)
+    pararnn_debug_set(ctx.ctx, 2, 1)
+    try:
+        _run(ctx, w, inp, max_iters=10)
+        assert ctx.status() == PARARNN_ETIMEOUT
+    finally:
+        pararnn_debug_set(ctx.ctx, 2, -1)
+        pararnn_debug_set(ctx.ctx, 1, 1_000_000_000)
+    out = _run(ctx, w, inp)
+    assert ctx.status() == 0
+    _check(ctx, w, inp, out)
+
+
 @pytest.mark.parametrize("quasi", [False, True])
 def test_fixed_iterations_match_oracle_iterates(ctx, quasi):
     w = wl.WORKLOADS["tanh_b16_t65536_in4_n8_deer"].resized(H=24, B=2, T=3000, quasi=quasi, seed=9)

@@ -462,6 +462,8 @@ constexpr int kTabMaxFloats = 12288;  // shared-memory table limit (48 KB)
 }  // namespace
 
 int adjoint_plan(const AdjointReq &r, int num_sms, Plan *plan) {
+    const int wide = adjoint_wide_plan(r, num_sms, plan);  // TMA-fed tiles for H % 32 == 0
+    if (wide <= 0) return wide;
     const int S = r.cell == 1 ? 2 : 1;
     const int L = S == 1 ? 8 : 4;
     const int C = pick_C(r.H);
@@ -498,6 +500,7 @@ int adjoint_plan(const AdjointReq &r, int num_sms, Plan *plan) {
 
 cudaError_t adjoint_launch(const AdjointReq &r, const Plan &plan, const Work &w, const DbgHost &dbg,
                            cudaStream_t st) {
+    if (plan.staged == 2) return adjoint_wide_launch(r, plan, w, dbg, st);
     AdjArgs A;
     A.B = r.B;
     A.T = r.T;

@@ -116,6 +116,10 @@ struct AdjointReq {
     float *grad_xproj, *grad_params, *grad_h0;
 };
 int adjoint_plan(const AdjointReq &r, int num_sms, Plan *plan);
+// TMA-fed tiles for H % 32 == 0 (adjoint_wide.cu); 1: shape not covered
+int adjoint_wide_plan(const AdjointReq &r, int num_sms, Plan *plan);
+cudaError_t adjoint_wide_launch(const AdjointReq &r, const Plan &plan, const Work &w, const DbgHost &dbg,
+                                cudaStream_t st);
 cudaError_t adjoint_launch(const AdjointReq &r, const Plan &plan, const Work &w, const DbgHost &dbg,
                            cudaStream_t st);
 

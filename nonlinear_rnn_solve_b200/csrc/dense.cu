@@ -1026,6 +1026,8 @@ int newton_tanh_plan(const NewtonTanhReq &r, int num_sms, Plan *plan) {
     if (!r.xproj && (r.in < 1 || r.in > 8)) return 1;
     const int q8 = tanh_quasi8_plan(r, num_sms, plan);  // warp-per-unit kernel for n == 8
     if (q8 <= 0) return q8;
+    const int tc = deer_tc_plan(r, num_sms, plan);  // tensor-core chain products for 32 < n <= 64
+    if (tc <= 0) return tc;
     switch (pad_n(r.n)) {
         case 8: return tanh_plan_n<8>(r, num_sms, plan);
         case 16: return tanh_plan_n<16>(r, num_sms, plan);
@@ -1037,6 +1039,7 @@ int newton_tanh_plan(const NewtonTanhReq &r, int num_sms, Plan *plan) {
 cudaError_t newton_tanh_launch(const NewtonTanhReq &r, const Plan &plan, const Work &w, const DbgHost &dbg,
                                cudaStream_t st) {
     if (plan.variant == 1108) return tanh_quasi8_launch(r, plan, w, dbg, st);
+    if (plan.variant == 1164) return deer_tc_launch(r, plan, w, dbg, st);
     TanhArgs A;
     A.B = r.B;
     A.T = r.T;

@@ -93,6 +93,10 @@ cudaError_t newton_tanh_launch(const NewtonTanhReq &r, const Plan &plan, const W
 int tanh_quasi8_plan(const NewtonTanhReq &r, int num_sms, Plan *plan);
 cudaError_t tanh_quasi8_launch(const NewtonTanhReq &r, const Plan &plan, const Work &w, const DbgHost &dbg,
                                cudaStream_t st);
+// full DEER at 32 < n <= 64 with the Jacobian products on the tensor cores (deer_tc.cu); 1: not covered
+int deer_tc_plan(const NewtonTanhReq &r, int num_sms, Plan *plan);
+cudaError_t deer_tc_launch(const NewtonTanhReq &r, const Plan &plan, const Work &w, const DbgHost &dbg,
+                           cudaStream_t st);
 
 // ---- standalone linear scan -------------------------------------------------------
 struct ScanReq {

@@ -165,3 +165,52 @@ def test_fixed_iterations_match_oracle_iterates(ctx, quasi):
         scale = max(1.0, float(np.abs(h_ref).max()))
         assert int(out["iters"].item()) == k
         assert max_abs(host(out["h"]), h_ref) <= TOL_STATE * scale
+
+
+TC_CASES = [  # (n, B, T, in, use_xproj): the tensor-core DEER kernel, 128-step tiles of four 32-step chains
+    (64, 3, 5 * 128 + 37, 4, False), (33, 2, 3 * 128, 2, True), (64, 1, 1, 4, False), (48, 2, 129, 8, False),
+    (64, 2, 2 * 128 + 64, 1, True),
+]
+
+
+@pytest.mark.parametrize("case", TC_CASES)
+def test_deer_tensor_core_tiles(ctx, case):
+    """Full DEER at 32 < n <= 64 with the Jacobian products on the tensor cores: several
+    sequences, ragged last tiles (chains partly filled or empty), raw and projected
+    inputs, a non-zero h0; iteration count, states and residual against the oracle."""
+    n, B, T, inp_w, use_xp = case
+    w = wl.WORKLOADS["tanh_b16_t65536_in4_n64_deer"].resized(H=n, B=B, T=T, inp=inp_w, seed=n + 7 * T,
+                                                              max_iters=T + 1)
+    inp = wl.generate(w)
+    rng = np.random.default_rng(T)
+    inp["h0"] = (rng.standard_normal(inp["h0"].shape) * 0.3).astype(np.float32)
+    xp = oracle.input_proj(inp["x"], inp["W"], inp["bias"]).astype(np.float32) if use_xp else None
+    out = _run(ctx, w, inp, xproj=xp, residual=True)
+    assert ctx.status() == 0
+    if use_xp:
+        m = oracle.Model("tanh", xp.reshape(B, T, 1, n), A=inp["A"])
+        h_ref, it_ref, _ = m.newton(inp["h0"], max_iters=w.max_iters, tol=w.tol)
+        assert int(out["iters"].item()) == it_ref
+        assert max_abs(host(out["h"]), h_ref) <= TOL_STATE
+    else:
+        m = _check(ctx, w, inp, out)
+    assert abs(float(out["residual"].item()) - m.residual(host(out["h"]), inp["h0"])) <= 2e-6
+
+
+def test_deer_tensor_core_withheld_publication_times_out(ctx):
+    """A tile of the tensor-core DEER kernel withholds its published delta (knob 2): its
+    successor's bounded wait runs out, the status reads ETIMEOUT, the context recovers."""
+    from nonlinear_rnn_solve_b200 import PARARNN_ETIMEOUT
+    w = wl.WORKLOADS["tanh_b16_t65536_in4_n64_deer"].resized(B=1, T=4 * 128, seed=78, max_iters=4 * 128)
+    inp = wl.generate(w)
+    pararnn_debug_set(ctx.ctx, 1, 50_000_000)
+    pararnn_debug_set(ctx.ctx, 2, 1)
+    try:
+        _run(ctx, w, inp, max_iters=10)
+        assert ctx.status() == PARARNN_ETIMEOUT
+    finally:
+        pararnn_debug_set(ctx.ctx, 2, -1)
+        pararnn_debug_set(ctx.ctx, 1, 1_000_000_000)
+    out = _run(ctx, w, inp)
+    assert ctx.status() == 0
+    _check(ctx, w, inp, out)

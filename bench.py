@@ -398,7 +398,14 @@ def measure_workload(L, w, inp, parts=None):
         nb = forward_bytes(w, it, False)
         if w.cell == wl.TANH:
             fl = tanh_flops(w, it, w.quasi)
-            e["roofline"] = _alu_entry(ms, fl, _fp32_peak_tflops()) if not w.quasi else _hbm_entry(ms, nb, hbm)
+            if not w.quasi and w.H > 32:
+                # chain products on the tensor cores as three TF32 products each: the fp32
+                # work against a third of the TF32 peak (measured bf16 x the nominal 1/2)
+                bf, how = _bf16_peak_tflops()
+                e["roofline"] = _tensor_entry(ms, fl, bf * 0.5 / 3.0,
+                                              f"tf32 / 3 (three-product split), tf32 = bf16 {how} x 1/2")
+            else:
+                e["roofline"] = _alu_entry(ms, fl, _fp32_peak_tflops()) if not w.quasi else _hbm_entry(ms, nb, hbm)
             e["roofline_other"] = _hbm_entry(ms, nb, hbm) if not w.quasi else _alu_entry(ms, fl, _fp32_peak_tflops())
         else:
             e["roofline"] = dict(_hbm_entry(ms, nb, hbm), bound="latency",

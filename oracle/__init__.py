@@ -82,6 +82,28 @@ def get_threads() -> int:
     return int(_L().orc_get_threads())
 
 
+def elk_block2(J, r, lam):
+    """The damped step of one unit with 2x2 Jacobian blocks (Kalman filter + RTS smoother
+    in oracle.c): J [T, 2, 2], r [T, 2] -> x [T, 2]."""
+    J = _f64(J).reshape(-1, 4)
+    r = _f64(r).reshape(-1, 2)
+    T = J.shape[0]
+    xs = np.zeros((T, 2))
+    rc = _L().orc_elk_block2(ctypes.c_long(T), _ptr(J), _ptr(r), ctypes.c_double(float(lam)), _ptr(xs))
+    assert rc == 0
+    return xs
+
+
+def elk_scalar(a, r, lam):
+    """The damped step of one scalar component (Kalman filter + RTS smoother in oracle.c):
+    a [T], r [T] -> x [T]."""
+    a, r = _f64(a).ravel(), _f64(r).ravel()
+    xs = np.zeros(a.shape[0])
+    rc = _L().orc_elk_scalar(ctypes.c_long(a.shape[0]), _ptr(a), _ptr(r), ctypes.c_double(float(lam)), _ptr(xs))
+    assert rc == 0
+    return xs
+
+
 class Model:
     """Cell + parameters + projected inputs, all widened exactly to float64.
 

@@ -57,9 +57,11 @@ typedef struct {
     int solver;          /* linearisation used by orc_newton: ORC_NEWTON (the cell's
                           * Jacobian, or its diagonal with quasi), ORC_JACOBI (J = 0),
                           * ORC_PICARD (J = I) ["Para-Seq" README, Main features], or
-                          * ORC_ELK (diagonal Jacobian, damped step, see orc_newton;
-                          * for the tanh RNN the diagonal of its dense Jacobian) */
-    double lambda;       /* ELK damping (>= 0; 0 gives the quasi-Newton step) */
+                          * ORC_ELK (damped step, see orc_newton: the LSTM's full 2x2
+                          * blocks, or their diagonals with quasi; GRU's diagonal; for
+                          * the tanh RNN the diagonal of its dense Jacobian) */
+    double lambda;       /* ELK damping (>= 0; 0 gives the Newton step of the same
+                          * linearisation) */
 } orc_model;
 
 enum { ORC_NEWTON = 0, ORC_JACOBI = 1, ORC_PICARD = 2, ORC_ELK = 3 };
@@ -309,6 +311,97 @@ static void elk_component(long T, const double *a, const double *r, double lambd
     }
 }
 
+/* ELK with a 2x2 block linearisation [ELK, Abstract: ELK with the Jacobian itself,
+ * quasi-ELK with its diagonal]: the same objective with x_t, r_t in R^2 and J_t the
+ * unit's 2x2 Jacobian block (row-major),
+ *     sum_t |x_t - J_t x_{t-1} - r_t|^2 + lambda sum_t |x_t|^2,    x_{-1} = 0,
+ * the MAP path of x_t = J_t x_{t-1} + r_t + w_t, w_t ~ N(0, I), observed as
+ * 0 = x_t + v_t, v_t ~ N(0, I / lambda).  Kalman filter with 2x2 covariances:
+ *     Pm_t = J_t P_{t-1} J_t^T + I,  mm_t = J_t m_{t-1} + r_t,
+ *     K_t = lambda Pm_t (I + lambda Pm_t)^{-1},  P_t = (I - K_t) Pm_t,  m_t = (I - K_t) mm_t,
+ * then the Rauch-Tung-Striebel smoother
+ *     x_{T-1} = m_{T-1},  x_t = m_t + G_t (x_{t+1} - mm_{t+1}),  G_t = P_t J_{t+1}^T Pm_{t+1}^{-1}.
+ * lambda = 0 gives K = 0 and x = the forward recursion (the Newton step).  Scratch: 12 T. */
+static void inv2(const double *M, double *R)
+{
+    const double det = M[0] * M[3] - M[1] * M[2];
+    R[0] = M[3] / det;
+    R[1] = -M[1] / det;
+    R[2] = -M[2] / det;
+    R[3] = M[0] / det;
+}
+static void mul2(const double *X, const double *Y, double *R) /* R = X Y (2x2, row-major) */
+{
+    const double r0 = X[0] * Y[0] + X[1] * Y[2], r1 = X[0] * Y[1] + X[1] * Y[3];
+    const double r2 = X[2] * Y[0] + X[3] * Y[2], r3 = X[2] * Y[1] + X[3] * Y[3];
+    R[0] = r0;
+    R[1] = r1;
+    R[2] = r2;
+    R[3] = r3;
+}
+static void elk_block2(long T, const double *J, const double *r, double lambda, double *xs, double *work)
+{
+    double *Pm = work, *mm = work + 4 * T, *P = work + 6 * T, *mf = work + 10 * T;
+    double Pp[4] = {0.0, 0.0, 0.0, 0.0}, mp[2] = {0.0, 0.0};
+    for (long t = 0; t < T; ++t) {
+        const double *Jt = J + 4 * t;
+        double JP[4], Jtr[4] = {Jt[0], Jt[2], Jt[1], Jt[3]};
+        mul2(Jt, Pp, JP);
+        mul2(JP, Jtr, Pm + 4 * t);
+        Pm[4 * t] += 1.0;
+        Pm[4 * t + 3] += 1.0;
+        mm[2 * t] = Jt[0] * mp[0] + Jt[1] * mp[1] + r[2 * t];
+        mm[2 * t + 1] = Jt[2] * mp[0] + Jt[3] * mp[1] + r[2 * t + 1];
+        double Sm[4] = {lambda * Pm[4 * t] + 1.0, lambda * Pm[4 * t + 1], lambda * Pm[4 * t + 2],
+                        lambda * Pm[4 * t + 3] + 1.0}, Si[4], K[4], IK[4];
+        inv2(Sm, Si);                       /* (I + lambda Pm)^{-1} */
+        mul2(Pm + 4 * t, Si, K);            /* Pm (I + lambda Pm)^{-1} */
+        for (int q = 0; q < 4; ++q) K[q] *= lambda;
+        IK[0] = 1.0 - K[0];
+        IK[1] = -K[1];
+        IK[2] = -K[2];
+        IK[3] = 1.0 - K[3];
+        mul2(IK, Pm + 4 * t, P + 4 * t);
+        mf[2 * t] = IK[0] * mm[2 * t] + IK[1] * mm[2 * t + 1];
+        mf[2 * t + 1] = IK[2] * mm[2 * t] + IK[3] * mm[2 * t + 1];
+        for (int q = 0; q < 4; ++q) Pp[q] = P[4 * t + q];
+        mp[0] = mf[2 * t];
+        mp[1] = mf[2 * t + 1];
+    }
+    xs[2 * (T - 1)] = mf[2 * (T - 1)];
+    xs[2 * (T - 1) + 1] = mf[2 * (T - 1) + 1];
+    for (long t = T - 2; t >= 0; --t) {
+        const double *Jn = J + 4 * (t + 1);
+        double Jnt[4] = {Jn[0], Jn[2], Jn[1], Jn[3]}, PJ[4], Pmi[4], G[4];
+        mul2(P + 4 * t, Jnt, PJ);
+        inv2(Pm + 4 * (t + 1), Pmi);
+        mul2(PJ, Pmi, G);
+        const double e0 = xs[2 * (t + 1)] - mm[2 * (t + 1)], e1 = xs[2 * (t + 1) + 1] - mm[2 * (t + 1) + 1];
+        xs[2 * t] = mf[2 * t] + G[0] * e0 + G[1] * e1;
+        xs[2 * t + 1] = mf[2 * t + 1] + G[2] * e0 + G[3] * e1;
+    }
+}
+
+/* Exported for the CPU pins of the block smoother: J [T][4], r [T][2] -> xs [T][2]. */
+int orc_elk_block2(long T, const double *J, const double *r, double lambda, double *xs)
+{
+    double *work = malloc(sizeof(double) * 12 * (T > 0 ? T : 1));
+    if (!work) return -1;
+    if (T > 0) elk_block2(T, J, r, lambda, xs, work);
+    free(work);
+    return 0;
+}
+
+/* Exported for the CPU pins of the scalar smoother: a [T], r [T] -> xs [T]. */
+int orc_elk_scalar(long T, const double *a, const double *r, double lambda, double *xs)
+{
+    double *work = malloc(sizeof(double) * 5 * (T > 0 ? T : 1));
+    if (!work) return -1;
+    if (T > 0) elk_component(T, a, r, lambda, xs, work);
+    free(work);
+    return 0;
+}
+
 int orc_newton(const orc_model *m, const double *h0, int max_iters, double tol, double *h_out,
                int *iters_out, double *delta_log, int log_len)
 {
@@ -392,7 +485,42 @@ int orc_newton(const orc_model *m, const double *h0, int max_iters, double tol, 
                 free(bt);
                 free(z0);
             }
+        } else if (m->solver == ORC_ELK && S == 2 && !m->quasi) {
+            /* ELK with each unit's full 2x2 Jacobian block */
+#pragma omp parallel for schedule(static) reduction(max : delta)
+            for (long bu = 0; bu < B * H; ++bu) {
+                long b = bu / H, u = bu % H;
+                double *Jb = malloc(sizeof(double) * T * 4), *r = malloc(sizeof(double) * T * 2);
+                double *xs = malloc(sizeof(double) * T * 2), *work = malloc(sizeof(double) * 12 * T);
+                double pk[2] = {0.0, 0.0}, f[2], J[4];
+                if (h0)
+                    for (long s = 0; s < 2; ++s) pk[s] = h0[(b * H + u) * 2 + s];
+                for (long t = 0; t < T; ++t) { /* linearise at h^(k): the block, the residual */
+                    unit_eval(m, b, t, u, pk, f, J, NULL, NULL);
+                    long idx = ((b * T + t) * H + u) * 2;
+                    for (int q = 0; q < 4; ++q) Jb[4 * t + q] = J[q];
+                    for (long s = 0; s < 2; ++s) {
+                        r[2 * t + s] = f[s] - hk[idx + s];
+                        pk[s] = hk[idx + s];
+                    }
+                }
+                elk_block2(T, Jb, r, m->lambda, xs, work);
+                double dloc = 0.0;
+                for (long t = 0; t < T; ++t)
+                    for (long s = 0; s < 2; ++s) {
+                        long idx = ((b * T + t) * H + u) * 2 + s;
+                        hn[idx] = hk[idx] + xs[2 * t + s];
+                        dloc = absmax_update(dloc, xs[2 * t + s]);
+                    }
+                if (dloc > delta) delta = dloc;
+                free(Jb);
+                free(r);
+                free(xs);
+                free(work);
+            }
         } else if (m->solver == ORC_ELK) {
+            /* ELK on a diagonal linearisation (ParaGRU; the ParaLSTM's block diagonal with
+             * quasi set): one scalar smoother per state component */
 #pragma omp parallel for schedule(static) reduction(max : delta)
             for (long bu = 0; bu < B * H; ++bu) {
                 long b = bu / H, u = bu % H;

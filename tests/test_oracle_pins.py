@@ -329,10 +329,11 @@ def test_fixed_point_sweeps_match_their_definition(cell, solver):
     np.testing.assert_allclose(h, R, atol=1e-12)
 
 
-def _lm_stacked(lib, xp, h0, iters, lam, state_shape):
+def _lm_stacked(lib, xp, h0, iters, lam, state_shape, diag_only=True):
     """Levenberg-Marquardt on the stacked residual F(h) = 0 with a dense solve:
-    h <- h - (Jd^T Jd + lam I)^{-1} Jd^T F, where Jd is dF/dh (autograd) with only the
-    diagonal of each sub-diagonal block kept (the diagonal linearisation)."""
+    h <- h - (Jd^T Jd + lam I)^{-1} Jd^T F, where Jd is dF/dh (autograd), with only the
+    diagonal of each sub-diagonal block kept (the diagonal linearisation) when
+    diag_only, else the whole Jacobian (full 2x2 blocks for the LSTM)."""
     xpt, h0t = torch.tensor(xp), torch.tensor(h0)
     hs = torch.zeros(state_shape, dtype=f64)
     B, T = hs.shape[:2]
@@ -343,11 +344,12 @@ def _lm_stacked(lib, xp, h0, iters, lam, state_shape):
         Jf = torch.autograd.functional.jacobian(
             lambda v: tc.stacked_residual(lib, xpt, h0t, v.reshape(hs.shape)).reshape(-1), hs.reshape(-1))
         Jm = Jf.reshape(B, T, D, B, T, D).clone()
-        off = ~torch.eye(D, dtype=torch.bool)
-        for b in range(B):
-            for t in range(1, T):
-                blk = Jm[b, t, :, b, t - 1, :]
-                blk[off] = 0.0
+        if diag_only:
+            off = ~torch.eye(D, dtype=torch.bool)
+            for b in range(B):
+                for t in range(1, T):
+                    blk = Jm[b, t, :, b, t - 1, :]
+                    blk[off] = 0.0
         Jd = Jm.reshape(B * T * D, B * T * D)
         step = torch.linalg.solve(Jd.T @ Jd + lam * torch.eye(Jd.shape[0], dtype=f64), Jd.T @ F)
         hs = hs - step.reshape(hs.shape)
@@ -355,39 +357,100 @@ def _lm_stacked(lib, xp, h0, iters, lam, state_shape):
     return out
 
 
-@pytest.mark.parametrize("cell", ["gru", "lstm", "tanh"])
+ELK_VARIANTS = [("gru", False), ("lstm", False), ("lstm", True), ("tanh", False)]
+
+
+@pytest.mark.parametrize("cell,quasi", ELK_VARIANTS)
 @pytest.mark.parametrize("lam", [0.3, 2.0])
-def test_elk_step_is_levenberg_marquardt_on_stacked_system(cell, lam):
-    """The Kalman-smoother step equals the dense Levenberg-Marquardt step."""
+def test_elk_step_is_levenberg_marquardt_on_stacked_system(cell, quasi, lam):
+    """The Kalman-smoother step equals the dense Levenberg-Marquardt step: with the
+    LSTM's full 2x2 blocks (ELK), or each block's diagonal (quasi-ELK; the tanh RNN's
+    ELK always takes the diagonal of its dense Jacobian)."""
     H = 3
     m, xp, prm, h0 = _rand_model(cell, B=2, T=8, H=H, seed=71)
-    m = oracle.Model(cell, xp, solver="elk", damping=lam, **prm)
-    refs = _lm_stacked(_lib(cell, H, prm), xp, h0, 3, lam, m.state_shape)
+    m = oracle.Model(cell, xp, solver="elk", damping=lam, quasi=quasi, **prm)
+    full = cell == "lstm" and not quasi
+    refs = _lm_stacked(_lib(cell, H, prm), xp, h0, 3, lam, m.state_shape, diag_only=not full)
     for k, ref in enumerate(refs, start=1):
         h, iters, _ = m.newton(h0, max_iters=k, tol=0.0)
         assert iters == k
         np.testing.assert_allclose(h, ref.numpy(), atol=1e-11)
 
 
-@pytest.mark.parametrize("cell", ["gru", "lstm", "tanh"])
-def test_elk_without_damping_is_the_diagonal_newton_step(cell):
+@pytest.mark.parametrize("cell,quasi", ELK_VARIANTS)
+def test_elk_without_damping_is_the_newton_step(cell, quasi):
+    """lambda = 0: the step of the same linearisation without damping (the full-block
+    Newton step for ELK on the LSTM, the diagonal quasi-Newton step otherwise)."""
     m, xp, prm, h0 = _rand_model(cell, B=2, T=30, H=4, seed=72)
-    e = oracle.Model(cell, xp, solver="elk", damping=0.0, **prm)
-    q = oracle.Model(cell, xp, quasi=True, **prm)  # GRU: its Jacobian is already diagonal
+    e = oracle.Model(cell, xp, solver="elk", damping=0.0, quasi=quasi, **prm)
+    q = oracle.Model(cell, xp, quasi=quasi or cell == "tanh", **prm)  # GRU: its Jacobian is already diagonal
     for k in (1, 2, 4):
         np.testing.assert_allclose(e.newton(h0, max_iters=k, tol=0.0)[0], q.newton(h0, max_iters=k, tol=0.0)[0],
                                    atol=1e-12)
 
 
-@pytest.mark.parametrize("cell", ["gru", "lstm", "tanh"])
-def test_elk_converges_to_rollout_and_damping_shortens_steps(cell):
+@pytest.mark.parametrize("cell,quasi", ELK_VARIANTS)
+def test_elk_converges_to_rollout_and_damping_shortens_steps(cell, quasi):
     m, xp, prm, h0 = _rand_model(cell, B=2, T=40, H=4, seed=73, scale=1.5)
     R = m.rollout(h0)
-    h, iters, d = oracle.Model(cell, xp, solver="elk", damping=0.5, **prm).newton(h0, max_iters=400, tol=1e-12)
+    h, iters, d = oracle.Model(cell, xp, solver="elk", damping=0.5, quasi=quasi, **prm).newton(
+        h0, max_iters=400, tol=1e-12)
     np.testing.assert_allclose(h, R, atol=1e-10)
-    first = [oracle.Model(cell, xp, solver="elk", damping=lam, **prm).newton(h0, max_iters=1, tol=0.0)[2][0]
-             for lam in (0.0, 0.5, 5.0)]
+    first = [oracle.Model(cell, xp, solver="elk", damping=lam, quasi=quasi, **prm).newton(
+        h0, max_iters=1, tol=0.0)[2][0] for lam in (0.0, 0.5, 5.0)]
     assert first[0] > first[1] > first[2]
+
+
+def _block_lm_dense(J, r, lam):
+    """argmin_x sum_t |x_t - J_t x_{t-1} - r_t|^2 + lam |x|^2 (x_{-1} = 0), solved densely."""
+    T = J.shape[0]
+    L = np.eye(2 * T)
+    for t in range(1, T):
+        L[2 * t:2 * t + 2, 2 * t - 2:2 * t] = -J[t]
+    return np.linalg.solve(L.T @ L + lam * np.eye(2 * T), L.T @ r.reshape(-1)).reshape(T, 2)
+
+
+@pytest.mark.parametrize("T", [1, 7, 40])
+@pytest.mark.parametrize("lam", [0.0, 0.4, 3.0])
+def test_block_smoother_is_the_dense_lm_solution(T, lam):
+    """The 2x2 Kalman filter + RTS smoother against the normal equations of its objective."""
+    rng = np.random.default_rng(T * 10 + int(lam * 10))
+    J = rng.standard_normal((T, 2, 2)) * 0.8
+    r = rng.standard_normal((T, 2))
+    np.testing.assert_allclose(oracle.elk_block2(J, r, lam), _block_lm_dense(J, r, lam), atol=1e-11)
+
+
+def test_block_smoother_without_damping_is_the_forward_recursion():
+    rng = np.random.default_rng(5)
+    T = 50
+    J = rng.standard_normal((T, 2, 2)) * 0.5
+    r = rng.standard_normal((T, 2))
+    x, ref = np.zeros(2), []
+    for t in range(T):
+        x = J[t] @ x + r[t]
+        ref.append(x)
+    np.testing.assert_allclose(oracle.elk_block2(J, r, 0.0), np.array(ref), atol=1e-12)
+
+
+def test_block_smoother_with_diagonal_blocks_is_two_scalar_smoothers():
+    rng = np.random.default_rng(6)
+    T = 60
+    a = rng.uniform(-1.2, 1.2, (T, 2))
+    r = rng.standard_normal((T, 2))
+    J = np.zeros((T, 2, 2))
+    J[:, 0, 0], J[:, 1, 1] = a[:, 0], a[:, 1]
+    x = oracle.elk_block2(J, r, 0.8)
+    for s in range(2):
+        np.testing.assert_allclose(x[:, s], oracle.elk_scalar(a[:, s], r[:, s], 0.8), atol=1e-12)
+
+
+def test_scalar_smoother_is_the_dense_lm_solution():
+    rng = np.random.default_rng(7)
+    T = 30
+    a, r = rng.uniform(-1.5, 1.5, T), rng.standard_normal(T)
+    L = np.eye(T) - np.diag(a[1:], -1)
+    ref = np.linalg.solve(L.T @ L + 1.3 * np.eye(T), L.T @ r)
+    np.testing.assert_allclose(oracle.elk_scalar(a, r, 1.3), ref, atol=1e-12)
 
 
 def test_newton_zero_iterations_returns_initial_guess():

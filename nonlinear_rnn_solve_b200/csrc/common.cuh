@@ -154,6 +154,9 @@ template <> struct Aff<1> {
     }
     __device__ __forceinline__ void to_floats(float *v) const { v[0] = a; v[1] = d; }
     __device__ __forceinline__ static Aff from_floats(const float *v) { return {v[0], v[1]}; }
+    // a published aggregate that is a constant map (its value does not depend on the carry)
+    __device__ __forceinline__ static bool const_floats(const float *v) { return v[0] == 0.f; }
+    __device__ __forceinline__ static void const_value(const float *v, float *x) { x[0] = v[1]; }
     static constexpr int kFloats = 2;
 };
 template <> struct Aff<2> {
@@ -180,6 +183,13 @@ template <> struct Aff<2> {
         v[0] = a00; v[1] = a01; v[2] = a10; v[3] = a11; v[4] = d0; v[5] = d1;
     }
     __device__ __forceinline__ static Aff from_floats(const float *v) { return {v[0], v[1], v[2], v[3], v[4], v[5]}; }
+    __device__ __forceinline__ static bool const_floats(const float *v) {
+        return v[0] == 0.f && v[1] == 0.f && v[2] == 0.f && v[3] == 0.f;
+    }
+    __device__ __forceinline__ static void const_value(const float *v, float *x) {
+        x[0] = v[4];
+        x[1] = v[5];
+    }
     static constexpr int kFloats = 6;
 };
 
@@ -383,7 +393,7 @@ __device__ bool resolve_carry(const LookBack<S> &lb, long tile, int chunk, long 
                     v = E::cst(iv);
                 } else if (agg_ok) {
                     v = E::from_floats(av);
-                    st = aff_is_const<S>(av) ? 2u : 1u;
+                    st = E::const_floats(av) ? 2u : 1u;
                 } else {
                     st = 0u;
                 }
@@ -467,11 +477,8 @@ __device__ bool look_back(const LookBack<S> &lb, ScanSmem<S, C, NT, E> &sm, cons
     if (halo != nullptr && chunk > 0) {
         float hv[E::kFloats];
         halo->to_floats(hv);
-        known = __all_sync(0xffffffffu, lane >= C || aff_is_const<S>(hv));
-        if (known) {
-#pragma unroll
-            for (int q = 0; q < S; ++q) carry[q] = hv[S * S + q];
-        }
+        known = __all_sync(0xffffffffu, lane >= C || E::const_floats(hv));
+        if (known) E::const_value(hv, carry);
     }
     if (!known && !resolve_carry<S, C, E>(lb, tile, chunk, nseq, epoch, base, carry, ctl, sticky, dbg)) return false;
     publish_inc<S, C, E>(lb, total, carry, tile, epoch, dbg);

@@ -70,6 +70,13 @@ struct PAff2 {
         v[0] = a00; v[1] = a01; v[2] = a10; v[3] = a11; v[4] = d0; v[5] = d1;
     }
     __device__ __forceinline__ static PAff2 from_floats(const float *v) { return {v[0], v[1], v[2], v[3], v[4], v[5]}; }
+    __device__ __forceinline__ static bool const_floats(const float *v) {
+        return v[0] == 0.f && v[1] == 0.f && v[2] == 0.f && v[3] == 0.f;
+    }
+    __device__ __forceinline__ static void const_value(const float *v, float *x) {
+        x[0] = v[4];
+        x[1] = v[5];
+    }
 };
 __device__ __forceinline__ PAff2 compose(const PAff2 &i, const PAff2 &o) {
     PAff2 r;
@@ -535,16 +542,6 @@ cudaError_t elk_launch_common(ElkArgs &E, long D, float lambda, const Plan &plan
 
 }  // namespace
 
-int elk_plan(const NewtonDiagReq &r, int num_sms, Plan *plan) {
-    const int S = r.cell == 1 ? 2 : 1;
-    const int D = r.H * S;
-    const int C = pick_C(D);
-    const bool fused = r.xproj == nullptr;
-    const void *k = S == 1 ? (fused ? elk_by_C<GruCell, -1>(C) : elk_by_C<GruCell, 0>(C))
-                           : (fused ? elk_by_C<LstmCell, -1>(C) : elk_by_C<LstmCell, 0>(C));
-    return elk_plan_common(k, r.B, r.T, D, C, r.max_iters, num_sms, plan);
-}
-
 int elk_tanh_plan(const NewtonTanhReq &r, int num_sms, Plan *plan) {
     if (r.n > kElkMaxN) return 1;
     const int C = pick_C(r.n);
@@ -574,32 +571,6 @@ cudaError_t elk_tanh_launch(const NewtonTanhReq &r, float lambda, const Plan &pl
     A.residual_out = r.residual_out;
     E.Amat = r.A;
     return elk_launch_common(E, r.n, lambda, plan, w, dbg, st);
-}
-
-cudaError_t elk_launch(const NewtonDiagReq &r, float lambda, const Plan &plan, const Work &w, const DbgHost &dbg,
-                       cudaStream_t st) {
-    ElkArgs E;
-    NewtonDiagArgs &A = E.A;
-    memset(&E, 0, sizeof(E));
-    A.B = r.B;
-    A.T = r.T;
-    A.H = r.H;
-    A.in = r.in;
-    A.jmode = 0;
-    A.xproj = r.xproj;
-    A.x = r.x;
-    A.W = r.W;
-    A.bias = r.bias;
-    A.a = r.a;
-    A.peep = r.peep;
-    A.h0 = r.h0;
-    A.h = r.h;
-    A.max_iters = r.max_iters;
-    A.tol = r.tol;
-    A.iters_out = r.iters_out;
-    A.delta_out = r.delta_out;
-    A.residual_out = r.residual_out;
-    return elk_launch_common(E, (long)r.H * (r.cell == 1 ? 2 : 1), lambda, plan, w, dbg, st);
 }
 
 }  // namespace prn

@@ -411,6 +411,23 @@ def measure_workload(L, w, inp, parts=None):
             e["roofline"] = dict(_hbm_entry(ms, nb, hbm), bound="latency",
                                  note="8,192 state elements: launch and iteration latency, no bandwidth claim")
         out["forward"] = e
+        if w.cell == wl.GRU:
+            # ELK (damping 1) on the same shape: per-iteration algorithmic bytes as the
+            # Newton solve's, over its own time; the ratio compares bytes/s
+            lam = 1.0
+            fe = lambda: solve.newton_forward(ctx.ctx, cell, w.B, w.T, w.H, h0=t["h0"],  # noqa: E731
+                                              max_iters=w.max_iters, tol=w.tol, h_out=h_out, scalars=sc,
+                                              solver="elk", damping=lam, **kw)
+            ms_e = L.time(fe)
+            it_e = int(sc["iters"].item())
+            nb_e = forward_bytes(w, it_e, False)
+            ee = {"ms": ms_e, "iters": it_e, "damping": lam, "device_status": _ctx_status(ctx)}
+            ee["roofline"] = _hbm_entry(ms_e, nb_e, hbm)
+            ee["bytes_per_s_vs_newton"] = (nb_e / ms_e) / (nb / ms)
+            if w.H <= 8 and w.elems < 1 << 20:
+                ee["roofline"] = dict(ee["roofline"], bound="latency",
+                                      note="8,192 state elements: launch and iteration latency, no bandwidth claim")
+            out["elk"] = ee
         return out
     # the LLM-width layers: projection GEMM, forward on xproj, adjoint, projection backward
     parts = parts or LAYER_PARTS
@@ -701,6 +718,10 @@ def run_ours(args, w):
             allc, one = cpu_baselines(w, inp)
             line["cpu_baseline"] = dict(allc, one_core=one, oracle_newton=cpu_newton(w, inp, allc["cores"]))
             line["per_config"] = per_config(ctx, dev, stream, flush)
+            if w.cell == wl.GRU:
+                # ELK on the headline shape, its bytes/s against the Newton solve's
+                line["elk_same_shape"] = measure_workload(_Legs(ctx, dev, stream, flush, reps=5, warmup=3), w,
+                                                          inp).get("elk")
         print(json.dumps(line), flush=True)
     ctx.close()
     if ws > 1:

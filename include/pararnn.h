@@ -107,10 +107,12 @@ typedef enum {
     /* ELK ("Towards Scalable and Stable Parallelization of Nonlinear RNNs", Abstract):
      * the Levenberg-Marquardt step of the stacked system, i.e. the minimiser of
      * sum_t |x_t - J_t x_{t-1} - r_t|^2 + damping sum_t |x_t|^2 (x = h^(k+1) - h^(k),
-     * r_t = f_t - h^(k)_t), computed by a parallel Kalman filter and smoother; J_t is
-     * diagonal: ParaGRU (ELK), ParaLSTM with each block's diagonal and the tanh RNN
-     * (either tanh cell id, n <= 64) with the diagonal of its Jacobian (quasi-ELK).
-     * damping = 0 gives the quasi-Newton step; larger damping shortens the steps. */
+     * r_t = f_t - h^(k)_t), computed by a parallel Kalman filter and smoother.  J_t is
+     * the ParaGRU's diagonal Jacobian, the ParaLSTM's full 2x2 block per unit
+     * (PARARNN_LSTM_CIFG_PEEP: ELK) or its diagonal (PARARNN_LSTM_CIFG_PEEP_QUASI:
+     * quasi-ELK), and the diagonal of the tanh RNN's Jacobian (either tanh cell id,
+     * n <= 64: quasi-ELK).  damping = 0 gives the undamped step of the same
+     * linearisation; larger damping shortens the steps. */
     PARARNN_SOLVER_ELK = 3
 } pararnn_solver;
 

@@ -407,9 +407,11 @@ def measure_workload(L, w, inp, parts=None):
             else:
                 e["roofline"] = _alu_entry(ms, fl, _fp32_peak_tflops()) if not w.quasi else _hbm_entry(ms, nb, hbm)
             e["roofline_other"] = _hbm_entry(ms, nb, hbm) if not w.quasi else _alu_entry(ms, fl, _fp32_peak_tflops())
-        else:
+        elif w.elems < 1 << 20:
             e["roofline"] = dict(_hbm_entry(ms, nb, hbm), bound="latency",
                                  note="8,192 state elements: launch and iteration latency, no bandwidth claim")
+        else:
+            e["roofline"] = _hbm_entry(ms, nb, hbm)
         out["forward"] = e
         if w.cell == wl.GRU:
             # ELK (damping 1) on the same shape: per-iteration algorithmic bytes as the

@@ -80,11 +80,13 @@ template <int S> __device__ __forceinline__ void mat_tvec(const float *X, const 
         r[0] = r0, r[S - 1] = r1;
     }
 }
-template <int S> __device__ __forceinline__ void mat_inv(const float *X, float *R) {  // R = X^{-1}
+// R = X^{-1}, with the hardware reciprocal (a few ulp; the matrices inverted here are
+// I + (positive semi-definite) x (positive semi-definite) products, far from singular)
+template <int S> __device__ __forceinline__ void mat_inv(const float *X, float *R) {
     if (S == 1) {
-        R[0] = 1.f / X[0];
+        R[0] = rcp_hw(X[0]);
     } else {
-        const float id = 1.f / fmaf(X[0], X[3 % (S * S)], -X[1] * X[2 % (S * S)]);
+        const float id = rcp_hw(fmaf(X[0], X[3 % (S * S)], -X[1] * X[2 % (S * S)]));
         const float r0 = X[3 % (S * S)] * id, r1 = -X[1] * id, r2 = -X[2 % (S * S)] * id, r3 = X[0] * id;
         R[0] = r0, R[1 % (S * S)] = r1, R[2 % (S * S)] = r2, R[3 % (S * S)] = r3;
     }

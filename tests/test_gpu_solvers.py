@@ -63,6 +63,8 @@ CASES = [  # (cell, B, T, H, in, xproj)
     ("lstm", 1, 4096, 1, 2, False),
     ("lstm", 2, 400, 64, 4, True),
     ("tanh", 3, 700, 8, 4, False),
+    ("tanh", 2, 600, 48, 4, False),   # 32 < n <= 64: the tensor-core cell product
+    ("tanh", 2, 300, 64, 4, True),
 ]
 
 

@@ -173,14 +173,17 @@ TC_CASES = [  # (n, B, T, in, use_xproj): the tensor-core DEER kernel, 128-step 
 ]
 
 
+@pytest.mark.parametrize("quasi", [False, True])
 @pytest.mark.parametrize("case", TC_CASES)
-def test_deer_tensor_core_tiles(ctx, case):
-    """Full DEER at 32 < n <= 64 with the Jacobian products on the tensor cores: several
-    sequences, ragged last tiles (chains partly filled or empty), raw and projected
-    inputs, a non-zero h0; iteration count, states and residual against the oracle."""
+def test_deer_tensor_core_tiles(ctx, case, quasi):
+    """The tanh RNN at 32 < n <= 64 with the cell product on the tensor cores: full DEER
+    (Jacobian products on the tensor cores too) and quasi-DEER (per-unit scans with the
+    decoupled look-back); several sequences, ragged last tiles (chains partly filled or
+    empty), raw and projected inputs, a non-zero h0; iteration count, states and residual
+    against the oracle."""
     n, B, T, inp_w, use_xp = case
     w = wl.WORKLOADS["tanh_b16_t65536_in4_n64_deer"].resized(H=n, B=B, T=T, inp=inp_w, seed=n + 7 * T,
-                                                              max_iters=T + 1)
+                                                              max_iters=T + 1, quasi=quasi)
     inp = wl.generate(w)
     rng = np.random.default_rng(T)
     inp["h0"] = (rng.standard_normal(inp["h0"].shape) * 0.3).astype(np.float32)
@@ -188,7 +191,7 @@ def test_deer_tensor_core_tiles(ctx, case):
     out = _run(ctx, w, inp, xproj=xp, residual=True)
     assert ctx.status() == 0
     if use_xp:
-        m = oracle.Model("tanh", xp.reshape(B, T, 1, n), A=inp["A"])
+        m = oracle.Model("tanh", xp.reshape(B, T, 1, n), A=inp["A"], quasi=quasi)
         h_ref, it_ref, _ = m.newton(inp["h0"], max_iters=w.max_iters, tol=w.tol)
         assert int(out["iters"].item()) == it_ref
         assert max_abs(host(out["h"]), h_ref) <= TOL_STATE
@@ -202,6 +205,26 @@ def test_deer_tensor_core_withheld_publication_times_out(ctx):
     successor's bounded wait runs out, the status reads ETIMEOUT, the context recovers."""
     from nonlinear_rnn_solve_b200 import PARARNN_ETIMEOUT
     w = wl.WORKLOADS["tanh_b16_t65536_in4_n64_deer"].resized(B=1, T=4 * 128, seed=78, max_iters=4 * 128)
+    inp = wl.generate(w)
+    pararnn_debug_set(ctx.ctx, 1, 50_000_000)
+    pararnn_debug_set(ctx.ctx, 2, 1)
+    try:
+        _run(ctx, w, inp, max_iters=10)
+        assert ctx.status() == PARARNN_ETIMEOUT
+    finally:
+        pararnn_debug_set(ctx.ctx, 2, -1)
+        pararnn_debug_set(ctx.ctx, 1, 1_000_000_000)
+    out = _run(ctx, w, inp)
+    assert ctx.status() == 0
+    _check(ctx, w, inp, out)
+
+
+def test_quasi_tensor_core_withheld_publication_times_out(ctx):
+    """Quasi-DEER at n = 64 (tensor-core cell product, per-unit look-back): a tile withholds
+    its published values (knob 2); the successor's bounded look-back wait runs out, the
+    status reads ETIMEOUT, the context recovers."""
+    from nonlinear_rnn_solve_b200 import PARARNN_ETIMEOUT
+    w = wl.WORKLOADS["tanh_b16_t65536_in4_n64_quasi"].resized(B=1, T=4 * 128, seed=79, max_iters=4 * 128)
     inp = wl.generate(w)
     pararnn_debug_set(ctx.ctx, 1, 50_000_000)
     pararnn_debug_set(ctx.ctx, 2, 1)

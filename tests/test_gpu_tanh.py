@@ -224,7 +224,8 @@ def test_quasi_tensor_core_withheld_publication_times_out(ctx):
     its published values (knob 2); the successor's bounded look-back wait runs out, the
     status reads ETIMEOUT, the context recovers."""
     from nonlinear_rnn_solve_b200 import PARARNN_ETIMEOUT
-    w = wl.WORKLOADS["tanh_b16_t65536_in4_n64_quasi"].resized(B=1, T=4 * 128, seed=79, max_iters=4 * 128)
+    # seed 80: the deltas around the stopping iteration sit 1.3x from the tolerance
+    w = wl.WORKLOADS["tanh_b16_t65536_in4_n64_quasi"].resized(B=1, T=4 * 128, seed=80, max_iters=4 * 128)
     inp = wl.generate(w)
     pararnn_debug_set(ctx.ctx, 1, 50_000_000)
     pararnn_debug_set(ctx.ctx, 2, 1)

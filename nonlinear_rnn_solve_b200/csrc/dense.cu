@@ -373,53 +373,38 @@ template <int N> __device__ void quasi_stage_params(const TanhArgs &A, QuasiSmem
     for (int i = threadIdx.x; i < N; i += kThreads) sm.diag[i] = i < A.n ? A.A[(size_t)i * A.n + i] : 0.f;
 }
 
-// Stage the tile's states (h^(k) rows t0-1 .. t0+TCH-1: h0 before t = 0, the side
-// value for the preceding tile's last step, zeros on the first iteration) and raw
-// inputs, transposed so that four consecutive steps of one unit are one 128-bit read.
-template <int N>
-__device__ void quasi_stage_tile(const TanhArgs &A, QuasiSmem<N> &sm, int b, int t0, bool have_h,
-                                 const float *prev_side) {
-    constexpr int TCH = QuasiSmem<N>::TCH, HS = QuasiSmem<N>::HS;
-    for (int e = threadIdx.x; e < (TCH + 1) * N; e += kThreads) {
-        const int r = e / N, i = e % N, t = t0 + r - 1;
-        float v = 0.f;
-        if (i < A.n) {
-            if (t < 0)
-                v = A.h0 ? A.h0[(size_t)b * A.n + i] : 0.f;
-            else if (t < A.T && have_h)
-                v = (r == 0 && prev_side) ? prev_side[i] : A.h[((size_t)b * A.T + t) * A.n + i];
-        }
-        sm.hT[i * HS + r] = v;
-        sm.hr[e] = v;
-    }
-    if (!A.xproj) {
-        for (int e = threadIdx.x; e < TCH * 8; e += kThreads) {
-            const int r = e / 8, q = e % 8, t = t0 + r;
-            sm.xT[q * HS + r] = (q < A.in && t < A.T) ? A.x[((size_t)b * A.T + t) * A.in + q] : 0.f;
-        }
-    }
+// h^(k) of unit i at tile row r (the state before step t0 + r): h0 before the sequence,
+// the side value for the preceding tile's last step, zeros on the first iteration.
+__device__ __forceinline__ float quasi_state(const TanhArgs &A, int b, int t0, int r, int i, bool have_h,
+                                             const float *prev_side) {
+    const int t = t0 + r - 1;
+    if (i >= A.n) return 0.f;
+    if (t < 0) return A.h0 ? A.h0[(size_t)b * A.n + i] : 0.f;
+    if (t < A.T && have_h) return (r == 0 && prev_side) ? prev_side[i] : A.h[((size_t)b * A.T + t) * A.n + i];
+    return 0.f;
 }
 
-// The next tile's states and inputs, loaded into registers while the current tile
-// computes, and written to shared memory (as quasi_stage_tile does) when it starts.
+// A tile's states (rows 0 .. TCH: the states before steps t0 .. t0 + TCH) and raw inputs,
+// loaded into registers -- the next tile's while the current one computes -- and then
+// written to shared memory, transposed (hT: four consecutive steps of one unit are one
+// 128-bit word) and by rows (hr).  A thread holds 4-row groups of one unit, so each
+// transposed write is one 128-bit store: a quarter-warp writes eight units' groups at
+// unit strides of HS floats (HS % 32 == 4), eight distinct 16-byte bank groups.
 template <int N> struct QuasiPrefetch {
     static constexpr int TCH = QuasiSmem<N>::TCH, HS = QuasiSmem<N>::HS;
-    static constexpr int HPT = ((TCH + 1) * N + kThreads - 1) / kThreads;
+    static constexpr int G4 = TCH * N / 4 / kThreads;  // 4-row groups per thread
     static constexpr int XPT = TCH * 8 / kThreads;
-    float hv[HPT], xv[XPT];
+    static_assert(G4 * 4 * kThreads == TCH * N, "whole 4-row groups per thread");
+    static_assert(HS % 4 == 0 && HS % 32 == 4, "float4 rows, conflict-free transposed stores");
+    float hv[G4][4], hx, xv[XPT];
     __device__ __forceinline__ void load(const TanhArgs &A, int b, int t0, bool have_h, const float *prev_side) {
 #pragma unroll
-        for (int j = 0; j < HPT; ++j) {
-            const int e = threadIdx.x + j * kThreads, r = e / N, i = e % N, t = t0 + r - 1;
-            float v = 0.f;
-            if (e < (TCH + 1) * N && i < A.n) {
-                if (t < 0)
-                    v = A.h0 ? A.h0[(size_t)b * A.n + i] : 0.f;
-                else if (t < A.T && have_h)
-                    v = (r == 0 && prev_side) ? prev_side[i] : A.h[((size_t)b * A.T + t) * A.n + i];
-            }
-            hv[j] = v;
+        for (int j = 0; j < G4; ++j) {
+            const int e4 = threadIdx.x + j * kThreads, g = e4 / N, i = e4 % N;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) hv[j][q] = quasi_state(A, b, t0, 4 * g + q, i, have_h, prev_side);
         }
+        hx = threadIdx.x < N ? quasi_state(A, b, t0, TCH, threadIdx.x, have_h, prev_side) : 0.f;
         if (!A.xproj) {
 #pragma unroll
             for (int j = 0; j < XPT; ++j) {
@@ -430,12 +415,15 @@ template <int N> struct QuasiPrefetch {
     }
     __device__ __forceinline__ void store(const TanhArgs &A, QuasiSmem<N> &sm) const {
 #pragma unroll
-        for (int j = 0; j < HPT; ++j) {
-            const int e = threadIdx.x + j * kThreads;
-            if (e < (TCH + 1) * N) {
-                sm.hT[(e % N) * HS + e / N] = hv[j];
-                sm.hr[e] = hv[j];
-            }
+        for (int j = 0; j < G4; ++j) {
+            const int e4 = threadIdx.x + j * kThreads, g = e4 / N, i = e4 % N;
+            *reinterpret_cast<float4 *>(sm.hT + i * HS + 4 * g) = make_float4(hv[j][0], hv[j][1], hv[j][2], hv[j][3]);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) sm.hr[(4 * g + q) * N + i] = hv[j][q];
+        }
+        if (threadIdx.x < N) {
+            sm.hT[threadIdx.x * HS + TCH] = hx;
+            sm.hr[TCH * N + threadIdx.x] = hx;
         }
         if (!A.xproj) {
 #pragma unroll
@@ -446,6 +434,15 @@ template <int N> struct QuasiPrefetch {
         }
     }
 };
+
+// Stage a tile directly (the first tile of an iteration, the residual pass).
+template <int N>
+__device__ __forceinline__ void quasi_stage_tile(const TanhArgs &A, QuasiSmem<N> &sm, int b, int t0, bool have_h,
+                                                 const float *prev_side) {
+    QuasiPrefetch<N> p;
+    p.load(A, b, t0, have_h, prev_side);
+    p.store(A, sm);
+}
 
 // Phase A: f = tanh(A h_{t-1} + p_t) for the thread's 4 x 4 block; J = (1 - f^2) A_ii
 // (identity outside the sequence), r = f - h^(k)_t; returns max |r| over valid entries.

@@ -9,8 +9,10 @@
 //   warp 1  allocates 2 x 256 TMEM columns and (one elected thread) issues
 //           tcgen05.mma.cta_group::1.kind::f16 (M = 128, N = 256, K = 16, bf16 x bf16 ->
 //           fp32 in TMEM), releasing each stage with tcgen05.commit;
-//   warps 2-5 read the accumulator with tcgen05.ld (32 lanes x 16 columns per load), add
-//           the bias and store fp32 rows.
+//   warps 2-9 drain the other accumulator: warp w owns TMEM lanes 32 (w % 4) .. + 31 (tile
+//           rows) and columns 128 ((w - 2) / 4) .. + 127; a thread pulls its 128 columns
+//           out of TMEM with one wait, hands the accumulator back at once, then adds the
+//           bias and stores fp32 rows (so the next tile's MMAs never wait on the stores).
 // Every mbarrier wait is bounded (%globaltimer); on a timeout the CTA raises the
 // status bit, frees its TMEM and returns.
 // fp32 path: a CUDA-core tiled GEMM (x and W both fp32).
@@ -31,7 +33,7 @@ namespace gemm {
 constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
 constexpr int A_BYTES = BM * BK * 2, B_BYTES = BN * BK * 2, STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int TMEM_COLS = 256;
-constexpr int THREADS = 192;
+constexpr int THREADS = 320;  // TMA warp, MMA warp, 8 epilogue warps
 constexpr unsigned long long WAIT_NS = 2000000000ull;
 
 __device__ __forceinline__ unsigned smem_u32(const void *p) { return (unsigned)__cvta_generic_to_shared(p); }
@@ -70,6 +72,22 @@ __device__ __forceinline__ void tma_load_2d(unsigned dst, const CUtensorMap *map
         "l"(reinterpret_cast<unsigned long long>(map)), "r"(x), "r"(y), "r"(bar)
         : "memory");
 }
+// 128 consecutive TMEM columns of this thread's lane (four 32-column loads, one wait).
+__device__ __forceinline__ void tmem_ld128(unsigned taddr, float (&v)[128]) {
+    unsigned r[128];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%128];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, %48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63}, [%129];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%64, %65, %66, %67, %68, %69, %70, %71, %72, %73, %74, %75, %76, %77, %78, %79, %80, %81, %82, %83, %84, %85, %86, %87, %88, %89, %90, %91, %92, %93, %94, %95}, [%130];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%96, %97, %98, %99, %100, %101, %102, %103, %104, %105, %106, %107, %108, %109, %110, %111, %112, %113, %114, %115, %116, %117, %118, %119, %120, %121, %122, %123, %124, %125, %126, %127}, [%131];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]), "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]), "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63]), "=r"(r[64]), "=r"(r[65]), "=r"(r[66]), "=r"(r[67]), "=r"(r[68]), "=r"(r[69]), "=r"(r[70]), "=r"(r[71]), "=r"(r[72]), "=r"(r[73]), "=r"(r[74]), "=r"(r[75]), "=r"(r[76]), "=r"(r[77]), "=r"(r[78]), "=r"(r[79]), "=r"(r[80]), "=r"(r[81]), "=r"(r[82]), "=r"(r[83]), "=r"(r[84]), "=r"(r[85]), "=r"(r[86]), "=r"(r[87]), "=r"(r[88]), "=r"(r[89]), "=r"(r[90]), "=r"(r[91]), "=r"(r[92]), "=r"(r[93]), "=r"(r[94]), "=r"(r[95]), "=r"(r[96]), "=r"(r[97]), "=r"(r[98]), "=r"(r[99]), "=r"(r[100]), "=r"(r[101]), "=r"(r[102]), "=r"(r[103]), "=r"(r[104]), "=r"(r[105]), "=r"(r[106]), "=r"(r[107]), "=r"(r[108]), "=r"(r[109]), "=r"(r[110]), "=r"(r[111]), "=r"(r[112]), "=r"(r[113]), "=r"(r[114]), "=r"(r[115]), "=r"(r[116]), "=r"(r[117]), "=r"(r[118]), "=r"(r[119]), "=r"(r[120]), "=r"(r[121]), "=r"(r[122]), "=r"(r[123]), "=r"(r[124]), "=r"(r[125]), "=r"(r[126]), "=r"(r[127])
+        : "r"(taddr), "r"(taddr + 32), "r"(taddr + 64), "r"(taddr + 96)
+        : "memory");
+#pragma unroll
+    for (int j = 0; j < 128; ++j) v[j] = __uint_as_float(r[j]);
+}
+
 // Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups 1024 B apart.
 __device__ __forceinline__ unsigned long long smem_desc(unsigned addr) {
     return (unsigned long long)((addr >> 4) & 0x3FFF) | (1ull << 16) | (64ull << 32) | (1ull << 46) |
@@ -106,7 +124,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(smem_u32(&acc_full[a]), 1);
-            mbar_init(smem_u32(&acc_empty[a]), 4);  // one arrival per epilogue warp
+            mbar_init(smem_u32(&acc_empty[a]), 8);  // one arrival per epilogue warp
         }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -177,12 +195,13 @@ __global__ void __launch_bounds__(THREADS, 1)
             }
         }
     } else {
-        // epilogue: warps 2..5 own TMEM lanes 32*(warp % 4) .. +31, i.e. tile rows
-        const int q = warp & 3;
+        // epilogue: warps 2..9 own TMEM lanes 32*(warp % 4) .. +31 (tile rows) and one
+        // 128-column half of the tile
+        const int q = warp & 3, hcol = (warp - 2) >> 2;
         int ti = 0;
         for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++ti) {
             const int a = ti & 1;
-            const int m0 = (tile / ntiles_n) * BM, n0 = (tile % ntiles_n) * BN;
+            const int m0 = (tile / ntiles_n) * BM, n0 = (tile % ntiles_n) * BN + 128 * hcol;
             const int row = m0 + q * 32 + lane;
             const bool ok =
                 __all_sync(0xffffffffu, mbar_wait(smem_u32(&acc_full[a]), (unsigned)(ti >> 1) & 1u, &abort_flag));
@@ -191,63 +210,46 @@ __global__ void __launch_bounds__(THREADS, 1)
                 break;
             }
             asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-#pragma unroll 1
-            for (int c = 0; c < BN; c += 16) {
-                unsigned r[16];
-                const unsigned taddr = tmem + ((unsigned)(q * 32) << 16) + (unsigned)(a * TMEM_COLS + c);
-                asm volatile(
-                    "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, "
-                    "%13, %14, %15}, [%16];"
-                    : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-                      "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
-                      "=r"(r[15])
-                    : "r"(taddr));
-                asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-                if (c + 16 >= BN) {
-                    // every column of this accumulator is in registers: hand it back
-                    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-                    __syncwarp();
-                    if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&acc_empty[a])) : "memory");
-                }
-                const int col = n0 + c;
-                if (row < M) {
-                    float v[16];
+            float v[128];
+            tmem_ld128(tmem + ((unsigned)(q * 32) << 16) + (unsigned)(a * TMEM_COLS + 128 * hcol), v);
+            // this half of the accumulator is in registers: hand it back
+            asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+            __syncwarp();
+            if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&acc_empty[a])) : "memory");
+            if (row < M) {
+                float *yr = y + (size_t)row * N;
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(r[j]);
-                    const bool full = col + 16 <= N;
+                for (int c = 0; c < 128; c += 8) {
+                    const int col = n0 + c;
+                    const bool full = col + 8 <= N;
+                    float w[8];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) w[j] = v[c + j];
                     if (bias) {
                         if (full) {
-#pragma unroll
-                            for (int j = 0; j < 16; j += 4) {
-                                const float4 bv = __ldg(reinterpret_cast<const float4 *>(bias + col + j));
-                                v[j] += bv.x;
-                                v[j + 1] += bv.y;
-                                v[j + 2] += bv.z;
-                                v[j + 3] += bv.w;
-                            }
+                            const float4 b0 = __ldg(reinterpret_cast<const float4 *>(bias + col));
+                            const float4 b1 = __ldg(reinterpret_cast<const float4 *>(bias + col + 4));
+                            w[0] += b0.x, w[1] += b0.y, w[2] += b0.z, w[3] += b0.w;
+                            w[4] += b1.x, w[5] += b1.y, w[6] += b1.z, w[7] += b1.w;
                         } else {
 #pragma unroll
-                            for (int j = 0; j < 16; ++j)
-                                if (col + j < N) v[j] += __ldg(bias + col + j);
+                            for (int j = 0; j < 8; ++j)
+                                if (col + j < N) w[j] += __ldg(bias + col + j);
                         }
                     }
-                    float *yr = y + (size_t)row * N + col;
                     if (full && vec8) {
                         // whole 32-byte sectors per lane
-#pragma unroll
-                        for (int j = 0; j < 16; j += 8)
-                            asm volatile("st.global.v8.f32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(yr + j),
-                                         "f"(v[j]), "f"(v[j + 1]), "f"(v[j + 2]), "f"(v[j + 3]), "f"(v[j + 4]),
-                                         "f"(v[j + 5]), "f"(v[j + 6]), "f"(v[j + 7])
-                                         : "memory");
+                        asm volatile("st.global.v8.f32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(yr + col),
+                                     "f"(w[0]), "f"(w[1]), "f"(w[2]), "f"(w[3]), "f"(w[4]), "f"(w[5]), "f"(w[6]),
+                                     "f"(w[7])
+                                     : "memory");
                     } else if (full && (N & 3) == 0) {
-#pragma unroll
-                        for (int j = 0; j < 16; j += 4)
-                            *reinterpret_cast<float4 *>(yr + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+                        *reinterpret_cast<float4 *>(yr + col) = make_float4(w[0], w[1], w[2], w[3]);
+                        *reinterpret_cast<float4 *>(yr + col + 4) = make_float4(w[4], w[5], w[6], w[7]);
                     } else {
 #pragma unroll
-                        for (int j = 0; j < 16; ++j)
-                            if (col + j < N) yr[j] = v[j];
+                        for (int j = 0; j < 8; ++j)
+                            if (col + j < N) yr[col + j] = w[j];
                     }
                 }
             }

@@ -397,7 +397,7 @@ int adjoint_wide_plan(const AdjointReq &r, int num_sms, Plan *plan) {
     if (r.H % 32 || (long)np * r.H > kTabMax || !encode_fn()) return 1;
     if ((long)r.B * r.T >= (1L << 31)) return 1;
     const int rc = S == 1 ? choose<GruCell, 8>(plan, num_sms, r.B, r.T, r.H)
-                          : choose<LstmCell, 4>(plan, num_sms, r.B, r.T, r.H);
+                          : choose<LstmCell, 5>(plan, num_sms, r.B, r.T, r.H);
     if (rc) return -1;
     if (plan->ntiles > 0x7fffffffL) return 1;
     plan->variant = 300 + S;

@@ -260,7 +260,7 @@ def cpu_newton(w, inp, threads, budget_s=3.0):
 PER_CONFIG = ["gru_b1_t1024_in4_h8", "gru_b8_t4096_h2048_bf16", "lstm_b4_t8192_h1024_bf16",
               "tanh_b16_t65536_in4_n8_quasi", "tanh_b16_t65536_in4_n8_deer",
               "tanh_b16_t65536_in4_n64_deer", "tanh_b16_t65536_in4_n64_quasi"]
-LAYER_PARTS = ["proj", "forward", "backward", "proj_backward"]
+LAYER_PARTS = ["proj", "forward", "backward", "proj_backward", "layer_backward"]
 
 
 def _fp32_peak_tflops():
@@ -465,7 +465,7 @@ def measure_workload(L, w, inp, parts=None):
         out["forward"] = e
     else:
         fwd()
-    if "backward" in parts or "proj_backward" in parts:
+    if "backward" in parts or "proj_backward" in parts or "layer_backward" in parts:
         g = f32("g")
         gx = torch.empty(B, T, 3, H, device=dev)
         gp = torch.empty(5 if w.cell == wl.LSTM else 3, H, device=dev)
@@ -481,6 +481,17 @@ def measure_workload(L, w, inp, parts=None):
                                "roofline": _hbm_entry(ms, nb, hbm)}
         else:
             bwd()
+        if "layer_backward" in parts:
+            # the same two passes in one call, grad_xproj handed from the adjoint to the
+            # products in bf16 (no fp32 copy written or read)
+            from nonlinear_rnn_solve_b200 import pararnn_layer_backward
+            lx, lW, lb = torch.empty(M, K, device=dev), torch.empty(N, K, device=dev), torch.empty(N, device=dev)
+            lp, lh0 = torch.empty_like(gp), torch.empty_like(h0)
+            ms = L.time(lambda: pararnn_layer_backward(ctx.ctx, xp4, prm, h0, h, g, x, W, lx, lW, lb, lp, lh0))
+            out["layer_backward"] = {"ms": ms, "device_status": _ctx_status(ctx),
+                                     "shape": "adjoint + grad_x, grad_W, grad_bias in one call (bf16 grad_xproj)",
+                                     "roofline": _tensor_entry(ms, 4 * M * N * K, bf_peak, bf_kind)}
+            del lx, lW, lb, lp, lh0
         del g
         if "proj_backward" in parts:
             from nonlinear_rnn_solve_b200 import pararnn_input_proj_backward
@@ -740,7 +751,8 @@ def main():
     ap.add_argument("--skip-extras", action="store_true",
                     help="skip the e2e, CPU-baseline and per-config legs (for profiler runs)")
     ap.add_argument("--leg", default=None,
-                    help="WORKLOAD[:PART]: time one leg alone (PART: proj, forward, backward, proj_backward)")
+                    help="WORKLOAD[:PART]: time one leg alone (PART: proj, forward, backward, proj_backward, "
+                         "layer_backward)")
     args = ap.parse_args()
     w = wl.WORKLOADS[args.workload]
     if args.leg:

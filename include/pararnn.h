@@ -230,6 +230,28 @@ int pararnn_adjoint_backward(pararnn_ctx *ctx, const float *xproj, const pararnn
                              const float *h0, const float *h, const float *grad_h,
                              float *grad_xproj, float *grad_params, float *grad_h0);
 
+/* Backward pass of a whole trainable layer, input projection included: the adjoint of
+ * pararnn_adjoint_backward followed by the reverse pass of pararnn_input_proj_backward
+ * for bf16 x and W ("Para-Seq" README, Main features: trainable layers with adjoint
+ * backward), with grad_xproj never stored in fp32: the adjoint rounds it to bf16
+ * (nearest even, the operand the two tensor-core products read, exactly as
+ * pararnn_input_proj_backward rounds it) and sums its fp32 values into grad_bias.
+ *   xproj, p, h0, h, grad_h, grad_params, grad_h0 as for pararnn_adjoint_backward
+ *   x [B*T, K] bf16, W [3H, K] bf16 (the projection of pararnn_input_proj)
+ *   grad_x [B*T, K], grad_W [3H, K], grad_bias [3H]: fp32, each may be NULL (not computed)
+ * grad_x and grad_W equal those of pararnn_adjoint_backward + pararnn_input_proj_backward
+ * bit for bit; grad_bias sums the same fp32 terms with one float atomic per lane, gate
+ * and tile, so its last bits can differ between runs.  Shapes without the adjoint's
+ * TMA-fed tiles (H not a multiple of 32, or a parameter table over 12288 floats) take
+ * those two calls' path through an fp32 buffer in the scratch.
+ * Shapes: B*T, K and 3H multiples of 8, as for pararnn_input_proj_backward.  The
+ * context's scratch grows to the projection backward's plus, on the fallback path,
+ * 4 * B*T * 3H bytes.  Returns EINVAL, EALIGN, EUNSUPPORTED, ENOMEM or ECUDA. */
+int pararnn_layer_backward(pararnn_ctx *ctx, const float *xproj, const pararnn_params *p, const float *h0,
+                           const float *h, const float *grad_h, const void *x, const void *W, int K,
+                           float *grad_x, float *grad_W, float *grad_bias, float *grad_params,
+                           float *grad_h0);
+
 /* Synchronise the context's stream and report (then clear) device-side conditions:
  * *device_status = PARARNN_OK, PARARNN_ENONFINITE or PARARNN_ETIMEOUT (first seen). */
 int pararnn_get_status(pararnn_ctx *ctx, int *device_status);

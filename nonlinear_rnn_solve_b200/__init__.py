@@ -48,6 +48,7 @@ EXPORTED = [
     "pararnn_newton_forward", "pararnn_linear_scan", "pararnn_adjoint_backward",
     "pararnn_get_status", "pararnn_strerror", "pararnn_debug_set", "pararnn_last_launch_count",
     "pararnn_linear_scan_noalloc", "pararnn_input_proj_backward", "pararnn_lsim",
+    "pararnn_layer_backward",
 ]
 
 
@@ -94,6 +95,8 @@ def lib() -> ctypes.CDLL:
         L.pararnn_linear_scan_noalloc.argtypes = [i, vp, vp, vp, vp, i, i, i, i, vp, vp]
         L.pararnn_input_proj_backward.argtypes = [vp, vp, vp, i, vp, vp, vp, vp, i, i, i]
         L.pararnn_lsim.argtypes = [vp, vp, vp, vp, vp, i, i, i, vp, vp, ctypes.c_double, i, i, i, vp, vp]
+        L.pararnn_layer_backward.argtypes = [vp, vp, ctypes.POINTER(pararnn_params), vp, vp, vp, vp, vp, i,
+                                             vp, vp, vp, vp, vp]
         for name in EXPORTED:
             if getattr(L, name).restype is None and name != "pararnn_strerror":
                 getattr(L, name).restype = i
@@ -216,6 +219,19 @@ def pararnn_adjoint_backward(ctx, xproj, params, h0, h, grad_h, grad_xproj, grad
                                           _p(h, f32), _p(grad_h, f32), _p(grad_xproj, f32),
                                           _p(grad_params, f32), _p(grad_h0, f32)),
            "pararnn_adjoint_backward")
+
+
+def pararnn_layer_backward(ctx, xproj, params, h0, h, grad_h, x, W, grad_x, grad_W, grad_bias,
+                           grad_params, grad_h0=None) -> None:
+    """Adjoint plus projection backward of a layer with bf16 x [B*T, K] and W [3H, K]
+    (grad_x, grad_W, grad_bias may each be None)."""
+    if x.dtype != torch.bfloat16 or W.dtype != torch.bfloat16:
+        raise TypeError("x and W must both be bf16")
+    f32 = torch.float32
+    _check(lib().pararnn_layer_backward(ctx, _p(xproj, f32), ctypes.byref(params), _p(h0, f32), _p(h, f32),
+                                        _p(grad_h, f32), _p(x), _p(W), int(x.shape[-1]), _p(grad_x, f32),
+                                        _p(grad_W, f32), _p(grad_bias, f32), _p(grad_params, f32),
+                                        _p(grad_h0, f32)), "pararnn_layer_backward")
 
 
 def pararnn_get_status(ctx) -> int:

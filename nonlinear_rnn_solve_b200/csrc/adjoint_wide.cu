@@ -14,7 +14,12 @@
 //   - the epilogue forms grad_xproj (each warp stores 128 contiguous bytes per gate and
 //     step) and accumulates the recurrent-parameter gradients in a shared table per CTA,
 //     summed over CTAs in a fixed order after a grid barrier.
+// For the backward pass of a whole layer (input projection included) a variant stores
+// grad_xproj rounded to bf16, the operand type of the projection's tensor-core products,
+// and adds its column sums (the bias gradient, from the fp32 values) with one global
+// atomic per lane, gate and tile.
 #include <cuda.h>
+#include <cuda_bf16.h>
 #include <string.h>
 
 #include "cells.cuh"
@@ -28,6 +33,8 @@ struct AdjWArgs {
     int B, T, H;
     const float *xproj, *a, *peep, *h0, *h, *g;
     float *gx, *gp, *gh0;
+    unsigned short *gxb;  // bf16 grad_xproj (the BF variant)
+    float *gbias;         // bias gradient [3][H] (the BF variant; may be null)
     float *gws;  // per-CTA parameter-gradient partials [grid][NPAR][H]
     Ctl *ctl;
     int *sticky;
@@ -51,7 +58,7 @@ template <class Cell, int LL> struct AdjWCfg {
     static_assert(TCH + 1 <= 256, "TMA box height");
 };
 
-template <class Cell, int L>
+template <class Cell, int L, bool BF>
 __global__ void __launch_bounds__(kThreads, 2)
     adjoint_wide_kernel(const AdjWArgs A, const __grid_constant__ AdjWMaps M) {
     using G = AdjWCfg<Cell, L>;
@@ -268,8 +275,9 @@ __global__ void __launch_bounds__(kThreads, 2)
         float gpv[NP];
 #pragma unroll
         for (int k = 0; k < NP; ++k) gpv[k] = 0.f;
-        float *o = A.gx + ((size_t)b * A.T + t_lo + rbase + L - 1) * 3 * A.H + h;  // scan step 0
+        const size_t obase = ((size_t)b * A.T + t_lo + rbase + L - 1) * 3 * A.H + h;  // scan step 0
         const size_t ostep = (size_t)3 * A.H;
+        float gbv[3] = {0.f, 0.f, 0.f};  // bias-gradient terms (BF)
 #pragma unroll
         for (int i = 0; i < L; ++i) {
             const int t = t_lo + rbase + (L - 1 - i);
@@ -303,10 +311,19 @@ __global__ void __launch_bounds__(kThreads, 2)
                 mu[r] = acc;
             }
             if (t < A.T) {
-                float *oi = o - i * ostep;
-                oi[0] = gxv[0];
-                oi[A.H] = gxv[1];
-                oi[2 * A.H] = gxv[2];
+                if (BF) {
+                    unsigned short *oi = A.gxb + (obase - i * ostep);
+#pragma unroll
+                    for (int qg = 0; qg < 3; ++qg) {
+                        oi[qg * A.H] = __bfloat16_as_ushort(__float2bfloat16_rn(gxv[qg]));
+                        gbv[qg] += gxv[qg];
+                    }
+                } else {
+                    float *oi = A.gx + (obase - i * ostep);
+                    oi[0] = gxv[0];
+                    oi[A.H] = gxv[1];
+                    oi[2 * A.H] = gxv[2];
+                }
                 if (t == 0 && A.gh0) {
 #pragma unroll
                     for (int k = 0; k < S; ++k) A.gh0[((size_t)b * A.H + h) * S + k] = mu[k];
@@ -315,6 +332,10 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
 #pragma unroll
         for (int k = 0; k < NP; ++k) atomicAdd(gp_tab + k * A.H + h, gpv[k]);
+        if (BF && A.gbias) {
+#pragma unroll
+            for (int qg = 0; qg < 3; ++qg) atomicAdd(A.gbias + qg * A.H + h, gbv[qg]);
+        }
         // this warp is done with the stage; the last warp to finish refills it with the
         // tile NST places ahead (acquire-release add on the counter)
         const bool more = j + NST < ntile_cta;
@@ -370,11 +391,11 @@ EncodeTiledFn encode_fn() {
 
 constexpr int kTabMax = 12288;  // shared-memory gradient table limit (floats)
 
-template <class Cell, int L> int choose(Plan *plan, int num_sms, long B, long T, long H) {
+template <class Cell, int L, bool BF> int choose(Plan *plan, int num_sms, long B, long T, long H) {
     using G = AdjWCfg<Cell, L>;
     const int np = Cell::NPAR;
     const int smem = (G::NST * G::STAGE + np * (int)H) * (int)sizeof(float) + 1024;
-    const void *f = reinterpret_cast<const void *>(&adjoint_wide_kernel<Cell, L>);
+    const void *f = reinterpret_cast<const void *>(&adjoint_wide_kernel<Cell, L, BF>);
     if (cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess ||
         cudaFuncSetAttribute(f, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess)
         return -1;
@@ -396,8 +417,11 @@ int adjoint_wide_plan(const AdjointReq &r, int num_sms, Plan *plan) {
     const int np = S == 1 ? GruCell::NPAR : LstmCell::NPAR;
     if (r.H % 32 || (long)np * r.H > kTabMax || !encode_fn()) return 1;
     if ((long)r.B * r.T >= (1L << 31)) return 1;
-    const int rc = S == 1 ? choose<GruCell, 8>(plan, num_sms, r.B, r.T, r.H)
-                          : choose<LstmCell, 5>(plan, num_sms, r.B, r.T, r.H);
+    const bool bf = r.out_bf16;
+    const int rc = S == 1 ? (bf ? choose<GruCell, 8, true>(plan, num_sms, r.B, r.T, r.H)
+                                : choose<GruCell, 8, false>(plan, num_sms, r.B, r.T, r.H))
+                          : (bf ? choose<LstmCell, 5, true>(plan, num_sms, r.B, r.T, r.H)
+                                : choose<LstmCell, 5, false>(plan, num_sms, r.B, r.T, r.H));
     if (rc) return -1;
     if (plan->ntiles > 0x7fffffffL) return 1;
     plan->variant = 300 + S;
@@ -449,6 +473,8 @@ cudaError_t adjoint_wide_launch(const AdjointReq &r, const Plan &plan, const Wor
     A.h = r.h;
     A.g = r.g;
     A.gx = r.grad_xproj;
+    A.gxb = r.grad_xproj_bf16;
+    A.gbias = r.grad_bias;
     A.gp = r.grad_params;
     A.gh0 = r.grad_h0;
     A.gws = w.side;

@@ -279,6 +279,62 @@ int pararnn_adjoint_backward(pararnn_ctx *ctx, const float *xproj, const pararnn
     return rc;
 }
 
+int pararnn_layer_backward(pararnn_ctx *ctx, const float *xproj, const pararnn_params *p, const float *h0,
+                           const float *h, const float *grad_h, const void *x, const void *W, int K, float *grad_x,
+                           float *grad_W, float *grad_bias, float *grad_params, float *grad_h0) {
+    if (!ctx || !p || !xproj || !h || !grad_h || !x || !W || !grad_params || K < 1) return PARARNN_EINVAL;
+    if (p->B < 1 || p->T < 1 || p->H < 1) return PARARNN_EINVAL;
+    if (p->cell != PARARNN_GRU_DIAG && p->cell != PARARNN_LSTM_CIFG_PEEP && p->cell != PARARNN_LSTM_CIFG_PEEP_QUASI)
+        return PARARNN_EUNSUPPORTED;
+    const int lstm = p->cell != PARARNN_GRU_DIAG;
+    if (!p->a || (lstm && !p->peep)) return PARARNN_EINVAL;
+    if ((long long)p->B * p->T > 0x7fffffffLL || 3LL * p->H > 0x7fffffffLL) return PARARNN_EINVAL;
+    const int M = p->B * p->T, N = 3 * p->H;
+    if (int chk = prn::proj_bwd_check(PARARNN_BF16, M, K, N)) return chk;
+    if (misaligned(xproj) || misaligned(h) || misaligned(grad_h) || misaligned(h0) || misaligned(grad_h0) ||
+        misaligned(x) || misaligned(W) || misaligned(grad_x) || misaligned(grad_W) || misaligned(grad_bias))
+        return PARARNN_EALIGN;
+    DeviceGuard g(ctx->device);
+    if (!g.ok) return PARARNN_ECUDA;
+    ctx->last_launches = 0;
+    prn::AdjointReq r{lstm, p->B, p->T, p->H, xproj, p->a, p->peep, h0, h, grad_h, nullptr, grad_params, grad_h0};
+    prn::Plan plan;
+    // the adjoint writes bf16 grad_xproj straight into the projection's scratch when its
+    // TMA-fed tiles cover the shape; otherwise fp32 grad_xproj goes through the scratch
+    r.out_bf16 = true;
+    const int wide = prn::adjoint_wide_plan(r, ctx->num_sms, &plan);
+    if (wide < 0) return PARARNN_ECUDA;
+    const size_t pbytes = prn::proj_bwd_scratch_bytes(PARARNN_BF16, M, K, N);
+    int rc = ensure_scratch(ctx, pbytes + (wide ? (size_t)M * N * sizeof(float) : 0));
+    if (rc) return rc;
+    if (wide == 0) {
+        r.grad_xproj_bf16 = prn::proj_bwd_gb(ctx->scratch, M, N);
+        r.grad_bias = grad_bias;
+    } else {
+        r.out_bf16 = false;
+        r.grad_xproj = reinterpret_cast<float *>(static_cast<char *>(ctx->scratch) + pbytes);
+        if (prn::adjoint_plan(r, ctx->num_sms, &plan)) return PARARNN_ECUDA;
+    }
+    prn::Work w;
+    if ((rc = prepare(ctx, plan, &w))) return rc;
+    const size_t np = (size_t)(lstm ? 5 : 3) * p->H;
+    if (cudaMemsetAsync(grad_params, 0, np * sizeof(float), ctx->stream) != cudaSuccess) return PARARNN_ECUDA;
+    int launches = 1;
+    if (wide == 0 && grad_bias) {
+        if (cudaMemsetAsync(grad_bias, 0, (size_t)N * sizeof(float), ctx->stream) != cudaSuccess) return PARARNN_ECUDA;
+    }
+    if ((rc = cuda_rc(prn::adjoint_launch(r, plan, w, ctx->dbg, ctx->stream)))) return rc;
+    int l = 0;
+    if (wide == 0)
+        rc = cuda_rc(prn::proj_bwd_from_bf16_launch(x, W, grad_x, grad_W, M, K, N, ctx->scratch, ctx->num_sms,
+                                                    ctx->stream, &l, ctx->sticky));
+    else
+        rc = cuda_rc(prn::proj_bwd_launch(PARARNN_BF16, r.grad_xproj, x, W, grad_x, grad_W, grad_bias, M, K, N,
+                                          ctx->scratch, ctx->num_sms, ctx->stream, &l, ctx->sticky));
+    if (rc == PARARNN_OK) ctx->last_launches = launches + l;
+    return rc;
+}
+
 int pararnn_input_proj(pararnn_ctx *ctx, const void *x, int x_dtype, const void *W, const float *bias,
                        float *xproj, int M, int K, int N) {
     if (!ctx || !x || !W || !xproj || M < 1 || K < 1 || N < 1) return PARARNN_EINVAL;

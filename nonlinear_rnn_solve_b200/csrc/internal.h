@@ -118,6 +118,12 @@ struct AdjointReq {
     int B, T, H;
     const float *xproj, *a, *peep, *h0, *h, *g;
     float *grad_xproj, *grad_params, *grad_h0;
+    // layer backward: grad_xproj rounded to bf16 (nearest even) instead of fp32, and its
+    // column sums (fp32 values) added into grad_bias [3 H] (zeroed by the caller); the
+    // TMA-fed tiles only (H % 32 == 0)
+    bool out_bf16 = false;
+    unsigned short *grad_xproj_bf16 = nullptr;
+    float *grad_bias = nullptr;
 };
 int adjoint_plan(const AdjointReq &r, int num_sms, Plan *plan);
 // TMA-fed tiles for H % 32 == 0 (adjoint_wide.cu); 1: shape not covered
@@ -131,10 +137,21 @@ cudaError_t adjoint_launch(const AdjointReq &r, const Plan &plan, const Work &w,
 int proj_check(int x_dtype, int M, int K, int N);
 cudaError_t proj_launch(int x_dtype, const void *x, const void *W, const float *bias, float *y, int M,
                         int K, int N, int num_sms, cudaStream_t st, int *launches, int *sticky);
+// The same, allowed to split K into up to kMaxKsplit parts summed through `ws` (ws_floats
+// floats) when the output has too few tiles for the SMs.
+constexpr int kMaxKsplit = 4;
+cudaError_t proj_launch_split(int x_dtype, const void *x, const void *W, const float *bias, float *y, int M, int K,
+                              int N, int num_sms, cudaStream_t st, int *launches, int *sticky, float *ws,
+                              size_t ws_floats);
 
 // ---- input projection backward ------------------------------------------------------
 int proj_bwd_check(int x_dtype, int M, int K, int N);
 size_t proj_bwd_scratch_bytes(int x_dtype, int M, int K, int N);
+// The bf16 path from a bf16 grad_xproj that the caller wrote at proj_bwd_gb(scratch, M, N)
+// (no fp32 copy, no bias sums): grad_x and grad_W only.
+unsigned short *proj_bwd_gb(void *scratch, int M, int N);
+cudaError_t proj_bwd_from_bf16_launch(const void *x, const void *W, float *grad_x, float *grad_W, int M, int K, int N,
+                                      void *scratch, int num_sms, cudaStream_t st, int *launches, int *sticky);
 cudaError_t proj_bwd_launch(int x_dtype, const float *gx, const void *x, const void *W, float *grad_x, float *grad_W,
                             float *grad_bias, int M, int K, int N, void *scratch, int num_sms, cudaStream_t st,
                             int *launches, int *sticky);

@@ -102,7 +102,8 @@ constexpr unsigned IDESC = (1u << 4) | (1u << 7) | (1u << 10) | ((unsigned)(BN >
 // MMA thread accumulates tile i + 1, and the TMA producer runs ahead across tiles.
 __global__ void __launch_bounds__(THREADS, 1)
     proj_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                     const float *__restrict__ bias, float *__restrict__ y, int M, int N, int K, int *sticky) {
+                     const float *__restrict__ bias, float *__restrict__ y, int M, int N, int K, int ksplit,
+                     int *sticky) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     // 1024-byte alignment for the swizzled tiles
     unsigned char *smem = reinterpret_cast<unsigned char *>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -113,6 +114,10 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int kblocks = (K + BK - 1) / BK;
     const int mtiles = (M + BM - 1) / BM, ntiles_n = (N + BN - 1) / BN;
     const int ntiles = mtiles * ntiles_n;
+    // work item = tile * ksplit + part: part p accumulates K blocks [p kblocks / ksplit,
+    // (p + 1) kblocks / ksplit) into its own M x N slab of y (summed afterwards in a
+    // fixed order); ksplit = 1 is the plain product
+    const int nitems = ntiles * ksplit;
     // 32-byte vector stores need 32-byte aligned rows
     const bool vec8 = (N & 7) == 0 && ((uintptr_t)y & 31) == 0;
 
@@ -142,9 +147,11 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (warp == 0) {
         if (lane == 0) {  // TMA producer, continuous over this CTA's tiles
             int it = 0;
-            for (int tile = blockIdx.x; tile < ntiles && !abort_flag; tile += gridDim.x) {
+            for (int item = blockIdx.x; item < nitems && !abort_flag; item += gridDim.x) {
+                const int tile = item / ksplit, part = item % ksplit;
                 const int m0 = (tile / ntiles_n) * BM, n0 = (tile % ntiles_n) * BN;
-                for (int kb = 0; kb < kblocks; ++kb, ++it) {
+                const int kb0 = part * kblocks / ksplit, kb1 = (part + 1) * kblocks / ksplit;
+                for (int kb = kb0; kb < kb1; ++kb, ++it) {
                     const int s = it % STAGES;
                     const unsigned ph = (unsigned)(it / STAGES) & 1u;
                     if (!mbar_wait(smem_u32(&bar_empty[s]), ph ^ 1u, &abort_flag)) { abort_flag = 1; break; }
@@ -159,7 +166,9 @@ __global__ void __launch_bounds__(THREADS, 1)
     } else if (warp == 1) {
         if (lane == 0) {  // MMA issuer
             int it = 0, ti = 0;
-            for (int tile = blockIdx.x; tile < ntiles && !abort_flag; tile += gridDim.x, ++ti) {
+            for (int item = blockIdx.x; item < nitems && !abort_flag; item += gridDim.x, ++ti) {
+                const int part = item % ksplit;
+                const int kb0 = part * kblocks / ksplit, kb1 = (part + 1) * kblocks / ksplit;
                 const int a = ti & 1;
                 const unsigned acc = tmem + (unsigned)(a * TMEM_COLS);
                 // the epilogue has drained this accumulator (its previous tile)
@@ -168,7 +177,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                     break;
                 }
                 asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-                for (int kb = 0; kb < kblocks; ++kb, ++it) {
+                for (int kb = kb0; kb < kb1; ++kb, ++it) {
                     const int s = it % STAGES;
                     const unsigned ph = (unsigned)(it / STAGES) & 1u;
                     if (!mbar_wait(smem_u32(&bar_full[s]), ph, &abort_flag)) { abort_flag = 1; break; }
@@ -177,7 +186,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
                     for (int k = 0; k < BK / 16; ++k) {
                         const unsigned long long ad = smem_desc(a0 + k * 32), bd = smem_desc(b0 + k * 32);
-                        const unsigned accum = (kb > 0 || k > 0) ? 1u : 0u;
+                        const unsigned accum = (kb > kb0 || k > 0) ? 1u : 0u;
                         asm volatile(
                             "{\n\t.reg .pred p;\n\t"
                             "setp.ne.b32 p, %4, 0;\n\t"
@@ -199,7 +208,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         // 128-column half of the tile
         const int q = warp & 3, hcol = (warp - 2) >> 2;
         int ti = 0;
-        for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++ti) {
+        for (int item = blockIdx.x; item < nitems; item += gridDim.x, ++ti) {
+            const int tile = item / ksplit, part = item % ksplit;
             const int a = ti & 1;
             const int m0 = (tile / ntiles_n) * BM, n0 = (tile % ntiles_n) * BN + 128 * hcol;
             const int row = m0 + q * 32 + lane;
@@ -217,7 +227,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             __syncwarp();
             if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&acc_empty[a])) : "memory");
             if (row < M) {
-                float *yr = y + (size_t)row * N;
+                float *yr = y + (size_t)part * M * N + (size_t)row * N;
 #pragma unroll
                 for (int c = 0; c < 128; c += 8) {
                     const int col = n0 + c;
@@ -350,8 +360,46 @@ int proj_check(int x_dtype, int M, int K, int N) {
     return PARARNN_OK;
 }
 
-cudaError_t proj_launch(int x_dtype, const void *x, const void *W, const float *bias, float *y, int M, int K, int N,
-                        int, cudaStream_t st, int *launches, int *sticky) {
+namespace {
+
+// y[i] = sum_p parts[p][i] (+ bias[i % N]), the parts added in order p = 0, 1, ...
+__global__ void split_sum_kernel(const float *__restrict__ parts, int ksplit, size_t n, const float *__restrict__ bias,
+                                 int N, float *__restrict__ y) {
+    for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
+        float acc = parts[i];
+        for (int p = 1; p < ksplit; ++p) acc += parts[(size_t)p * n + i];
+        if (bias) acc += bias[i % N];
+        y[i] = acc;
+    }
+}
+
+// K blocks split into ksplit parts when the output has fewer tiles than there are SMs and
+// that shortens the product: the work items fill ceil(tiles * s / SMs) waves of kblocks / s
+// blocks each (about 0.3 us per block on the layer shapes), and the parts cost (s + 1) M N
+// 4 bytes of HBM traffic to sum.  (With a wave or more of tiles the extra epilogue and
+// summing traffic outweighed the better balance on the 6144 x 2048 weight gradient.)
+int choose_ksplit(int M, int N, int K, int sms, size_t ws_floats) {
+    const long tiles = (long)((M + gemm::BM - 1) / gemm::BM) * ((N + gemm::BN - 1) / gemm::BN);
+    const int kblocks = (K + gemm::BK - 1) / gemm::BK;
+    if (tiles >= sms) return 1;
+    int best = 1;
+    double best_us = 1e300;
+    for (int s = 1; s <= kMaxKsplit; ++s) {
+        if (s > 1 && (kblocks / s < 8 || (size_t)s * M * N > ws_floats)) break;
+        const long waves = (tiles * s + sms - 1) / sms;
+        const double us = waves * ((kblocks + s - 1) / s) * 0.3 + (s > 1 ? (s + 1) * 4.0 * M * N / 6.5e6 : 0.0);
+        if (us < best_us) {
+            best_us = us;
+            best = s;
+        }
+    }
+    return best;
+}
+
+}  // namespace
+
+cudaError_t proj_launch_split(int x_dtype, const void *x, const void *W, const float *bias, float *y, int M, int K,
+                              int N, int, cudaStream_t st, int *launches, int *sticky, float *ws, size_t ws_floats) {
     *launches = 0;
     if (x_dtype == PARARNN_F32) {
         dim3 grid((M + 63) / 64, (N + 63) / 64);
@@ -368,11 +416,25 @@ cudaError_t proj_launch(int x_dtype, const void *x, const void *W, const float *
     int dev = 0, sms = 0;
     if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
     if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    const int ksplit = ws ? choose_ksplit(M, N, K, sms, ws_floats) : 1;
     const long tiles = (long)((M + gemm::BM - 1) / gemm::BM) * ((N + gemm::BN - 1) / gemm::BN);
-    const int grid = (int)std::min<long>(tiles, sms);  // persistent: one CTA per SM
-    gemm::proj_bf16_kernel<<<grid, gemm::THREADS, smem, st>>>(ta, tb, bias, y, M, N, K, sticky);
-    *launches = 1;
+    const int grid = (int)std::min<long>(tiles * ksplit, sms);  // persistent: one CTA per SM
+    if (ksplit == 1) {
+        gemm::proj_bf16_kernel<<<grid, gemm::THREADS, smem, st>>>(ta, tb, bias, y, M, N, K, 1, sticky);
+        *launches = 1;
+        return cudaGetLastError();
+    }
+    gemm::proj_bf16_kernel<<<grid, gemm::THREADS, smem, st>>>(ta, tb, nullptr, ws, M, N, K, ksplit, sticky);
+    const size_t n = (size_t)M * N;
+    split_sum_kernel<<<(int)std::min<size_t>((n + 255) / 256, (size_t)sms * 16), 256, 0, st>>>(ws, ksplit, n, bias, N,
+                                                                                              y);
+    *launches = 2;
     return cudaGetLastError();
+}
+
+cudaError_t proj_launch(int x_dtype, const void *x, const void *W, const float *bias, float *y, int M, int K, int N,
+                        int num_sms, cudaStream_t st, int *launches, int *sticky) {
+    return proj_launch_split(x_dtype, x, W, bias, y, M, K, N, num_sms, st, launches, sticky, nullptr, 0);
 }
 
 }  // namespace prn

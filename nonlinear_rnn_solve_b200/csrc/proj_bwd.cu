@@ -103,7 +103,7 @@ __global__ void colsum_reduce_kernel(const float *__restrict__ part, float *__re
 __global__ void __launch_bounds__(256) transpose_u16_kernel(const unsigned short *__restrict__ a,
                                                             unsigned short *__restrict__ at, int R, int C) {
     __shared__ unsigned short tile[TT][TT + 2];
-    const int r0 = blockIdx.y * TT, c0 = blockIdx.x * TT;
+    const int r0 = blockIdx.x * TT, c0 = blockIdx.y * TT;  // row tiles on x: no 65535 limit
     for (int e = threadIdx.x; e < TT * TT; e += 256) {
         const int r = e / TT, c = e % TT;
         tile[r][c] = (r0 + r < R && c0 + c < C) ? a[(size_t)(r0 + r) * C + c0 + c] : (unsigned short)0;
@@ -113,6 +113,42 @@ __global__ void __launch_bounds__(256) transpose_u16_kernel(const unsigned short
         const int c = e / TT, r = e % TT;
         if (c0 + c < C && r0 + r < R) at[(size_t)(c0 + c) * R + r0 + r] = tile[r][c];
     }
+}
+
+// The same for R and C multiples of 4 (every bf16 operand here): 8-byte loads and stores,
+// a warp moving two 128-byte row pieces per access.  Lane l of a store takes column
+// c = 2 w + l / 16 (w the warp's pair) and rows 4 (l % 16) .. + 3 of the tile, read
+// from shared memory with a row pitch of 33 words (two-way conflicts at most).
+__global__ void __launch_bounds__(256) transpose_u16x4_kernel(const unsigned short *__restrict__ a,
+                                                              unsigned short *__restrict__ at, int R, int C) {
+    __shared__ unsigned short tile[TT][TT + 2];
+    const int r0 = blockIdx.x * TT, c0 = blockIdx.y * TT;  // row tiles on x: no 65535 limit
+    for (int e = threadIdx.x; e < TT * TT / 4; e += 256) {
+        const int r = e / (TT / 4), c = 4 * (e % (TT / 4));
+        uint2 v = make_uint2(0u, 0u);
+        if (r0 + r < R && c0 + c < C) v = *reinterpret_cast<const uint2 *>(a + (size_t)(r0 + r) * C + c0 + c);
+        unsigned *d = reinterpret_cast<unsigned *>(&tile[r][c]);  // 4-byte aligned: even pitch, c % 4 == 0
+        d[0] = v.x;
+        d[1] = v.y;
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < TT * TT / 4; e += 256) {
+        const int c = e / (TT / 4), r = 4 * (e % (TT / 4));
+        if (c0 + c < C && r0 + r < R) {
+            const unsigned lo = tile[r][c] | ((unsigned)tile[r + 1][c] << 16);
+            const unsigned hi = tile[r + 2][c] | ((unsigned)tile[r + 3][c] << 16);
+            *reinterpret_cast<uint2 *>(at + (size_t)(c0 + c) * R + r0 + r) = make_uint2(lo, hi);
+        }
+    }
+}
+
+// at = a^T with the vector kernel when the rows allow it
+void transpose_u16(const unsigned short *a, unsigned short *at, int R, int C, cudaStream_t st) {
+    const dim3 grid((R + TT - 1) / TT, (C + TT - 1) / TT);
+    if (R % 4 == 0 && C % 4 == 0 && ((uintptr_t)a & 7) == 0 && ((uintptr_t)at & 7) == 0)
+        transpose_u16x4_kernel<<<grid, 256, 0, st>>>(a, at, R, C);
+    else
+        transpose_u16_kernel<<<grid, 256, 0, st>>>(a, at, R, C);
 }
 
 // fp32 C [M, N] = sum_k A(m, k) B(n, k) with A(m, k) = A[m sam + k sak] and
@@ -167,12 +203,52 @@ int row_blocks(int M) {
     return std::max(1, std::min(tiles, 64));
 }
 
+// grad_x = gb W and grad_W = gbt x on the tensor cores, from the bf16 copies gb [M, N]
+// and gbt [N, M] already in the scratch (layout: column-sum parts, gb, gbt, x^T, W^T,
+// K-split parts of grad_W).
+cudaError_t bf16_products(const void *x, const void *W, float *grad_x, float *grad_W, int M, int K, int N,
+                          void *scratch, int num_sms, cudaStream_t st, int *launches, int *sticky) {
+    *launches = 0;
+    char *ws = static_cast<char *>(scratch) + up256((size_t)row_blocks(M) * N * sizeof(float));
+    const unsigned short *gb = reinterpret_cast<const unsigned short *>(ws);
+    ws += up256((size_t)M * N * 2);
+    const unsigned short *gbt = reinterpret_cast<const unsigned short *>(ws);
+    ws += up256((size_t)M * N * 2);
+    unsigned short *xT = reinterpret_cast<unsigned short *>(ws);
+    ws += up256((size_t)M * K * 2);
+    unsigned short *WT = reinterpret_cast<unsigned short *>(ws);
+    ws += up256((size_t)N * K * 2);
+    float *kws = reinterpret_cast<float *>(ws);  // K-split parts of grad_W
+    cudaError_t e;
+    int l = 0;
+    if (grad_x) {
+        transpose_u16(static_cast<const unsigned short *>(W), WT, N, K, st);
+        ++*launches;
+        if ((e = proj_launch(PARARNN_BF16, gb, WT, nullptr, grad_x, M, N, K, num_sms, st, &l, sticky)) != cudaSuccess)
+            return e;
+        *launches += l;
+    }
+    if (grad_W) {
+        transpose_u16(static_cast<const unsigned short *>(x), xT, M, K, st);
+        ++*launches;
+        // an N x K output over a long contraction (M): few tiles, so the K blocks may be
+        // split across more CTAs and the parts summed in order
+        if ((e = proj_launch_split(PARARNN_BF16, gbt, xT, nullptr, grad_W, N, M, K, num_sms, st, &l, sticky, kws,
+                                   (size_t)kMaxKsplit * N * K)) != cudaSuccess)
+            return e;
+        *launches += l;
+    }
+    return cudaGetLastError();
+}
+
 }  // namespace
 
 size_t proj_bwd_scratch_bytes(int x_dtype, int M, int K, int N) {
     const size_t part = up256((size_t)row_blocks(M) * N * sizeof(float));
     if (x_dtype != PARARNN_BF16) return part;
-    return part + 2 * up256((size_t)M * N * 2) + up256((size_t)M * K * 2) + up256((size_t)N * K * 2);
+    // + the parts of a K-split grad_W product (N x K each)
+    return part + 2 * up256((size_t)M * N * 2) + up256((size_t)M * K * 2) + up256((size_t)N * K * 2) +
+           up256((size_t)kMaxKsplit * N * K * sizeof(float));
 }
 
 int proj_bwd_check(int x_dtype, int M, int K, int N) {
@@ -214,13 +290,7 @@ cudaError_t proj_bwd_launch(int x_dtype, const float *gx, const void *x, const v
         return cudaGetLastError();
     }
     unsigned short *gb = reinterpret_cast<unsigned short *>(ws);
-    ws += up256((size_t)M * N * 2);
-    unsigned short *gbt = reinterpret_cast<unsigned short *>(ws);
-    ws += up256((size_t)M * N * 2);
-    unsigned short *xT = reinterpret_cast<unsigned short *>(ws);
-    ws += up256((size_t)M * K * 2);
-    unsigned short *WT = reinterpret_cast<unsigned short *>(ws);
-    gx_prep_kernel<true><<<prep_grid, 256, 0, st>>>(gx, gb, gbt, part, M, N, rpb);
+    gx_prep_kernel<true><<<prep_grid, 256, 0, st>>>(gx, gb, gb + up256((size_t)M * N * 2) / 2, part, M, N, rpb);
     ++*launches;
     if (grad_bias) {
         colsum_reduce_kernel<<<(N + 255) / 256, 256, 0, st>>>(part, grad_bias, R, N);
@@ -228,23 +298,28 @@ cudaError_t proj_bwd_launch(int x_dtype, const float *gx, const void *x, const v
     }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     int l = 0;
-    if (grad_x) {
-        transpose_u16_kernel<<<dim3((K + TT - 1) / TT, (N + TT - 1) / TT), 256, 0, st>>>(
-            static_cast<const unsigned short *>(W), WT, N, K);
-        ++*launches;
-        if ((e = proj_launch(PARARNN_BF16, gb, WT, nullptr, grad_x, M, N, K, num_sms, st, &l, sticky)) != cudaSuccess)
-            return e;
-        *launches += l;
-    }
+    e = bf16_products(x, W, grad_x, grad_W, M, K, N, scratch, num_sms, st, &l, sticky);
+    *launches += l;
+    return e;
+}
+
+unsigned short *proj_bwd_gb(void *scratch, int M, int N) {
+    return reinterpret_cast<unsigned short *>(static_cast<char *>(scratch) +
+                                              up256((size_t)row_blocks(M) * N * sizeof(float)));
+}
+
+cudaError_t proj_bwd_from_bf16_launch(const void *x, const void *W, float *grad_x, float *grad_W, int M, int K, int N,
+                                      void *scratch, int num_sms, cudaStream_t st, int *launches, int *sticky) {
+    *launches = 0;
+    unsigned short *gb = proj_bwd_gb(scratch, M, N), *gbt = gb + up256((size_t)M * N * 2) / 2;
     if (grad_W) {
-        transpose_u16_kernel<<<dim3((K + TT - 1) / TT, (M + TT - 1) / TT), 256, 0, st>>>(
-            static_cast<const unsigned short *>(x), xT, M, K);
+        transpose_u16(gb, gbt, M, N, st);
         ++*launches;
-        if ((e = proj_launch(PARARNN_BF16, gbt, xT, nullptr, grad_W, N, M, K, num_sms, st, &l, sticky)) != cudaSuccess)
-            return e;
-        *launches += l;
     }
-    return cudaGetLastError();
+    int l = 0;
+    const cudaError_t e = bf16_products(x, W, grad_x, grad_W, M, K, N, scratch, num_sms, st, &l, sticky);
+    *launches += l;
+    return e;
 }
 
 }  // namespace prn

@@ -188,3 +188,30 @@ def adjoint_backward(ctx, cell, B, T, H, *, xproj, a, peep=None, h0=None, h, gra
     gh0 = torch.empty((B, H, 2) if lstm else (B, H), device=dev, dtype=torch.float32)
     pararnn_adjoint_backward(ctx, xproj, prm, h0, h, grad_h, gx, gp, gh0)
     return gx, gp, gh0
+
+
+def layer_backward(ctx, cell, B, T, H, *, xproj, a, peep=None, h0=None, h, grad_h, x, W):
+    """Backward pass of a layer with bf16 x [B, T, K] and W [3H, K]: the adjoint at states h
+    and the projection's reverse pass, grad_xproj handed over in bf16.  Returns
+    (grad_x, grad_W, grad_bias, grad_params, grad_h0)."""
+    from . import pararnn_layer_backward
+    dev = xproj.device
+    S = 2 if cell in ("lstm", "lstm_quasi") else 1
+    K = x.shape[-1]
+    _need(xproj, B * T * 3 * H, "xproj [B, T, 3, H]")
+    _need(a, 3 * H, "a [3, H]")
+    _need(peep, 2 * H, "peep [2, H]")
+    _need(h0, B * H * S, "h0")
+    _need(h, B * T * H * S, "h")
+    _need(grad_h, B * T * H * S, "grad_h")
+    _need(x, B * T * K, "x [B, T, K]")
+    _need(W, 3 * H * K, "W [3H, K]")
+    prm = make_params(CELLS[cell], B, T, H, 0, a=a, peep=peep)
+    lstm = cell in ("lstm", "lstm_quasi")
+    gxi = torch.empty(B, T, K, device=dev, dtype=torch.float32)
+    gW = torch.empty(3 * H, K, device=dev, dtype=torch.float32)
+    gb = torch.empty(3 * H, device=dev, dtype=torch.float32)
+    gp = torch.empty(5 if lstm else 3, H, device=dev, dtype=torch.float32)
+    gh0 = torch.empty((B, H, 2) if lstm else (B, H), device=dev, dtype=torch.float32)
+    pararnn_layer_backward(ctx, xproj, prm, h0, h, grad_h, x, W, gxi, gW, gb, gp, gh0)
+    return gxi, gW, gb, gp, gh0

@@ -10,8 +10,9 @@ max|delta| < tol.  Default workload: the DEER GRU benchmark shape (batch 16,
 
 Besides the headline, the line carries ``per_config``: every other workload of the
 path timed on the device (CUDA events, L2 flushed between repeats, median), leg by
-leg -- the projection GEMM, the Newton forward, the adjoint backward and the
-projection backward of the LLM-width ParaGRU / ParaLSTM layers; the tanh RNN with
+leg -- the projection GEMM, the Newton forward, the adjoint backward, the
+projection backward and the two backward passes in one call (grad_xproj handed over
+in bf16) of the LLM-width ParaGRU / ParaLSTM layers; the tanh RNN with
 full DEER and quasi-DEER at n = 8 and 64 -- each with its algorithmic bytes or flops
 and its fraction of the bound it sits on, next to the fp64 oracle's sequential
 rollout (the "naive sequential application") on all host cores and on one core.

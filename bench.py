@@ -13,7 +13,8 @@ path timed on the device (CUDA events, L2 flushed between repeats, median), leg 
 leg -- the projection GEMM, the Newton forward, the adjoint backward, the
 projection backward and the two backward passes in one call (grad_xproj handed over
 in bf16) of the LLM-width ParaGRU / ParaLSTM layers; the tanh RNN with
-full DEER and quasi-DEER at n = 8 and 64 -- each with its algorithmic bytes or flops
+full DEER and quasi-DEER at n = 8 and 64, and the standalone dense linear scan at the
+n = 64 shape -- each with its algorithmic bytes or flops
 and its fraction of the bound it sits on, next to the fp64 oracle's sequential
 rollout (the "naive sequential application") on all host cores and on one core.
 
@@ -391,6 +392,28 @@ def measure_workload(L, w, inp, parts=None):
             st = _ctx_status(ctx)
             return {"forward": {"diverges_from_zero_guess": True, "iters": int(sc["iters"].item()),
                                 "device_status": st}}
+        if w.cell == wl.TANH and not w.quasi and w.H > 32 and (parts is None or "scan" in parts):
+            # the standalone dense linear scan (pararnn_linear_scan, dense kind) at the
+            # workload's shape: out_t = J_t out_{t-1} + b_t, J_t [n, n] of N(0, 0.81 / n)
+            # entries and b_t of N(0, 1) drawn on the device (seeded)
+            from nonlinear_rnn_solve_b200 import PARARNN_SCAN_DENSE, pararnn_linear_scan
+            n = w.H
+            gen = torch.Generator(device=dev)
+            gen.manual_seed(7)
+            J = torch.randn(w.B, w.T, n, n, device=dev, generator=gen).mul_(0.9 / n ** 0.5)
+            bb = torch.randn(w.B, w.T, n, device=dev, generator=gen)
+            out_s = torch.empty_like(bb)
+            ms = L.time(lambda: pararnn_linear_scan(ctx.ctx, PARARNN_SCAN_DENSE, J, bb, None, out_s, w.B, w.T, n))
+            steps = w.B * w.T
+            # chain map 2 n^3 + its offset 2 n^2 per step, re-walk 2 n^2; J and b read twice
+            fl = steps * (2 * n ** 3 + 4 * n * n)
+            nb = steps * (2 * (n * n + n) + n) * 4
+            out["scan"] = {"ms": ms, "shape": f"J [B{w.B}, T{w.T}, {n}, {n}], forward",
+                           "device_status": _ctx_status(ctx), "roofline": _alu_entry(ms, fl, _fp32_peak_tflops()),
+                           "roofline_other": _hbm_entry(ms, nb, hbm)}
+            del J, bb, out_s
+            if parts is not None and "forward" not in parts:
+                return out
         fn = lambda: solve.newton_forward(ctx.ctx, cell, w.B, w.T, w.H, h0=t["h0"],  # noqa: E731
                                           max_iters=w.max_iters, tol=w.tol, h_out=h_out, scalars=sc, **kw)
         ms = L.time(fn)
@@ -753,7 +776,7 @@ def main():
                     help="skip the e2e, CPU-baseline and per-config legs (for profiler runs)")
     ap.add_argument("--leg", default=None,
                     help="WORKLOAD[:PART]: time one leg alone (PART: proj, forward, backward, proj_backward, "
-                         "layer_backward)")
+                         "layer_backward; scan for the n = 64 tanh DEER workload)")
     args = ap.parse_args()
     w = wl.WORKLOADS[args.workload]
     if args.leg:

@@ -683,93 +683,178 @@ struct DScanArgs {
 
 template <int N> struct DScanSmem {
     static constexpr int MS = N + 4;
-    float MT[2][N * MS];  // MT[k][i] = M_t[i][k], double buffered per step
+    // the matrix that defines scan step t, row-major with padded rows: J_t (forward:
+    // M_t = J_t) or J_{t+1} (reverse: M_t = J_{t+1}^T); double buffered per step
+    float Js[2][N * MS];
     float P[2][N * N];
     float D[2][N];
     float carry[N];
     float v[2][N];
 };
 
-// Stage MT for scan step t (time index) of sequence b into buffer mt.
+// Stage the matrix of scan step t (time index) of sequence b into buffer js: with
+// 16-byte cp.async copies when n % 4 == 0 (the padding rows and columns, zeroed once,
+// are never written), else with plain loads that also write the padding; the identity
+// after the last step of a reverse scan.  Copies are committed by the caller.
 template <int N>
-__device__ __forceinline__ void dscan_stage_M(const DScanArgs &A, float *mt, int b, int t) {
+__device__ __forceinline__ void dscan_stage_M(const DScanArgs &A, float *js, int b, int t, bool vec) {
     constexpr int MS = DScanSmem<N>::MS;
-    const size_t row = (size_t)b * A.T;
-    for (int e = threadIdx.x; e < N * N; e += kThreads) {
-        const int i = e / N, k = e % N;
-        float v;
-        if (!A.reverse) {  // M = J_t, stored MT[k][i] = J_t[i][k]
-            v = (i < A.n && k < A.n) ? A.J[((row + t) * A.n + i) * A.n + k] : 0.f;
-            mt[k * MS + i] = v;
-        } else if (t + 1 < A.T) {  // M = J_{t+1}^T, MT[k][i] = J_{t+1}[k][i]; read row-major (k = row)
-            v = (i < A.n && k < A.n) ? A.J[((row + t + 1) * A.n + i) * A.n + k] : 0.f;
-            mt[i * MS + k] = v;
-        } else {
-            mt[i * MS + k] = (i == k && i < A.n) ? 1.f : 0.f;
+    const int tt = A.reverse ? t + 1 : t;
+    if (tt >= A.T) {  // reverse, last step: M = I
+        for (int e = threadIdx.x; e < N * N; e += kThreads) {
+            const int i = e / N, k = e % N;
+            js[i * MS + k] = (i == k && i < A.n) ? 1.f : 0.f;
+        }
+        return;
+    }
+    const float *src = A.J + ((size_t)b * A.T + tt) * A.n * A.n;
+    if (vec) {
+        const int cpr = A.n >> 2;  // 16-byte chunks per row
+        for (int e = threadIdx.x; e < A.n * cpr; e += kThreads) {
+            const int i = e / cpr, c = e - i * cpr;
+            cp_async16(js + i * MS + 4 * c, src + i * A.n + 4 * c, 16);
+        }
+    } else {
+        for (int e = threadIdx.x; e < N * N; e += kThreads) {
+            const int i = e / N, k = e % N;
+            js[i * MS + k] = (i < A.n && k < A.n) ? src[i * A.n + k] : 0.f;
         }
     }
 }
 
-template <int N>
-__global__ void __launch_bounds__(kThreads, 1) dense_scan_kernel(const DScanArgs A) {
+// One step of the chain map, P <- M_t P, for the thread's BR x BR block (rows i0.., columns
+// j0..): forward M_t[i][k] = js[i][k], reverse M_t[i][k] = js[k][i].
+template <int N, bool REV>
+__device__ __forceinline__ void dscan_chain_step(const float *js, const float *P, float *Pn, int i0, int j0) {
+    constexpr int MS = DScanSmem<N>::MS, BR = DeerCfg<N>::BR;
+    float acc[BR][BR];
+#pragma unroll
+    for (int a = 0; a < BR; ++a)
+#pragma unroll
+        for (int c = 0; c < BR; ++c) acc[a][c] = 0.f;
+    if constexpr (BR == 4) {
+        if constexpr (REV) {
+#pragma unroll 8
+            for (int kk = 0; kk < N; ++kk) {
+                const float4 m = *reinterpret_cast<const float4 *>(js + kk * MS + i0);  // M_t[i0 + a][kk]
+                const float4 p = *reinterpret_cast<const float4 *>(P + kk * N + j0);
+                const float mv[4] = {m.x, m.y, m.z, m.w}, pv[4] = {p.x, p.y, p.z, p.w};
+#pragma unroll
+                for (int a = 0; a < 4; ++a)
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) acc[a][c] = fmaf(mv[a], pv[c], acc[a][c]);
+            }
+        } else {
+#pragma unroll 2
+            for (int k4 = 0; k4 < N; k4 += 4) {
+                float mv[4][4], pv[4][4];
+#pragma unroll
+                for (int a = 0; a < 4; ++a) {  // M_t[i0 + a][k4 .. k4 + 3]
+                    const float4 m = *reinterpret_cast<const float4 *>(js + (i0 + a) * MS + k4);
+                    mv[a][0] = m.x;
+                    mv[a][1] = m.y;
+                    mv[a][2] = m.z;
+                    mv[a][3] = m.w;
+                }
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {  // P[k4 + q][j0 .. j0 + 3]
+                    const float4 v = *reinterpret_cast<const float4 *>(P + (k4 + q) * N + j0);
+                    pv[q][0] = v.x;
+                    pv[q][1] = v.y;
+                    pv[q][2] = v.z;
+                    pv[q][3] = v.w;
+                }
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+#pragma unroll
+                    for (int a = 0; a < 4; ++a)
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) acc[a][c] = fmaf(mv[a][q], pv[q][c], acc[a][c]);
+            }
+        }
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+            *reinterpret_cast<float4 *>(Pn + (i0 + a) * N + j0) = make_float4(acc[a][0], acc[a][1], acc[a][2], acc[a][3]);
+    } else {
+#pragma unroll 8
+        for (int kk = 0; kk < N; ++kk) {
+            float av[BR], pv[BR];
+#pragma unroll
+            for (int a = 0; a < BR; ++a) av[a] = REV ? js[kk * MS + i0 + a] : js[(i0 + a) * MS + kk];
+#pragma unroll
+            for (int c = 0; c < BR; ++c) pv[c] = P[kk * N + j0 + c];
+#pragma unroll
+            for (int a = 0; a < BR; ++a)
+#pragma unroll
+                for (int c = 0; c < BR; ++c) acc[a][c] = fmaf(av[a], pv[c], acc[a][c]);
+        }
+#pragma unroll
+        for (int a = 0; a < BR; ++a)
+#pragma unroll
+            for (int c = 0; c < BR; ++c) Pn[(i0 + a) * N + j0 + c] = acc[a][c];
+    }
+}
+
+// Row r of M_t times the vector x (N entries): forward reads row r of js (16-byte
+// loads), reverse column r.
+template <int N, bool REV> __device__ __forceinline__ float dscan_row_dot(const float *js, int r, const float *x) {
+    constexpr int MS = DScanSmem<N>::MS;
+    float acc = 0.f;
+    if constexpr (REV) {
+#pragma unroll 8
+        for (int kk = 0; kk < N; ++kk) acc = fmaf(js[kk * MS + r], x[kk], acc);
+    } else {
+#pragma unroll 4
+        for (int k4 = 0; k4 < N; k4 += 4) {
+            const float4 m = *reinterpret_cast<const float4 *>(js + r * MS + k4);
+            const float4 v = *reinterpret_cast<const float4 *>(x + k4);
+            acc = fmaf(m.x, v.x, acc);
+            acc = fmaf(m.y, v.y, acc);
+            acc = fmaf(m.z, v.z, acc);
+            acc = fmaf(m.w, v.w, acc);
+        }
+    }
+    return acc;
+}
+
+// Two CTAs per SM: each step's matrix is copied into the other buffer while the current
+// one is used (cp.async, waited for before the step's barrier), so the copies' latency
+// overlaps the chain product.
+template <int N, bool REV>
+__device__ __forceinline__ void dense_scan_body(const DScanArgs &A, DScanSmem<N> &sm, int *s_fail, bool vec) {
     constexpr int TCH = DeerCfg<N>::TCH, BR = DeerCfg<N>::BR, TG = DeerCfg<N>::TG, MS = DScanSmem<N>::MS;
-    extern __shared__ __align__(16) unsigned char smraw[];
-    DScanSmem<N> &sm = *reinterpret_cast<DScanSmem<N> *>(smraw);
-    __shared__ int s_fail;
     const int tid = threadIdx.x;
     const int nchunk = (A.T + TCH - 1) / TCH;
     const long nseq = A.B;
     const long ntiles = nseq * nchunk;
     const unsigned epoch = A.epoch0 + 1u;
-    if (tid == 0) s_fail = 0;
     TileWalk tw(nseq);
     for (long tile = blockIdx.x; tile < ntiles; tile += gridDim.x, tw.next()) {
         const int chunk = tw.chunk;  // scan order
         const int b = tw.seq;
-        const int tch = A.reverse ? nchunk - 1 - chunk : chunk;
+        const int tch = REV ? nchunk - 1 - chunk : chunk;
         const int tbeg = tch * TCH;
         const int steps = min(TCH, A.T - tbeg);
-        auto time_of = [&](int i) { return A.reverse ? tbeg + steps - 1 - i : tbeg + i; };
+        auto time_of = [&](int i) { return REV ? tbeg + steps - 1 - i : tbeg + i; };
         for (int e = tid; e < N * N; e += kThreads) sm.P[0][e] = (e / N == e % N) ? 1.f : 0.f;
         if (tid < N) sm.D[0][tid] = 0.f;
-        __syncthreads();
-        dscan_stage_M<N>(A, sm.MT[0], b, time_of(0));
+        dscan_stage_M<N>(A, sm.Js[0], b, time_of(0), vec);
+        cp_async_commit();
+        cp_async_wait_all();
         __syncthreads();
         int cur = 0;
         for (int i = 0; i < steps; ++i) {
             const int t = time_of(i);
-            if (i + 1 < steps) dscan_stage_M<N>(A, sm.MT[(i + 1) & 1], b, time_of(i + 1));
-            const float *mt = sm.MT[i & 1];
-            if (tid < TG * TG) {
-                const int i0 = (tid / TG) * BR, j0 = (tid % TG) * BR;
-                float acc[BR][BR];
-#pragma unroll
-                for (int a = 0; a < BR; ++a)
-#pragma unroll
-                    for (int c = 0; c < BR; ++c) acc[a][c] = 0.f;
-#pragma unroll 8
-                for (int kk = 0; kk < N; ++kk) {
-                    float av[BR], pv[BR];
-#pragma unroll
-                    for (int a = 0; a < BR; ++a) av[a] = mt[kk * MS + i0 + a];
-#pragma unroll
-                    for (int c = 0; c < BR; ++c) pv[c] = sm.P[cur][kk * N + j0 + c];
-#pragma unroll
-                    for (int a = 0; a < BR; ++a)
-#pragma unroll
-                        for (int c = 0; c < BR; ++c) acc[a][c] = fmaf(av[a], pv[c], acc[a][c]);
-                }
-#pragma unroll
-                for (int a = 0; a < BR; ++a)
-#pragma unroll
-                    for (int c = 0; c < BR; ++c) sm.P[cur ^ 1][(i0 + a) * N + j0 + c] = acc[a][c];
-            }
+            if (i + 1 < steps) dscan_stage_M<N>(A, sm.Js[(i + 1) & 1], b, time_of(i + 1), vec);
+            cp_async_commit();
+            const float *js = sm.Js[i & 1];
+            if (tid < TG * TG) dscan_chain_step<N, REV>(js, sm.P[cur], sm.P[cur ^ 1], (tid / TG) * BR, (tid % TG) * BR);
             if (tid >= kThreads - N) {
                 const int r = tid - (kThreads - N);
-                float acc = (r < A.n) ? A.b[((size_t)b * A.T + t) * A.n + r] : 0.f;
-                for (int kk = 0; kk < N; ++kk) acc = fmaf(mt[kk * MS + r], sm.D[cur][kk], acc);
-                sm.D[cur ^ 1][r] = acc;
+                const float acc = dscan_row_dot<N, REV>(js, r, sm.D[cur]);
+                sm.D[cur ^ 1][r] = (r < A.n) ? acc + A.b[((size_t)b * A.T + t) * A.n + r] : acc;
             }
+            cp_async_wait_all();
             __syncthreads();
             cur ^= 1;
         }
@@ -778,30 +863,32 @@ __global__ void __launch_bounds__(kThreads, 1) dense_scan_kernel(const DScanArgs
             if (chunk == 0) {
                 cv = (A.h0 && tid < A.n) ? A.h0[(size_t)b * A.n + tid] : 0.f;
             } else if (!wait_word(A.inc + (tile - nseq) * N + tid, epoch, &cv, A.ctl, A.sticky, A.dbg)) {
-                s_fail = 1;
+                *s_fail = 1;
             }
             sm.carry[tid] = cv;
         }
         __syncthreads();
-        if (s_fail) return;
+        if (*s_fail) return;
         if (tid < N) {
             float acc = sm.D[cur][tid];
             for (int j = 0; j < N; ++j) acc = fmaf(sm.P[cur][tid * N + j], sm.carry[j], acc);
             if (A.dbg.skip_tile != tile) st_relaxed_u64(A.inc + tile * N + tid, pack_tag(acc, epoch));
             sm.v[0][tid] = sm.carry[tid];
         }
-        __syncthreads();
-        dscan_stage_M<N>(A, sm.MT[0], b, time_of(0));
+        dscan_stage_M<N>(A, sm.Js[0], b, time_of(0), vec);
+        cp_async_commit();
+        cp_async_wait_all();
         __syncthreads();
         int vc = 0;
         for (int i = 0; i < steps; ++i) {
             const int t = time_of(i);
-            if (i + 1 < steps) dscan_stage_M<N>(A, sm.MT[(i + 1) & 1], b, time_of(i + 1));
-            const float *mt = sm.MT[i & 1];
+            if (i + 1 < steps) dscan_stage_M<N>(A, sm.Js[(i + 1) & 1], b, time_of(i + 1), vec);
+            cp_async_commit();
+            const float *js = sm.Js[i & 1];
             if (tid < 4 * N) {
                 const int r = tid >> 2, q = tid & 3;
                 float acc = 0.f;
-                for (int kk = q; kk < N; kk += 4) acc = fmaf(mt[kk * MS + r], sm.v[vc][kk], acc);
+                for (int kk = q; kk < N; kk += 4) acc = fmaf(REV ? js[kk * MS + r] : js[r * MS + kk], sm.v[vc][kk], acc);
                 acc += __shfl_xor_sync(0xffffffffu, acc, 1);
                 acc += __shfl_xor_sync(0xffffffffu, acc, 2);
                 if (q == 0) {
@@ -810,10 +897,29 @@ __global__ void __launch_bounds__(kThreads, 1) dense_scan_kernel(const DScanArgs
                     if (r < A.n) A.out[((size_t)b * A.T + t) * A.n + r] = acc;
                 }
             }
+            cp_async_wait_all();
             __syncthreads();
             vc ^= 1;
         }
     }
+}
+
+template <int N>
+__global__ void __launch_bounds__(kThreads, 2) dense_scan_kernel(const DScanArgs A) {
+    extern __shared__ __align__(16) unsigned char smraw[];
+    DScanSmem<N> &sm = *reinterpret_cast<DScanSmem<N> *>(smraw);
+    __shared__ int s_fail;
+    const int tid = threadIdx.x;
+    // 16-byte copies of whole rows: n % 4 == 0 (then every row start is 16-byte aligned)
+    const bool vec = (A.n & 3) == 0 && ((uintptr_t)A.J & 15) == 0;
+    if (tid == 0) s_fail = 0;
+    // the padding of both staging buffers stays zero: the 16-byte copies never write it
+    for (int e = tid; e < 2 * N * DScanSmem<N>::MS; e += kThreads) (&sm.Js[0][0])[e] = 0.f;
+    __syncthreads();
+    if (A.reverse)
+        dense_scan_body<N, true>(A, sm, &s_fail, vec);
+    else
+        dense_scan_body<N, false>(A, sm, &s_fail, vec);
 }
 
 // Small states (n <= 8): one warp per tile, so the sequential walks synchronise with

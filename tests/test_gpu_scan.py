@@ -54,7 +54,9 @@ def test_scan_matches_oracle(ctx, kind, reverse, shape):
     assert max_abs(host(out), ref) <= TOL
 
 
-@pytest.mark.parametrize("N", [1, 5, 8, 13, 32, 64])
+# N = 20, 44: rows of a multiple of 4 floats copied in 16-byte pieces into the 32- and
+# 64-wide padded tiles, whose padding stays zero; N = 13: the element-wise staging
+@pytest.mark.parametrize("N", [1, 5, 8, 13, 20, 32, 44, 64])
 @pytest.mark.parametrize("reverse", [False, True])
 @pytest.mark.parametrize("BT", [(2, 300), (1, 1), (3, 1025)])
 def test_dense_scan_matches_oracle(ctx, N, reverse, BT):

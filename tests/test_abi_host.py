@@ -60,6 +60,8 @@ def test_null_context_and_pointers_are_rejected():
     assert L.pararnn_input_proj(None, None, 0, None, None, None, 1, 1, 1) == EINVAL
     assert L.pararnn_input_proj_backward(None, None, None, 0, None, None, None, None, 1, 1, 1) == EINVAL
     assert L.pararnn_lsim(None, None, None, None, None, 1, 1, 1, None, None, 0.1, 0, 1, 1, None, None) == EINVAL
+    assert L.pararnn_layer_backward(None, None, ctypes.byref(p), None, None, None, None, None, 8, None, None, None,
+                                    None, None) == EINVAL
     st = ctypes.c_int()
     assert L.pararnn_get_status(None, ctypes.byref(st)) == EINVAL
     assert L.pararnn_debug_set(None, 1, 5) == EINVAL
@@ -125,6 +127,12 @@ def test_wrappers_check_operand_sizes_before_the_pointer_only_calls():
         solve.input_proj(None, z(6, 8), z(16, 7))
     with pytest.raises(ValueError):  # grad_xproj [M, N]
         solve.input_proj_backward(None, z(6, 15), z(6, 8), z(16, 8))
+    with pytest.raises(ValueError):  # layer backward: x [B, T, K]
+        solve.layer_backward(None, "gru", 2, 8, 32, xproj=z(2, 8, 3, 32), a=z(3, 32), h=z(2, 8, 32),
+                             grad_h=z(2, 8, 32), x=z(2, 7, 16), W=z(96, 16))
+    with pytest.raises(ValueError):  # layer backward: W [3H, K]
+        solve.layer_backward(None, "lstm", 2, 8, 32, xproj=z(2, 8, 3, 32), a=z(3, 32), peep=z(2, 32),
+                             h=z(2, 8, 32, 2), grad_h=z(2, 8, 32, 2), x=z(2, 8, 16), W=z(64, 16))
     with pytest.raises(ValueError):  # allocation-free scan: block2 J [B, T, N, 2, 2]
         solve.linear_scan_noalloc("block2", z(2, 5, 3, 2), z(2, 5, 3, 2))
     with pytest.raises(ValueError):  # allocation-free scan: h_out like b

@@ -569,6 +569,8 @@ def run_leg(args):
     from nonlinear_rnn_solve_b200 import Context
     name, _, part = args.leg.partition(":")
     w = wl.WORKLOADS[name]
+    if args.leg_batch:
+        w = w.resized(B=args.leg_batch)  # a smaller case of the same shape (ncu captures)
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream(dev)
@@ -777,6 +779,8 @@ def main():
     ap.add_argument("--leg", default=None,
                     help="WORKLOAD[:PART]: time one leg alone (PART: proj, forward, backward, proj_backward, "
                          "layer_backward; scan for the n = 64 tanh DEER workload)")
+    ap.add_argument("--leg-batch", type=int, default=0,
+                    help="with --leg: the workload's batch replaced by this one (a smaller case for profiling)")
     args = ap.parse_args()
     w = wl.WORKLOADS[args.workload]
     if args.leg:

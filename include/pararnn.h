@@ -149,7 +149,9 @@ int pararnn_input_proj(pararnn_ctx *ctx, const void *x, int x_dtype, const void 
  * Shapes: M, K, N >= 1; bf16 needs M, K, N multiples of 8 (16-byte rows of every
  * operand, including the transposed copies); M * N and M * K <= 2^40.  All pointers
  * 16-byte aligned.  The context keeps a scratch buffer of the bf16 copies
- * (4 M N + 2 M K + 2 N K bytes) for later calls.
+ * (4 M N + 2 M K + 2 N K bytes) and of the parts of a weight gradient whose product is
+ * split along M (16 N K bytes; taken when grad_W has fewer 128 x 256 output tiles than
+ * the GPU has SMs, the parts summed in a fixed order) for later calls.
  * Returns EINVAL, EALIGN, ENOMEM or ECUDA. */
 int pararnn_input_proj_backward(pararnn_ctx *ctx, const float *grad_xproj, const void *x, int x_dtype,
                                 const void *W, float *grad_x, float *grad_W, float *grad_bias, int M, int K,

@@ -33,8 +33,9 @@ struct AdjWArgs {
     int B, T, H;
     const float *xproj, *a, *peep, *h0, *h, *g;
     float *gx, *gp, *gh0;
-    unsigned short *gxb;  // bf16 grad_xproj (the BF variant)
-    float *gbias;         // bias gradient [3][H] (the BF variant; may be null)
+    unsigned short *gxb;   // bf16 grad_xproj (the BF variant)
+    unsigned short *gxbt;  // its transpose [3 H][B T] (the BF variant, 8 steps per thread; may be null)
+    float *gbias;          // bias gradient [3][H] (the BF variant; may be null)
     float *gws;  // per-CTA parameter-gradient partials [grid][NPAR][H]
     Ctl *ctl;
     int *sticky;
@@ -278,6 +279,10 @@ __global__ void __launch_bounds__(kThreads, 2)
         const size_t obase = ((size_t)b * A.T + t_lo + rbase + L - 1) * 3 * A.H + h;  // scan step 0
         const size_t ostep = (size_t)3 * A.H;
         float gbv[3] = {0.f, 0.f, 0.f};  // bias-gradient terms (BF)
+        // the transposed copy (BF, 8 steps per thread): gate q's 8 values of this thread's
+        // steps, in time order, packed two per word for one 16-byte store
+        constexpr bool kT8 = BF && L == 8;
+        unsigned pk[3][4] = {{0u, 0u, 0u, 0u}, {0u, 0u, 0u, 0u}, {0u, 0u, 0u, 0u}};
 #pragma unroll
         for (int i = 0; i < L; ++i) {
             const int t = t_lo + rbase + (L - 1 - i);
@@ -315,7 +320,9 @@ __global__ void __launch_bounds__(kThreads, 2)
                     unsigned short *oi = A.gxb + (obase - i * ostep);
 #pragma unroll
                     for (int qg = 0; qg < 3; ++qg) {
-                        oi[qg * A.H] = __bfloat16_as_ushort(__float2bfloat16_rn(gxv[qg]));
+                        const unsigned short bits = __bfloat16_as_ushort(__float2bfloat16_rn(gxv[qg]));
+                        oi[qg * A.H] = bits;
+                        if (kT8) pk[qg][(L - 1 - i) >> 1] |= (unsigned)bits << (16 * ((L - 1 - i) & 1));
                         gbv[qg] += gxv[qg];
                     }
                 } else {
@@ -335,6 +342,16 @@ __global__ void __launch_bounds__(kThreads, 2)
         if (BF && A.gbias) {
 #pragma unroll
             for (int qg = 0; qg < 3; ++qg) atomicAdd(A.gbias + qg * A.H + h, gbv[qg]);
+        }
+        if (kT8 && A.gxbt && t_lo + rbase + L <= A.T) {
+            // row q H + h of the transpose, columns b T + t_lo + rbase .. + 7: 16-byte aligned
+            // (T is a multiple of 8, so an 8-step run lies wholly inside the sequence or
+            // wholly past its end)
+            const size_t M = (size_t)A.B * A.T, col = (size_t)b * A.T + t_lo + rbase;
+#pragma unroll
+            for (int qg = 0; qg < 3; ++qg)
+                *reinterpret_cast<uint4 *>(A.gxbt + (size_t)(qg * A.H + h) * M + col) =
+                    make_uint4(pk[qg][0], pk[qg][1], pk[qg][2], pk[qg][3]);
         }
         // this warp is done with the stage; the last warp to finish refills it with the
         // tile NST places ahead (acquire-release add on the counter)
@@ -411,6 +428,10 @@ template <class Cell, int L, bool BF> int choose(Plan *plan, int num_sms, long B
 
 }  // namespace
 
+// The bf16 variant's transposed copy: ParaGRU (8 steps per thread), whole 8-step runs
+// of every sequence 16-byte aligned in the transpose's rows (T % 8 == 0).
+bool adjoint_wide_writes_transpose(const AdjointReq &r) { return r.cell == 0 && r.out_bf16 && r.T % 8 == 0; }
+
 // H % 32 == 0 and a shared-memory gradient table that fits; 1: not covered.
 int adjoint_wide_plan(const AdjointReq &r, int num_sms, Plan *plan) {
     const int S = r.cell == 1 ? 2 : 1;
@@ -474,6 +495,7 @@ cudaError_t adjoint_wide_launch(const AdjointReq &r, const Plan &plan, const Wor
     A.g = r.g;
     A.gx = r.grad_xproj;
     A.gxb = r.grad_xproj_bf16;
+    A.gxbt = r.grad_xproj_bf16_t;
     A.gbias = r.grad_bias;
     A.gp = r.grad_params;
     A.gh0 = r.grad_h0;

@@ -307,9 +307,13 @@ int pararnn_layer_backward(pararnn_ctx *ctx, const float *xproj, const pararnn_p
     const size_t pbytes = prn::proj_bwd_scratch_bytes(PARARNN_BF16, M, K, N);
     int rc = ensure_scratch(ctx, pbytes + (wide ? (size_t)M * N * sizeof(float) : 0));
     if (rc) return rc;
+    bool have_gbt = false;
     if (wide == 0) {
         r.grad_xproj_bf16 = prn::proj_bwd_gb(ctx->scratch, M, N);
         r.grad_bias = grad_bias;
+        // ParaGRU: the adjoint also writes the transposed copy that grad_W's product reads
+        have_gbt = grad_W && prn::adjoint_wide_writes_transpose(r);
+        if (have_gbt) r.grad_xproj_bf16_t = prn::proj_bwd_gbt(ctx->scratch, M, N);
     } else {
         r.out_bf16 = false;
         r.grad_xproj = reinterpret_cast<float *>(static_cast<char *>(ctx->scratch) + pbytes);
@@ -326,8 +330,8 @@ int pararnn_layer_backward(pararnn_ctx *ctx, const float *xproj, const pararnn_p
     if ((rc = cuda_rc(prn::adjoint_launch(r, plan, w, ctx->dbg, ctx->stream)))) return rc;
     int l = 0;
     if (wide == 0)
-        rc = cuda_rc(prn::proj_bwd_from_bf16_launch(x, W, grad_x, grad_W, M, K, N, ctx->scratch, ctx->num_sms,
-                                                    ctx->stream, &l, ctx->sticky));
+        rc = cuda_rc(prn::proj_bwd_from_bf16_launch(x, W, grad_x, grad_W, M, K, N, have_gbt, ctx->scratch,
+                                                    ctx->num_sms, ctx->stream, &l, ctx->sticky));
     else
         rc = cuda_rc(prn::proj_bwd_launch(PARARNN_BF16, r.grad_xproj, x, W, grad_x, grad_W, grad_bias, M, K, N,
                                           ctx->scratch, ctx->num_sms, ctx->stream, &l, ctx->sticky));

@@ -123,8 +123,12 @@ struct AdjointReq {
     // TMA-fed tiles only (H % 32 == 0)
     bool out_bf16 = false;
     unsigned short *grad_xproj_bf16 = nullptr;
+    // and its transpose [3 H][B T] (ParaGRU tiles of 8 steps per thread, T % 8 == 0); null: none
+    unsigned short *grad_xproj_bf16_t = nullptr;
     float *grad_bias = nullptr;
 };
+// Whether the wide adjoint's bf16 variant writes the transposed copy for this shape.
+bool adjoint_wide_writes_transpose(const AdjointReq &r);
 int adjoint_plan(const AdjointReq &r, int num_sms, Plan *plan);
 // TMA-fed tiles for H % 32 == 0 (adjoint_wide.cu); 1: shape not covered
 int adjoint_wide_plan(const AdjointReq &r, int num_sms, Plan *plan);
@@ -149,9 +153,12 @@ int proj_bwd_check(int x_dtype, int M, int K, int N);
 size_t proj_bwd_scratch_bytes(int x_dtype, int M, int K, int N);
 // The bf16 path from a bf16 grad_xproj that the caller wrote at proj_bwd_gb(scratch, M, N)
 // (no fp32 copy, no bias sums): grad_x and grad_W only.
+// have_gbt: the transposed copy is there too (proj_bwd_gbt(scratch, M, N)).
 unsigned short *proj_bwd_gb(void *scratch, int M, int N);
+unsigned short *proj_bwd_gbt(void *scratch, int M, int N);
 cudaError_t proj_bwd_from_bf16_launch(const void *x, const void *W, float *grad_x, float *grad_W, int M, int K, int N,
-                                      void *scratch, int num_sms, cudaStream_t st, int *launches, int *sticky);
+                                      bool have_gbt, void *scratch, int num_sms, cudaStream_t st, int *launches,
+                                      int *sticky);
 cudaError_t proj_bwd_launch(int x_dtype, const float *gx, const void *x, const void *W, float *grad_x, float *grad_W,
                             float *grad_bias, int M, int K, int N, void *scratch, int num_sms, cudaStream_t st,
                             int *launches, int *sticky);

@@ -308,11 +308,14 @@ unsigned short *proj_bwd_gb(void *scratch, int M, int N) {
                                               up256((size_t)row_blocks(M) * N * sizeof(float)));
 }
 
+unsigned short *proj_bwd_gbt(void *scratch, int M, int N) { return proj_bwd_gb(scratch, M, N) + up256((size_t)M * N * 2) / 2; }
+
 cudaError_t proj_bwd_from_bf16_launch(const void *x, const void *W, float *grad_x, float *grad_W, int M, int K, int N,
-                                      void *scratch, int num_sms, cudaStream_t st, int *launches, int *sticky) {
+                                      bool have_gbt, void *scratch, int num_sms, cudaStream_t st, int *launches,
+                                      int *sticky) {
     *launches = 0;
-    unsigned short *gb = proj_bwd_gb(scratch, M, N), *gbt = gb + up256((size_t)M * N * 2) / 2;
-    if (grad_W) {
+    unsigned short *gb = proj_bwd_gb(scratch, M, N), *gbt = proj_bwd_gbt(scratch, M, N);
+    if (grad_W && !have_gbt) {
         transpose_u16(gb, gbt, M, N, st);
         ++*launches;
     }

@@ -905,7 +905,7 @@ __device__ __forceinline__ void dense_scan_body(const DScanArgs &A, DScanSmem<N>
 }
 
 template <int N>
-__global__ void __launch_bounds__(kThreads, 2) dense_scan_kernel(const DScanArgs A) {
+__global__ void __launch_bounds__(kThreads, 3) dense_scan_kernel(const DScanArgs A) {
     extern __shared__ __align__(16) unsigned char smraw[];
     DScanSmem<N> &sm = *reinterpret_cast<DScanSmem<N> *>(smraw);
     __shared__ int s_fail;

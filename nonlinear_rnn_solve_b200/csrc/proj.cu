@@ -34,6 +34,11 @@ constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
 constexpr int A_BYTES = BM * BK * 2, B_BYTES = BN * BK * 2, STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int TMEM_COLS = 256;
 constexpr int THREADS = 320;  // TMA warp, MMA warp, 8 epilogue warps
+// The bias is copied into shared memory after the stage ring when it has at most this
+// many entries (the ring leaves about 34 KB of the 227 KB): the epilogue then reads it as
+// shared-memory broadcasts instead of global loads that the output stream keeps evicting
+// from L1.
+constexpr int BIAS_SMEM = 8192;
 constexpr unsigned long long WAIT_NS = 2000000000ull;
 
 __device__ __forceinline__ unsigned smem_u32(const void *p) { return (unsigned)__cvta_generic_to_shared(p); }
@@ -120,6 +125,10 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int nitems = ntiles * ksplit;
     // 32-byte vector stores need 32-byte aligned rows
     const bool vec8 = (N & 7) == 0 && ((uintptr_t)y & 31) == 0;
+    const bool bias_sm = bias && N <= BIAS_SMEM;
+    float *const bias_s = reinterpret_cast<float *>(smem + STAGES * STAGE_BYTES);  // [N] when bias_sm
+    if (bias_sm)
+        for (int i = threadIdx.x; i < N; i += THREADS) bias_s[i] = __ldg(bias + i);
 
     if (threadIdx.x == 0) {
         abort_flag = 0;
@@ -237,8 +246,14 @@ __global__ void __launch_bounds__(THREADS, 1)
                     for (int j = 0; j < 8; ++j) w[j] = v[c + j];
                     if (bias) {
                         if (full) {
-                            const float4 b0 = __ldg(reinterpret_cast<const float4 *>(bias + col));
-                            const float4 b1 = __ldg(reinterpret_cast<const float4 *>(bias + col + 4));
+                            float4 b0, b1;
+                            if (bias_sm) {  // 16-byte aligned: the ring is 1024-byte aligned, col % 8 == 0
+                                b0 = *reinterpret_cast<const float4 *>(bias_s + col);
+                                b1 = *reinterpret_cast<const float4 *>(bias_s + col + 4);
+                            } else {
+                                b0 = __ldg(reinterpret_cast<const float4 *>(bias + col));
+                                b1 = __ldg(reinterpret_cast<const float4 *>(bias + col + 4));
+                            }
                             w[0] += b0.x, w[1] += b0.y, w[2] += b0.z, w[3] += b0.w;
                             w[4] += b1.x, w[5] += b1.y, w[6] += b1.z, w[7] += b1.w;
                         } else {
@@ -410,8 +425,12 @@ cudaError_t proj_launch_split(int x_dtype, const void *x, const void *W, const f
     }
     CUtensorMap ta, tb;
     if (!make_map(&ta, x, M, K, gemm::BM) || !make_map(&tb, W, N, K, gemm::BN)) return cudaErrorInvalidValue;
-    const int smem = gemm::STAGES * gemm::STAGE_BYTES + 1024;
-    cudaError_t e = cudaFuncSetAttribute(gemm::proj_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    // the stage ring, its 1024-byte alignment slack and the bias table (when it is used)
+    const int smem_max = gemm::STAGES * gemm::STAGE_BYTES + 1024 + gemm::BIAS_SMEM * (int)sizeof(float);
+    const int smem = gemm::STAGES * gemm::STAGE_BYTES + 1024 +
+                     ((bias && N <= gemm::BIAS_SMEM) ? N * (int)sizeof(float) : 0);
+    cudaError_t e =
+        cudaFuncSetAttribute(gemm::proj_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_max);
     if (e != cudaSuccess) return e;
     int dev = 0, sms = 0;
     if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;

@@ -13,10 +13,12 @@
 // product reads the previous iterate's state rows from shared memory), composes them, and
 // the warp scans its 32 lanes with shuffles: no CTA barrier in the scan.  The carry
 // entering the tile comes from the tile's own evaluation of the 128 steps before it (the
-// halo): the quasi-Jacobian is contractive here, and when the composed map of those steps
-// has a matrix part that is exactly zero in fp32 it is a constant whose value is the
-// carry (the same value the scan would carry in, up to rounding order).  Otherwise the
-// warp waits (bounded) for the predecessor tile's published value of its unit.
+// halo): the quasi-Jacobian is contractive here, so the composed map of those steps,
+// delta -> a delta + d, has a tiny matrix part a, and when |a| <= 2^-40 its offset d is
+// taken as the carry: the dropped term a delta is at most 2^-40 times the delta entering
+// the halo, far below the fp32 resolution of the states it updates (with a = 0 exactly,
+// d is the value the scan would carry in, up to rounding order).  Otherwise the warp waits
+// (bounded) for the predecessor tile's published value of its unit.
 //
 // Data movement is by bulk copies (cp.async.bulk, no multicast), one per 16-row segment,
 // the issue shared by all warps: a tile's state and input rows arrive in padded shared-memory segments
@@ -304,7 +306,7 @@ __device__ __forceinline__ void q8_tile(const Q8Args &A, const Q8Unit &U, const 
             if (v + off < 32) eh = compose(eh, o);
         }
         const float ha = __shfl_sync(0xffffffffu, eh.a, 0), hd = __shfl_sync(0xffffffffu, eh.d, 0);
-        if (ha == 0.f) {
+        if (fabsf(ha) <= 0x1p-40f) {  // the halo's map is a constant up to 2^-40 |delta|
             known = true;
             carry = hd;
         }

@@ -1,9 +1,9 @@
 """GPU parity of the two ways a long ParaGRU tile (H = 1, raw inputs) gets its carry.
 
-A tile evaluates the 255 steps before it itself; when their composed map has an
-exactly zero Jacobian part it is a constant, and that constant is the carry (no
-predecessor is read).  Otherwise the tile takes the carry from the decoupled
-look-back.  Both must give the oracle's Newton iteration count and states within
+A tile evaluates the 63 steps before it itself; when their composed map's Jacobian
+part is at most 2^-40 in magnitude its offset is the carry (no predecessor is read; the
+dropped term is at most 2^-40 times the delta entering the halo).  Otherwise the tile
+takes the carry from the decoupled look-back.  Both must give the oracle's Newton iteration count and states within
 1e-4, on a contractive case (halo constant almost everywhere) and on a near-identity
 case (z-gate bias -8: Jacobians near 1, halo never constant, look-back only).
 Shapes: several tiles with a ragged last one; T a multiple of 32 so the inputs are

@@ -173,7 +173,14 @@ int pararnn_input_proj_backward(pararnn_ctx *ctx, const float *grad_xproj, const
  *   final_delta_out  device float or NULL: delta of the last iteration
  *   residual_out     device float or NULL: max |h_t - f(h_{t-1}, x_t)| at the result
  * Supported: GRU and LSTM any H; tanh RNN with n <= 64 (EUNSUPPORTED above), every
- * solver for every cell.  B, T >= 1. */
+ * solver for every cell.  B, T >= 1.
+ * Carries across tiles: the long-sequence tiles (ParaGRU with H = 1 and raw inputs; the
+ * tanh RNN at n = 8 with inputs of width 4, quasi) first evaluate the steps just before
+ * them (63 and 128) and, when every entry of those steps' composed Jacobian is at most
+ * 2^-40 in magnitude, take that map's offset as the carry; the neglected term is at most
+ * 2^-40 times the update entering those steps.  Otherwise, and in every other layout,
+ * the carry is the scan's own (a look-back over the preceding tiles).  Debug knob 5
+ * turns the first way off. */
 int pararnn_newton_forward(pararnn_ctx *ctx, const float *xproj, const pararnn_params *p,
                            const float *h0, float *h_out, int max_iters, float tol,
                            int *iters_out, float *final_delta_out, float *residual_out);
